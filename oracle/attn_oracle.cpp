@@ -1,0 +1,410 @@
+// Exact-attention oracle: plain, slow, fp64, CPU only.
+//
+// TEST INFRASTRUCTURE. Only the test suite, the package smoke check and the
+// benchmark's CPU-baseline leg may load this code. It shares nothing with the
+// CUDA library (no header, helper, table or constant): it is the definition of
+// the operation written out, so a reader can check it against the sources by eye.
+//
+// Sources, cited by title and section:
+//   [jsqmd]   "From GPU memory access to code: how FlashAttention makes large-model
+//             training 3x faster" (jsqmd.com news 754333)
+//   [intelli] "FlashAttention optimisation: breaking the performance bottleneck of
+//             standard attention" (intelliparadigm.com)
+//   [yunthe]  "Flash Attention-2: acceleration principle and GPU memory optimisation
+//             in deployment" (yunthe.com)
+//   [jos]     "A survey of key techniques of large language model pre-training
+//             systems", Journal of Software 2026(1), p.218
+//
+// What it computes (per batch b and head h, with X[b,h] an N x d row-major matrix):
+//   S = scale * Q K^T          [jos] attention definition (S = QK^T, P = Softmax(S),
+//                              O = PV); the scaling by 1/sqrt(d) is [intelli] section 1
+//                              step 2 and [yunthe] "standard attention" section; the
+//                              scale is an argument here.
+//   S[i][j] = -inf if causal and j > i   [yunthe] "causal mask" troubleshooting item
+//                              (is_causal=True); the key at the query's own position
+//                              is kept.
+//   m_i = max_j S[i][j]        [jsqmd] section 2.1, safe softmax
+//   P[i][j] = exp(S[i][j] - m_i) / sum_j exp(S[i][j] - m_i)
+//   O = P V
+//   L_i = m_i + ln sum_j exp(S[i][j] - m_i)   natural-log log-sum-exp of the scaled
+//                              logits: the normalisation statistics of [intelli]
+//                              section 4.1, kept in log space as [intelli] 3.3 says.
+//
+// Backward, for the scalar loss l = <dO, O> (the sources only say "recompute",
+// [intelli] section 4.2; the gradient is plain calculus of the definition above):
+//   dV = P^T dO
+//   dP = dO V^T
+//   D_i = sum_j P[i][j] dP[i][j]   (equal to sum_k dO[i][k] O[i][k])
+//   dS = P o (dP - D)              (softmax Jacobian, row by row)
+//   dQ = scale * dS K
+//   dK = scale * dS^T Q
+//
+// Every function materialises what the definition names (S, P, dP, dS) for one
+// head, or one row, at a time; there is no blocking, no fusion and no online
+// rescaling here. Parallelism is OpenMP over independent rows, which does not
+// change the order of any sum within a row.
+//
+// Layout: all matrices contiguous, row-major [B, H, N, d]; L and D are [B, H, N].
+// Every entry point returns 0 on success, nonzero on a bad argument or a failed
+// allocation.
+
+#include <cmath>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <limits>
+#include <vector>
+
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+namespace {
+
+const double kNegInf = -std::numeric_limits<double>::infinity();
+
+bool bad_shape(int64_t B, int64_t H, int64_t N, int64_t d) {
+  return B < 0 || H < 0 || N < 0 || d <= 0;
+}
+
+// One row of scaled, masked logits: s[j] = scale * <q_i, k_j>, -inf above the
+// diagonal when causal.
+void logits_row(const double* q, const double* K, int64_t N, int64_t d, double scale,
+                int causal, int64_t i, double* s) {
+  for (int64_t j = 0; j < N; ++j) {
+    if (causal && j > i) {
+      s[j] = kNegInf;
+      continue;
+    }
+    const double* k = K + j * d;
+    double acc = 0.0;
+    for (int64_t c = 0; c < d; ++c) acc += q[c] * k[c];
+    s[j] = scale * acc;
+  }
+}
+
+// Safe softmax of one row ([jsqmd] section 2.1): subtract the row max,
+// exponentiate, divide by the sum. Writes p and returns the natural-log
+// log-sum-exp m + ln(sum). A row with every entry masked gets p = 0 and -inf.
+double safe_softmax_row(const double* s, int64_t N, double* p) {
+  double m = kNegInf;
+  for (int64_t j = 0; j < N; ++j) m = s[j] > m ? s[j] : m;
+  if (m == kNegInf) {
+    for (int64_t j = 0; j < N; ++j) p[j] = 0.0;
+    return kNegInf;
+  }
+  double sum = 0.0;
+  for (int64_t j = 0; j < N; ++j) {
+    p[j] = std::exp(s[j] - m);
+    sum += p[j];
+  }
+  for (int64_t j = 0; j < N; ++j) p[j] /= sum;
+  return m + std::log(sum);
+}
+
+}  // namespace
+
+extern "C" {
+
+// Number of OpenMP threads the oracle will use (1 without OpenMP).
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}
+
+void oracle_set_num_threads(int n) {
+#ifdef _OPENMP
+  if (n > 0) omp_set_num_threads(n);
+#else
+  (void)n;
+#endif
+}
+
+// The row-stochastic matrix P = softmax(S) of one head, N x N, into P.
+int oracle_attention_probs(const double* Q, const double* K, int64_t N, int64_t d,
+                           double scale, int causal, double* P) {
+  if (bad_shape(1, 1, N, d) || !Q || !K || !P) return 1;
+#pragma omp parallel
+  {
+    std::vector<double> s(N);
+#pragma omp for schedule(static)
+    for (int64_t i = 0; i < N; ++i) {
+      logits_row(Q + i * d, K, N, d, scale, causal, i, s.data());
+      safe_softmax_row(s.data(), N, P + i * N);
+    }
+  }
+  return 0;
+}
+
+// Full forward: O [B,H,N,d] and L [B,H,N]. Materialises S and P (N x N) of one
+// head at a time.
+int oracle_attention_forward(const double* Q, const double* K, const double* V, int64_t B,
+                             int64_t H, int64_t N, int64_t d, double scale, int causal,
+                             double* O, double* L) {
+  if (bad_shape(B, H, N, d) || !Q || !K || !V || !O || !L) return 1;
+  if (N == 0) return 0;
+  std::vector<double> P;
+  try {
+    P.resize(static_cast<size_t>(N) * N);
+  } catch (...) {
+    return 2;
+  }
+  for (int64_t bh = 0; bh < B * H; ++bh) {
+    const double* q = Q + bh * N * d;
+    const double* k = K + bh * N * d;
+    const double* v = V + bh * N * d;
+    double* o = O + bh * N * d;
+    double* l = L + bh * N;
+    // S then P, row by row (P overwrites S in place).
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < N; ++i) {
+      double* row = P.data() + i * N;
+      logits_row(q + i * d, k, N, d, scale, causal, i, row);
+      std::vector<double> s(row, row + N);
+      l[i] = safe_softmax_row(s.data(), N, row);
+    }
+    // O = P V
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < N; ++i) {
+      const double* p = P.data() + i * N;
+      double* oi = o + i * d;
+      for (int64_t c = 0; c < d; ++c) oi[c] = 0.0;
+      for (int64_t j = 0; j < N; ++j) {
+        const double pij = p[j];
+        const double* vj = v + j * d;
+        for (int64_t c = 0; c < d; ++c) oi[c] += pij * vj[c];
+      }
+    }
+  }
+  return 0;
+}
+
+// Full backward by calculus: dQ, dK, dV [B,H,N,d] and D [B,H,N] (D = rowsum(P o dP)).
+// Materialises P, dP and dS (N x N) of one head at a time. If Dcheck is non-null it
+// receives, per row, sum_k dO[i][k] * O[i][k] computed from O = P V, the second
+// way of forming D; the two must agree.
+int oracle_attention_backward(const double* Q, const double* K, const double* V,
+                              const double* dO, int64_t B, int64_t H, int64_t N, int64_t d,
+                              double scale, int causal, double* dQ, double* dK, double* dV,
+                              double* D, double* Dcheck) {
+  if (bad_shape(B, H, N, d) || !Q || !K || !V || !dO || !dQ || !dK || !dV || !D) return 1;
+  if (N == 0) return 0;
+  std::vector<double> P, dS;
+  try {
+    P.resize(static_cast<size_t>(N) * N);
+    dS.resize(static_cast<size_t>(N) * N);
+  } catch (...) {
+    return 2;
+  }
+  for (int64_t bh = 0; bh < B * H; ++bh) {
+    const double* q = Q + bh * N * d;
+    const double* k = K + bh * N * d;
+    const double* v = V + bh * N * d;
+    const double* go = dO + bh * N * d;
+    double* gq = dQ + bh * N * d;
+    double* gk = dK + bh * N * d;
+    double* gv = dV + bh * N * d;
+    double* Dh = D + bh * N;
+    // P = softmax(S)
+#pragma omp parallel
+    {
+      std::vector<double> s(N);
+#pragma omp for schedule(static)
+      for (int64_t i = 0; i < N; ++i) {
+        logits_row(q + i * d, k, N, d, scale, causal, i, s.data());
+        safe_softmax_row(s.data(), N, P.data() + i * N);
+      }
+    }
+    // dP = dO V^T, D_i = sum_j P_ij dP_ij, dS = P o (dP - D); dS holds dP first.
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < N; ++i) {
+      const double* goi = go + i * d;
+      double* dsi = dS.data() + i * N;
+      const double* pi = P.data() + i * N;
+      double Di = 0.0;
+      for (int64_t j = 0; j < N; ++j) {
+        const double* vj = v + j * d;
+        double acc = 0.0;
+        for (int64_t c = 0; c < d; ++c) acc += goi[c] * vj[c];
+        dsi[j] = acc;
+        Di += pi[j] * acc;
+      }
+      Dh[i] = Di;
+      for (int64_t j = 0; j < N; ++j) dsi[j] = pi[j] * (dsi[j] - Di);
+      if (Dcheck) {
+        // O_i = sum_j P_ij V_j, then sum_k dO_ik O_ik
+        double Dc = 0.0;
+        for (int64_t c = 0; c < d; ++c) {
+          double oic = 0.0;
+          for (int64_t j = 0; j < N; ++j) oic += pi[j] * v[j * d + c];
+          Dc += goi[c] * oic;
+        }
+        Dcheck[bh * N + i] = Dc;
+      }
+    }
+    // dQ = scale * dS K
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < N; ++i) {
+      const double* dsi = dS.data() + i * N;
+      double* gqi = gq + i * d;
+      for (int64_t c = 0; c < d; ++c) gqi[c] = 0.0;
+      for (int64_t j = 0; j < N; ++j) {
+        const double* kj = k + j * d;
+        for (int64_t c = 0; c < d; ++c) gqi[c] += dsi[j] * kj[c];
+      }
+      for (int64_t c = 0; c < d; ++c) gqi[c] *= scale;
+    }
+    // dK = scale * dS^T Q, dV = P^T dO
+#pragma omp parallel for schedule(static)
+    for (int64_t j = 0; j < N; ++j) {
+      double* gkj = gk + j * d;
+      double* gvj = gv + j * d;
+      for (int64_t c = 0; c < d; ++c) {
+        gkj[c] = 0.0;
+        gvj[c] = 0.0;
+      }
+      for (int64_t i = 0; i < N; ++i) {
+        const double ds = dS[i * N + j];
+        const double p = P[i * N + j];
+        const double* qi = q + i * d;
+        const double* goi = go + i * d;
+        for (int64_t c = 0; c < d; ++c) {
+          gkj[c] += ds * qi[c];
+          gvj[c] += p * goi[c];
+        }
+      }
+      for (int64_t c = 0; c < d; ++c) gkj[c] *= scale;
+    }
+  }
+  return 0;
+}
+
+// Forward restricted to selected query rows: for r in [0, R), row rows[r] of head
+// heads[r] (head index bh = b * H + h). Writes O_r [R, d] and L_r [R]. The same
+// definition as oracle_attention_forward, one materialised row of S and P each.
+int oracle_attention_forward_rows(const double* Q, const double* K, const double* V,
+                                  int64_t B, int64_t H, int64_t N, int64_t d, double scale,
+                                  int causal, int64_t R, const int64_t* heads,
+                                  const int64_t* rows, double* O_r, double* L_r) {
+  if (bad_shape(B, H, N, d) || R < 0 || (R > 0 && (!heads || !rows || !O_r || !L_r)))
+    return 1;
+  for (int64_t r = 0; r < R; ++r)
+    if (heads[r] < 0 || heads[r] >= B * H || rows[r] < 0 || rows[r] >= N) return 1;
+#pragma omp parallel
+  {
+    std::vector<double> s(N), p(N);
+#pragma omp for schedule(dynamic, 4)
+    for (int64_t r = 0; r < R; ++r) {
+      const int64_t bh = heads[r], i = rows[r];
+      const double* k = K + bh * N * d;
+      const double* v = V + bh * N * d;
+      logits_row(Q + (bh * N + i) * d, k, N, d, scale, causal, i, s.data());
+      L_r[r] = safe_softmax_row(s.data(), N, p.data());
+      double* o = O_r + r * d;
+      for (int64_t c = 0; c < d; ++c) o[c] = 0.0;
+      for (int64_t j = 0; j < N; ++j)
+        for (int64_t c = 0; c < d; ++c) o[c] += p[j] * v[j * d + c];
+    }
+  }
+  return 0;
+}
+
+// dQ restricted to selected query rows (same selection convention as
+// oracle_attention_forward_rows). Row i needs only its own P row and dP row:
+// D_i = sum_j P_ij dP_ij, dQ_i = scale * sum_j P_ij (dP_ij - D_i) K_j.
+int oracle_attention_backward_dq_rows(const double* Q, const double* K, const double* V,
+                                      const double* dO, int64_t B, int64_t H, int64_t N,
+                                      int64_t d, double scale, int causal, int64_t R,
+                                      const int64_t* heads, const int64_t* rows,
+                                      double* dQ_r, double* D_r) {
+  if (bad_shape(B, H, N, d) || R < 0 || (R > 0 && (!heads || !rows || !dQ_r || !D_r)))
+    return 1;
+  for (int64_t r = 0; r < R; ++r)
+    if (heads[r] < 0 || heads[r] >= B * H || rows[r] < 0 || rows[r] >= N) return 1;
+#pragma omp parallel
+  {
+    std::vector<double> s(N), p(N), dp(N);
+#pragma omp for schedule(dynamic, 4)
+    for (int64_t r = 0; r < R; ++r) {
+      const int64_t bh = heads[r], i = rows[r];
+      const double* k = K + bh * N * d;
+      const double* v = V + bh * N * d;
+      const double* goi = dO + (bh * N + i) * d;
+      logits_row(Q + (bh * N + i) * d, k, N, d, scale, causal, i, s.data());
+      safe_softmax_row(s.data(), N, p.data());
+      double Di = 0.0;
+      for (int64_t j = 0; j < N; ++j) {
+        double acc = 0.0;
+        for (int64_t c = 0; c < d; ++c) acc += goi[c] * v[j * d + c];
+        dp[j] = acc;
+        Di += p[j] * acc;
+      }
+      D_r[r] = Di;
+      double* g = dQ_r + r * d;
+      for (int64_t c = 0; c < d; ++c) g[c] = 0.0;
+      for (int64_t j = 0; j < N; ++j) {
+        const double ds = p[j] * (dp[j] - Di);
+        for (int64_t c = 0; c < d; ++c) g[c] += ds * k[j * d + c];
+      }
+      for (int64_t c = 0; c < d; ++c) g[c] *= scale;
+    }
+  }
+  return 0;
+}
+
+// dK and dV restricted to selected key rows j of one head bh. Column j of P needs
+// every row's normaliser and every row's D, so the caller passes L [N] and D [N]
+// of that head as this oracle computed them (oracle_attention_forward_rows over all
+// rows for L; oracle_attention_backward_dq_rows for D):
+//   P_ij = exp(S_ij - L_i), dS_ij = P_ij (dO_i . V_j - D_i),
+//   dV_j = sum_i P_ij dO_i,  dK_j = scale * sum_i dS_ij Q_i.
+int oracle_attention_backward_dkdv_rows(const double* Q, const double* K, const double* V,
+                                        const double* dO, int64_t B, int64_t H, int64_t N,
+                                        int64_t d, double scale, int causal, int64_t bh,
+                                        const double* L, const double* D, int64_t R,
+                                        const int64_t* keys, double* dK_r, double* dV_r) {
+  if (bad_shape(B, H, N, d) || bh < 0 || bh >= B * H || R < 0 || !L || !D ||
+      (R > 0 && (!keys || !dK_r || !dV_r)))
+    return 1;
+  for (int64_t r = 0; r < R; ++r)
+    if (keys[r] < 0 || keys[r] >= N) return 1;
+  const double* q = Q + bh * N * d;
+  const double* k = K + bh * N * d;
+  const double* v = V + bh * N * d;
+  const double* go = dO + bh * N * d;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t r = 0; r < R; ++r) {
+    const int64_t j = keys[r];
+    const double* kj = k + j * d;
+    const double* vj = v + j * d;
+    double* gk = dK_r + r * d;
+    double* gv = dV_r + r * d;
+    for (int64_t c = 0; c < d; ++c) {
+      gk[c] = 0.0;
+      gv[c] = 0.0;
+    }
+    for (int64_t i = 0; i < N; ++i) {
+      if (causal && j > i) continue;
+      const double* qi = q + i * d;
+      const double* goi = go + i * d;
+      double sij = 0.0, dpij = 0.0;
+      for (int64_t c = 0; c < d; ++c) {
+        sij += qi[c] * kj[c];
+        dpij += goi[c] * vj[c];
+      }
+      const double pij = std::exp(scale * sij - L[i]);
+      const double dsij = pij * (dpij - D[i]);
+      for (int64_t c = 0; c < d; ++c) {
+        gv[c] += pij * goi[c];
+        gk[c] += dsij * qi[c];
+      }
+    }
+    for (int64_t c = 0; c < d; ++c) gk[c] *= scale;
+  }
+  return 0;
+}
+
+}  // extern "C"

@@ -1,0 +1,326 @@
+"""Pins of the fp64 oracle against facts that do not come from the oracle itself.
+
+Each ``pin_*`` takes an oracle object (``oracle.Oracle``) and raises AssertionError
+when the oracle disagrees with:
+  * the two-block softmax decomposition m = max(m1, m2),
+    l = e^(m1-m) l1 + e^(m2-m) l2 of "A survey of key techniques of large language
+    model pre-training systems" (Journal of Software 2026(1), p.218), and the
+    two-pass tiled softmax of "From GPU memory access to code: how FlashAttention
+    makes large-model training 3x faster", section 2.1;
+  * closed forms (rows of P sum to 1; a constant key gives the mean of V; one key
+    gives O = V; a two-level logit pattern has an exact weighted mean);
+  * the blockwise online loop of "Flash Attention-2: acceleration principle and
+    GPU memory optimisation in deployment" (its "Flash Attention-2 blockwise
+    computation" listing, restated here in numpy), which that page says equals
+    standard attention exactly;
+  * a library routine computing the same function (torch fp64 CPU
+    scaled_dot_product_attention and its autograd backward);
+  * central finite differences of the loss <dO, O>;
+  * invariants of the gradient (sum_j dK_j = 0, sum_i dV_i = sum_i dO_i, D two ways).
+
+The same pins run against variants of the oracle with a planted mistake
+(tests/test_oracle_mutants.py); each such variant must fail at least one pin.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+
+import numpy as np
+import torch
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _close(a, b, tol, what):
+    a = np.asarray(a, dtype=np.float64)
+    b = np.asarray(b, dtype=np.float64)
+    assert a.shape == b.shape, f"{what}: shape {a.shape} != {b.shape}"
+    assert np.all(np.isfinite(a)), f"{what}: non-finite values"
+    err = float(np.max(np.abs(a - b))) if a.size else 0.0
+    assert err <= tol, f"{what}: max abs error {err:.3e} > {tol:.1e}"
+
+
+# --------------------------------------------------------------------------- softmax
+
+
+def pin_two_block_decomposition(orc):
+    """The oracle's softmax row equals the two-block decomposition and the two-pass
+    tiled softmax, for unequal splits and logits up to +-800 (where skipping the
+    max subtraction overflows fp64)."""
+    rng = _rng(11)
+    cases = [(7, 3, 1.0), (16, 1, 50.0), (33, 20, 300.0), (64, 63, 300.0), (9, 4, 800.0)]
+    for N, split, spread in cases:
+        x = rng.uniform(-spread, spread, N)
+        # d = 1, q = 1, k_j = x_j, scale = 1: every row's logits are exactly x.
+        q = np.ones((N, 1))
+        k = x.reshape(N, 1)
+        P = orc.probs(q, k, 1.0, False)
+        x1, x2 = x[:split], x[split:]
+        m1, m2 = x1.max(), x2.max()
+        f1, f2 = np.exp(x1 - m1), np.exp(x2 - m2)
+        l1, l2 = f1.sum(), f2.sum()
+        m = max(m1, m2)
+        f = np.concatenate([np.exp(m1 - m) * f1, np.exp(m2 - m) * f2])
+        l = np.exp(m1 - m) * l1 + np.exp(m2 - m) * l2
+        want = f / l
+        for i in (0, N // 2, N - 1):
+            _close(P[i], want, 1e-14, f"two-block softmax N={N} split={split}")
+        # two-pass tiled softmax: global max over blocks, then the sum, then divide
+        blocks = [x[a:a + 5] for a in range(0, N, 5)]
+        gmax = max(b.max() for b in blocks)
+        total = sum(np.exp(b - gmax).sum() for b in blocks)
+        tiled = np.concatenate([np.exp(b - gmax) / total for b in blocks])
+        _close(P[0], tiled, 1e-14, "two-pass tiled softmax")
+        # the log-sum-exp the forward returns is m + ln l of the decomposition
+        V = rng.standard_normal((1, 1, N, 1))
+        _, L = orc.forward(q.reshape(1, 1, N, 1), k.reshape(1, 1, N, 1), V, 1.0, False)
+        _close(L[0, 0], np.full(N, m + math.log(l)), 1e-12 * max(1.0, abs(m)),
+               "log-sum-exp from the decomposition")
+
+
+def pin_rows_sum_to_one(orc):
+    """Softmax = f / l: every row of P sums to 1; causal rows put no weight above
+    the diagonal and some weight on it."""
+    rng = _rng(12)
+    N, d = 50, 8
+    q = rng.standard_normal((N, d)) * 3
+    k = rng.standard_normal((N, d)) * 3
+    for causal in (False, True):
+        P = orc.probs(q, k, 0.5, causal)
+        _close(P.sum(axis=1), np.ones(N), 1e-12, "row sums")
+        assert np.all(P >= 0)
+        if causal:
+            assert np.all(np.triu(P, 1) == 0.0), "weight above the diagonal"
+            assert np.all(np.diag(P) > 0.0), "no weight on the diagonal"
+
+
+# --------------------------------------------------------------------------- forward
+
+
+def pin_constant_key(orc):
+    """All keys equal: P is uniform over the visible keys, so O_i is the mean of
+    V_0..V_{N-1} (causal: of V_0..V_i) and L_i = scale <q_i, k> + ln(count)."""
+    rng = _rng(13)
+    B, H, N, d = 2, 2, 24, 8
+    scale = 0.3
+    Q = rng.standard_normal((B, H, N, d))
+    k = rng.standard_normal((B, H, 1, d))
+    K = np.repeat(k, N, axis=2)
+    V = rng.standard_normal((B, H, N, d))
+    for causal in (False, True):
+        O, L = orc.forward(Q, K, V, scale, causal)
+        if causal:
+            counts = np.arange(1, N + 1, dtype=np.float64)
+            want_O = np.cumsum(V, axis=2) / counts[None, None, :, None]
+        else:
+            counts = np.full(N, float(N))
+            want_O = np.broadcast_to(V.mean(axis=2, keepdims=True), V.shape)
+        want_L = scale * np.einsum("bhnd,bhd->bhn", Q, k[:, :, 0, :]) + np.log(counts)
+        _close(O, want_O, 1e-12, f"constant key O (causal={causal})")
+        _close(L, want_L, 1e-12, f"constant key L (causal={causal})")
+
+
+def pin_single_key(orc):
+    """N = 1: O = V, L = scale <q, k>; the gradient is dQ = dK = 0, dV = dO."""
+    rng = _rng(14)
+    B, H, N, d = 3, 2, 1, 16
+    Q, K, V, dO = (rng.standard_normal((B, H, N, d)) for _ in range(4))
+    for causal in (False, True):
+        O, L = orc.forward(Q, K, V, 0.7, causal)
+        _close(O, V, 1e-15, "N=1 O")
+        _close(L, 0.7 * np.sum(Q * K, axis=-1), 1e-13, "N=1 L")
+        dQ, dK, dV, D = orc.backward(Q, K, V, dO, 0.7, causal)
+        _close(dQ, np.zeros_like(dQ), 1e-15, "N=1 dQ")
+        _close(dK, np.zeros_like(dK), 1e-15, "N=1 dK")
+        _close(dV, dO, 1e-15, "N=1 dV")
+
+
+def pin_two_level_logits(orc):
+    """Logits a on one key pi(i) per row and 0 elsewhere (pi a permutation):
+    O_i = (e^a V_pi(i) + sum_{j != pi(i)} V_j) / (e^a + N - 1), L_i = ln(e^a + N - 1)."""
+    rng = _rng(15)
+    N = 12
+    perm = rng.permutation(N)
+    V = rng.standard_normal((1, 1, N, N))  # the oracle takes one head width for Q, K, V
+    for a in (3.0, 60.0):
+        scale = 0.5
+        Q = np.zeros((1, 1, N, N))
+        Q[0, 0, np.arange(N), perm] = a / scale
+        K = np.eye(N).reshape(1, 1, N, N)
+        O, L = orc.forward(Q, K, V, scale, False)
+        total = V[0, 0].sum(axis=0)
+        ea = math.exp(a)
+        want = (ea * V[0, 0, perm] + (total[None, :] - V[0, 0, perm])) / (ea + N - 1)
+        _close(O[0, 0], want, 1e-13, f"two-level logits O (a={a})")
+        _close(L[0, 0], np.full(N, math.log(ea + N - 1)), 1e-13, f"two-level logits L (a={a})")
+
+
+def blockwise_forward(Q, K, V, scale, causal, Br, Bc):
+    """The blockwise online-softmax loop (outer loop over query blocks, inner over
+    key/value blocks, running max m and sum l, rescale by exp(m_old - m_new), divide
+    by l at the end), in fp64 numpy. Independent of the oracle's code."""
+    B, H, N, d = Q.shape
+    O = np.zeros_like(Q)
+    L = np.zeros((B, H, N))
+    for b in range(B):
+        for h in range(H):
+            for i0 in range(0, N, Br):
+                qi = Q[b, h, i0:i0 + Br]
+                r = qi.shape[0]
+                rows = np.arange(i0, i0 + r)
+                m = np.full(r, -np.inf)
+                l = np.zeros(r)
+                acc = np.zeros((r, d))
+                for j0 in range(0, N, Bc):
+                    if causal and j0 > rows[-1]:
+                        break
+                    kj = K[b, h, j0:j0 + Bc]
+                    vj = V[b, h, j0:j0 + Bc]
+                    s = (qi @ kj.T) * scale
+                    if causal:
+                        cols = np.arange(j0, j0 + kj.shape[0])
+                        s = np.where(cols[None, :] > rows[:, None], -np.inf, s)
+                    m_new = np.maximum(m, s.max(axis=1))
+                    p = np.exp(s - m_new[:, None])
+                    alpha = np.exp(m - m_new)
+                    l = l * alpha + p.sum(axis=1)
+                    acc = acc * alpha[:, None] + p @ vj
+                    m = m_new
+                O[b, h, i0:i0 + r] = acc / l[:, None]
+                L[b, h, i0:i0 + r] = m + np.log(l)
+    return O, L
+
+
+def pin_blockwise_loop(orc):
+    """The oracle equals the blockwise online loop (ragged last blocks, unequal
+    Br and Bc, causal and not) to 1e-12."""
+    rng = _rng(16)
+    B, H, N, d = 2, 3, 100, 16
+    Q, K, V = (rng.standard_normal((B, H, N, d)) * 2 for _ in range(3))
+    for causal in (False, True):
+        O, L = orc.forward(Q, K, V, 0.25, causal)
+        Ob, Lb = blockwise_forward(Q, K, V, 0.25, causal, Br=32, Bc=48)
+        _close(O, Ob, 1e-12, f"blockwise O (causal={causal})")
+        _close(L, Lb, 1e-12, f"blockwise L (causal={causal})")
+
+
+# --------------------------------------------------------------------------- library
+
+
+def pin_torch_sdpa(orc):
+    """fp64 torch SDPA on the CPU (forward and autograd backward) agrees to 1e-12."""
+    rng = _rng(17)
+    B, H, N, d = 2, 2, 40, 16
+    Q, K, V, dO = (rng.standard_normal((B, H, N, d)) for _ in range(4))
+    for causal in (False, True):
+        scale = 1.0 / math.sqrt(d)
+        O, L = orc.forward(Q, K, V, scale, causal)
+        qt, kt, vt = (torch.tensor(x, requires_grad=True) for x in (Q, K, V))
+        ot = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, is_causal=causal,
+                                                              scale=scale)
+        ot.backward(torch.tensor(dO))
+        _close(O, ot.detach().numpy(), 1e-12, "SDPA O")
+        # L against the library's logsumexp of the masked logits
+        s = torch.einsum("bhid,bhjd->bhij", torch.tensor(Q), torch.tensor(K)) * scale
+        if causal:
+            s = s.masked_fill(torch.triu(torch.ones(N, N, dtype=torch.bool), 1), -math.inf)
+        _close(L, torch.logsumexp(s, dim=-1).numpy(), 1e-12, "logsumexp L")
+        dQ, dK, dV, D = orc.backward(Q, K, V, dO, scale, causal)
+        _close(dQ, qt.grad.numpy(), 1e-12, "SDPA dQ")
+        _close(dK, kt.grad.numpy(), 1e-12, "SDPA dK")
+        _close(dV, vt.grad.numpy(), 1e-12, "SDPA dV")
+
+
+# --------------------------------------------------------------------------- backward
+
+
+def pin_finite_differences(orc):
+    """Central differences (h = 1e-6) of l = <dO, O> over every element of Q, K, V
+    at N <= 16, d <= 8, causal and not: relative error <= 1e-6 of max|grad|."""
+    rng = _rng(18)
+    for (N, d, causal) in ((16, 8, False), (13, 4, True), (5, 8, True)):
+        B, H = 1, 2
+        Q, K, V, dO = (rng.standard_normal((B, H, N, d)) for _ in range(4))
+        scale = 1.0 / math.sqrt(d)
+        dQ, dK, dV, _ = orc.backward(Q, K, V, dO, scale, causal)
+
+        def loss(q, k, v):
+            O, _ = orc.forward(q, k, v, scale, causal)
+            return float(np.sum(O * dO))
+
+        h = 1e-6
+        for which, grad in ((0, dQ), (1, dK), (2, dV)):
+            num = np.zeros_like(grad)
+            for idx in np.ndindex(*grad.shape):
+                args_p = [Q.copy(), K.copy(), V.copy()]
+                args_m = [Q.copy(), K.copy(), V.copy()]
+                args_p[which][idx] += h
+                args_m[which][idx] -= h
+                num[idx] = (loss(*args_p) - loss(*args_m)) / (2 * h)
+            ref = max(1e-3, float(np.max(np.abs(num))))
+            err = float(np.max(np.abs(num - grad)))
+            assert err <= 1e-6 * ref, (
+                f"finite differences of {'QKV'[which]} (N={N}, d={d}, causal={causal}): "
+                f"{err:.3e} > 1e-6 * {ref:.3e}")
+
+
+def pin_gradient_invariants(orc):
+    """Rows of dS sum to 0, so sum_j dK_j = 0; sum_i dV_i = sum_i dO_i (columns of
+    P^T sum to 1); D = rowsum(P o dP) equals rowsum(dO o O)."""
+    rng = _rng(19)
+    B, H, N, d = 2, 2, 48, 16
+    Q, K, V, dO = (rng.standard_normal((B, H, N, d)) * 1.5 for _ in range(4))
+    for causal in (False, True):
+        dQ, dK, dV, D, Dc = orc.backward(Q, K, V, dO, 0.25, causal, with_check=True)
+        _close(dK.sum(axis=2), np.zeros((B, H, d)), 1e-12 * N * max(1.0, np.abs(dK).max()),
+               "sum_j dK_j")
+        _close(dV.sum(axis=2), dO.sum(axis=2), 1e-12 * N, "sum_i dV_i")
+        _close(D, Dc, 1e-12 * max(1.0, np.abs(D).max()), "D two ways")
+        O, _ = orc.forward(Q, K, V, 0.25, causal)
+        _close(D, np.sum(dO * O, axis=-1), 1e-12 * max(1.0, np.abs(D).max()), "D = rowsum(dO o O)")
+
+
+# --------------------------------------------------------------------------- golden
+
+
+def pin_golden_fixtures(orc):
+    """Hand-worked examples stored under tests/golden/ (each with its derivation)."""
+    for name in sorted(os.listdir(GOLDEN)):
+        if not name.endswith(".json"):
+            continue
+        with open(os.path.join(GOLDEN, name)) as f:
+            fx = json.load(f)
+        env = {"math": math, "ln": math.log, "exp": math.exp}
+
+        def ev(x):
+            if isinstance(x, list):
+                return [ev(y) for y in x]
+            return float(eval(x, env)) if isinstance(x, str) else float(x)
+
+        for case in fx["cases"]:
+            Q = np.array(ev(case["Q"]), dtype=np.float64)[None, None]
+            K = np.array(ev(case["K"]), dtype=np.float64)[None, None]
+            V = np.array(ev(case["V"]), dtype=np.float64)[None, None]
+            O, L = orc.forward(Q, K, V, float(case["scale"]), bool(case["causal"]))
+            _close(O[0, 0], np.array(ev(case["O"])), 1e-13, f"{name}:{case['name']} O")
+            _close(L[0, 0], np.array(ev(case["L"])), 1e-13, f"{name}:{case['name']} L")
+
+
+ALL_PINS = [
+    pin_two_block_decomposition,
+    pin_rows_sum_to_one,
+    pin_constant_key,
+    pin_single_key,
+    pin_two_level_logits,
+    pin_blockwise_loop,
+    pin_torch_sdpa,
+    pin_finite_differences,
+    pin_gradient_invariants,
+    pin_golden_fixtures,
+]
