@@ -1,0 +1,133 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) IO-aware exact-attention library.
+ *
+ * The operation (per batch b and head h; X[b,h] is an N x d row-major matrix):
+ *   S = scale * Q K^T, with S[i][j] = -inf when causal and j > i,
+ *   P = softmax(S) row by row, O = P V, LSE[i] = ln sum_j exp(S[i][j]).
+ * Definition: "A survey of key techniques of large language model pre-training
+ * systems", Journal of Software 2026(1), p.218 (attention definition S = QK^T,
+ * P = Softmax(S), O = PV, and the two-block softmax decomposition the kernels use
+ * to process keys tile by tile); scaling by 1/sqrt(d): "FlashAttention
+ * optimisation: breaking the performance bottleneck of standard attention",
+ * section 1; causal masking: "Flash Attention-2: acceleration principle and GPU
+ * memory optimisation in deployment", causal-mask item. The forward is the fused,
+ * tiled, online-softmax pass of "FlashAttention optimisation ...", section 4.1;
+ * the backward recomputes P from LSE ("... ", section 4.2; "From GPU memory access
+ * to code: how FlashAttention makes large-model training 3x faster", section 2.2)
+ * and forms the gradient of the loss <dO, O>:
+ *   dV = P^T dO, dP = dO V^T, D = rowsum(dO o O), dS = P o (dP - D),
+ *   dQ = scale * dS K, dK = scale * dS^T Q.
+ * No N x N matrix is ever written to device memory.
+ *
+ * Conventions shared by every entry point:
+ *   - Tensors are contiguous row-major [B, H, N, d] (LSE and D are [B, H, N]),
+ *     in DEVICE memory, base addresses 16-byte aligned. Q, K and V share one N
+ *     (self-attention shape).
+ *   - The caller owns every buffer, including the backward workspace; the
+ *     library allocates no device memory. It holds one device status word per
+ *     GPU and a host-side cache of nothing that outlives a call.
+ *   - Calls are asynchronous on `stream` (0 = the legacy default stream).
+ *     Argument errors are returned synchronously and launch nothing. A failed
+ *     launch returns FA_ERR_CUDA.
+ *   - Every wait inside a kernel is bounded (default 10 s, environment variable
+ *     FA_WATCHDOG_MS). A wait that runs out makes the kernel record the error in
+ *     the device status word and return early, leaving its outputs undefined;
+ *     fa_get_status() reports it as FA_ERR_TIMEOUT.
+ *   - Supported: B, H >= 1; N >= 0 (N = 0 is a no-op); d in {64, 128};
+ *     causal in {0, 1}; scale finite and > 0; B*H*N*d < 2^31.
+ *   - Outputs are overwritten, never accumulated into.
+ */
+#ifndef FA_B200_FA_H
+#define FA_B200_FA_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as the CUDA runtime's cudaStream_t. */
+typedef struct CUstream_st* fa_stream_t;
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad shape, bad scale */
+  FA_ERR_UNSUPPORTED = 2, /* valid arguments outside what this build implements */
+  FA_ERR_CUDA = 3,        /* a CUDA call or launch failed (no device, bad context) */
+  FA_ERR_TIMEOUT = 4      /* a kernel's bounded wait ran out (see fa_get_status) */
+} fa_status;
+
+/*
+ * Forward, bf16 in / bf16 out, fp32 accumulation (tcgen05 tensor cores).
+ *   Q, K, V : bf16 [B,H,N,d], read only.
+ *   O       : bf16 [B,H,N,d], written: softmax(S) V rounded to nearest-even.
+ *   LSE     : fp32 [B,H,N], written: natural-log log-sum-exp of the scaled,
+ *             masked logits of each query row.
+ */
+fa_status fa_forward(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                     int B, int H, int N, int d, float scale, int causal,
+                     fa_stream_t stream);
+
+/*
+ * Workspace bytes fa_backward and fa_backward_f32 need for this shape:
+ *   D (fp32 [B,H,N]) + dQ accumulator (fp32 [B,H,N,d]), each rounded up to 256 B.
+ * Returns 0 for a shape that is invalid or empty.
+ */
+size_t fa_backward_workspace_size(int B, int H, int N, int d);
+
+/*
+ * Backward, bf16 in / bf16 out, fp32 accumulation (tcgen05 tensor cores).
+ *   Q, K, V, O, dO : bf16 [B,H,N,d], read only (O and LSE from fa_forward on the
+ *                    same Q, K, V, scale and causal).
+ *   LSE            : fp32 [B,H,N], read only.
+ *   dQ, dK, dV     : bf16 [B,H,N,d], written (gradients of <dO, O>).
+ *   workspace      : device memory of at least fa_backward_workspace_size bytes,
+ *                    16-byte aligned; its contents on entry do not matter and are
+ *                    undefined on return.
+ * dQ is accumulated in fp32 with atomic adds, so its last bits may differ from
+ * run to run; dK and dV are deterministic.
+ */
+fa_status fa_backward(const void* Q, const void* K, const void* V, const void* O,
+                      const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
+                      int B, int H, int N, int d, float scale, int causal,
+                      void* workspace, size_t workspace_bytes, fa_stream_t stream);
+
+/*
+ * fp32 entry points: the same operation and arguments with fp32 tensors
+ * (float [B,H,N,d]), computed in fp32 on the CUDA cores (FFMA), for callers that
+ * need fp32 accuracy; tensor-core fp32 (tf32) cannot reach it. The backward is
+ * deterministic. workspace as for fa_backward.
+ */
+fa_status fa_forward_f32(const float* Q, const float* K, const float* V, float* O,
+                         float* LSE, int B, int H, int N, int d, float scale, int causal,
+                         fa_stream_t stream);
+fa_status fa_backward_f32(const float* Q, const float* K, const float* V, const float* O,
+                          const float* dO, const float* LSE, float* dQ, float* dK,
+                          float* dV, int B, int H, int N, int d, float scale, int causal,
+                          void* workspace, size_t workspace_bytes, fa_stream_t stream);
+
+/*
+ * Synchronises `stream`, reads and clears the device status word of the current
+ * GPU. Returns FA_ERR_TIMEOUT if a kernel since the last call gave up on a wait,
+ * FA_ERR_CUDA if the synchronisation itself failed, else FA_OK.
+ */
+fa_status fa_get_status(fa_stream_t stream);
+
+/*
+ * Launches one kernel that waits, bounded by `timeout_ms`, on a barrier nothing
+ * ever completes, so the watchdog path can be exercised without a fault or hang.
+ * Afterwards fa_get_status() must return FA_ERR_TIMEOUT.
+ */
+fa_status fa_watchdog_selftest(int timeout_ms, fa_stream_t stream);
+
+/* Static English text for a status code. */
+const char* fa_status_string(fa_status status);
+
+/* Library version string, e.g. "fa-b200 0.1.0 sm_100a". */
+const char* fa_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_FA_H */

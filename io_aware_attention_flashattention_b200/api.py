@@ -1,0 +1,186 @@
+"""Python binding of the C ABI in include/fa.h (argument marshalling only).
+
+The ``fa_*`` functions mirror the C entry points one to one: they take torch
+tensors that already live on the GPU, check dtype/shape/contiguity, and pass raw
+pointers, sizes and the current CUDA stream to libfa_b200.so. Every arithmetic
+step runs in the library's kernels; there is no CPU or PyTorch fallback.
+
+``forward``, ``backward`` and ``attention`` are conveniences on top: they allocate
+outputs (and the backward workspace) with torch and call the entry points;
+``attention`` is differentiable through ``FlashAttentionFunction``.
+
+Operation (see include/fa.h): O = softmax(scale * Q K^T [causal mask]) V and
+LSE = natural-log log-sum-exp per query row, for [B, H, N, d] tensors, d in
+{64, 128}; backward gives dQ, dK, dV of the loss <dO, O>.
+"""
+from __future__ import annotations
+
+import math
+
+import torch
+
+from ._lib import FAError, check, lib
+
+__all__ = [
+    "FAError", "fa_forward", "fa_backward", "fa_backward_workspace_size", "fa_forward_f32",
+    "fa_backward_f32", "fa_get_status", "fa_watchdog_selftest", "fa_version",
+    "forward", "backward", "attention", "FlashAttentionFunction",
+]
+
+
+def _stream(stream) -> int:
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return int(getattr(stream, "cuda_stream", stream))
+
+
+def _shape(t: torch.Tensor):
+    if t.dim() != 4:
+        raise ValueError(f"expected a [B, H, N, d] tensor, got shape {tuple(t.shape)}")
+    return tuple(int(x) for x in t.shape)
+
+
+def _need(name: str, t: torch.Tensor, dtype: torch.dtype, shape) -> int:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def fa_version() -> str:
+    return lib().fa_version().decode()
+
+
+def fa_backward_workspace_size(B: int, H: int, N: int, d: int) -> int:
+    return int(lib().fa_backward_workspace_size(B, H, N, d))
+
+
+def fa_forward(Q, K, V, O, LSE, scale: float, causal: bool, stream=None) -> None:
+    B, H, N, d = _shape(Q)
+    bf = torch.bfloat16
+    args = [_need("Q", Q, bf, (B, H, N, d)), _need("K", K, bf, (B, H, N, d)),
+            _need("V", V, bf, (B, H, N, d)), _need("O", O, bf, (B, H, N, d)),
+            _need("LSE", LSE, torch.float32, (B, H, N))]
+    check("fa_forward", lib().fa_forward(*args, B, H, N, d, float(scale), int(bool(causal)),
+                                         _stream(stream)))
+
+
+def fa_forward_f32(Q, K, V, O, LSE, scale: float, causal: bool, stream=None) -> None:
+    B, H, N, d = _shape(Q)
+    f = torch.float32
+    args = [_need("Q", Q, f, (B, H, N, d)), _need("K", K, f, (B, H, N, d)),
+            _need("V", V, f, (B, H, N, d)), _need("O", O, f, (B, H, N, d)),
+            _need("LSE", LSE, f, (B, H, N))]
+    check("fa_forward_f32", lib().fa_forward_f32(*args, B, H, N, d, float(scale),
+                                                 int(bool(causal)), _stream(stream)))
+
+
+def _bwd_args(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, dtype):
+    B, H, N, d = _shape(Q)
+    s4 = (B, H, N, d)
+    ptrs = [_need("Q", Q, dtype, s4), _need("K", K, dtype, s4), _need("V", V, dtype, s4),
+            _need("O", O, dtype, s4), _need("dO", dO, dtype, s4),
+            _need("LSE", LSE, torch.float32, (B, H, N)),
+            _need("dQ", dQ, dtype, s4), _need("dK", dK, dtype, s4), _need("dV", dV, dtype, s4)]
+    if not (isinstance(workspace, torch.Tensor) and workspace.is_cuda and workspace.is_contiguous()):
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    return ptrs, (B, H, N, d), workspace.data_ptr(), workspace.numel() * workspace.element_size()
+
+
+def fa_backward(Q, K, V, O, dO, LSE, dQ, dK, dV, scale: float, causal: bool, workspace,
+                stream=None) -> None:
+    ptrs, (B, H, N, d), ws, nbytes = _bwd_args(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace,
+                                               torch.bfloat16)
+    check("fa_backward", lib().fa_backward(*ptrs, B, H, N, d, float(scale), int(bool(causal)),
+                                           ws, nbytes, _stream(stream)))
+
+
+def fa_backward_f32(Q, K, V, O, dO, LSE, dQ, dK, dV, scale: float, causal: bool, workspace,
+                    stream=None) -> None:
+    ptrs, (B, H, N, d), ws, nbytes = _bwd_args(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace,
+                                               torch.float32)
+    check("fa_backward_f32", lib().fa_backward_f32(*ptrs, B, H, N, d, float(scale),
+                                                   int(bool(causal)), ws, nbytes,
+                                                   _stream(stream)))
+
+
+def fa_get_status(stream=None) -> int:
+    """Synchronises the stream; returns the library status code (0 = ok, 4 = a
+    kernel's bounded wait ran out since the last call)."""
+    return int(lib().fa_get_status(_stream(stream)))
+
+
+def fa_watchdog_selftest(timeout_ms: int, stream=None) -> None:
+    check("fa_watchdog_selftest", lib().fa_watchdog_selftest(int(timeout_ms), _stream(stream)))
+
+
+# ---------------------------------------------------------------- conveniences
+
+
+def _default_scale(d: int, scale):
+    return 1.0 / math.sqrt(d) if scale is None else float(scale)
+
+
+def forward(q, k, v, causal: bool = False, scale=None):
+    """(O, LSE) for bf16 or fp32 q, k, v of shape [B, H, N, d] on the GPU."""
+    B, H, N, d = _shape(q)
+    scale = _default_scale(d, scale)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    if q.dtype == torch.bfloat16:
+        fa_forward(q, k, v, o, lse, scale, causal)
+    elif q.dtype == torch.float32:
+        fa_forward_f32(q, k, v, o, lse, scale, causal)
+    else:
+        raise TypeError(f"unsupported dtype {q.dtype}: bf16 or fp32")
+    return o, lse
+
+
+def workspace_for(q) -> torch.Tensor:
+    B, H, N, d = _shape(q)
+    n = max(1, fa_backward_workspace_size(B, H, N, d))
+    return torch.empty(n, dtype=torch.uint8, device=q.device)
+
+
+def backward(q, k, v, o, lse, do, causal: bool = False, scale=None, workspace=None):
+    """(dQ, dK, dV) of the loss <dO, O>."""
+    B, H, N, d = _shape(q)
+    scale = _default_scale(d, scale)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = workspace_for(q) if workspace is None else workspace
+    if q.dtype == torch.bfloat16:
+        fa_backward(q, k, v, o, do, lse, dq, dk, dv, scale, causal, ws)
+    elif q.dtype == torch.float32:
+        fa_backward_f32(q, k, v, o, do, lse, dq, dk, dv, scale, causal, ws)
+    else:
+        raise TypeError(f"unsupported dtype {q.dtype}: bf16 or fp32")
+    return dq, dk, dv
+
+
+class FlashAttentionFunction(torch.autograd.Function):
+    """Differentiable exact attention through the library's forward and backward."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, causal: bool = False, scale=None):
+        q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+        o, lse = forward(q, k, v, causal, scale)
+        ctx.save_for_backward(q, k, v, o, lse)
+        ctx.causal, ctx.scale = causal, scale
+        return o
+
+    @staticmethod
+    def backward(ctx, do):
+        q, k, v, o, lse = ctx.saved_tensors
+        dq, dk, dv = backward(q, k, v, o, lse, do.contiguous(), ctx.causal, ctx.scale)
+        return dq, dk, dv, None, None
+
+
+def attention(q, k, v, causal: bool = False, scale=None):
+    return FlashAttentionFunction.apply(q, k, v, causal, scale)

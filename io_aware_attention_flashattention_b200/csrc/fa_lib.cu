@@ -1,0 +1,343 @@
+// fa_lib.cu -- the C ABI of include/fa.h: argument validation, TMA tensor-map
+// construction, kernel launches and the device status word. All kernels are in
+// this one translation unit (they share the status word without relocatable
+// device code). The library allocates no device memory.
+
+#include "fa.h"
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <algorithm>
+#include <cstdlib>
+#include <mutex>
+
+#include "fa_ptx.cuh"
+#include "fa_fwd_sm100.cuh"
+#include "fa_bwd_sm100.cuh"
+#include "fa_simt_f32.cuh"
+
+namespace fa {
+namespace {
+
+// ------------------------------------------------------------------ watchdog kernel
+
+__global__ void watchdog_selftest_kernel(unsigned long long timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  // Nothing ever arrives on `bar`: the wait must run out and record the timeout.
+  const Watchdog wd{&abort_flag, timeout_ns};
+  mbar_wait(smem_u32(&bar), 0, wd);
+}
+
+// ------------------------------------------------------------------ host helpers
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+unsigned long long watchdog_ns() {
+  static const unsigned long long v = [] {
+    const char* e = std::getenv("FA_WATCHDOG_MS");
+    long long ms = e ? std::atoll(e) : 5000;
+    if (ms <= 0) ms = 5000;
+    return static_cast<unsigned long long>(ms) * 1000000ull;
+  }();
+  return v;
+}
+
+constexpr int kMaxDevices = 64;
+struct DeviceState {
+  bool checked = false;
+  bool supported = false;
+  bool attrs_done = false;
+};
+DeviceState g_devices[kMaxDevices];
+std::mutex g_mutex;
+
+template <typename Kern>
+cudaError_t set_smem(Kern k, size_t bytes) {
+  return cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              static_cast<int>(bytes));
+}
+
+// Checks that the current device is an sm_100 part and sets the kernels'
+// shared-memory limits once per device.
+fa_status prepare_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  DeviceState& st = g_devices[dev];
+  if (!st.checked) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return FA_ERR_CUDA;
+    st.supported = (major == 10 && minor == 0);
+    st.checked = true;
+  }
+  if (!st.supported) return FA_ERR_UNSUPPORTED;
+  if (!st.attrs_done) {
+    cudaError_t e = cudaSuccess;
+    e = e ? e : set_smem(fwd::fa_fwd_kernel<64>, fwd::Cfg<64>::kSmemBytes);
+    e = e ? e : set_smem(fwd::fa_fwd_kernel<128>, fwd::Cfg<128>::kSmemBytes);
+    e = e ? e : set_smem(bwd::fa_bwd_kernel<64>, bwd::Cfg<64>::kSmemBytes);
+    e = e ? e : set_smem(bwd::fa_bwd_kernel<128>, bwd::Cfg<128>::kSmemBytes);
+    e = e ? e : set_smem(f32::fa_f32_bwd_dkdv_kernel<64>, f32::dkdv_smem_bytes<64>());
+    e = e ? e : set_smem(f32::fa_f32_bwd_dkdv_kernel<128>, f32::dkdv_smem_bytes<128>());
+    e = e ? e : set_smem(f32::fa_f32_bwd_dq_kernel<64>, f32::dq_smem_bytes<64>());
+    e = e ? e : set_smem(f32::fa_f32_bwd_dq_kernel<128>, f32::dq_smem_bytes<128>());
+    if (e != cudaSuccess) return FA_ERR_CUDA;
+    st.attrs_done = true;
+  }
+  return FA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+fa_status check_shape(int B, int H, int N, int d, float scale, int causal) {
+  if (B < 1 || H < 1 || N < 0) return FA_ERR_INVALID_ARG;
+  if (!(std::isfinite(scale) && scale > 0.0f)) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  const long long total = static_cast<long long>(B) * H * N * d;
+  if (total >= (1ll << 31)) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+fa_status check_ptrs(std::initializer_list<const void*> ptrs) {
+  for (const void* p : ptrs)
+    if (p == nullptr || !aligned16(p)) return FA_ERR_INVALID_ARG;
+  return FA_OK;
+}
+
+size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+// 3-D view [B*H, N, d] of a bf16 tensor with boxes of 64 columns x `box_rows`
+// rows x 1 head, 128-byte swizzle. Rows beyond N read as zero, per head.
+bool make_map_bf16(CUtensorMap* map, const void* ptr, int BH, int N, int d, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
+                              static_cast<cuuint64_t>(BH)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 2,
+                                 static_cast<cuuint64_t>(N) * d * 2};
+  const cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_rows), 1u};
+  const cuuint32_t estr[3] = {1u, 1u, 1u};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+fa_status launch_status() {
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace fa
+
+using namespace fa;
+
+extern "C" {
+
+const char* fa_version(void) { return "fa-b200 0.1.0 sm_100a"; }
+
+const char* fa_status_string(fa_status s) {
+  switch (s) {
+    case FA_OK: return "ok";
+    case FA_ERR_INVALID_ARG: return "invalid argument";
+    case FA_ERR_UNSUPPORTED: return "unsupported configuration or device";
+    case FA_ERR_CUDA: return "CUDA error";
+    case FA_ERR_TIMEOUT: return "kernel watchdog timeout";
+  }
+  return "unknown status";
+}
+
+size_t fa_backward_workspace_size(int B, int H, int N, int d) {
+  if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
+  const size_t bh = static_cast<size_t>(B) * H;
+  const size_t npad = (static_cast<size_t>(N) + 127) / 128 * 128;
+  return 2 * round256(bh * npad * sizeof(float)) + round256(bh * N * d * sizeof(float));
+}
+
+fa_status fa_get_status(fa_stream_t stream) {
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return FA_ERR_CUDA;
+  unsigned int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(v)) != cudaSuccess) return FA_ERR_CUDA;
+  if (v != 0 && cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess)
+    return FA_ERR_CUDA;
+  return (v & kStatusTimeout) ? FA_ERR_TIMEOUT : FA_OK;
+}
+
+fa_status fa_watchdog_selftest(int timeout_ms, fa_stream_t stream) {
+  if (timeout_ms < 1 || timeout_ms > 60000) return FA_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_CUDA;
+  int major = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+    return FA_ERR_CUDA;
+  if (major != 10) return FA_ERR_UNSUPPORTED;
+  watchdog_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      static_cast<unsigned long long>(timeout_ms) * 1000000ull);
+  return launch_status();
+}
+
+fa_status fa_forward(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
+                     int H, int N, int d, float scale, int causal, fa_stream_t stream) {
+  fa_status st = check_shape(B, H, N, d, scale, causal);
+  if (st != FA_OK) return st;
+  if (N == 0) return FA_OK;
+  if ((st = check_ptrs({Q, K, V, O, LSE})) != FA_OK) return st;
+  if ((st = prepare_device()) != FA_OK) return st;
+  const int BH = B * H;
+  CUtensorMap mq, mk, mv;
+  if (!make_map_bf16(&mq, Q, BH, N, d, fwd::BM) || !make_map_bf16(&mk, K, BH, N, d, fwd::BN) ||
+      !make_map_bf16(&mv, V, BH, N, d, fwd::BN))
+    return FA_ERR_CUDA;
+  fwd::Params p;
+  p.O = static_cast<__nv_bfloat16*>(O);
+  p.LSE = LSE;
+  p.N = N;
+  p.BH = BH;
+  p.n_qblk = (N + 2 * fwd::BM - 1) / (2 * fwd::BM);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.causal = causal;
+  p.timeout_ns = watchdog_ns();
+  const dim3 grid(static_cast<unsigned>(p.n_qblk) * BH);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 64)
+    fwd::fa_fwd_kernel<64><<<grid, fwd::kThreads, fwd::Cfg<64>::kSmemBytes, s>>>(mq, mk, mv, p);
+  else
+    fwd::fa_fwd_kernel<128><<<grid, fwd::kThreads, fwd::Cfg<128>::kSmemBytes, s>>>(mq, mk, mv, p);
+  return launch_status();
+}
+
+fa_status fa_backward(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                      const float* LSE, void* dQ, void* dK, void* dV, int B, int H, int N, int d,
+                      float scale, int causal, void* workspace, size_t workspace_bytes,
+                      fa_stream_t stream) {
+  fa_status st = check_shape(B, H, N, d, scale, causal);
+  if (st != FA_OK) return st;
+  if (N == 0) return FA_OK;
+  if ((st = check_ptrs({Q, K, V, O, dO, LSE, dQ, dK, dV, workspace})) != FA_OK) return st;
+  if (workspace_bytes < fa_backward_workspace_size(B, H, N, d)) return FA_ERR_INVALID_ARG;
+  if ((st = prepare_device()) != FA_OK) return st;
+  const int BH = B * H;
+  const int Npad = (N + 127) / 128 * 128;
+  CUtensorMap mq, mk, mv, mdo;
+  if (!make_map_bf16(&mq, Q, BH, N, d, bwd::BM) || !make_map_bf16(&mk, K, BH, N, d, bwd::BN) ||
+      !make_map_bf16(&mv, V, BH, N, d, bwd::BN) || !make_map_bf16(&mdo, dO, BH, N, d, bwd::BM))
+    return FA_ERR_CUDA;
+  // workspace: L2 [BH, Npad] | D [BH, Npad] | dQ accumulator [BH, N, d] (fp32)
+  char* ws = static_cast<char*>(workspace);
+  const size_t vec_bytes = round256(static_cast<size_t>(BH) * Npad * sizeof(float));
+  float* L2 = reinterpret_cast<float*>(ws);
+  float* Dv = reinterpret_cast<float*>(ws + vec_bytes);
+  float* dQacc = reinterpret_cast<float*>(ws + 2 * vec_bytes);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const long long pre_rows = static_cast<long long>(BH) * Npad;
+  const unsigned pre_blocks = static_cast<unsigned>((pre_rows + 7) / 8);
+  bwd::Params p;
+  p.dK = static_cast<__nv_bfloat16*>(dK);
+  p.dV = static_cast<__nv_bfloat16*>(dV);
+  p.L2 = L2;
+  p.Dv = Dv;
+  p.dQacc = dQacc;
+  p.N = N;
+  p.Npad = Npad;
+  p.BH = BH;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.causal = causal;
+  p.timeout_ns = watchdog_ns();
+  const dim3 grid(static_cast<unsigned>(Npad / bwd::BN) * BH);
+  const long long n4 = static_cast<long long>(BH) * N * d / 4;
+  const unsigned cvt_blocks = static_cast<unsigned>(std::min<long long>((n4 + 255) / 256, 148 * 16));
+  const auto* O16 = static_cast<const __nv_bfloat16*>(O);
+  const auto* dO16 = static_cast<const __nv_bfloat16*>(dO);
+  if (d == 64) {
+    bwd::fa_bwd_pre_kernel<64><<<pre_blocks, 256, 0, s>>>(O16, dO16, LSE, L2, Dv, dQacc, N, Npad, pre_rows);
+    bwd::fa_bwd_kernel<64><<<grid, bwd::kThreads, bwd::Cfg<64>::kSmemBytes, s>>>(mq, mk, mv, mdo, p);
+    bwd::fa_bwd_dq_kernel<64><<<cvt_blocks, 256, 0, s>>>(dQacc, static_cast<__nv_bfloat16*>(dQ), n4, scale);
+  } else {
+    bwd::fa_bwd_pre_kernel<128><<<pre_blocks, 256, 0, s>>>(O16, dO16, LSE, L2, Dv, dQacc, N, Npad, pre_rows);
+    bwd::fa_bwd_kernel<128><<<grid, bwd::kThreads, bwd::Cfg<128>::kSmemBytes, s>>>(mq, mk, mv, mdo, p);
+    bwd::fa_bwd_dq_kernel<128><<<cvt_blocks, 256, 0, s>>>(dQacc, static_cast<__nv_bfloat16*>(dQ), n4, scale);
+  }
+  return launch_status();
+}
+
+fa_status fa_forward_f32(const float* Q, const float* K, const float* V, float* O, float* LSE,
+                         int B, int H, int N, int d, float scale, int causal,
+                         fa_stream_t stream) {
+  fa_status st = check_shape(B, H, N, d, scale, causal);
+  if (st != FA_OK) return st;
+  if (N == 0) return FA_OK;
+  if ((st = check_ptrs({Q, K, V, O, LSE})) != FA_OK) return st;
+  if ((st = prepare_device()) != FA_OK) return st;
+  const dim3 grid((N + f32::kRowsPerBlock - 1) / f32::kRowsPerBlock, B * H);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 64)
+    f32::fa_f32_fwd_kernel<64><<<grid, f32::kWarps * 32, 0, s>>>(Q, K, V, O, LSE, N, scale, causal);
+  else
+    f32::fa_f32_fwd_kernel<128><<<grid, f32::kWarps * 32, 0, s>>>(Q, K, V, O, LSE, N, scale, causal);
+  return launch_status();
+}
+
+fa_status fa_backward_f32(const float* Q, const float* K, const float* V, const float* O,
+                          const float* dO, const float* LSE, float* dQ, float* dK, float* dV,
+                          int B, int H, int N, int d, float scale, int causal, void* workspace,
+                          size_t workspace_bytes, fa_stream_t stream) {
+  fa_status st = check_shape(B, H, N, d, scale, causal);
+  if (st != FA_OK) return st;
+  if (N == 0) return FA_OK;
+  if ((st = check_ptrs({Q, K, V, O, dO, LSE, dQ, dK, dV, workspace})) != FA_OK) return st;
+  if (workspace_bytes < fa_backward_workspace_size(B, H, N, d)) return FA_ERR_INVALID_ARG;
+  if ((st = prepare_device()) != FA_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  float* Dvec = static_cast<float*>(workspace);
+  const long long rows = static_cast<long long>(B) * H * N;
+  const unsigned dot_blocks = static_cast<unsigned>((rows + f32::kWarps - 1) / f32::kWarps);
+  const dim3 grid((N + f32::kRowsPerBlock - 1) / f32::kRowsPerBlock, B * H);
+  if (d == 64) {
+    f32::fa_f32_bwd_dot_kernel<64><<<dot_blocks, f32::kWarps * 32, 0, s>>>(O, dO, Dvec, rows);
+    f32::fa_f32_bwd_dkdv_kernel<64><<<grid, f32::kWarps * 32, f32::dkdv_smem_bytes<64>(), s>>>(
+        Q, K, V, dO, LSE, Dvec, dK, dV, N, scale, causal);
+    f32::fa_f32_bwd_dq_kernel<64><<<grid, f32::kWarps * 32, f32::dq_smem_bytes<64>(), s>>>(
+        Q, K, V, dO, LSE, Dvec, dQ, N, scale, causal);
+  } else {
+    f32::fa_f32_bwd_dot_kernel<128><<<dot_blocks, f32::kWarps * 32, 0, s>>>(O, dO, Dvec, rows);
+    f32::fa_f32_bwd_dkdv_kernel<128><<<grid, f32::kWarps * 32, f32::dkdv_smem_bytes<128>(), s>>>(
+        Q, K, V, dO, LSE, Dvec, dK, dV, N, scale, causal);
+    f32::fa_f32_bwd_dq_kernel<128><<<grid, f32::kWarps * 32, f32::dq_smem_bytes<128>(), s>>>(
+        Q, K, V, dO, LSE, Dvec, dQ, N, scale, causal);
+  }
+  return launch_status();
+}
+
+}  // extern "C"
