@@ -1,0 +1,439 @@
+#!/usr/bin/env python
+"""Benchmark of the exact-attention hot path: one step = forward + backward
+(fa_forward, then the three backward stages that fa_backward runs) over one batch
+of seeded synthetic inputs already resident in HBM.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+  python bench.py --impl reference ...   # the fp64 CPU oracle on the host cores
+
+Metric: attention fwd+bwd TFLOP/s, counting 4*B*H*N^2*d for the forward (halved
+when causal) and 2.5x that for the backward. Timing: CUDA events on the launching
+stream around every kernel of every step; L2 is flushed (a 256 MiB write) before
+each timed step, outside the events; W untimed warm-up steps; a barrier and a
+device synchronise on both sides of the K timed steps; max over ranks. With N > 1
+each rank runs its own replica of the workload (independent heads; no collective
+on the data path), so the scaling is weak.
+
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd/bwd TFLOP/s (bf16, d=128) and % of B200 dense BF16 peak"
+DEFAULT_WORKLOAD = "long_b1h8_n16384_d128"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse():
+    ap = argparse.ArgumentParser(description=__doc__.split("\n\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target CPU time of the oracle sample")
+    return ap.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            return json.load(f), "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_source_sha():
+    """Hash of the CUDA sources; ncu traffic figures are only reported while the
+    kernels are the ones they were taken on."""
+    csrc = os.path.join(ROOT, "io_aware_attention_flashattention_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def profiled_traffic(kernel: str, workload: str):
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        table = json.load(f)
+    ent = table.get(kernel)
+    if not ent or ent.get("workload") != workload or ent.get("source_sha") != kernel_source_sha():
+        return None
+    return ent.get("bytes_per_launch")
+
+
+class ClockSampler:
+    """nvidia-smi clock and throttle-reason samples while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50", "-i", str(self.index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, power, reasons = [], [], [], set()
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for name, val in zip(self.NAMES, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(power) if power else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- CPU oracle sample
+
+
+def oracle_sample(w, seconds: float, rng_seed: int = 0, inputs=None):
+    """The fp64 oracle, as it stands, on a bounded sample of the workload: R random
+    (head, query row) pairs through the forward (O, LSE) and the dQ backward rows,
+    each with all visible keys. Returns (flops, seconds, rows, threads). Flops count
+    what the oracle's definition computes per visible (row, key) pair and head
+    dimension element: 4 for the forward (S and PV), 6 for the dQ rows (S, dP and
+    dS K)."""
+    import numpy as np
+
+    import oracle
+    from io_aware_attention_flashattention_b200.inputs import workload_inputs
+
+    q, k, v, do = inputs if inputs is not None else workload_inputs(w)
+    # fp64 copies made once, outside the timed calls
+    q, k, v, do = (np.ascontiguousarray(t.double().numpy()) for t in (q, k, v, do))
+    BH = w.B * w.H
+    rng = np.random.default_rng(rng_seed)
+
+    def run(R):
+        heads = rng.integers(0, BH, R)
+        rows = rng.integers(0, w.N, R)
+        order = np.lexsort((rows, heads))
+        heads, rows = heads[order], rows[order]
+        t0 = time.perf_counter()
+        oracle.forward_rows(q, k, v, w.scale, w.causal, heads, rows)
+        oracle.backward_dq_rows(q, k, v, do, w.scale, w.causal, heads, rows)
+        dt = time.perf_counter() - t0
+        visible = (rows + 1) if w.causal else np.full(R, w.N)
+        return float(np.sum(visible)) * w.d * 10.0, dt
+
+    r0 = max(32, 4 * oracle.num_threads())
+    _, t0 = run(r0)  # calibration: enough rows to occupy every thread
+    per_row = t0 / r0
+    R = int(max(1, seconds / max(per_row, 1e-9)))
+    flops, dt = run(R)
+    return flops, dt, R, oracle.num_threads()
+
+
+def reference_arm(args, w):
+    """--impl reference: the oracle on the host cores, each step a bounded sample."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    from io_aware_attention_flashattention_b200.inputs import workload_inputs
+
+    inputs = workload_inputs(w)
+    budget = 150.0 / max(1, args.steps + args.warmup)
+    for i in range(args.warmup):
+        oracle_sample(w, budget, rng_seed=i, inputs=inputs)
+    flops = secs = 0.0
+    rows = threads = 0
+    for i in range(args.steps):
+        f, t, R, threads = oracle_sample(w, budget, rng_seed=1000 + i, inputs=inputs)
+        flops += f
+        secs += t
+        rows += R
+    value = flops / secs / 1e12
+    sample = (f"{rows // max(1, args.steps)} random (head, query row) pairs per step of "
+              f"{w.name}, all visible keys: oracle forward rows + dQ rows, fp64")
+    out = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "impl": "reference",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                   "causal": w.causal, "scale": w.scale},
+        "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out))
+    return 0
+
+
+# ---------------------------------------------------------------- our arm
+
+
+def main():
+    args = parse()
+    from io_aware_attention_flashattention_b200.inputs import WORKLOADS
+
+    w = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return reference_arm(args, w)
+
+    import torch
+    import torch.distributed as dist
+
+    from io_aware_attention_flashattention_b200 import api
+    from io_aware_attention_flashattention_b200.inputs import make_inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    # inputs: this rank's replica of the workload (seed offset by rank)
+    q, k, v, do = make_inputs(w.B, w.H, w.N, w.d, w.dtype, w.seed + 7919 * rank, w.qk_gain)
+    Q, K, V, dO = (t.to(dev) for t in (q, k, v, do))
+    O = torch.empty_like(Q)
+    LSE = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+    dQ, dK, dV = torch.empty_like(Q), torch.empty_like(K), torch.empty_like(V)
+    ws = api.workspace_for(Q)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    bf16 = w.dtype == torch.bfloat16
+    if not bf16:
+        raise SystemExit("the benchmark times the bf16 tensor-core path")
+
+    names = ["fa_fwd_kernel", "fa_bwd_pre_kernel", "fa_bwd_kernel", "fa_bwd_dq_kernel"]
+    nev = len(names) + 1
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        api.fa_forward(Q, K, V, O, LSE, w.scale, w.causal)
+        if ev is not None:
+            ev[1].record(stream)
+        api.fa_backward_preprocess(O, dO, LSE, w.scale, w.causal, ws)
+        if ev is not None:
+            ev[2].record(stream)
+        api.fa_backward_main(Q, K, V, dO, dK, dV, w.scale, w.causal, ws)
+        if ev is not None:
+            ev[3].record(stream)
+        api.fa_backward_dq_convert(dQ, w.scale, ws)
+        if ev is not None:
+            ev[4].record(stream)
+
+    for _ in range(max(3, args.warmup)):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if api.fa_get_status() != 0:
+        raise SystemExit("kernel watchdog fired during warm-up")
+
+    events = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
+    sampler = ClockSampler(torch.cuda.current_device())
+    barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.2)  # let the sampler start before the timed region
+    wall0 = time.perf_counter()
+    for s in range(args.steps):
+        flush.zero_()
+        step(events[s])
+    torch.cuda.synchronize()
+    wall = time.perf_counter() - wall0
+    barrier()
+    clocks = sampler.stop()
+    status = api.fa_get_status()
+    per_kernel = [[events[s][i].elapsed_time(events[s][i + 1]) for s in range(args.steps)]
+                  for i in range(len(names))]
+    step_ms = [events[s][0].elapsed_time(events[s][-1]) for s in range(args.steps)]
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+
+    fwd_f, bwd_f = w.fwd_flops(), w.bwd_flops()
+    flops_step = fwd_f + bwd_f
+    value = flops_step * world * args.steps / (total_ms * 1e-3) / 1e12
+
+    # per-kernel figures and the dominant kernel's roofline
+    BH, N, d = w.B * w.H, w.N, w.d
+    npad = (N + 127) // 128 * 128
+    kern = {
+        "fa_fwd_kernel": {"flops": fwd_f, "bytes": 4 * BH * N * d * 2 + 4 * BH * N},
+        "fa_bwd_pre_kernel": {"bytes": 2 * BH * N * d * 2 + 4 * BH * N + 8 * BH * npad
+                              + 4 * BH * N * d},
+        # reads Q, K, V, dO and L2/D; writes dK, dV; read-modify-write of the fp32 dQ accumulator
+        "fa_bwd_kernel": {"flops": bwd_f, "bytes": 6 * BH * N * d * 2 + 8 * BH * npad
+                          + 2 * 4 * BH * N * d},
+        "fa_bwd_dq_kernel": {"bytes": 4 * BH * N * d + 2 * BH * N * d},
+    }
+    kernels = {}
+    for name, times in zip(names, per_kernel):
+        avg = sum(times) / len(times)
+        ent = {"avg_ms": avg, "share": sum(times) / total_ms if world == 1 else None}
+        if "flops" in kern[name]:
+            ent["tflops"] = kern[name]["flops"] / (avg * 1e-3) / 1e12
+        ent["gbs"] = kern[name]["bytes"] / (avg * 1e-3) / 1e9
+        kernels[name] = ent
+    peaks, peak_src = load_peaks()
+    dom = max(names, key=lambda n: kernels[n]["avg_ms"])
+    if "flops" in kern[dom]:
+        achieved = kernels[dom]["tflops"]
+        peak = float(peaks["bf16_tflops"])
+        roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak}
+    else:
+        achieved = kernels[dom]["gbs"]
+        peak = float(peaks["hbm_gbs"])
+        roof = {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak}
+    roof.update({"traffic": profiled_traffic(dom, w.name), "kernel": dom,
+                 "peak_source": f"{peak_src} (burst bf16 GEMM)" if roof["bound"] == "tensor"
+                 else f"{peak_src} (copy)"})
+
+    # end to end through the public C-ABI calls with host buffers
+    e2e = None
+    if not args.no_e2e:
+        hq, hk, hv, hdo = (t.pin_memory() for t in (q, k, v, do))
+        hO = torch.empty(q.shape, dtype=q.dtype).pin_memory()
+        hL = torch.empty((w.B, w.H, w.N), dtype=torch.float32).pin_memory()
+        hdQ, hdK, hdV = (torch.empty(q.shape, dtype=q.dtype).pin_memory() for _ in range(3))
+        h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hdo))
+        d2h = sum(t.numel() * t.element_size() for t in (hO, hL, hdQ, hdK, hdV))
+
+        def e2e_step():
+            for dst, src in ((Q, hq), (K, hk), (V, hv), (dO, hdo)):
+                dst.copy_(src, non_blocking=True)
+            api.fa_forward(Q, K, V, O, LSE, w.scale, w.causal)
+            api.fa_backward(Q, K, V, O, dO, LSE, dQ, dK, dV, w.scale, w.causal, ws)
+            for dst, src in ((hO, O), (hL, LSE), (hdQ, dQ), (hdK, dK), (hdV, dV)):
+                dst.copy_(src, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        n_e2e = max(3, min(args.steps, 20))
+        barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(n_e2e):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        barrier()
+        e_ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        e2e = {"value": flops_step * world * n_e2e / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
+               "ms_per_step": e_ms / n_e2e}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        f, t, R, threads = oracle_sample(w, args.cpu_seconds)
+        cpu = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+               "sample": f"{R} random (head, query row) pairs of {w.name}, all visible keys: "
+                         f"oracle forward rows + dQ rows, fp64, {t:.1f} s"}
+
+    if world > 1:
+        barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    out = {
+        "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": max(3, args.warmup),
+        "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
+                   "causal": w.causal, "scale": w.scale, "parallelism": f"replicas{world}",
+                   "l2": "flushed (256 MiB write) before every timed step"},
+        "fwd_tflops": fwd_f / (kernels["fa_fwd_kernel"]["avg_ms"] * 1e-3) / 1e12,
+        "bwd_tflops": bwd_f / (sum(kernels[n]["avg_ms"] for n in names[1:]) * 1e-3) / 1e12,
+        "frac_of_peak": {"fwd": None, "bwd": None, "peak_tflops": float(peaks["bf16_tflops"])},
+        "roofline": roof,
+        "kernels": kernels,
+        "gpu_launches": len(names) * args.steps,
+        "clocks": clocks,
+        "e2e": e2e,
+        "cpu_baseline": cpu,
+        "watchdog_status": status,
+        "wall_s_timed_region": wall,
+    }
+    pk = float(peaks["bf16_tflops"])
+    out["frac_of_peak"]["fwd"] = out["fwd_tflops"] / pk
+    out["frac_of_peak"]["bwd"] = out["bwd_tflops"] / pk
+    print(json.dumps(out))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

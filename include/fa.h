@@ -29,10 +29,11 @@
  *   - Calls are asynchronous on `stream` (0 = the legacy default stream).
  *     Argument errors are returned synchronously and launch nothing. A failed
  *     launch returns FA_ERR_CUDA.
- *   - Every wait inside a kernel is bounded (default 10 s, environment variable
- *     FA_WATCHDOG_MS). A wait that runs out makes the kernel record the error in
- *     the device status word and return early, leaving its outputs undefined;
- *     fa_get_status() reports it as FA_ERR_TIMEOUT.
+ *   - Every wait inside a kernel is bounded (default 5 s; the environment
+ *     variable FA_WATCHDOG_MS, read once per process, overrides it). A wait that
+ *     runs out makes the kernel record the error in the device status word and
+ *     return early, leaving its outputs undefined; fa_get_status() reports it as
+ *     FA_ERR_TIMEOUT.
  *   - Supported: B, H >= 1; N >= 0 (N = 0 is a no-op); d in {64, 128};
  *     causal in {0, 1}; scale finite and > 0; B*H*N*d < 2^31.
  *   - Outputs are overwritten, never accumulated into.
@@ -69,8 +70,10 @@ fa_status fa_forward(const void* Q, const void* K, const void* V, void* O, float
                      fa_stream_t stream);
 
 /*
- * Workspace bytes fa_backward and fa_backward_f32 need for this shape:
- *   D (fp32 [B,H,N]) + dQ accumulator (fp32 [B,H,N,d]), each rounded up to 256 B.
+ * Workspace bytes fa_backward and fa_backward_f32 need for this shape, with
+ * Npad = N rounded up to a multiple of 128:
+ *   LSE*log2(e) (fp32 [B*H, Npad]) + D (fp32 [B*H, Npad]) + dQ accumulator
+ *   (fp32 [B,H,N,d]), each region rounded up to 256 bytes.
  * Returns 0 for a shape that is invalid or empty.
  */
 size_t fa_backward_workspace_size(int B, int H, int N, int d);
@@ -91,6 +94,29 @@ fa_status fa_backward(const void* Q, const void* K, const void* V, const void* O
                       const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
                       int B, int H, int N, int d, float scale, int causal,
                       void* workspace, size_t workspace_bytes, fa_stream_t stream);
+
+/*
+ * The three stages fa_backward runs, in order, on the same stream and workspace
+ * (exposed so that each stage can be timed or scheduled on its own; calling the
+ * three in order is exactly fa_backward):
+ *   fa_backward_preprocess: D = rowsum(dO o O) and LSE*log2(e) into the workspace
+ *                           (rows padded to a multiple of 128), and zeroes the fp32
+ *                           dQ accumulator in the workspace.
+ *   fa_backward_main      : the fused recomputation kernel: writes dK, dV and adds
+ *                           the unscaled dQ into the workspace accumulator.
+ *   fa_backward_dq_convert: dQ = bf16(scale * accumulator).
+ * Arguments mean what they mean for fa_backward; `causal` is not used by the
+ * convert stage. Argument errors are returned before any launch.
+ */
+fa_status fa_backward_preprocess(const void* O, const void* dO, const float* LSE, int B, int H,
+                                 int N, int d, float scale, int causal, void* workspace,
+                                 size_t workspace_bytes, fa_stream_t stream);
+fa_status fa_backward_main(const void* Q, const void* K, const void* V, const void* dO,
+                           void* dK, void* dV, int B, int H, int N, int d, float scale,
+                           int causal, void* workspace, size_t workspace_bytes,
+                           fa_stream_t stream);
+fa_status fa_backward_dq_convert(void* dQ, int B, int H, int N, int d, float scale,
+                                 void* workspace, size_t workspace_bytes, fa_stream_t stream);
 
 /*
  * fp32 entry points: the same operation and arguments with fp32 tensors

@@ -22,7 +22,8 @@ import torch
 from ._lib import FAError, check, lib
 
 __all__ = [
-    "FAError", "fa_forward", "fa_backward", "fa_backward_workspace_size", "fa_forward_f32",
+    "FAError", "fa_forward", "fa_backward", "fa_backward_workspace_size",
+    "fa_backward_preprocess", "fa_backward_main", "fa_backward_dq_convert", "fa_forward_f32",
     "fa_backward_f32", "fa_get_status", "fa_watchdog_selftest", "fa_version",
     "forward", "backward", "attention", "FlashAttentionFunction",
 ]
@@ -100,6 +101,40 @@ def fa_backward(Q, K, V, O, dO, LSE, dQ, dK, dV, scale: float, causal: bool, wor
                                                torch.bfloat16)
     check("fa_backward", lib().fa_backward(*ptrs, B, H, N, d, float(scale), int(bool(causal)),
                                            ws, nbytes, _stream(stream)))
+
+
+def _ws(workspace):
+    if not (isinstance(workspace, torch.Tensor) and workspace.is_cuda and workspace.is_contiguous()):
+        raise ValueError("workspace must be a contiguous CUDA tensor")
+    return workspace.data_ptr(), workspace.numel() * workspace.element_size()
+
+
+def fa_backward_preprocess(O, dO, LSE, scale: float, causal: bool, workspace, stream=None):
+    B, H, N, d = _shape(O)
+    bf = torch.bfloat16
+    ws, nbytes = _ws(workspace)
+    check("fa_backward_preprocess", lib().fa_backward_preprocess(
+        _need("O", O, bf, (B, H, N, d)), _need("dO", dO, bf, (B, H, N, d)),
+        _need("LSE", LSE, torch.float32, (B, H, N)), B, H, N, d, float(scale),
+        int(bool(causal)), ws, nbytes, _stream(stream)))
+
+
+def fa_backward_main(Q, K, V, dO, dK, dV, scale: float, causal: bool, workspace, stream=None):
+    B, H, N, d = _shape(Q)
+    s4, bf = (B, H, N, d), torch.bfloat16
+    ws, nbytes = _ws(workspace)
+    check("fa_backward_main", lib().fa_backward_main(
+        _need("Q", Q, bf, s4), _need("K", K, bf, s4), _need("V", V, bf, s4),
+        _need("dO", dO, bf, s4), _need("dK", dK, bf, s4), _need("dV", dV, bf, s4),
+        B, H, N, d, float(scale), int(bool(causal)), ws, nbytes, _stream(stream)))
+
+
+def fa_backward_dq_convert(dQ, scale: float, workspace, stream=None):
+    B, H, N, d = _shape(dQ)
+    ws, nbytes = _ws(workspace)
+    check("fa_backward_dq_convert", lib().fa_backward_dq_convert(
+        _need("dQ", dQ, torch.bfloat16, (B, H, N, d)), B, H, N, d, float(scale), ws, nbytes,
+        _stream(stream)))
 
 
 def fa_backward_f32(Q, K, V, O, dO, LSE, dQ, dK, dV, scale: float, causal: bool, workspace,

@@ -237,59 +237,123 @@ fa_status fa_forward(const void* Q, const void* K, const void* V, void* O, float
   return launch_status();
 }
 
-fa_status fa_backward(const void* Q, const void* K, const void* V, const void* O, const void* dO,
-                      const float* LSE, void* dQ, void* dK, void* dV, int B, int H, int N, int d,
-                      float scale, int causal, void* workspace, size_t workspace_bytes,
-                      fa_stream_t stream) {
+// Shared validation and set-up of the three backward stages. Fills the tensor maps
+// only when `maps` is set (the main stage is the only one that needs them).
+struct BwdPlan {
+  int BH, N, Npad, d;
+  float* L2;
+  float* Dv;
+  float* dQacc;
+};
+
+static fa_status bwd_plan(const void* const* ptrs, int nptrs, int B, int H, int N, int d,
+                          float scale, int causal, void* workspace, size_t workspace_bytes,
+                          BwdPlan* plan) {
   fa_status st = check_shape(B, H, N, d, scale, causal);
   if (st != FA_OK) return st;
+  plan->BH = B * H;
+  plan->N = N;
+  plan->d = d;
+  plan->Npad = (N + 127) / 128 * 128;
   if (N == 0) return FA_OK;
-  if ((st = check_ptrs({Q, K, V, O, dO, LSE, dQ, dK, dV, workspace})) != FA_OK) return st;
+  for (int i = 0; i < nptrs; ++i)
+    if (ptrs[i] == nullptr || !aligned16(ptrs[i])) return FA_ERR_INVALID_ARG;
+  if (workspace == nullptr || !aligned16(workspace)) return FA_ERR_INVALID_ARG;
   if (workspace_bytes < fa_backward_workspace_size(B, H, N, d)) return FA_ERR_INVALID_ARG;
   if ((st = prepare_device()) != FA_OK) return st;
-  const int BH = B * H;
-  const int Npad = (N + 127) / 128 * 128;
-  CUtensorMap mq, mk, mv, mdo;
-  if (!make_map_bf16(&mq, Q, BH, N, d, bwd::BM) || !make_map_bf16(&mk, K, BH, N, d, bwd::BN) ||
-      !make_map_bf16(&mv, V, BH, N, d, bwd::BN) || !make_map_bf16(&mdo, dO, BH, N, d, bwd::BM))
-    return FA_ERR_CUDA;
   // workspace: L2 [BH, Npad] | D [BH, Npad] | dQ accumulator [BH, N, d] (fp32)
   char* ws = static_cast<char*>(workspace);
-  const size_t vec_bytes = round256(static_cast<size_t>(BH) * Npad * sizeof(float));
-  float* L2 = reinterpret_cast<float*>(ws);
-  float* Dv = reinterpret_cast<float*>(ws + vec_bytes);
-  float* dQacc = reinterpret_cast<float*>(ws + 2 * vec_bytes);
+  const size_t vec_bytes = round256(static_cast<size_t>(plan->BH) * plan->Npad * sizeof(float));
+  plan->L2 = reinterpret_cast<float*>(ws);
+  plan->Dv = reinterpret_cast<float*>(ws + vec_bytes);
+  plan->dQacc = reinterpret_cast<float*>(ws + 2 * vec_bytes);
+  return FA_OK;
+}
+
+fa_status fa_backward_preprocess(const void* O, const void* dO, const float* LSE, int B, int H,
+                                 int N, int d, float scale, int causal, void* workspace,
+                                 size_t workspace_bytes, fa_stream_t stream) {
+  const void* ptrs[] = {O, dO, LSE};
+  BwdPlan pl;
+  fa_status st = bwd_plan(ptrs, 3, B, H, N, d, scale, causal, workspace, workspace_bytes, &pl);
+  if (st != FA_OK || N == 0) return st;
+  const long long rows = static_cast<long long>(pl.BH) * pl.Npad;
+  const unsigned blocks = static_cast<unsigned>((rows + 7) / 8);
+  const auto* O16 = static_cast<const __nv_bfloat16*>(O);
+  const auto* dO16 = static_cast<const __nv_bfloat16*>(dO);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const long long pre_rows = static_cast<long long>(BH) * Npad;
-  const unsigned pre_blocks = static_cast<unsigned>((pre_rows + 7) / 8);
+  if (d == 64)
+    bwd::fa_bwd_pre_kernel<64><<<blocks, 256, 0, s>>>(O16, dO16, LSE, pl.L2, pl.Dv, pl.dQacc, N,
+                                                      pl.Npad, rows);
+  else
+    bwd::fa_bwd_pre_kernel<128><<<blocks, 256, 0, s>>>(O16, dO16, LSE, pl.L2, pl.Dv, pl.dQacc, N,
+                                                       pl.Npad, rows);
+  return launch_status();
+}
+
+fa_status fa_backward_main(const void* Q, const void* K, const void* V, const void* dO, void* dK,
+                           void* dV, int B, int H, int N, int d, float scale, int causal,
+                           void* workspace, size_t workspace_bytes, fa_stream_t stream) {
+  const void* ptrs[] = {Q, K, V, dO, dK, dV};
+  BwdPlan pl;
+  fa_status st = bwd_plan(ptrs, 6, B, H, N, d, scale, causal, workspace, workspace_bytes, &pl);
+  if (st != FA_OK || N == 0) return st;
+  CUtensorMap mq, mk, mv, mdo;
+  if (!make_map_bf16(&mq, Q, pl.BH, N, d, bwd::BM) || !make_map_bf16(&mk, K, pl.BH, N, d, bwd::BN) ||
+      !make_map_bf16(&mv, V, pl.BH, N, d, bwd::BN) || !make_map_bf16(&mdo, dO, pl.BH, N, d, bwd::BM))
+    return FA_ERR_CUDA;
   bwd::Params p;
   p.dK = static_cast<__nv_bfloat16*>(dK);
   p.dV = static_cast<__nv_bfloat16*>(dV);
-  p.L2 = L2;
-  p.Dv = Dv;
-  p.dQacc = dQacc;
+  p.L2 = pl.L2;
+  p.Dv = pl.Dv;
+  p.dQacc = pl.dQacc;
   p.N = N;
-  p.Npad = Npad;
-  p.BH = BH;
+  p.Npad = pl.Npad;
+  p.BH = pl.BH;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.causal = causal;
   p.timeout_ns = watchdog_ns();
-  const dim3 grid(static_cast<unsigned>(Npad / bwd::BN) * BH);
-  const long long n4 = static_cast<long long>(BH) * N * d / 4;
-  const unsigned cvt_blocks = static_cast<unsigned>(std::min<long long>((n4 + 255) / 256, 148 * 16));
-  const auto* O16 = static_cast<const __nv_bfloat16*>(O);
-  const auto* dO16 = static_cast<const __nv_bfloat16*>(dO);
-  if (d == 64) {
-    bwd::fa_bwd_pre_kernel<64><<<pre_blocks, 256, 0, s>>>(O16, dO16, LSE, L2, Dv, dQacc, N, Npad, pre_rows);
+  const dim3 grid(static_cast<unsigned>(pl.Npad / bwd::BN) * pl.BH);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 64)
     bwd::fa_bwd_kernel<64><<<grid, bwd::kThreads, bwd::Cfg<64>::kSmemBytes, s>>>(mq, mk, mv, mdo, p);
-    bwd::fa_bwd_dq_kernel<64><<<cvt_blocks, 256, 0, s>>>(dQacc, static_cast<__nv_bfloat16*>(dQ), n4, scale);
-  } else {
-    bwd::fa_bwd_pre_kernel<128><<<pre_blocks, 256, 0, s>>>(O16, dO16, LSE, L2, Dv, dQacc, N, Npad, pre_rows);
+  else
     bwd::fa_bwd_kernel<128><<<grid, bwd::kThreads, bwd::Cfg<128>::kSmemBytes, s>>>(mq, mk, mv, mdo, p);
-    bwd::fa_bwd_dq_kernel<128><<<cvt_blocks, 256, 0, s>>>(dQacc, static_cast<__nv_bfloat16*>(dQ), n4, scale);
-  }
   return launch_status();
+}
+
+fa_status fa_backward_dq_convert(void* dQ, int B, int H, int N, int d, float scale, void* workspace,
+                                 size_t workspace_bytes, fa_stream_t stream) {
+  const void* ptrs[] = {dQ};
+  BwdPlan pl;
+  fa_status st = bwd_plan(ptrs, 1, B, H, N, d, scale, 0, workspace, workspace_bytes, &pl);
+  if (st != FA_OK || N == 0) return st;
+  const long long n4 = static_cast<long long>(pl.BH) * N * d / 4;
+  const unsigned blocks = static_cast<unsigned>(std::min<long long>((n4 + 255) / 256, 148 * 16));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 64)
+    bwd::fa_bwd_dq_kernel<64><<<blocks, 256, 0, s>>>(pl.dQacc, static_cast<__nv_bfloat16*>(dQ), n4, scale);
+  else
+    bwd::fa_bwd_dq_kernel<128><<<blocks, 256, 0, s>>>(pl.dQacc, static_cast<__nv_bfloat16*>(dQ), n4, scale);
+  return launch_status();
+}
+
+fa_status fa_backward(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                      const float* LSE, void* dQ, void* dK, void* dV, int B, int H, int N, int d,
+                      float scale, int causal, void* workspace, size_t workspace_bytes,
+                      fa_stream_t stream) {
+  const void* ptrs[] = {Q, K, V, O, dO, LSE, dQ, dK, dV};
+  BwdPlan pl;
+  fa_status st = bwd_plan(ptrs, 9, B, H, N, d, scale, causal, workspace, workspace_bytes, &pl);
+  if (st != FA_OK || N == 0) return st;
+  st = fa_backward_preprocess(O, dO, LSE, B, H, N, d, scale, causal, workspace, workspace_bytes, stream);
+  if (st != FA_OK) return st;
+  st = fa_backward_main(Q, K, V, dO, dK, dV, B, H, N, d, scale, causal, workspace, workspace_bytes,
+                        stream);
+  if (st != FA_OK) return st;
+  return fa_backward_dq_convert(dQ, B, H, N, d, scale, workspace, workspace_bytes, stream);
 }
 
 fa_status fa_forward_f32(const float* Q, const float* K, const float* V, float* O, float* LSE,
