@@ -119,6 +119,32 @@ fa_status fa_backward_dq_convert(void* dQ, int B, int H, int N, int d, float sca
                                  void* workspace, size_t workspace_bytes, fa_stream_t stream);
 
 /*
+ * fa_backward without a workspace argument, for callers that cannot allocate
+ * device memory (for example code that must not call cudaMalloc because it may
+ * synchronise the device, plugins whose host application owns every allocation,
+ * or programs whose memory is all reserved by their own pool). The sources this
+ * library follows have no counterpart: it is a deployment convenience.
+ *   Arguments, outputs and numerics: as for fa_backward.
+ *   Scratch: a 32 MiB array built into the library, one per GPU, placed in device
+ *     memory when the library's module is loaded on that GPU and held until the
+ *     process exits. The call allocates nothing.
+ *   Limit: shapes whose fa_backward_workspace_size exceeds 32 MiB (33554432
+ *     bytes) return FA_ERR_UNSUPPORTED and launch nothing.
+ *   Set-up: the first call on a GPU looks up the array's device address with
+ *     that GPU current (and may load the library's module there); make that first
+ *     call before any stream capture.
+ *   Sharing: every call on a GPU uses the same array. Each call rewrites all of
+ *     it that it reads (the dQ accumulator is zeroed by the call itself), but two
+ *     calls whose kernels can overlap on the GPU (different streams without an
+ *     ordering between them, or different host threads) race on it and give
+ *     wrong results. Order such calls on one stream.
+ */
+fa_status fa_backward_noalloc(const void* Q, const void* K, const void* V, const void* O,
+                              const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
+                              int B, int H, int N, int d, float scale, int causal,
+                              fa_stream_t stream);
+
+/*
  * fp32 entry points: the same operation and arguments with fp32 tensors
  * (float [B,H,N,d]), computed in fp32 on the CUDA cores (FFMA), for callers that
  * need fp32 accuracy; tensor-core fp32 (tf32) cannot reach it. The backward is

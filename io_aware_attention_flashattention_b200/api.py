@@ -23,7 +23,8 @@ from ._lib import FAError, check, lib
 
 __all__ = [
     "FAError", "fa_forward", "fa_backward", "fa_backward_workspace_size",
-    "fa_backward_preprocess", "fa_backward_main", "fa_backward_dq_convert", "fa_forward_f32",
+    "fa_backward_preprocess", "fa_backward_main", "fa_backward_dq_convert",
+    "fa_backward_noalloc", "fa_forward_f32",
     "fa_backward_f32", "fa_get_status", "fa_watchdog_selftest", "fa_version",
     "forward", "backward", "attention", "FlashAttentionFunction",
 ]
@@ -135,6 +136,23 @@ def fa_backward_dq_convert(dQ, scale: float, workspace, stream=None):
     check("fa_backward_dq_convert", lib().fa_backward_dq_convert(
         _need("dQ", dQ, torch.bfloat16, (B, H, N, d)), B, H, N, d, float(scale), ws, nbytes,
         _stream(stream)))
+
+
+def fa_backward_noalloc(Q, K, V, O, dO, LSE, dQ, dK, dV, scale: float, causal: bool,
+                        stream=None) -> None:
+    """fa_backward for callers that cannot allocate device memory: the workspace
+    is a fixed 32 MiB array inside the library (one per GPU). Shapes needing more
+    raise FAError (FA_ERR_UNSUPPORTED). Calls on one GPU share the array, so they
+    must not overlap: keep them on one stream. The first call on a GPU does a
+    one-time look-up of the array's address; make it before any stream capture."""
+    B, H, N, d = _shape(Q)
+    s4, bf = (B, H, N, d), torch.bfloat16
+    ptrs = [_need("Q", Q, bf, s4), _need("K", K, bf, s4), _need("V", V, bf, s4),
+            _need("O", O, bf, s4), _need("dO", dO, bf, s4),
+            _need("LSE", LSE, torch.float32, (B, H, N)),
+            _need("dQ", dQ, bf, s4), _need("dK", dK, bf, s4), _need("dV", dV, bf, s4)]
+    check("fa_backward_noalloc", lib().fa_backward_noalloc(
+        *ptrs, B, H, N, d, float(scale), int(bool(causal)), _stream(stream)))
 
 
 def fa_backward_f32(Q, K, V, O, dO, LSE, dQ, dK, dV, scale: float, causal: bool, workspace,

@@ -356,6 +356,52 @@ fa_status fa_backward(const void* Q, const void* K, const void* V, const void* O
   return fa_backward_dq_convert(dQ, B, H, N, d, scale, workspace, workspace_bytes, stream);
 }
 
+// ---------------------------------------------------------------- backward without allocation
+//
+// fa_backward needs a caller-provided device workspace. Some callers cannot make
+// one: code that must not call cudaMalloc because the call can synchronise the
+// whole device in the middle of latency-critical work, plugins whose host
+// application owns every device allocation, or programs that reserved all of the
+// device's memory up front for their own pool. For them, fa_backward_noalloc
+// keeps the workspace in this fixed array, which the CUDA runtime places in device
+// memory when the library's module is loaded on a GPU; it stays there, on every
+// GPU that loads the library, until the process exits.
+constexpr size_t kNoAllocScratchBytes = 32ull << 20;  // 32 MiB per GPU
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+// Device address of g_noalloc_scratch on each GPU. In host code the array's name
+// only stands in for the symbol; the address a kernel may use comes from
+// cudaGetSymbolAddress with that GPU current.
+static void* g_noalloc_ptr[kMaxDevices];
+
+fa_status fa_backward_noalloc(const void* Q, const void* K, const void* V, const void* O,
+                              const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
+                              int B, int H, int N, int d, float scale, int causal,
+                              fa_stream_t stream) {
+  fa_status st = check_shape(B, H, N, d, scale, causal);
+  if (st != FA_OK) return st;
+  if (N == 0) return FA_OK;
+  if (fa_backward_workspace_size(B, H, N, d) > kNoAllocScratchBytes) return FA_ERR_UNSUPPORTED;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
+  void* scratch = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_mutex);
+    if (g_noalloc_ptr[dev] == nullptr) {
+      void* p = nullptr;
+      if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
+        return FA_ERR_CUDA;
+      g_noalloc_ptr[dev] = p;
+    }
+    scratch = g_noalloc_ptr[dev];
+  }
+  // The preprocess stage rewrites every byte of scratch the later stages read
+  // (LSE*log2e, D, and the dQ accumulator it zeroes), so whatever an earlier call
+  // left in the array does not matter.
+  return fa_backward(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, scale, causal, scratch,
+                     kNoAllocScratchBytes, stream);
+}
+
 fa_status fa_forward_f32(const float* Q, const float* K, const float* V, float* O, float* LSE,
                          int B, int H, int N, int d, float scale, int causal,
                          fa_stream_t stream) {
