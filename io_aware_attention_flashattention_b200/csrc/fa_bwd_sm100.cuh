@@ -12,22 +12,29 @@
 //   1. fa_bwd_pre_kernel: D_i and L2_i = LSE_i*log2(e) into [B*H, Npad] (padding
 //      rows get D = 0, L2 = +inf so that they contribute nothing), and zero the
 //      fp32 dQ accumulator.
-//   2. fa_bwd_kernel (one CTA per SM, 320 threads): the CTA owns one tile of 128
+//   2. fa_bwd_kernel (one CTA per SM, 512 threads): the CTA owns one tile of 128
 //      keys K_j, V_j and streams the query tiles Q_i, dO_i (128 rows) through a
-//      ring of shared-memory slots with TMA.
-//        warp 9 (MMA, one thread): S^T = K_j Q_i^T and dP^T = V_j dO_i^T into TMEM;
-//          dV += P^T dO_i and dK += dS^T Q_i with P^T and dS^T read from TMEM;
-//          dQ_i = dS K_j with dS read from shared memory.
-//        warps 0-3 (one thread per key row): P^T = 2^(S^T c - L2), masked;
-//          dS^T = P^T (dP^T - D); both rounded to bf16 and stored back into TMEM
-//          over S^T and dP^T, and dS also into shared memory for the dQ MMA.
-//          At the end they write dK (times scale) and dV once.
-//        warps 4-7 (one thread per query row): read dQ_i from TMEM and add it into
-//          the fp32 accumulator with vector reductions (red.global.add.v4.f32).
-//        warp 8: TMA producer.
-//      TMEM (512 columns): dK [0,D), dV [D,2D), S^T [2D,2D+128), dP^T [2D+128,2D+256);
-//      P^T and dS^T (bf16 pairs) alias the first 64 columns of S^T and dP^T. dQ_i
-//      uses S^T's columns when D = 128 and its own columns [384,448) when D = 64.
+//      ring of shared-memory slots with TMA. Each query tile is processed as two
+//      halves of 64 queries (h = 0, 1) so that the MMAs of one half overlap the
+//      elementwise work of the other.
+//        warp 13 (MMA, one thread), per half h: S^T_h = K_j Q_ih^T and
+//          dP^T_h = V_j dO_ih^T into TMEM; dV += P^T_h dO_ih and dK += dS^T_h Q_ih
+//          with P^T_h and dS^T_h read from TMEM; for D = 128, dQ^T_h = K_j^T dS^T_h
+//          (M = 128 head-dimension rows, N = 64 queries) into the columns S^T_h
+//          used; for D = 64, after both halves, dQ_i = dS K_j into its own columns.
+//        warps 4h..4h+3 (one thread per key row, queries of half h): P^T = 2^(S^T c
+//          - L2), masked on diagonal and ragged tiles only; dS^T = P^T (dP^T - D);
+//          both rounded to bf16 and stored back into TMEM over S^T_h and dP^T_h, and
+//          dS also into a 128-byte-swizzled shared tile for the dQ MMA. At the end
+//          warps 0-3 write dK (times scale) and warps 4-7 write dV, once.
+//        warps 8-11: read dQ from TMEM and add it into the fp32 accumulator. For
+//          D = 128 a thread owns one head-dimension element, so a warp's 32 adds
+//          for one query hit 128 contiguous bytes; for D = 64 a thread owns a query
+//          row and uses 16-byte vector adds.
+//        warp 12: TMA producer.
+//      TMEM (512 columns): dK [0,D), dV [D,2D), S^T [2D,2D+128), dP^T [2D+128,2D+256),
+//      half h at +64h; P^T_h and dS^T_h (bf16 pairs) alias the first 32 columns of
+//      their half.
 //   3. fa_bwd_dq_kernel: dQ = bf16(scale * accumulator).
 // No N x N matrix is written to device memory.
 #pragma once
@@ -39,38 +46,42 @@ namespace bwd {
 
 constexpr int BM = 128;        // query rows per step
 constexpr int BN = 128;        // key rows per CTA
-constexpr int kThreads = 320;
-constexpr int kWarpTma = 8;
-constexpr int kWarpMma = 9;
+constexpr int kThreads = 512;
+constexpr int kWarpDq = 8;     // first of the 4 dQ warps
+constexpr int kWarpTma = 12;
+constexpr int kWarpMma = 13;
 
 template <int D>
 struct Cfg {
-  static constexpr int kChunkBytes = 128 * 128;  // 128 rows x 64 bf16
+  static constexpr int kChunkBytes = 128 * 128;  // 128 rows x 64 bf16 (K, V, dS)
   static constexpr int kChunks = D / 64;
   static constexpr int kTileBytes = kChunks * kChunkBytes;  // 128 x D bf16
-  static constexpr int kSlots = (D == 128) ? 3 : 6;         // Q/dO ring
-  static constexpr int kVecBytes = BM * 4;                   // 128 fp32 (L2 or D)
+  // Q and dO stream in half tiles (64 rows x D): 64-row chunks of 8 KB
+  static constexpr int kHalfChunkBytes = 64 * 128;
+  static constexpr int kHalfBytes = kChunks * kHalfChunkBytes;
+  static constexpr int kSlots = (D == 128) ? 6 : 12;  // half-tile ring
+  static constexpr int kVecBytes = 64 * 4;             // 64 fp32 (L2 or D of a half)
   static constexpr int kKOff = 0;
   static constexpr int kVOff = kTileBytes;
   static constexpr int kRingOff = 2 * kTileBytes;
-  static constexpr int kDSOff = kRingOff + kSlots * kTileBytes;  // dS, 128 x 128 bf16
+  static constexpr int kDSOff = kRingOff + kSlots * kHalfBytes;  // dS: 2 chunks of 64 queries
   static constexpr int kDSBytes = 2 * kChunkBytes;
-  static constexpr int kVecOff = kDSOff + kDSBytes;  // per slot: L2[128], D[128]
+  static constexpr int kVecOff = kDSOff + kDSBytes;  // per slot: L2[64], D[64]
   static constexpr int kBarOff = kVecOff + kSlots * 2 * kVecBytes;
   static constexpr int kBarKV = 0;
   static constexpr int kBarFull = 1;
   static constexpr int kBarEmpty = 1 + kSlots;
-  static constexpr int kBarS = 1 + 2 * kSlots;
-  static constexpr int kBarP = kBarS + 1;
-  static constexpr int kBarDQFull = kBarP + 1;
-  static constexpr int kBarDQEmpty = kBarDQFull + 1;
-  static constexpr int kBarDKDV = kBarDQEmpty + 1;
+  static constexpr int kBarS = 1 + 2 * kSlots;  // [2]
+  static constexpr int kBarP = kBarS + 2;       // [2]
+  static constexpr int kBarDQFull = kBarP + 2;  // [2]
+  static constexpr int kBarDQEmpty = kBarDQFull + 2;  // [2]
+  static constexpr int kBarDKDV = kBarDQEmpty + 2;
   static constexpr int kBarDrain = kBarDKDV + 1;
   static constexpr int kNumBars = kBarDrain + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kSmemBytes = kMiscOff + 16 + 1024;
   static constexpr uint32_t kTmDK = 0, kTmDV = D, kTmS = 2 * D, kTmDP = 2 * D + 128;
-  static constexpr uint32_t kTmDQ = (D == 128) ? kTmS : 384;
+  static constexpr uint32_t kTmDQ64 = 384;  // D = 64 only
   static constexpr uint32_t kTmCols = 512;
 };
 
@@ -108,6 +119,10 @@ __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float 
                : "memory");
 }
 
+__device__ __forceinline__ void red_add(float* addr, float a) {
+  asm volatile("red.global.add.f32 [%0], %1;" ::"l"(addr), "f"(a) : "memory");
+}
+
 __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
   const uint64_t t0 = globaltimer_ns();
   while (!mbar_try_wait(bar, parity)) {
@@ -118,40 +133,53 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
   }
 }
 
-// S^T (or dP^T) = X_j Y_i^T: M = 128 rows of X, N = 128 rows of Y, K = D; both
-// operands K-major in 128-byte-swizzled tiles.
+// X_j Y_h^T: M = 128 rows of X, N = 64 rows of the half tile Y_h, K = D; both
+// operands K-major (rows of 64 bf16 per 128-byte-swizzled chunk).
 template <int D>
-__device__ __forceinline__ void issue_xyT(uint32_t tm_d, uint32_t x_smem, uint32_t y_smem) {
-  constexpr uint32_t idesc = idesc_bf16_f32(128, 128, 0, 0);
+__device__ __forceinline__ void issue_xyT_half(uint32_t tm_d, uint32_t x_smem, uint32_t yh_smem) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, 64, 0, 0);
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t off = (kk / 4) * Cfg<D>::kChunkBytes + (kk % 4) * 32;
-    mma_ss(tm_d, sdesc_sw128(x_smem + off, 16, 1024), sdesc_sw128(y_smem + off, 16, 1024), idesc,
+    const uint32_t xo = (kk / 4) * Cfg<D>::kChunkBytes + (kk % 4) * 32;
+    const uint32_t yo = (kk / 4) * Cfg<D>::kHalfChunkBytes + (kk % 4) * 32;
+    mma_ss(tm_d, sdesc_sw128(x_smem + xo, 16, 1024), sdesc_sw128(yh_smem + yo, 16, 1024), idesc,
            kk > 0 ? 1u : 0u);
   }
 }
 
-// acc[128 x D] (+)= A_tmem[128 x 128] * Y[128 x D], Y a row-major tile in shared
-// memory used as the MN-major B operand.
+// acc[128 keys x D] (+)= A_tmem[128 keys x 64 queries] * Y_h[64 queries x D] (the half
+// tile, row-major in shared memory, used as the MN-major B operand).
 template <int D>
-__device__ __forceinline__ void issue_ts_acc(uint32_t tm_acc, uint32_t tm_a, uint32_t y_smem,
-                                             bool accumulate) {
+__device__ __forceinline__ void issue_acc_half(uint32_t tm_acc, uint32_t tm_a, uint32_t yh_smem,
+                                               bool accumulate) {
   constexpr uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);
 #pragma unroll
-  for (int kk = 0; kk < 128 / 16; ++kk)
-    mma_ts(tm_acc, tm_a + kk * 8, sdesc_sw128(y_smem + kk * 2048, Cfg<D>::kChunkBytes, 1024), idesc,
+  for (int kk = 0; kk < 64 / 16; ++kk)
+    mma_ts(tm_acc, tm_a + kk * 8,
+           sdesc_sw128(yh_smem + kk * 2048, Cfg<D>::kHalfChunkBytes, 1024), idesc,
            (accumulate || kk > 0) ? 1u : 0u);
 }
 
-// dQ_i[128 queries x D] = dS[queries x keys] * K_j[keys x D]: A is the dS tile
-// (stored key-row-major, i.e. MN-major for A), B is K_j (MN-major).
-template <int D>
-__device__ __forceinline__ void issue_dq(uint32_t tm_dq, uint32_t ds_smem, uint32_t k_smem) {
-  constexpr uint32_t idesc = idesc_bf16_f32(128, D, 1, 1);
+// D = 128: dQ^T_h[128 dims x 64 queries] = K_j^T[dims x keys] * dS_h^T[keys x queries]:
+// A = K_j read MN-major (dims contiguous), B = dS chunk h read MN-major (queries
+// contiguous in each key row).
+__device__ __forceinline__ void issue_dqT_half(uint32_t tm_d, uint32_t k_smem, uint32_t ds_chunk) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, 64, 1, 1);
 #pragma unroll
   for (int kk = 0; kk < 128 / 16; ++kk)
-    mma_ss(tm_dq, sdesc_sw128(ds_smem + kk * 2048, Cfg<D>::kChunkBytes, 1024),
-           sdesc_sw128(k_smem + kk * 2048, Cfg<D>::kChunkBytes, 1024), idesc, kk > 0 ? 1u : 0u);
+    mma_ss(tm_d, sdesc_sw128(k_smem + kk * 2048, Cfg<128>::kChunkBytes, 1024),
+           sdesc_sw128(ds_chunk + kk * 2048, Cfg<128>::kChunkBytes, 1024), idesc,
+           kk > 0 ? 1u : 0u);
+}
+
+// D = 64: dQ_i[128 queries x 64] = dS[queries x keys] * K_j[keys x 64]: A = the whole
+// dS tile (MN-major, two 64-query chunks), B = K_j (MN-major).
+__device__ __forceinline__ void issue_dq64(uint32_t tm_d, uint32_t ds_smem, uint32_t k_smem) {
+  constexpr uint32_t idesc = idesc_bf16_f32(128, 64, 1, 1);
+#pragma unroll
+  for (int kk = 0; kk < 128 / 16; ++kk)
+    mma_ss(tm_d, sdesc_sw128(ds_smem + kk * 2048, Cfg<64>::kChunkBytes, 1024),
+           sdesc_sw128(k_smem + kk * 2048, Cfg<64>::kChunkBytes, 1024), idesc, kk > 0 ? 1u : 0u);
 }
 
 // ------------------------------------------------------------------ preprocess
@@ -253,10 +281,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(C::kBarFull + s), 1);
       mbar_init(bar(C::kBarEmpty + s), 1);
     }
-    mbar_init(bar(C::kBarS), 1);
-    mbar_init(bar(C::kBarP), 4);
-    mbar_init(bar(C::kBarDQFull), 1);
-    mbar_init(bar(C::kBarDQEmpty), 4);
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(bar(C::kBarS + h), 1);
+      mbar_init(bar(C::kBarP + h), 4);        // the 4 warps of half h
+      mbar_init(bar(C::kBarDQFull + h), 1);
+      mbar_init(bar(C::kBarDQEmpty + h), 4);  // the 4 dQ warps
+    }
     mbar_init(bar(C::kBarDKDV), 1);
     mbar_init(bar(C::kBarDrain), 1);
     *abort_flag = 0;
@@ -272,11 +302,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const Watchdog wd{abort_flag, p.timeout_ns};
 
-  // ring sequence: seq = 2*step + w, w = 0 for Q_i (with L2_i, D_i), 1 for dO_i
+  // ring of half tiles: seq = 4*step + 2*h + w, w = 0 for dO (rows 64h.. of query
+  // tile i), w = 1 for Q (with L2 and D of those 64 queries)
+  auto seq_of = [](int s, int h, int w) { return 4 * s + 2 * h + w; };
   auto slot_of = [&](int seq) { return seq % C::kSlots; };
   auto round_of = [&](int seq) { return seq / C::kSlots; };
   auto slot_smem = [&](int seq) -> uint32_t {
-    return base + C::kRingOff + slot_of(seq) * C::kTileBytes;
+    return base + C::kRingOff + slot_of(seq) * C::kHalfBytes;
   };
 
   if (warp == kWarpTma) {
@@ -295,8 +327,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       for (int s = 0; s < nsteps && ok; ++s) {
         const int i = i_begin + s;
-        for (int w = 0; w < 2; ++w) {
-          const int seq = 2 * s + w;
+        for (int hw = 0; hw < 4 && ok; ++hw) {
+          const int h = hw >> 1, w = hw & 1;
+          const int seq = seq_of(s, h, w);
           const int slot = slot_of(seq);
           const int rnd = round_of(seq);
           if (rnd > 0 && !mbar_wait(bar(C::kBarEmpty + slot), (rnd - 1) & 1, wd)) {
@@ -305,17 +338,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           const uint32_t full = bar(C::kBarFull + slot);
           const uint32_t dst = slot_smem(seq);
-          if (w == 0) {
-            mbar_arrive_expect_tx(full, C::kTileBytes + 2 * C::kVecBytes);
+          const int row0 = i * BM + 64 * h;
+          if (w == 1) {
+            mbar_arrive_expect_tx(full, C::kHalfBytes + 2 * C::kVecBytes);
             const uint32_t vec = base + C::kVecOff + slot * 2 * C::kVecBytes;
-            const size_t off = static_cast<size_t>(bh) * p.Npad + static_cast<size_t>(i) * BM;
+            const size_t off = static_cast<size_t>(bh) * p.Npad + static_cast<size_t>(row0);
             bulk_load(vec, p.L2 + off, C::kVecBytes, full);
             bulk_load(vec + C::kVecBytes, p.Dv + off, C::kVecBytes, full);
           } else {
-            mbar_arrive_expect_tx(full, C::kTileBytes);
+            mbar_arrive_expect_tx(full, C::kHalfBytes);
           }
           for (int c = 0; c < C::kChunks; ++c)
-            tma_load_3d(dst + c * C::kChunkBytes, w ? &tmdO : &tmQ, full, c * 64, i * BM, bh);
+            tma_load_3d(dst + c * C::kHalfChunkBytes, w ? &tmQ : &tmdO, full, c * 64, row0, bh);
           issued = seq + 1;
         }
       }
@@ -334,167 +368,206 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto wait_full = [&](int seq) -> bool {
         return mbar_wait(bar(C::kBarFull + slot_of(seq)), round_of(seq) & 1, wd);
       };
-      if (ok && nsteps > 0) {
-        ok = wait_full(0) && wait_full(1);
-        if (ok) {
+      // S^T and dP^T of both halves of step s (dP^T first: its columns free up earlier)
+      auto issue_sdp = [&](int s) -> bool {
+        for (int h = 0; h < 2; ++h) {
+          const int seqO = seq_of(s, h, 0), seqQ = seq_of(s, h, 1);
+          if (!(wait_full(seqO) && wait_full(seqQ))) return false;
           tc_fence_after();
-          issue_xyT<D>(tm_s, k_smem, slot_smem(0));   // S^T = K Q^T
-          issue_xyT<D>(tm_dp, v_smem, slot_smem(1));  // dP^T = V dO^T
-          tc_commit(bar(C::kBarS));
-        }
-      }
-      for (int s = 0; s < nsteps && ok; ++s) {
-        const int seqQ = 2 * s, seqO = 2 * s + 1;
-        if (!mbar_wait(bar(C::kBarP), s & 1, wd)) { ok = false; break; }
-        tc_fence_after();
-        issue_ts_acc<D>(tmem + C::kTmDV, tm_s, slot_smem(seqO), s > 0);   // dV += P^T dO
-        issue_ts_acc<D>(tmem + C::kTmDK, tm_dp, slot_smem(seqQ), s > 0);  // dK += dS^T Q
-        if (D == 64 && s > 0) {  // dQ region reused: the previous dQ must have been read
-          if (!mbar_wait(bar(C::kBarDQEmpty), (s - 1) & 1, wd)) { ok = false; break; }
-          tc_fence_after();
-        }
-        issue_dq<D>(tmem + C::kTmDQ, ds_smem, k_smem);
-        tc_commit(bar(C::kBarDQFull));
-        tc_commit(bar(C::kBarEmpty + slot_of(seqQ)));
-        tc_commit(bar(C::kBarEmpty + slot_of(seqO)));
-        if (s + 1 < nsteps) {
-          if (!(wait_full(seqQ + 2) && wait_full(seqO + 2))) { ok = false; break; }
-          tc_fence_after();
-          issue_xyT<D>(tm_dp, v_smem, slot_smem(seqO + 2));  // dP^T for the next step
-          if (D == 128) {  // S^T shares columns with dQ: wait until dQ has been read
-            if (!mbar_wait(bar(C::kBarDQEmpty), s & 1, wd)) { ok = false; break; }
+          issue_xyT_half<D>(tm_dp + 64 * h, v_smem, slot_smem(seqO));
+          if (D == 128 && s > 0) {  // S^T_h shares columns with dQ^T_h of the last step
+            if (!mbar_wait(bar(C::kBarDQEmpty + h), (s - 1) & 1, wd)) return false;
             tc_fence_after();
           }
-          issue_xyT<D>(tm_s, k_smem, slot_smem(seqQ + 2));
-          tc_commit(bar(C::kBarS));
+          issue_xyT_half<D>(tm_s + 64 * h, k_smem, slot_smem(seqQ));
+          tc_commit(bar(C::kBarS + h));
         }
+        return true;
+      };
+      if (ok && nsteps > 0) ok = issue_sdp(0);
+      for (int s = 0; s < nsteps && ok; ++s) {
+        for (int h = 0; h < 2 && ok; ++h) {
+          const int seqO = seq_of(s, h, 0), seqQ = seq_of(s, h, 1);
+          if (!mbar_wait(bar(C::kBarP + h), s & 1, wd)) { ok = false; break; }
+          tc_fence_after();
+          const bool acc = (s > 0) || (h > 0);
+          issue_acc_half<D>(tmem + C::kTmDV, tm_s + 64 * h, slot_smem(seqO), acc);   // dV
+          issue_acc_half<D>(tmem + C::kTmDK, tm_dp + 64 * h, slot_smem(seqQ), acc);  // dK
+          if constexpr (D == 128) {
+            issue_dqT_half(tm_s + 64 * h, k_smem, ds_smem + h * C::kChunkBytes);
+            tc_commit(bar(C::kBarDQFull + h));
+          }
+          tc_commit(bar(C::kBarEmpty + slot_of(seqO)));
+          tc_commit(bar(C::kBarEmpty + slot_of(seqQ)));
+        }
+        if (!ok) break;
+        if constexpr (D == 64) {
+          if (s > 0) {  // the dQ columns are reused: the previous dQ must have been read
+            if (!mbar_wait(bar(C::kBarDQEmpty), (s - 1) & 1, wd)) { ok = false; break; }
+            tc_fence_after();
+          }
+          issue_dq64(tmem + C::kTmDQ64, ds_smem, k_smem);
+          tc_commit(bar(C::kBarDQFull));
+        }
+        if (s + 1 < nsteps) ok = issue_sdp(s + 1);
       }
       if (ok) tc_commit(bar(C::kBarDKDV));
       tc_commit(bar(C::kBarDrain));
       drain_wait(bar(C::kBarDrain), 0, p.timeout_ns);
     }
     __syncwarp();
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ P^T, dS^T (key rows)
-    const int krow = warp * 32 + lane;  // key row within the tile = TMEM lane
+    const int h = warp >> 2;                  // query half
+    const int krow = (warp & 3) * 32 + lane;  // key row within the tile = TMEM lane
     const int key = k0 + krow;
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-    const uint32_t tm_s = tmem + lane_off + C::kTmS;
-    const uint32_t tm_dp = tmem + lane_off + C::kTmDP;
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tm_s = tmem + lane_off + C::kTmS + 64 * h;
+    const uint32_t tm_dp = tmem + lane_off + C::kTmDP + 64 * h;
     const float c = p.scale_log2;
-    uint8_t* ds_row = base_ptr + C::kDSOff + krow * 128;
+    uint8_t* ds_row = base_ptr + C::kDSOff + h * C::kChunkBytes + krow * 128;
+    const bool ragged_keys = k0 + BN > p.N;
+    const int dq_bar = (D == 128) ? C::kBarDQFull + h : C::kBarDQFull;
     bool ok = true;
     for (int s = 0; s < nsteps && ok; ++s) {
       const int i = i_begin + s;
-      const int q0 = i * BM;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarS), s & 1, wd));
-      if (ok && s > 0)  // the previous dQ MMA has finished reading the dS tile
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarDQFull), (s - 1) & 1, wd));
-      // L2_i and D_i arrived with Q_i: observe that copy's barrier directly
+      const int qh0 = i * BM + 64 * h;  // first query of this half
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarS + h), s & 1, wd));
+      if (ok && s > 0)  // the dQ MMA of the last step has finished reading this dS chunk
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(dq_bar), (s - 1) & 1, wd));
+      // L2 and D of this half arrived with its Q rows: observe that copy's barrier
+      const int seqQ = seq_of(s, h, 1);
       if (ok)
         ok = __all_sync(0xffffffffu,
-                        mbar_wait(bar(C::kBarFull + slot_of(2 * s)), round_of(2 * s) & 1, wd));
+                        mbar_wait(bar(C::kBarFull + slot_of(seqQ)), round_of(seqQ) & 1, wd));
       if (!ok) break;
       tc_fence_after();
-      const int slot = slot_of(2 * s);
-      const float* Lv = reinterpret_cast<const float*>(base_ptr + C::kVecOff + slot * 2 * C::kVecBytes);
-      const float* Dvv = Lv + BM;
-      // query columns q0 + [lim, 128) are visible to this key: causal needs q >= key
-      const int lim = p.causal ? max(0, key - q0) : 0;
-      const bool key_valid = key < p.N;
-#pragma unroll 1
+      const float4* Lv = reinterpret_cast<const float4*>(
+          base_ptr + C::kVecOff + slot_of(seqQ) * 2 * C::kVecBytes);
+      const float4* Dv4 = Lv + 64 / 4;
+      // masking is needed only on the causal diagonal step and on a ragged key tile
+      const bool mask = (p.causal && i == j) || ragged_keys;
+      const int lim = !(key < p.N) ? 1 << 30 : (p.causal ? key - qh0 : -1);  // q index < lim masked
+      uint32_t sv[2][16], dv[2][16];
+      tmem_ld16(tm_s, sv[0]);
+      tmem_ld16(tm_dp, dv[0]);
+      tmem_wait_ld();
+#pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
-        uint32_t sv[32], dv[32];
-        tmem_ld32(tm_s + cc * 32, sv);
-        tmem_ld32(tm_dp + cc * 32, dv);
-        tmem_wait_ld();
-        uint32_t pk[16], dk[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const int qa = cc * 32 + 2 * k, qb = qa + 1;
-          float pa = ex2_approx(fmaf(__uint_as_float(sv[2 * k]), c, -Lv[qa]));
-          float pb = ex2_approx(fmaf(__uint_as_float(sv[2 * k + 1]), c, -Lv[qb]));
-          if (!key_valid || qa < lim) pa = 0.f;
-          if (!key_valid || qb < lim) pb = 0.f;
-          const float da = pa * (__uint_as_float(dv[2 * k]) - Dvv[qa]);
-          const float db = pb * (__uint_as_float(dv[2 * k + 1]) - Dvv[qb]);
-          pk[k] = pack_bf16x2(pa, pb);
-          dk[k] = pack_bf16x2(da, db);
+        const int cur = cc & 1;
+        if (cc + 1 < 4) {  // the next chunk's loads overlap this chunk's arithmetic
+          tmem_ld16(tm_s + 16 * (cc + 1), sv[cur ^ 1]);
+          tmem_ld16(tm_dp + 16 * (cc + 1), dv[cur ^ 1]);
         }
-        tmem_st16(tm_s + cc * 16, pk);
-        tmem_st16(tm_dp + cc * 16, dk);
-        // dS tile in shared memory: chunk of 64 queries = cc/2, 16-byte units
-        // (cc%2)*4 .. +3 of this key's 128-byte row, 128-byte swizzle.
-        uint8_t* chunk = ds_row + (cc >> 1) * C::kChunkBytes;
+        uint32_t pk[8], dk[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int unit = ((cc & 1) * 4 + u) ^ (krow & 7);
-          *reinterpret_cast<uint4*>(chunk + unit * 16) =
-              make_uint4(dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
+        for (int v = 0; v < 4; ++v) {
+          const float4 L4 = Lv[cc * 4 + v];
+          const float4 D4 = Dv4[cc * 4 + v];
+          const float Ls[4] = {L4.x, L4.y, L4.z, L4.w};
+          const float Ds[4] = {D4.x, D4.y, D4.z, D4.w};
+          float pv[4], dsv[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int k = 4 * v + e;
+            float pe = ex2_approx(fmaf(__uint_as_float(sv[cur][k]), c, -Ls[e]));
+            if (mask && (cc * 16 + k) < lim) pe = 0.f;
+            pv[e] = pe;
+            dsv[e] = pe * (__uint_as_float(dv[cur][k]) - Ds[e]);
+          }
+          pk[2 * v] = pack_bf16x2(pv[0], pv[1]);
+          pk[2 * v + 1] = pack_bf16x2(pv[2], pv[3]);
+          dk[2 * v] = pack_bf16x2(dsv[0], dsv[1]);
+          dk[2 * v + 1] = pack_bf16x2(dsv[2], dsv[3]);
         }
+        tmem_st8(tm_s + 8 * cc, pk);
+        tmem_st8(tm_dp + 8 * cc, dk);
+        // dS into the swizzled shared chunk: 16 queries = 16-byte units 2cc, 2cc+1
+        *reinterpret_cast<uint4*>(ds_row + (((2 * cc) ^ (krow & 7)) * 16)) =
+            make_uint4(dk[0], dk[1], dk[2], dk[3]);
+        *reinterpret_cast<uint4*>(ds_row + (((2 * cc + 1) ^ (krow & 7)) * 16)) =
+            make_uint4(dk[4], dk[5], dk[6], dk[7]);
+        if (cc + 1 < 4) tmem_wait_ld();
       }
       tmem_wait_st();
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(bar(C::kBarP));
+      if (lane == 0) mbar_arrive(bar(C::kBarP + h));
     }
     if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarDKDV), 0, wd));
     if (ok && nsteps > 0) {
+      // warps 0-3 write dK (times scale), warps 4-7 write dV
       tc_fence_after();
-      const uint32_t tm_dk = tmem + lane_off + C::kTmDK;
-      const uint32_t tm_dv = tmem + lane_off + C::kTmDV;
+      const uint32_t tm_acc = tmem + lane_off + (h == 0 ? C::kTmDK : C::kTmDV);
+      __nv_bfloat16* out = (h == 0 ? p.dK : p.dV) + (static_cast<size_t>(bh) * p.N + key) * D;
+      const float mul = (h == 0) ? p.scale : 1.0f;
 #pragma unroll 1
-      for (int which = 0; which < 2; ++which) {
-        __nv_bfloat16* out = (which == 0 ? p.dK : p.dV) + (static_cast<size_t>(bh) * p.N + key) * D;
-        const float mul = (which == 0) ? p.scale : 1.0f;
-#pragma unroll 1
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t v[32];
-          tmem_ld32((which == 0 ? tm_dk : tm_dv) + cc * 32, v);
-          tmem_wait_ld();
-          uint32_t pk[16];
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t v[32];
+        tmem_ld32(tm_acc + cc * 32, v);
+        tmem_wait_ld();
+        uint32_t pk[16];
 #pragma unroll
-          for (int k = 0; k < 16; ++k)
-            pk[k] = pack_bf16x2(__uint_as_float(v[2 * k]) * mul, __uint_as_float(v[2 * k + 1]) * mul);
-          if (key < p.N) {
-            uint4* dst = reinterpret_cast<uint4*>(out + cc * 32);
+        for (int k = 0; k < 16; ++k)
+          pk[k] = pack_bf16x2(__uint_as_float(v[2 * k]) * mul, __uint_as_float(v[2 * k + 1]) * mul);
+        if (key < p.N) {
+          uint4* dst = reinterpret_cast<uint4*>(out + cc * 32);
 #pragma unroll
-            for (int u = 0; u < 4; ++u)
-              dst[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-          }
+          for (int u = 0; u < 4; ++u)
+            dst[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
         }
       }
-    } else if (ok && nsteps == 0) {
-      // no query tile sees this key tile (cannot happen for square causal attention)
     }
-  } else {
-    // ------------------------------------------------------------ dQ readout (query rows)
-    const int wq = warp - 4;
-    const int qrow = wq * 32 + lane;
+  } else if (warp < kWarpTma) {
+    // ------------------------------------------------------------ dQ readout
+    const int wq = warp - kWarpDq;
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
-    const uint32_t tm_dq = tmem + lane_off + C::kTmDQ;
+    const int row = wq * 32 + lane;  // TMEM lane: head-dim element (D = 128) or query (D = 64)
     bool ok = true;
     for (int s = 0; s < nsteps && ok; ++s) {
-      const int q = (i_begin + s) * BM + qrow;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarDQFull), s & 1, wd));
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t v[D / 32][32];
+      const int q0 = (i_begin + s) * BM;
+      if constexpr (D == 128) {
+        for (int h = 0; h < 2 && ok; ++h) {
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarDQFull + h), s & 1, wd));
+          if (!ok) break;
+          tc_fence_after();
+          uint32_t v[2][32];
+          tmem_ld32(tmem + lane_off + C::kTmS + 64 * h, v[0]);
+          tmem_ld32(tmem + lane_off + C::kTmS + 64 * h + 32, v[1]);
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(C::kBarDQEmpty + h));
+          // element `row` of the head dimension for 64 queries: a warp covers 32
+          // consecutive elements of one query row (128 contiguous bytes) per add
+          float* dst = p.dQacc + (static_cast<size_t>(bh) * p.N + q0 + 64 * h) * D + row;
+          const int nq = min(64, p.N - (q0 + 64 * h));
 #pragma unroll
-      for (int cc = 0; cc < D / 32; ++cc) tmem_ld32(tm_dq + cc * 32, v[cc]);
-      tmem_wait_ld();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(C::kBarDQEmpty));
-      if (q < p.N) {
-        float* dst = p.dQacc + (static_cast<size_t>(bh) * p.N + q) * D;
+          for (int qq = 0; qq < 64; ++qq)
+            if (qq < nq) red_add(dst + static_cast<size_t>(qq) * D, __uint_as_float(v[qq / 32][qq % 32]));
+        }
+      } else {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarDQFull), s & 1, wd));
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t v[2][32];
+        tmem_ld32(tmem + lane_off + C::kTmDQ64, v[0]);
+        tmem_ld32(tmem + lane_off + C::kTmDQ64 + 32, v[1]);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(C::kBarDQEmpty));
+        const int q = q0 + row;
+        if (q < p.N) {
+          float* dst = p.dQacc + (static_cast<size_t>(bh) * p.N + q) * D;
 #pragma unroll
-        for (int k = 0; k < D / 4; ++k)
-          red_add_v4(dst + 4 * k, __uint_as_float(v[k / 8][(4 * k) % 32]),
-                     __uint_as_float(v[k / 8][(4 * k + 1) % 32]),
-                     __uint_as_float(v[k / 8][(4 * k + 2) % 32]),
-                     __uint_as_float(v[k / 8][(4 * k + 3) % 32]));
+          for (int k = 0; k < 16; ++k)
+            red_add_v4(dst + 4 * k, __uint_as_float(v[k / 8][(4 * k) % 32]),
+                       __uint_as_float(v[k / 8][(4 * k + 1) % 32]),
+                       __uint_as_float(v[k / 8][(4 * k + 2) % 32]),
+                       __uint_as_float(v[k / 8][(4 * k + 3) % 32]));
+        }
       }
     }
   }

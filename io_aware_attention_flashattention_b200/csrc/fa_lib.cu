@@ -299,8 +299,9 @@ fa_status fa_backward_main(const void* Q, const void* K, const void* V, const vo
   fa_status st = bwd_plan(ptrs, 6, B, H, N, d, scale, causal, workspace, workspace_bytes, &pl);
   if (st != FA_OK || N == 0) return st;
   CUtensorMap mq, mk, mv, mdo;
-  if (!make_map_bf16(&mq, Q, pl.BH, N, d, bwd::BM) || !make_map_bf16(&mk, K, pl.BH, N, d, bwd::BN) ||
-      !make_map_bf16(&mv, V, pl.BH, N, d, bwd::BN) || !make_map_bf16(&mdo, dO, pl.BH, N, d, bwd::BM))
+  // Q and dO stream in half tiles of 64 rows; K and V are loaded as 128-row tiles
+  if (!make_map_bf16(&mq, Q, pl.BH, N, d, 64) || !make_map_bf16(&mk, K, pl.BH, N, d, bwd::BN) ||
+      !make_map_bf16(&mv, V, pl.BH, N, d, bwd::BN) || !make_map_bf16(&mdo, dO, pl.BH, N, d, 64))
     return FA_ERR_CUDA;
   bwd::Params p;
   p.dK = static_cast<__nv_bfloat16*>(dK);
