@@ -38,13 +38,19 @@ constexpr int kThreads = 320;  // 8 softmax warps + producer + MMA
 constexpr int kWarpTma = 8;
 constexpr int kWarpMma = 9;
 constexpr float kRescaleThreshold = 8.0f;  // log2 domain: rescale when max grows > 2^8
+// When kPolyPeriod > 0, one pair of exponentials in every kPolyPeriod goes to the
+// polynomial exp2 on the FMA pipe (exp2_poly2) instead of MUFU. Measured on B200
+// at d = 128 the forward is not MUFU-bound (timing is unchanged with the softmax
+// arithmetic removed), and moving 12.5% or 25% of the exponentials made it 1.5% and
+// 2% slower, so it is off.
+constexpr int kPolyPeriod = 0;
 
 template <int D>
 struct Cfg {
   static constexpr int kChunkBytes = 128 * 128;      // 128 rows x 64 bf16 (one TMA box)
   static constexpr int kChunks = D / 64;             // boxes per 128 x D tile
   static constexpr int kTileBytes = kChunks * kChunkBytes;
-  static constexpr int kSlots = (D == 128) ? 4 : 8;  // K/V ring slots
+  static constexpr int kSlots = (D == 128) ? 5 : 10;  // K/V ring slots
   static constexpr int kQOff = 0;
   static constexpr int kKVOff = 2 * kTileBytes;
   static constexpr int kBarOff = kKVOff + kSlots * kTileBytes;
@@ -218,6 +224,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto wait_full = [&](int seq) -> bool {
         return mbar_wait(bar(C::kBarKVFull + seq % C::kSlots), (seq / C::kSlots) & 1, wd);
       };
+      // Each K/V slot is released by a commit issued right after the last MMA that
+      // reads it (a commit fires once every earlier MMA is complete), so the
+      // producer can refill it as early as possible.
+      // K_j is read by S_t(j) for the tiles with j < nk[t]; V_j by PV_t(j). Tile 1
+      // never has fewer key tiles than tile 0 (causal) unless it is empty.
+      auto last_tile = [&](int jj) { return (jj < nk[1]) ? 1 : 0; };
       // prologue: S_t(0)
       if (ok && nkv > 0) {
         ok = wait_full(0);
@@ -228,33 +240,38 @@ __global__ void __launch_bounds__(kThreads, 1)
             issue_s<D>(tmem + C::kTmS0 + t * 128, q_smem[t], slot_smem(0));
             tc_commit(bar(C::kBarSFull + t));
           }
+          tc_commit(bar(C::kBarKVEmpty + 0));
         }
       }
+      bool have_v = false, have_k = false;
       for (int j = 0; j < nkv && ok; ++j) {
         const int seqK = 2 * j, seqV = 2 * j + 1;
-        ok = wait_full(seqV);
-        if (ok && j + 1 < nkv) ok = wait_full(seqK + 2);
-        if (!ok) break;
-        tc_fence_after();
+        have_v = false;
+        have_k = false;
         for (int t = 0; t < 2; ++t) {
           if (j >= nk[t]) continue;
-          if (!mbar_wait(bar(C::kBarPFull + t), j & 1, wd)) {
-            ok = false;
-            break;
+          if (!mbar_wait(bar(C::kBarPFull + t), j & 1, wd)) { ok = false; break; }
+          if (!have_v) {
+            if (!wait_full(seqV)) { ok = false; break; }
+            have_v = true;
           }
           tc_fence_after();
           const uint32_t tm_s = tmem + C::kTmS0 + t * 128;
           issue_pv<D>(tmem + C::kTmO0 + t * D, tm_s, slot_smem(seqV), j > 0);
+          if (t == last_tile(j)) tc_commit(bar(C::kBarKVEmpty + seqV % C::kSlots));
           if (j + 1 < nk[t]) {
+            if (!have_k) {
+              if (!wait_full(seqK + 2)) { ok = false; break; }
+              have_k = true;
+              tc_fence_after();
+            }
             issue_s<D>(tm_s, q_smem[t], slot_smem(seqK + 2));
             tc_commit(bar(C::kBarSFull + t));
+            if (t == last_tile(j + 1)) tc_commit(bar(C::kBarKVEmpty + (seqK + 2) % C::kSlots));
           } else {
             tc_commit(bar(C::kBarOFull + t));
           }
         }
-        if (!ok) break;
-        tc_commit(bar(C::kBarKVEmpty + seqK % C::kSlots));
-        tc_commit(bar(C::kBarKVEmpty + seqV % C::kSlots));
       }
       // No MMA may be in flight when TMEM is released.
       tc_commit(bar(C::kBarDrain));
@@ -291,9 +308,22 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int k = 0; k < 128; ++k)
           if (kv0 + k >= lim) s[k / 32][k % 32] = __float_as_uint(-INFINITY);
       }
-      float mx = __uint_as_float(s[0][0]);
+      // row max: per 32-column chunk a tree of three-input maxima (short dependency
+      // chains, few live temporaries), then across the four chunks
+      float cm[4];
 #pragma unroll
-      for (int k = 1; k < 128; ++k) mx = fmaxf(mx, __uint_as_float(s[k / 32][k % 32]));
+      for (int cc = 0; cc < 4; ++cc) {
+        float t1[11];
+#pragma unroll
+        for (int q = 0; q < 10; ++q)
+          t1[q] = fmax3(__uint_as_float(s[cc][3 * q]), __uint_as_float(s[cc][3 * q + 1]),
+                        __uint_as_float(s[cc][3 * q + 2]));
+        t1[10] = fmaxf(__uint_as_float(s[cc][30]), __uint_as_float(s[cc][31]));
+        const float a = fmax3(t1[0], t1[1], t1[2]), b = fmax3(t1[3], t1[4], t1[5]);
+        const float d2 = fmax3(t1[6], t1[7], t1[8]), e = fmaxf(t1[9], t1[10]);
+        cm[cc] = fmax3(a, b, fmaxf(d2, e));
+      }
+      const float mx = fmaxf(fmaxf(cm[0], cm[1]), fmaxf(cm[2], cm[3]));
       const float m_new = fmaxf(m_ref, mx * c);
       const bool need = m_new > m_ref + kRescaleThreshold;
       // The reference max moves for the whole warp when any row needs it (TMEM
@@ -306,19 +336,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         l *= alpha;
       }
       const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
-      float rowsum = 0.0f;
+      const float2 c2 = make_float2(c, c), nm2 = make_float2(-m_use, -m_use);
+      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                       make_float2(0.f, 0.f)};
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         uint32_t pk[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k) {
-          const float p0 = ex2_approx(fmaf(__uint_as_float(s[cc][2 * k]), c, -m_use));
-          const float p1 = ex2_approx(fmaf(__uint_as_float(s[cc][2 * k + 1]), c, -m_use));
-          rowsum += p0 + p1;
-          pk[k] = pack_bf16x2(p0, p1);
+          const float2 x = ffma2(make_float2(__uint_as_float(s[cc][2 * k]),
+                                             __uint_as_float(s[cc][2 * k + 1])), c2, nm2);
+          float2 pe;
+          if (kPolyPeriod > 0 && k % (kPolyPeriod > 0 ? kPolyPeriod : 1) == kPolyPeriod - 1) {
+            pe = exp2_poly2(x);  // a share of the exponentials on the FMA pipe
+          } else {
+            pe = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+          }
+          acc[k & 3] = fadd2(acc[k & 3], pe);
+          pk[k] = pack_bf16x2(pe.x, pe.y);
         }
         tmem_st16(tm_s + cc * 16, pk);
       }
+      const float rowsum = (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y) +
+                           (acc[2].x + acc[2].y) + (acc[3].x + acc[3].y);
       l += rowsum;
       if (move && j > 0) {
         // O_t holds the sum up to tile j-1 (PV_t(j-1) completed before S_t(j)'s

@@ -259,6 +259,66 @@ __device__ __forceinline__ float ex2_approx(float x) {
   return y;
 }
 
+// Packed fp32 pairs (Blackwell f32x2 arithmetic: one instruction for two lanes of
+// work on the FMA pipe).
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// Three-input maximum (one instruction on sm_100).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// 2^x for a pair, on the FMA and integer pipes instead of MUFU, for x <= 64.
+// Range reduction in the Cody-Waite manner: adding 1.5*2^23 rounds x to the
+// nearest integer j and leaves j in the low mantissa bits of the sum; f = x - j
+// lies in [-0.5, 0.5]. 2^f is a degree-3 polynomial fitted to 2^f on [-0.5, 0.5]
+// (least squares at Chebyshev nodes with Lawson reweighting toward the minimax
+// fit; maximum relative error 7.5e-5, about 1/26 of a bf16 ulp), and j is added
+// to its exponent field. x is clamped at -125 so the result stays a normal
+// number: inputs below that give 2^-125 (about 2.4e-38) instead of 0.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  x.x = fmaxf(x.x, -125.0f);
+  x.y = fmaxf(x.y, -125.0f);
+  const float2 t = fadd2(x, make_float2(kMagic, kMagic));
+  const float2 j = fadd2(t, make_float2(-kMagic, -kMagic));
+  const float2 f = ffma2(j, make_float2(-1.0f, -1.0f), x);
+  float2 q = ffma2(f, make_float2(0.0551716648f, 0.0551716648f),
+                   make_float2(0.2426111251f, 0.2426111251f));
+  q = ffma2(q, f, make_float2(0.6932609678f, 0.6932609678f));
+  q = ffma2(q, f, make_float2(0.9999280572f, 0.9999280572f));
+  return make_float2(__uint_as_float(__float_as_uint(q.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
+}
+
 // Two fp32 values to a packed bf16x2 word, round-to-nearest-even; `lo` lands in
 // the low half (the element with the smaller index).
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
