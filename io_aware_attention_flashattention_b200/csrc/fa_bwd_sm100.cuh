@@ -100,19 +100,6 @@ struct Params {
   unsigned long long timeout_ns;
 };
 
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
-                                          uint32_t bar) {
-  asm volatile(
-      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-          dst),
-      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
-      : "memory");
-}
-
-__device__ __forceinline__ void fence_proxy_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
 __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
                "f"(c), "f"(d)
@@ -142,8 +129,8 @@ __device__ __forceinline__ void issue_xyT_half(uint32_t tm_d, uint32_t x_smem, u
   for (int kk = 0; kk < D / 16; ++kk) {
     const uint32_t xo = (kk / 4) * Cfg<D>::kChunkBytes + (kk % 4) * 32;
     const uint32_t yo = (kk / 4) * Cfg<D>::kHalfChunkBytes + (kk % 4) * 32;
-    mma_ss(tm_d, sdesc_sw128(x_smem + xo, 16, 1024), sdesc_sw128(yh_smem + yo, 16, 1024), idesc,
-           kk > 0 ? 1u : 0u);
+    mma_ss_e(tm_d, sdesc_sw128(x_smem + xo, 16, 1024), sdesc_sw128(yh_smem + yo, 16, 1024),
+             idesc, kk > 0 ? 1u : 0u);
   }
 }
 
@@ -155,9 +142,9 @@ __device__ __forceinline__ void issue_acc_half(uint32_t tm_acc, uint32_t tm_a, u
   constexpr uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);
 #pragma unroll
   for (int kk = 0; kk < 64 / 16; ++kk)
-    mma_ts(tm_acc, tm_a + kk * 8,
-           sdesc_sw128(yh_smem + kk * 2048, Cfg<D>::kHalfChunkBytes, 1024), idesc,
-           (accumulate || kk > 0) ? 1u : 0u);
+    mma_ts_e(tm_acc, tm_a + kk * 8,
+             sdesc_sw128(yh_smem + kk * 2048, Cfg<D>::kHalfChunkBytes, 1024), idesc,
+             (accumulate || kk > 0) ? 1u : 0u);
 }
 
 // D = 128: dQ^T_h[128 dims x 64 queries] = K_j^T[dims x keys] * dS_h^T[keys x queries]:
@@ -167,9 +154,9 @@ __device__ __forceinline__ void issue_dqT_half(uint32_t tm_d, uint32_t k_smem, u
   constexpr uint32_t idesc = idesc_bf16_f32(128, 64, 1, 1);
 #pragma unroll
   for (int kk = 0; kk < 128 / 16; ++kk)
-    mma_ss(tm_d, sdesc_sw128(k_smem + kk * 2048, Cfg<128>::kChunkBytes, 1024),
-           sdesc_sw128(ds_chunk + kk * 2048, Cfg<128>::kChunkBytes, 1024), idesc,
-           kk > 0 ? 1u : 0u);
+    mma_ss_e(tm_d, sdesc_sw128(k_smem + kk * 2048, Cfg<128>::kChunkBytes, 1024),
+             sdesc_sw128(ds_chunk + kk * 2048, Cfg<128>::kChunkBytes, 1024), idesc,
+             kk > 0 ? 1u : 0u);
 }
 
 // D = 64: dQ_i[128 queries x 64] = dS[queries x keys] * K_j[keys x 64]: A = the whole
@@ -178,8 +165,8 @@ __device__ __forceinline__ void issue_dq64(uint32_t tm_d, uint32_t ds_smem, uint
   constexpr uint32_t idesc = idesc_bf16_f32(128, 64, 1, 1);
 #pragma unroll
   for (int kk = 0; kk < 128 / 16; ++kk)
-    mma_ss(tm_d, sdesc_sw128(ds_smem + kk * 2048, Cfg<64>::kChunkBytes, 1024),
-           sdesc_sw128(k_smem + kk * 2048, Cfg<64>::kChunkBytes, 1024), idesc, kk > 0 ? 1u : 0u);
+    mma_ss_e(tm_d, sdesc_sw128(ds_smem + kk * 2048, Cfg<64>::kChunkBytes, 1024),
+             sdesc_sw128(k_smem + kk * 2048, Cfg<64>::kChunkBytes, 1024), idesc, kk > 0 ? 1u : 0u);
 }
 
 // ------------------------------------------------------------------ preprocess
@@ -313,108 +300,108 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == kWarpTma) {
     // ------------------------------------------------------------ producer
+    // (the whole warp runs the loop; one elected lane issues each copy)
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmdO);
-      mbar_arrive_expect_tx(bar(C::kBarKV), 2 * C::kTileBytes);
-      for (int c = 0; c < C::kChunks; ++c) {
-        tma_load_3d(base + C::kKOff + c * C::kChunkBytes, &tmK, bar(C::kBarKV), c * 64, k0, bh);
-        tma_load_3d(base + C::kVOff + c * C::kChunkBytes, &tmV, bar(C::kBarKV), c * 64, k0, bh);
-      }
-      int issued = 0;
-      bool ok = true;
-      for (int s = 0; s < nsteps && ok; ++s) {
-        const int i = i_begin + s;
-        for (int hw = 0; hw < 4 && ok; ++hw) {
-          const int h = hw >> 1, w = hw & 1;
-          const int seq = seq_of(s, h, w);
-          const int slot = slot_of(seq);
-          const int rnd = round_of(seq);
-          if (rnd > 0 && !mbar_wait(bar(C::kBarEmpty + slot), (rnd - 1) & 1, wd)) {
-            ok = false;
-            break;
-          }
-          const uint32_t full = bar(C::kBarFull + slot);
-          const uint32_t dst = slot_smem(seq);
-          const int row0 = i * BM + 64 * h;
-          if (w == 1) {
-            mbar_arrive_expect_tx(full, C::kHalfBytes + 2 * C::kVecBytes);
-            const uint32_t vec = base + C::kVecOff + slot * 2 * C::kVecBytes;
-            const size_t off = static_cast<size_t>(bh) * p.Npad + static_cast<size_t>(row0);
-            bulk_load(vec, p.L2 + off, C::kVecBytes, full);
-            bulk_load(vec + C::kVecBytes, p.Dv + off, C::kVecBytes, full);
-          } else {
-            mbar_arrive_expect_tx(full, C::kHalfBytes);
-          }
-          for (int c = 0; c < C::kChunks; ++c)
-            tma_load_3d(dst + c * C::kHalfChunkBytes, w ? &tmQ : &tmdO, full, c * 64, row0, bh);
-          issued = seq + 1;
-        }
-      }
-      for (int seq = max(0, issued - C::kSlots); seq < issued; ++seq)
-        drain_wait(bar(C::kBarFull + slot_of(seq)), round_of(seq) & 1, p.timeout_ns);
-      drain_wait(bar(C::kBarKV), 0, p.timeout_ns);
     }
+    mbar_arrive_expect_tx_e(bar(C::kBarKV), 2 * C::kTileBytes);
+    for (int c = 0; c < C::kChunks; ++c) {
+      tma_load_3d_e(base + C::kKOff + c * C::kChunkBytes, &tmK, bar(C::kBarKV), c * 64, k0, bh);
+      tma_load_3d_e(base + C::kVOff + c * C::kChunkBytes, &tmV, bar(C::kBarKV), c * 64, k0, bh);
+    }
+    int issued = 0;
+    bool ok = true;
+    for (int s = 0; s < nsteps && ok; ++s) {
+      const int i = i_begin + s;
+      for (int hw = 0; hw < 4 && ok; ++hw) {
+        const int h = hw >> 1, w = hw & 1;
+        const int seq = seq_of(s, h, w);
+        const int slot = slot_of(seq);
+        const int rnd = round_of(seq);
+        if (rnd > 0 && !mbar_wait_warp(bar(C::kBarEmpty + slot), (rnd - 1) & 1, wd)) {
+          ok = false;
+          break;
+        }
+        const uint32_t full = bar(C::kBarFull + slot);
+        const uint32_t dst = slot_smem(seq);
+        const int row0 = i * BM + 64 * h;
+        if (w == 1) {
+          mbar_arrive_expect_tx_e(full, C::kHalfBytes + 2 * C::kVecBytes);
+          const uint32_t vec = base + C::kVecOff + slot * 2 * C::kVecBytes;
+          const size_t off = static_cast<size_t>(bh) * p.Npad + static_cast<size_t>(row0);
+          bulk_load_e(vec, p.L2 + off, C::kVecBytes, full);
+          bulk_load_e(vec + C::kVecBytes, p.Dv + off, C::kVecBytes, full);
+        } else {
+          mbar_arrive_expect_tx_e(full, C::kHalfBytes);
+        }
+        for (int c = 0; c < C::kChunks; ++c)
+          tma_load_3d_e(dst + c * C::kHalfChunkBytes, w ? &tmQ : &tmdO, full, c * 64, row0, bh);
+        issued = seq + 1;
+      }
+    }
+    for (int seq = max(0, issued - C::kSlots); seq < issued; ++seq)
+      drain_wait(bar(C::kBarFull + slot_of(seq)), round_of(seq) & 1, p.timeout_ns);
+    drain_wait(bar(C::kBarKV), 0, p.timeout_ns);
     __syncwarp();
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      const uint32_t k_smem = base + C::kKOff, v_smem = base + C::kVOff;
-      const uint32_t ds_smem = base + C::kDSOff;
-      const uint32_t tm_s = tmem + C::kTmS, tm_dp = tmem + C::kTmDP;
-      bool ok = mbar_wait(bar(C::kBarKV), 0, wd);
-      auto wait_full = [&](int seq) -> bool {
-        return mbar_wait(bar(C::kBarFull + slot_of(seq)), round_of(seq) & 1, wd);
-      };
-      // S^T and dP^T of both halves of step s (dP^T first: its columns free up earlier)
-      auto issue_sdp = [&](int s) -> bool {
-        for (int h = 0; h < 2; ++h) {
-          const int seqO = seq_of(s, h, 0), seqQ = seq_of(s, h, 1);
-          if (!(wait_full(seqO) && wait_full(seqQ))) return false;
+    // (the whole warp runs the loop; one elected lane issues each MMA and commit)
+    const uint32_t k_smem = base + C::kKOff, v_smem = base + C::kVOff;
+    const uint32_t ds_smem = base + C::kDSOff;
+    const uint32_t tm_s = tmem + C::kTmS, tm_dp = tmem + C::kTmDP;
+    bool ok = mbar_wait_warp(bar(C::kBarKV), 0, wd);
+    auto wait_full = [&](int seq) -> bool {
+      return mbar_wait_warp(bar(C::kBarFull + slot_of(seq)), round_of(seq) & 1, wd);
+    };
+    // S^T and dP^T of both halves of step s (dP^T first: its columns free up earlier)
+    auto issue_sdp = [&](int s) -> bool {
+      for (int h = 0; h < 2; ++h) {
+        const int seqO = seq_of(s, h, 0), seqQ = seq_of(s, h, 1);
+        if (!(wait_full(seqO) && wait_full(seqQ))) return false;
+        tc_fence_after();
+        issue_xyT_half<D>(tm_dp + 64 * h, v_smem, slot_smem(seqO));
+        if (D == 128 && s > 0) {  // S^T_h shares columns with dQ^T_h of the last step
+          if (!mbar_wait_warp(bar(C::kBarDQEmpty + h), (s - 1) & 1, wd)) return false;
           tc_fence_after();
-          issue_xyT_half<D>(tm_dp + 64 * h, v_smem, slot_smem(seqO));
-          if (D == 128 && s > 0) {  // S^T_h shares columns with dQ^T_h of the last step
-            if (!mbar_wait(bar(C::kBarDQEmpty + h), (s - 1) & 1, wd)) return false;
-            tc_fence_after();
-          }
-          issue_xyT_half<D>(tm_s + 64 * h, k_smem, slot_smem(seqQ));
-          tc_commit(bar(C::kBarS + h));
         }
-        return true;
-      };
-      if (ok && nsteps > 0) ok = issue_sdp(0);
-      for (int s = 0; s < nsteps && ok; ++s) {
-        for (int h = 0; h < 2 && ok; ++h) {
-          const int seqO = seq_of(s, h, 0), seqQ = seq_of(s, h, 1);
-          if (!mbar_wait(bar(C::kBarP + h), s & 1, wd)) { ok = false; break; }
-          tc_fence_after();
-          const bool acc = (s > 0) || (h > 0);
-          issue_acc_half<D>(tmem + C::kTmDV, tm_s + 64 * h, slot_smem(seqO), acc);   // dV
-          issue_acc_half<D>(tmem + C::kTmDK, tm_dp + 64 * h, slot_smem(seqQ), acc);  // dK
-          if constexpr (D == 128) {
-            issue_dqT_half(tm_s + 64 * h, k_smem, ds_smem + h * C::kChunkBytes);
-            tc_commit(bar(C::kBarDQFull + h));
-          }
-          tc_commit(bar(C::kBarEmpty + slot_of(seqO)));
-          tc_commit(bar(C::kBarEmpty + slot_of(seqQ)));
-        }
-        if (!ok) break;
-        if constexpr (D == 64) {
-          if (s > 0) {  // the dQ columns are reused: the previous dQ must have been read
-            if (!mbar_wait(bar(C::kBarDQEmpty), (s - 1) & 1, wd)) { ok = false; break; }
-            tc_fence_after();
-          }
-          issue_dq64(tmem + C::kTmDQ64, ds_smem, k_smem);
-          tc_commit(bar(C::kBarDQFull));
-        }
-        if (s + 1 < nsteps) ok = issue_sdp(s + 1);
+        issue_xyT_half<D>(tm_s + 64 * h, k_smem, slot_smem(seqQ));
+        tc_commit_e(bar(C::kBarS + h));
       }
-      if (ok) tc_commit(bar(C::kBarDKDV));
-      tc_commit(bar(C::kBarDrain));
-      drain_wait(bar(C::kBarDrain), 0, p.timeout_ns);
+      return true;
+    };
+    if (ok && nsteps > 0) ok = issue_sdp(0);
+    for (int s = 0; s < nsteps && ok; ++s) {
+      for (int h = 0; h < 2 && ok; ++h) {
+        const int seqO = seq_of(s, h, 0), seqQ = seq_of(s, h, 1);
+        if (!mbar_wait_warp(bar(C::kBarP + h), s & 1, wd)) { ok = false; break; }
+        tc_fence_after();
+        const bool acc = (s > 0) || (h > 0);
+        issue_acc_half<D>(tmem + C::kTmDV, tm_s + 64 * h, slot_smem(seqO), acc);   // dV
+        issue_acc_half<D>(tmem + C::kTmDK, tm_dp + 64 * h, slot_smem(seqQ), acc);  // dK
+        if constexpr (D == 128) {
+          issue_dqT_half(tm_s + 64 * h, k_smem, ds_smem + h * C::kChunkBytes);
+          tc_commit_e(bar(C::kBarDQFull + h));
+        }
+        tc_commit_e(bar(C::kBarEmpty + slot_of(seqO)));
+        tc_commit_e(bar(C::kBarEmpty + slot_of(seqQ)));
+      }
+      if (!ok) break;
+      if constexpr (D == 64) {
+        if (s > 0) {  // the dQ columns are reused: the previous dQ must have been read
+          if (!mbar_wait_warp(bar(C::kBarDQEmpty), (s - 1) & 1, wd)) { ok = false; break; }
+          tc_fence_after();
+        }
+        issue_dq64(tmem + C::kTmDQ64, ds_smem, k_smem);
+        tc_commit_e(bar(C::kBarDQFull));
+      }
+      if (s + 1 < nsteps) ok = issue_sdp(s + 1);
     }
+    if (ok) tc_commit_e(bar(C::kBarDKDV));
+    tc_commit_e(bar(C::kBarDrain));
+    drain_wait(bar(C::kBarDrain), 0, p.timeout_ns);
     __syncwarp();
   } else if (warp < 8) {
     // ------------------------------------------------------------ P^T, dS^T (key rows)

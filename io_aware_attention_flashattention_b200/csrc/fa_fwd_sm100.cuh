@@ -9,21 +9,25 @@
 // m2), l = e^(m1-m) l1 + e^(m2-m) l2). Causal tiles above the diagonal are skipped
 // ("Flash Attention-2: acceleration principle ...", causal-mask item).
 //
-// B200 mapping (one CTA per SM, 320 threads):
-//   * CTA = 2 query tiles of 128 rows (256 rows) of one (batch, head); the two
-//     tiles ping-pong so that one tile's softmax overlaps the other's MMAs.
-//   * warp 8: TMA producer. Q tiles once; K and V tiles of 128 rows through a ring
-//     of NSLOT shared-memory slots (128-byte swizzle), full/empty mbarriers.
-//   * warp 9: MMA issuer (one thread). S_t = Q_t K_j^T with tcgen05.mma into TMEM
-//     (128 fp32 columns per tile); O_t += P_t V_j with P_t read from TMEM.
-//   * warps 0-3 / 4-7: softmax of tile 0 / 1, one thread per query row (TMEM lane).
-//     Scores are read with tcgen05.ld, the running max and sum stay in registers,
-//     p = 2^(s*c - m) with c = scale*log2(e) folded into one FFMA before ex2, P is
-//     rounded to bf16 and stored over the S columns for the PV MMA. O is rescaled
-//     in TMEM only when the running max grew by more than 2^8 (exact: O and l
-//     always share the same reference max).
-//   * TMEM: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D); P_t
-//     (bf16 pairs) aliases the first 64 columns of S_t.
+// B200 mapping (one CTA per SM, 352 threads):
+//   * CTA = 2 query tiles of 128 rows (256 rows) of one (batch, head); the two tiles
+//     share every K/V tile that is loaded.
+//   * warp 8: TMA producer for the Q tiles (once) and the K tiles (128 rows) through
+//     a ring of kKSlots shared-memory slots; warp 10: TMA producer for the V tiles
+//     (ring of kVSlots). Separate rings let K run further ahead of the MMAs than V.
+//   * warp 9: MMA issuer (one thread), per key tile j:
+//       S_t(j+1) = Q_t K_{j+1}^T (tcgen05.mma, fp32 into TMEM columns [128t, 128t+128))
+//       as soon as the softmax of tile t has read S_t(j) out of TMEM; then
+//       O_t += P_t(j) V_j with P_t read from shared memory once it is written.
+//     So the tensor cores compute S for the next key tile while the softmax of the
+//     current one is still running.
+//   * warps 0-3 / 4-7: softmax of tile 0 / 1, one thread per query row (TMEM lane):
+//     read S with tcgen05.ld, row max (thread-local), p = 2^(s*c - m) with
+//     c = scale*log2(e) folded into one FFMA before ex2, row sum in registers, P
+//     rounded to bf16 into a 128-byte-swizzled shared tile (the K-major A operand of
+//     the PV MMA). O is rescaled in TMEM only when the running max grew by more than
+//     2^8 (exact: O and l always share the same reference max).
+//   * TMEM: S0 [0,128), S1 [128,256), O0 [256,256+D), O1 [256+D,256+2D).
 //   * Epilogue: O/l rounded to bf16 stored row per thread; LSE = (m + log2 l) ln 2.
 #pragma once
 
@@ -34,15 +38,13 @@ namespace fwd {
 
 constexpr int BM = 128;        // query rows per tile
 constexpr int BN = 128;        // key/value rows per tile
-constexpr int kThreads = 320;  // 8 softmax warps + producer + MMA
-constexpr int kWarpTma = 8;
+constexpr int kThreads = 352;  // 8 softmax warps, K/Q producer, MMA, V producer
+constexpr int kWarpTmaK = 8;
 constexpr int kWarpMma = 9;
+constexpr int kWarpTmaV = 10;
 constexpr float kRescaleThreshold = 8.0f;  // log2 domain: rescale when max grows > 2^8
 // When kPolyPeriod > 0, one pair of exponentials in every kPolyPeriod goes to the
-// polynomial exp2 on the FMA pipe (exp2_poly2) instead of MUFU. Measured on B200
-// at d = 128 the forward is not MUFU-bound (timing is unchanged with the softmax
-// arithmetic removed), and moving 12.5% or 25% of the exponentials made it 1.5% and
-// 2% slower, so it is off.
+// polynomial exp2 on the FMA pipe (exp2_poly2) instead of MUFU.
 constexpr int kPolyPeriod = 0;
 
 template <int D>
@@ -50,18 +52,24 @@ struct Cfg {
   static constexpr int kChunkBytes = 128 * 128;      // 128 rows x 64 bf16 (one TMA box)
   static constexpr int kChunks = D / 64;             // boxes per 128 x D tile
   static constexpr int kTileBytes = kChunks * kChunkBytes;
-  static constexpr int kSlots = (D == 128) ? 5 : 10;  // K/V ring slots
+  static constexpr int kPBytes = 2 * kChunkBytes;    // P: 128 x 128 bf16
+  static constexpr int kKSlots = (D == 128) ? 2 : 3;
+  static constexpr int kVSlots = (D == 128) ? 1 : 3;
   static constexpr int kQOff = 0;
-  static constexpr int kKVOff = 2 * kTileBytes;
-  static constexpr int kBarOff = kKVOff + kSlots * kTileBytes;
-  // barriers: q_full[2], kv_full[S], kv_empty[S], s_full[2], p_full[2], o_full[2], drain
-  static constexpr int kBarQFull = 0;
-  static constexpr int kBarKVFull = 2;
-  static constexpr int kBarKVEmpty = 2 + kSlots;
-  static constexpr int kBarSFull = 2 + 2 * kSlots;
-  static constexpr int kBarPFull = kBarSFull + 2;
-  static constexpr int kBarOFull = kBarPFull + 2;
-  static constexpr int kBarDrain = kBarOFull + 2;
+  static constexpr int kPOff = 2 * kTileBytes;
+  static constexpr int kKOff = kPOff + 2 * kPBytes;
+  static constexpr int kVOff = kKOff + kKSlots * kTileBytes;
+  static constexpr int kBarOff = kVOff + kVSlots * kTileBytes;
+  static constexpr int kBarQFull = 0;                             // [2]
+  static constexpr int kBarKFull = 2;                             // [kKSlots]
+  static constexpr int kBarKEmpty = kBarKFull + kKSlots;          // [kKSlots]
+  static constexpr int kBarVFull = kBarKEmpty + kKSlots;          // [kVSlots]
+  static constexpr int kBarVEmpty = kBarVFull + kVSlots;          // [kVSlots]
+  static constexpr int kBarSFull = kBarVEmpty + kVSlots;          // [2] S_t(j) in TMEM
+  static constexpr int kBarSFree = kBarSFull + 2;                 // [2] S_t(j) read out
+  static constexpr int kBarPFull = kBarSFree + 2;                 // [2] P_t(j) written
+  static constexpr int kBarPVDone = kBarPFull + 2;                // [2] PV_t(j) complete
+  static constexpr int kBarDrain = kBarPVDone + 2;
   static constexpr int kNumBars = kBarDrain + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem base, abort flag
   static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + 1024 for alignment
@@ -80,26 +88,29 @@ struct Params {
   unsigned long long timeout_ns;
 };
 
+// S = Q_t K_j^T: M = 128 query rows, N = 128 keys, K = D; both operands K-major.
 template <int D>
 __device__ __forceinline__ void issue_s(uint32_t tm_d, uint32_t q_smem, uint32_t k_smem) {
   constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, 0, 0);
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
     const uint32_t off = (kk / 4) * Cfg<D>::kChunkBytes + (kk % 4) * 32;
-    mma_ss(tm_d, sdesc_sw128(q_smem + off, 16, 1024), sdesc_sw128(k_smem + off, 16, 1024), idesc,
-           kk > 0 ? 1u : 0u);
+    mma_ss_e(tm_d, sdesc_sw128(q_smem + off, 16, 1024), sdesc_sw128(k_smem + off, 16, 1024),
+             idesc, kk > 0 ? 1u : 0u);
   }
 }
 
+// O += P V_j: A = P (128 x 128 keys, K-major in shared memory), B = V_j read MN-major.
 template <int D>
-__device__ __forceinline__ void issue_pv(uint32_t tm_o, uint32_t tm_p, uint32_t v_smem,
+__device__ __forceinline__ void issue_pv(uint32_t tm_o, uint32_t p_smem, uint32_t v_smem,
                                          bool accumulate) {
   constexpr uint32_t idesc = idesc_bf16_f32(BM, D, 0, 1);
 #pragma unroll
   for (int kk = 0; kk < BN / 16; ++kk) {
-    mma_ts(tm_o, tm_p + kk * 8,
-           sdesc_sw128(v_smem + kk * 16 * 128, Cfg<D>::kChunkBytes, 1024), idesc,
-           (accumulate || kk > 0) ? 1u : 0u);
+    const uint32_t poff = (kk / 4) * Cfg<D>::kChunkBytes + (kk % 4) * 32;
+    mma_ss_e(tm_o, sdesc_sw128(p_smem + poff, 16, 1024),
+             sdesc_sw128(v_smem + kk * 16 * 128, Cfg<D>::kChunkBytes, 1024), idesc,
+             (accumulate || kk > 0) ? 1u : 0u);
   }
 }
 
@@ -143,19 +154,24 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r0 = q0 + t * BM;
     nk[t] = (r0 < p.N) ? (p.causal ? min(r0 / BN + 1, n_kv_total) : n_kv_total) : 0;
   }
+  // Tile 1 never has fewer key tiles than tile 0 unless it is empty.
   const int nkv = max(nk[0], nk[1]);
 
   if (threadIdx.x == 0) {
-    mbar_init(bar(C::kBarQFull + 0), 1);
-    mbar_init(bar(C::kBarQFull + 1), 1);
-    for (int s = 0; s < C::kSlots; ++s) {
-      mbar_init(bar(C::kBarKVFull + s), 1);
-      mbar_init(bar(C::kBarKVEmpty + s), 1);
-    }
     for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(C::kBarQFull + t), 1);
       mbar_init(bar(C::kBarSFull + t), 1);
-      mbar_init(bar(C::kBarPFull + t), 4);  // one arrival per softmax warp
-      mbar_init(bar(C::kBarOFull + t), 1);
+      mbar_init(bar(C::kBarSFree + t), 4);  // one arrival per softmax warp
+      mbar_init(bar(C::kBarPFull + t), 4);
+      mbar_init(bar(C::kBarPVDone + t), 1);
+    }
+    for (int s = 0; s < C::kKSlots; ++s) {
+      mbar_init(bar(C::kBarKFull + s), 1);
+      mbar_init(bar(C::kBarKEmpty + s), 1);
+    }
+    for (int s = 0; s < C::kVSlots; ++s) {
+      mbar_init(bar(C::kBarVFull + s), 1);
+      mbar_init(bar(C::kBarVEmpty + s), 1);
     }
     mbar_init(bar(C::kBarDrain), 1);
     *abort_flag = 0;
@@ -171,112 +187,114 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const Watchdog wd{abort_flag, p.timeout_ns};
 
-  if (warp == kWarpTma) {
-    // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      tma_prefetch_desc(&tmQ);
-      tma_prefetch_desc(&tmK);
-      tma_prefetch_desc(&tmV);
+  auto k_smem = [&](int j) -> uint32_t {
+    return base + C::kKOff + (j % C::kKSlots) * C::kTileBytes;
+  };
+  auto v_smem = [&](int j) -> uint32_t {
+    return base + C::kVOff + (j % C::kVSlots) * C::kTileBytes;
+  };
+
+  if (warp == kWarpTmaK || warp == kWarpTmaV) {
+    // ------------------------------------------------------------ producers
+    // (the whole warp runs the loop; one elected lane issues each copy)
+    const bool is_k = (warp == kWarpTmaK);
+    const CUtensorMap* map = is_k ? &tmK : &tmV;
+    const int nslots = is_k ? C::kKSlots : C::kVSlots;
+    const int bfull = is_k ? C::kBarKFull : C::kBarVFull;
+    const int bempty = is_k ? C::kBarKEmpty : C::kBarVEmpty;
+    if (lane == 0) tma_prefetch_desc(map);
+    if (is_k) {
+      if (lane == 0) tma_prefetch_desc(&tmQ);
       for (int t = 0; t < 2; ++t) {
         if (nk[t] == 0) continue;
         const uint32_t dst = base + C::kQOff + t * C::kTileBytes;
-        mbar_arrive_expect_tx(bar(C::kBarQFull + t), C::kTileBytes);
+        mbar_arrive_expect_tx_e(bar(C::kBarQFull + t), C::kTileBytes);
         for (int c = 0; c < C::kChunks; ++c)
-          tma_load_3d(dst + c * C::kChunkBytes, &tmQ, bar(C::kBarQFull + t), c * 64, q0 + t * BM,
-                      bh);
+          tma_load_3d_e(dst + c * C::kChunkBytes, &tmQ, bar(C::kBarQFull + t), c * 64,
+                        q0 + t * BM, bh);
       }
-      int issued = 0;
-      bool ok = true;
-      for (int j = 0; j < nkv && ok; ++j) {
-        for (int w = 0; w < 2; ++w) {
-          const int seq = 2 * j + w;
-          const int slot = seq % C::kSlots;
-          const int rnd = seq / C::kSlots;
-          if (rnd > 0 && !mbar_wait(bar(C::kBarKVEmpty + slot), (rnd - 1) & 1, wd)) {
-            ok = false;
-            break;
-          }
-          const uint32_t dst = base + C::kKVOff + slot * C::kTileBytes;
-          mbar_arrive_expect_tx(bar(C::kBarKVFull + slot), C::kTileBytes);
-          for (int c = 0; c < C::kChunks; ++c)
-            tma_load_3d(dst + c * C::kChunkBytes, w ? &tmV : &tmK, bar(C::kBarKVFull + slot),
-                        c * 64, j * BN, bh);
-          issued = seq + 1;
-        }
-      }
-      // Every issued copy must land before the CTA may exit.
-      for (int seq = max(0, issued - C::kSlots); seq < issued; ++seq)
-        drain_wait(bar(C::kBarKVFull + seq % C::kSlots), (seq / C::kSlots) & 1, p.timeout_ns);
+    }
+    int issued = 0;
+    for (int j = 0; j < nkv; ++j) {
+      const int slot = j % nslots, rnd = j / nslots;
+      if (rnd > 0 && !mbar_wait_warp(bar(bempty + slot), (rnd - 1) & 1, wd)) break;
+      const uint32_t dst = is_k ? k_smem(j) : v_smem(j);
+      mbar_arrive_expect_tx_e(bar(bfull + slot), C::kTileBytes);
+      for (int c = 0; c < C::kChunks; ++c)
+        tma_load_3d_e(dst + c * C::kChunkBytes, map, bar(bfull + slot), c * 64, j * BN, bh);
+      issued = j + 1;
+    }
+    // Every issued copy must land before the CTA may exit.
+    for (int j = max(0, issued - nslots); j < issued; ++j)
+      drain_wait(bar(bfull + j % nslots), (j / nslots) & 1, p.timeout_ns);
+    if (is_k)
       for (int t = 0; t < 2; ++t)
         if (nk[t] > 0) drain_wait(bar(C::kBarQFull + t), 0, p.timeout_ns);
-    }
     __syncwarp();
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      bool ok = true;
-      for (int t = 0; t < 2 && ok; ++t)
-        if (nk[t] > 0) ok = mbar_wait(bar(C::kBarQFull + t), 0, wd);
-      const uint32_t q_smem[2] = {base + C::kQOff, base + C::kQOff + C::kTileBytes};
-      auto slot_smem = [&](int seq) -> uint32_t {
-        return base + C::kKVOff + (seq % C::kSlots) * C::kTileBytes;
-      };
-      auto wait_full = [&](int seq) -> bool {
-        return mbar_wait(bar(C::kBarKVFull + seq % C::kSlots), (seq / C::kSlots) & 1, wd);
-      };
-      // Each K/V slot is released by a commit issued right after the last MMA that
-      // reads it (a commit fires once every earlier MMA is complete), so the
-      // producer can refill it as early as possible.
-      // K_j is read by S_t(j) for the tiles with j < nk[t]; V_j by PV_t(j). Tile 1
-      // never has fewer key tiles than tile 0 (causal) unless it is empty.
-      auto last_tile = [&](int jj) { return (jj < nk[1]) ? 1 : 0; };
-      // prologue: S_t(0)
-      if (ok && nkv > 0) {
-        ok = wait_full(0);
-        if (ok) {
-          tc_fence_after();
-          for (int t = 0; t < 2; ++t) {
-            if (nk[t] == 0) continue;
-            issue_s<D>(tmem + C::kTmS0 + t * 128, q_smem[t], slot_smem(0));
-            tc_commit(bar(C::kBarSFull + t));
-          }
-          tc_commit(bar(C::kBarKVEmpty + 0));
-        }
-      }
-      bool have_v = false, have_k = false;
-      for (int j = 0; j < nkv && ok; ++j) {
-        const int seqK = 2 * j, seqV = 2 * j + 1;
-        have_v = false;
-        have_k = false;
+    // (the whole warp runs the loop; one elected lane issues each MMA and commit)
+    bool ok = true;
+    for (int t = 0; t < 2 && ok; ++t)
+      if (nk[t] > 0) ok = mbar_wait_warp(bar(C::kBarQFull + t), 0, wd);
+    const uint32_t q_smem0 = base + C::kQOff, q_smem1 = base + C::kQOff + C::kTileBytes;
+    const uint32_t p_smem0 = base + C::kPOff, p_smem1 = base + C::kPOff + C::kPBytes;
+    auto wait_k = [&](int j) {
+      return mbar_wait_warp(bar(C::kBarKFull + j % C::kKSlots), (j / C::kKSlots) & 1, wd);
+    };
+    auto wait_v = [&](int j) {
+      return mbar_wait_warp(bar(C::kBarVFull + j % C::kVSlots), (j / C::kVSlots) & 1, wd);
+    };
+    // prologue: S_t(0)
+    if (ok && nkv > 0) {
+      ok = wait_k(0);
+      if (ok) {
+        tc_fence_after();
         for (int t = 0; t < 2; ++t) {
-          if (j >= nk[t]) continue;
-          if (!mbar_wait(bar(C::kBarPFull + t), j & 1, wd)) { ok = false; break; }
-          if (!have_v) {
-            if (!wait_full(seqV)) { ok = false; break; }
-            have_v = true;
+          if (nk[t] == 0) continue;
+          issue_s<D>(tmem + C::kTmS0 + t * 128, t ? q_smem1 : q_smem0, k_smem(0));
+          tc_commit_e(bar(C::kBarSFull + t));
+        }
+        tc_commit_e(bar(C::kBarKEmpty + 0));
+      }
+    }
+    for (int j = 0; j < nkv && ok; ++j) {
+      // S_t(j+1) for both tiles, each as soon as S_t(j) has been read out
+      if (j + 1 < nkv) {
+        bool have_k = false;
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (j + 1 >= nk[t]) continue;
+          if (!mbar_wait_warp(bar(C::kBarSFree + t), j & 1, wd)) { ok = false; break; }
+          if (!have_k) {
+            if (!wait_k(j + 1)) { ok = false; break; }
+            have_k = true;
           }
           tc_fence_after();
-          const uint32_t tm_s = tmem + C::kTmS0 + t * 128;
-          issue_pv<D>(tmem + C::kTmO0 + t * D, tm_s, slot_smem(seqV), j > 0);
-          if (t == last_tile(j)) tc_commit(bar(C::kBarKVEmpty + seqV % C::kSlots));
-          if (j + 1 < nk[t]) {
-            if (!have_k) {
-              if (!wait_full(seqK + 2)) { ok = false; break; }
-              have_k = true;
-              tc_fence_after();
-            }
-            issue_s<D>(tm_s, q_smem[t], slot_smem(seqK + 2));
-            tc_commit(bar(C::kBarSFull + t));
-            if (t == last_tile(j + 1)) tc_commit(bar(C::kBarKVEmpty + (seqK + 2) % C::kSlots));
-          } else {
-            tc_commit(bar(C::kBarOFull + t));
-          }
+          issue_s<D>(tmem + C::kTmS0 + t * 128, t ? q_smem1 : q_smem0, k_smem(j + 1));
+          tc_commit_e(bar(C::kBarSFull + t));
         }
+        if (!ok) break;
+        tc_commit_e(bar(C::kBarKEmpty + (j + 1) % C::kKSlots));
       }
-      // No MMA may be in flight when TMEM is released.
-      tc_commit(bar(C::kBarDrain));
-      drain_wait(bar(C::kBarDrain), 0, p.timeout_ns);
+      // O_t += P_t(j) V_j
+      bool have_v = false;
+      for (int t = 0; t < 2 && ok; ++t) {
+        if (j >= nk[t]) continue;
+        if (!mbar_wait_warp(bar(C::kBarPFull + t), j & 1, wd)) { ok = false; break; }
+        if (!have_v) {
+          if (!wait_v(j)) { ok = false; break; }
+          have_v = true;
+        }
+        tc_fence_after();
+        issue_pv<D>(tmem + C::kTmO0 + t * D, t ? p_smem1 : p_smem0, v_smem(j), j > 0);
+        tc_commit_e(bar(C::kBarPVDone + t));
+      }
+      if (!ok) break;
+      tc_commit_e(bar(C::kBarVEmpty + j % C::kVSlots));
     }
+    // No MMA may be in flight when TMEM is released.
+    tc_commit_e(bar(C::kBarDrain));
+    drain_wait(bar(C::kBarDrain), 0, p.timeout_ns);
     __syncwarp();
   } else {
     // ------------------------------------------------------------ softmax
@@ -288,6 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const uint32_t tm_s = tmem + lane_off + C::kTmS0 + t * 128;
     const uint32_t tm_o = tmem + lane_off + C::kTmO0 + t * D;
+    uint8_t* p_row = base_ptr + C::kPOff + t * C::kPBytes + row_in_tile * 128;
     const float c = p.scale_log2;
     float m_ref = -INFINITY;
     float l = 0.0f;
@@ -300,6 +319,10 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) tmem_ld32(tm_s + cc * 32, s[cc]);
       tmem_wait_ld();
+      // S_t(j) is in registers: the MMA may overwrite it with S_t(j+1) now
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::kBarSFree + t));
       const int kv0 = j * BN;
       const bool need_mask = (p.causal && kv0 + BN - 1 > r0) || (kv0 + BN > p.N);
       if (need_mask) {
@@ -335,6 +358,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         m_ref = m_new;
         l *= alpha;
       }
+      // PV_t(j-1) must be complete before P_t is overwritten and O_t rescaled.
+      if (j > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarPVDone + t), (j - 1) & 1, wd));
+        if (!ok) break;
+        tc_fence_after();
+      }
       const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
       const float2 c2 = make_float2(c, c), nm2 = make_float2(-m_use, -m_use);
       float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
@@ -355,14 +384,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           acc[k & 3] = fadd2(acc[k & 3], pe);
           pk[k] = pack_bf16x2(pe.x, pe.y);
         }
-        tmem_st16(tm_s + cc * 16, pk);
+        // keys 32cc..32cc+31 = 16-byte units 4cc..4cc+3 of this row's 256 bytes:
+        // chunk (cc / 2), units (cc % 2) * 4 + u, 128-byte swizzle by the row
+        uint8_t* chunk = p_row + (cc >> 1) * C::kChunkBytes;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          *reinterpret_cast<uint4*>(chunk + ((((cc & 1) * 4 + u) ^ (row_in_tile & 7)) * 16)) =
+              make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
       }
-      const float rowsum = (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y) +
-                           (acc[2].x + acc[2].y) + (acc[3].x + acc[3].y);
-      l += rowsum;
+      l += (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y) + (acc[2].x + acc[2].y) +
+           (acc[3].x + acc[3].y);
       if (move && j > 0) {
-        // O_t holds the sum up to tile j-1 (PV_t(j-1) completed before S_t(j)'s
-        // commit fired); bring it to the new reference max before PV_t(j).
+        // bring the sum up to key tile j-1 to the new reference max before PV_t(j)
 #pragma unroll
         for (int cc = 0; cc < D / 32; ++cc) {
           uint32_t o[32];
@@ -372,14 +405,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
           tmem_st32(tm_o + cc * 32, o);
         }
+        tmem_wait_st();
       }
-      tmem_wait_st();
+      fence_proxy_async_smem();  // P (generic stores) before the MMA reads it
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(C::kBarPFull + t));
     }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarOFull + t), 0, wd));
-    if (ok) {
+    if (ok && nk[t] > 0)
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarPVDone + t), (nk[t] - 1) & 1, wd));
+    if (ok && nk[t] > 0) {
       tc_fence_after();
       const float inv_l = (l > 0.0f) ? 1.0f / l : 0.0f;
       __nv_bfloat16* orow = p.O + (static_cast<size_t>(bh) * p.N + row) * D;
