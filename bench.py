@@ -45,6 +45,8 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD)
+    ap.add_argument("--seq-len", type=int, default=None,
+                    help="override the workload's N (same B, H, d, dtype, mask and scale)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
@@ -230,6 +232,11 @@ def main():
     from io_aware_attention_flashattention_b200.inputs import WORKLOADS
 
     w = WORKLOADS[args.workload]
+    if args.seq_len is not None and args.seq_len != w.N:
+        import dataclasses
+
+        w = dataclasses.replace(w, N=int(args.seq_len),
+                                name=f"{w.name.rsplit('_n', 1)[0]}_n{args.seq_len}_d{w.d}")
     if args.impl == "reference":
         return reference_arm(args, w)
 

@@ -255,8 +255,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  const int j = static_cast<int>(blockIdx.x) / p.BH;  // key tile (heaviest first if causal)
-  const int bh = static_cast<int>(blockIdx.x) % p.BH;
+  // Work item: head-major (the resident CTAs share one or two heads' Q, dO and dQ
+  // accumulator in L2); within a head, key tile 0 (the heaviest if causal) first.
+  const int n_kt = p.Npad / BN;
+  const int bh = static_cast<int>(blockIdx.x) / n_kt;
+  const int j = static_cast<int>(blockIdx.x) % n_kt;
   const int k0 = j * BN;
   const int n_q = (p.N + BM - 1) / BM;
   const int i_begin = p.causal ? j : 0;  // BM == BN: query tiles i >= j see key tile j

@@ -143,9 +143,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // Work item: heaviest query blocks first (matters for causal).
-  const int qb = (p.n_qblk - 1) - static_cast<int>(blockIdx.x) / p.BH;
-  const int bh = static_cast<int>(blockIdx.x) % p.BH;
+  // Work item: head-major, so that the CTAs resident at any time cover about two
+  // heads and their K/V stay in L2; within a head the heaviest query blocks (causal)
+  // go first.
+  const int bh = static_cast<int>(blockIdx.x) / p.n_qblk;
+  const int qb = (p.n_qblk - 1) - static_cast<int>(blockIdx.x) % p.n_qblk;
   const int q0 = qb * 2 * BM;
   const int n_kv_total = (p.N + BN - 1) / BN;
   int nk[2];
