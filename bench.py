@@ -146,6 +146,32 @@ class ClockSampler:
                 "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# ---------------------------------------------------------------- ranks
+
+
+def replica_seed(w, rank: int) -> int:
+    """Each rank draws its own replica of the workload (independent heads)."""
+    return w.seed + 7919 * rank
+
+
+def max_over_ranks(value_ms: float, world: int, device=None) -> float:
+    """The slowest rank's time (the job's time); a no-op for one rank. Uses the
+    default process group (NCCL on GPUs; gloo works for host-side tests)."""
+    if world <= 1:
+        return float(value_ms)
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([float(value_ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(flops_per_step: float, world: int, steps: int, job_ms: float) -> float:
+    """Whole-job TFLOP/s: the work of all ranks divided by the slowest rank's time."""
+    return flops_per_step * world * steps / (job_ms * 1e-3) / 1e12
+
+
 # ---------------------------------------------------------------- CPU oracle sample
 
 
@@ -262,7 +288,7 @@ def main():
             dist.barrier()
 
     # inputs: this rank's replica of the workload (seed offset by rank)
-    q, k, v, do = make_inputs(w.B, w.H, w.N, w.d, w.dtype, w.seed + 7919 * rank, w.qk_gain)
+    q, k, v, do = make_inputs(w.B, w.H, w.N, w.d, w.dtype, replica_seed(w, rank), w.qk_gain)
     Q, K, V, dO = (t.to(dev) for t in (q, k, v, do))
     O = torch.empty_like(Q)
     LSE = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
@@ -318,15 +344,11 @@ def main():
     per_kernel = [[events[s][i].elapsed_time(events[s][i + 1]) for s in range(args.steps)]
                   for i in range(len(names))]
     step_ms = [events[s][0].elapsed_time(events[s][-1]) for s in range(args.steps)]
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), world, dev)
 
     fwd_f, bwd_f = w.fwd_flops(), w.bwd_flops()
     flops_step = fwd_f + bwd_f
-    value = flops_step * world * args.steps / (total_ms * 1e-3) / 1e12
+    value = job_throughput(flops_step, world, args.steps, total_ms)
 
     # per-kernel figures and the dominant kernel's roofline
     BH, N, d = w.B * w.H, w.N, w.d
@@ -394,12 +416,8 @@ def main():
         e1.record(stream)
         torch.cuda.synchronize()
         barrier()
-        e_ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([e_ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
-        e2e = {"value": flops_step * world * n_e2e / (e_ms * 1e-3) / 1e12, "unit": "TFLOP/s",
+        e_ms = max_over_ranks(e0.elapsed_time(e1), world, dev)
+        e2e = {"value": job_throughput(flops_step, world, n_e2e, e_ms), "unit": "TFLOP/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
                "ms_per_step": e_ms / n_e2e}
 
