@@ -145,6 +145,22 @@ fa_status fa_backward_noalloc(const void* Q, const void* K, const void* V, const
                               fa_stream_t stream);
 
 /*
+ * f16 entry points: fa_forward and fa_backward with IEEE half-precision (f16)
+ * tensors in place of bf16 -- Q, K, V, O, dO, dQ, dK, dV are f16 [B,H,N,d]; LSE
+ * and the workspace as for the bf16 calls. Same kernels and the same fp32
+ * accumulation; P and dS are rounded to f16 before their products (the tensor
+ * cores take both operands of one product in one 16-bit type). f16 holds values
+ * below 65504 in magnitude: O, dQ, dK and dV beyond that become infinite.
+ */
+fa_status fa_forward_f16(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                         int B, int H, int N, int d, float scale, int causal,
+                         fa_stream_t stream);
+fa_status fa_backward_f16(const void* Q, const void* K, const void* V, const void* O,
+                          const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
+                          int B, int H, int N, int d, float scale, int causal,
+                          void* workspace, size_t workspace_bytes, fa_stream_t stream);
+
+/*
  * fp32 entry points: the same operation and arguments with fp32 tensors
  * (float [B,H,N,d]), computed in fp32 on the CUDA cores (FFMA), for callers that
  * need fp32 accuracy; tensor-core fp32 (tf32) cannot reach it. The backward is

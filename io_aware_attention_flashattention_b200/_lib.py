@@ -27,6 +27,9 @@ SIGNATURES = {
     "fa_backward_dq_convert": (_i, [_vp, _i, _i, _i, _i, _f, _vp, _sz, _vp]),
     "fa_backward_noalloc": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                  _i, _i, _i, _i, _f, _i, _vp]),
+    "fa_forward_f16": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp]),
+    "fa_backward_f16": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                             _i, _i, _i, _i, _f, _i, _vp, _sz, _vp]),
     "fa_forward_f32": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp]),
     "fa_backward_f32": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                              _i, _i, _i, _i, _f, _i, _vp, _sz, _vp]),

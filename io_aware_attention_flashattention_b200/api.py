@@ -24,7 +24,7 @@ from ._lib import FAError, check, lib
 __all__ = [
     "FAError", "fa_forward", "fa_backward", "fa_backward_workspace_size",
     "fa_backward_preprocess", "fa_backward_main", "fa_backward_dq_convert",
-    "fa_backward_noalloc", "fa_forward_f32",
+    "fa_backward_noalloc", "fa_forward_f16", "fa_backward_f16", "fa_forward_f32",
     "fa_backward_f32", "fa_get_status", "fa_watchdog_selftest", "fa_version",
     "forward", "backward", "attention", "FlashAttentionFunction",
 ]
@@ -72,6 +72,16 @@ def fa_forward(Q, K, V, O, LSE, scale: float, causal: bool, stream=None) -> None
             _need("LSE", LSE, torch.float32, (B, H, N))]
     check("fa_forward", lib().fa_forward(*args, B, H, N, d, float(scale), int(bool(causal)),
                                          _stream(stream)))
+
+
+def fa_forward_f16(Q, K, V, O, LSE, scale: float, causal: bool, stream=None) -> None:
+    B, H, N, d = _shape(Q)
+    h = torch.float16
+    args = [_need("Q", Q, h, (B, H, N, d)), _need("K", K, h, (B, H, N, d)),
+            _need("V", V, h, (B, H, N, d)), _need("O", O, h, (B, H, N, d)),
+            _need("LSE", LSE, torch.float32, (B, H, N))]
+    check("fa_forward_f16", lib().fa_forward_f16(*args, B, H, N, d, float(scale),
+                                                 int(bool(causal)), _stream(stream)))
 
 
 def fa_forward_f32(Q, K, V, O, LSE, scale: float, causal: bool, stream=None) -> None:
@@ -155,6 +165,15 @@ def fa_backward_noalloc(Q, K, V, O, dO, LSE, dQ, dK, dV, scale: float, causal: b
         *ptrs, B, H, N, d, float(scale), int(bool(causal)), _stream(stream)))
 
 
+def fa_backward_f16(Q, K, V, O, dO, LSE, dQ, dK, dV, scale: float, causal: bool, workspace,
+                    stream=None) -> None:
+    ptrs, (B, H, N, d), ws, nbytes = _bwd_args(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace,
+                                               torch.float16)
+    check("fa_backward_f16", lib().fa_backward_f16(*ptrs, B, H, N, d, float(scale),
+                                                   int(bool(causal)), ws, nbytes,
+                                                   _stream(stream)))
+
+
 def fa_backward_f32(Q, K, V, O, dO, LSE, dQ, dK, dV, scale: float, causal: bool, workspace,
                     stream=None) -> None:
     ptrs, (B, H, N, d), ws, nbytes = _bwd_args(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace,
@@ -182,17 +201,19 @@ def _default_scale(d: int, scale):
 
 
 def forward(q, k, v, causal: bool = False, scale=None):
-    """(O, LSE) for bf16 or fp32 q, k, v of shape [B, H, N, d] on the GPU."""
+    """(O, LSE) for bf16, f16 or fp32 q, k, v of shape [B, H, N, d] on the GPU."""
     B, H, N, d = _shape(q)
     scale = _default_scale(d, scale)
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     if q.dtype == torch.bfloat16:
         fa_forward(q, k, v, o, lse, scale, causal)
+    elif q.dtype == torch.float16:
+        fa_forward_f16(q, k, v, o, lse, scale, causal)
     elif q.dtype == torch.float32:
         fa_forward_f32(q, k, v, o, lse, scale, causal)
     else:
-        raise TypeError(f"unsupported dtype {q.dtype}: bf16 or fp32")
+        raise TypeError(f"unsupported dtype {q.dtype}: bf16, f16 or fp32")
     return o, lse
 
 
@@ -210,10 +231,12 @@ def backward(q, k, v, o, lse, do, causal: bool = False, scale=None, workspace=No
     ws = workspace_for(q) if workspace is None else workspace
     if q.dtype == torch.bfloat16:
         fa_backward(q, k, v, o, do, lse, dq, dk, dv, scale, causal, ws)
+    elif q.dtype == torch.float16:
+        fa_backward_f16(q, k, v, o, do, lse, dq, dk, dv, scale, causal, ws)
     elif q.dtype == torch.float32:
         fa_backward_f32(q, k, v, o, do, lse, dq, dk, dv, scale, causal, ws)
     else:
-        raise TypeError(f"unsupported dtype {q.dtype}: bf16 or fp32")
+        raise TypeError(f"unsupported dtype {q.dtype}: bf16, f16 or fp32")
     return dq, dk, dv
 
 

@@ -1,4 +1,5 @@
-// fa_bwd_sm100.cuh -- attention backward for sm_100a (bf16 in/out, fp32 accumulate).
+// fa_bwd_sm100.cuh -- attention backward for sm_100a (bf16 or f16 in/out, fp32
+// accumulate; the element type is the template parameter E).
 //
 // Method: recomputation ("FlashAttention optimisation: breaking the performance
 // bottleneck of standard attention", section 4.2; "From GPU memory access to code:
@@ -86,8 +87,8 @@ struct Cfg {
 };
 
 struct Params {
-  __nv_bfloat16* dK;
-  __nv_bfloat16* dV;
+  uint16_t* dK;  // 16-bit elements (the kernel's element type)
+  uint16_t* dV;
   const float* L2;  // [BH, Npad], LSE * log2(e), +inf in padding
   const float* Dv;  // [BH, Npad]
   float* dQacc;     // [BH, N, D]
@@ -122,9 +123,9 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
 
 // X_j Y_h^T: M = 128 rows of X, N = 64 rows of the half tile Y_h, K = D; both
 // operands K-major (rows of 64 bf16 per 128-byte-swizzled chunk).
-template <int D>
+template <int D, Elt E>
 __device__ __forceinline__ void issue_xyT_half(uint32_t tm_d, uint32_t x_smem, uint32_t yh_smem) {
-  constexpr uint32_t idesc = idesc_bf16_f32(128, 64, 0, 0);
+  constexpr uint32_t idesc = idesc_f32acc<E>(128, 64, 0, 0);
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
     const uint32_t xo = (kk / 4) * Cfg<D>::kChunkBytes + (kk % 4) * 32;
@@ -136,10 +137,10 @@ __device__ __forceinline__ void issue_xyT_half(uint32_t tm_d, uint32_t x_smem, u
 
 // acc[128 keys x D] (+)= A_tmem[128 keys x 64 queries] * Y_h[64 queries x D] (the half
 // tile, row-major in shared memory, used as the MN-major B operand).
-template <int D>
+template <int D, Elt E>
 __device__ __forceinline__ void issue_acc_half(uint32_t tm_acc, uint32_t tm_a, uint32_t yh_smem,
                                                bool accumulate) {
-  constexpr uint32_t idesc = idesc_bf16_f32(128, D, 0, 1);
+  constexpr uint32_t idesc = idesc_f32acc<E>(128, D, 0, 1);
 #pragma unroll
   for (int kk = 0; kk < 64 / 16; ++kk)
     mma_ts_e(tm_acc, tm_a + kk * 8,
@@ -150,8 +151,9 @@ __device__ __forceinline__ void issue_acc_half(uint32_t tm_acc, uint32_t tm_a, u
 // D = 128: dQ^T_h[128 dims x 64 queries] = K_j^T[dims x keys] * dS_h^T[keys x queries]:
 // A = K_j read MN-major (dims contiguous), B = dS chunk h read MN-major (queries
 // contiguous in each key row).
+template <Elt E>
 __device__ __forceinline__ void issue_dqT_half(uint32_t tm_d, uint32_t k_smem, uint32_t ds_chunk) {
-  constexpr uint32_t idesc = idesc_bf16_f32(128, 64, 1, 1);
+  constexpr uint32_t idesc = idesc_f32acc<E>(128, 64, 1, 1);
 #pragma unroll
   for (int kk = 0; kk < 128 / 16; ++kk)
     mma_ss_e(tm_d, sdesc_sw128(k_smem + kk * 2048, Cfg<128>::kChunkBytes, 1024),
@@ -161,8 +163,9 @@ __device__ __forceinline__ void issue_dqT_half(uint32_t tm_d, uint32_t k_smem, u
 
 // D = 64: dQ_i[128 queries x 64] = dS[queries x keys] * K_j[keys x 64]: A = the whole
 // dS tile (MN-major, two 64-query chunks), B = K_j (MN-major).
+template <Elt E>
 __device__ __forceinline__ void issue_dq64(uint32_t tm_d, uint32_t ds_smem, uint32_t k_smem) {
-  constexpr uint32_t idesc = idesc_bf16_f32(128, 64, 1, 1);
+  constexpr uint32_t idesc = idesc_f32acc<E>(128, 64, 1, 1);
 #pragma unroll
   for (int kk = 0; kk < 128 / 16; ++kk)
     mma_ss_e(tm_d, sdesc_sw128(ds_smem + kk * 2048, Cfg<64>::kChunkBytes, 1024),
@@ -171,9 +174,9 @@ __device__ __forceinline__ void issue_dq64(uint32_t tm_d, uint32_t ds_smem, uint
 
 // ------------------------------------------------------------------ preprocess
 
-template <int D>
+template <int D, Elt E>
 __global__ void __launch_bounds__(256)
-    fa_bwd_pre_kernel(const __nv_bfloat16* __restrict__ O, const __nv_bfloat16* __restrict__ dO,
+    fa_bwd_pre_kernel(const uint16_t* __restrict__ O, const uint16_t* __restrict__ dO,
                       const float* __restrict__ LSE, float* __restrict__ L2,
                       float* __restrict__ Dv, float* __restrict__ dQacc, int N, int Npad,
                       long long total_rows) {
@@ -190,22 +193,18 @@ __global__ void __launch_bounds__(256)
     return;
   }
   const long long row = bh * N + i;
-  constexpr int PER = D / 32;  // bf16 per lane: 2 or 4
+  constexpr int WORDS = D / 64;  // 32-bit words (element pairs) per lane: 1 or 2
   float s = 0.f;
-  if (PER == 4) {
+  if (WORDS == 2) {
     const uint2 a = reinterpret_cast<const uint2*>(O + row * D)[lane];
     const uint2 b = reinterpret_cast<const uint2*>(dO + row * D)[lane];
-    const __nv_bfloat162* a2 = reinterpret_cast<const __nv_bfloat162*>(&a);
-    const __nv_bfloat162* b2 = reinterpret_cast<const __nv_bfloat162*>(&b);
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const float2 x = __bfloat1622float2(a2[k]), y = __bfloat1622float2(b2[k]);
-      s = fmaf(x.x, y.x, fmaf(x.y, y.y, s));
-    }
+    const float2 x0 = unpack2<E>(a.x), y0 = unpack2<E>(b.x);
+    const float2 x1 = unpack2<E>(a.y), y1 = unpack2<E>(b.y);
+    s = fmaf(x0.x, y0.x, fmaf(x0.y, y0.y, fmaf(x1.x, y1.x, x1.y * y1.y)));
   } else {
-    const __nv_bfloat162 a = reinterpret_cast<const __nv_bfloat162*>(O + row * D)[lane];
-    const __nv_bfloat162 b = reinterpret_cast<const __nv_bfloat162*>(dO + row * D)[lane];
-    const float2 x = __bfloat1622float2(a), y = __bfloat1622float2(b);
+    const uint32_t a = reinterpret_cast<const uint32_t*>(O + row * D)[lane];
+    const uint32_t b = reinterpret_cast<const uint32_t*>(dO + row * D)[lane];
+    const float2 x = unpack2<E>(a), y = unpack2<E>(b);
     s = fmaf(x.x, y.x, x.y * y.y);
   }
 #pragma unroll
@@ -221,23 +220,23 @@ __global__ void __launch_bounds__(256)
 
 // ------------------------------------------------------------------ dQ convert
 
-template <int D>
+template <int D, Elt E>
 __global__ void __launch_bounds__(256)
-    fa_bwd_dq_kernel(const float* __restrict__ dQacc, __nv_bfloat16* __restrict__ dQ,
-                     long long n4, float scale) {
+    fa_bwd_dq_kernel(const float* __restrict__ dQacc, uint16_t* __restrict__ dQ, long long n4,
+                     float scale) {
   for (long long k = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; k < n4;
        k += static_cast<long long>(gridDim.x) * blockDim.x) {
     const float4 v = reinterpret_cast<const float4*>(dQacc)[k];
     uint2 out;
-    out.x = pack_bf16x2(v.x * scale, v.y * scale);
-    out.y = pack_bf16x2(v.z * scale, v.w * scale);
+    out.x = pack2<E>(v.x * scale, v.y * scale);
+    out.y = pack2<E>(v.z * scale, v.w * scale);
     reinterpret_cast<uint2*>(dQ)[k] = out;
   }
 }
 
 // ------------------------------------------------------------------ main kernel
 
-template <int D>
+template <int D, Elt E>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -365,12 +364,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int seqO = seq_of(s, h, 0), seqQ = seq_of(s, h, 1);
         if (!(wait_full(seqO) && wait_full(seqQ))) return false;
         tc_fence_after();
-        issue_xyT_half<D>(tm_dp + 64 * h, v_smem, slot_smem(seqO));
+        issue_xyT_half<D, E>(tm_dp + 64 * h, v_smem, slot_smem(seqO));
         if (D == 128 && s > 0) {  // S^T_h shares columns with dQ^T_h of the last step
           if (!mbar_wait_warp(bar(C::kBarDQEmpty + h), (s - 1) & 1, wd)) return false;
           tc_fence_after();
         }
-        issue_xyT_half<D>(tm_s + 64 * h, k_smem, slot_smem(seqQ));
+        issue_xyT_half<D, E>(tm_s + 64 * h, k_smem, slot_smem(seqQ));
         tc_commit_e(bar(C::kBarS + h));
       }
       return true;
@@ -382,10 +381,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait_warp(bar(C::kBarP + h), s & 1, wd)) { ok = false; break; }
         tc_fence_after();
         const bool acc = (s > 0) || (h > 0);
-        issue_acc_half<D>(tmem + C::kTmDV, tm_s + 64 * h, slot_smem(seqO), acc);   // dV
-        issue_acc_half<D>(tmem + C::kTmDK, tm_dp + 64 * h, slot_smem(seqQ), acc);  // dK
+        issue_acc_half<D, E>(tmem + C::kTmDV, tm_s + 64 * h, slot_smem(seqO), acc);   // dV
+        issue_acc_half<D, E>(tmem + C::kTmDK, tm_dp + 64 * h, slot_smem(seqQ), acc);  // dK
         if constexpr (D == 128) {
-          issue_dqT_half(tm_s + 64 * h, k_smem, ds_smem + h * C::kChunkBytes);
+          issue_dqT_half<E>(tm_s + 64 * h, k_smem, ds_smem + h * C::kChunkBytes);
           tc_commit_e(bar(C::kBarDQFull + h));
         }
         tc_commit_e(bar(C::kBarEmpty + slot_of(seqO)));
@@ -397,7 +396,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (!mbar_wait_warp(bar(C::kBarDQEmpty), (s - 1) & 1, wd)) { ok = false; break; }
           tc_fence_after();
         }
-        issue_dq64(tmem + C::kTmDQ64, ds_smem, k_smem);
+        issue_dq64<E>(tmem + C::kTmDQ64, ds_smem, k_smem);
         tc_commit_e(bar(C::kBarDQFull));
       }
       if (s + 1 < nsteps) ok = issue_sdp(s + 1);
@@ -465,10 +464,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             pv[e] = pe;
             dsv[e] = pe * (__uint_as_float(dv[cur][k]) - Ds[e]);
           }
-          pk[2 * v] = pack_bf16x2(pv[0], pv[1]);
-          pk[2 * v + 1] = pack_bf16x2(pv[2], pv[3]);
-          dk[2 * v] = pack_bf16x2(dsv[0], dsv[1]);
-          dk[2 * v + 1] = pack_bf16x2(dsv[2], dsv[3]);
+          pk[2 * v] = pack2<E>(pv[0], pv[1]);
+          pk[2 * v + 1] = pack2<E>(pv[2], pv[3]);
+          dk[2 * v] = pack2<E>(dsv[0], dsv[1]);
+          dk[2 * v + 1] = pack2<E>(dsv[2], dsv[3]);
         }
         tmem_st8(tm_s + 8 * cc, pk);
         tmem_st8(tm_dp + 8 * cc, dk);
@@ -490,7 +489,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       // warps 0-3 write dK (times scale), warps 4-7 write dV
       tc_fence_after();
       const uint32_t tm_acc = tmem + lane_off + (h == 0 ? C::kTmDK : C::kTmDV);
-      __nv_bfloat16* out = (h == 0 ? p.dK : p.dV) + (static_cast<size_t>(bh) * p.N + key) * D;
+      uint16_t* out = (h == 0 ? p.dK : p.dV) + (static_cast<size_t>(bh) * p.N + key) * D;
       const float mul = (h == 0) ? p.scale : 1.0f;
 #pragma unroll 1
       for (int cc = 0; cc < D / 32; ++cc) {
@@ -500,7 +499,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t pk[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k)
-          pk[k] = pack_bf16x2(__uint_as_float(v[2 * k]) * mul, __uint_as_float(v[2 * k + 1]) * mul);
+          pk[k] = pack2<E>(__uint_as_float(v[2 * k]) * mul, __uint_as_float(v[2 * k + 1]) * mul);
         if (key < p.N) {
           uint4* dst = reinterpret_cast<uint4*>(out + cc * 32);
 #pragma unroll

@@ -1,4 +1,5 @@
-// fa_fwd_sm100.cuh -- fused attention forward for sm_100a (bf16 in, fp32 accumulate).
+// fa_fwd_sm100.cuh -- fused attention forward for sm_100a (bf16 or f16 in, fp32
+// accumulate; the element type is the template parameter E).
 //
 // Method: the blockwise forward of "FlashAttention optimisation: breaking the
 // performance bottleneck of standard attention", section 4.1 (for each query
@@ -78,7 +79,7 @@ struct Cfg {
 };
 
 struct Params {
-  __nv_bfloat16* O;
+  uint16_t* O;  // 16-bit elements (bf16 or f16, the kernel's element type)
   float* LSE;
   int N;
   int BH;
@@ -89,9 +90,9 @@ struct Params {
 };
 
 // S = Q_t K_j^T: M = 128 query rows, N = 128 keys, K = D; both operands K-major.
-template <int D>
+template <int D, Elt E>
 __device__ __forceinline__ void issue_s(uint32_t tm_d, uint32_t q_smem, uint32_t k_smem) {
-  constexpr uint32_t idesc = idesc_bf16_f32(BM, BN, 0, 0);
+  constexpr uint32_t idesc = idesc_f32acc<E>(BM, BN, 0, 0);
 #pragma unroll
   for (int kk = 0; kk < D / 16; ++kk) {
     const uint32_t off = (kk / 4) * Cfg<D>::kChunkBytes + (kk % 4) * 32;
@@ -101,10 +102,10 @@ __device__ __forceinline__ void issue_s(uint32_t tm_d, uint32_t q_smem, uint32_t
 }
 
 // O += P V_j: A = P (128 x 128 keys, K-major in shared memory), B = V_j read MN-major.
-template <int D>
+template <int D, Elt E>
 __device__ __forceinline__ void issue_pv(uint32_t tm_o, uint32_t p_smem, uint32_t v_smem,
                                          bool accumulate) {
-  constexpr uint32_t idesc = idesc_bf16_f32(BM, D, 0, 1);
+  constexpr uint32_t idesc = idesc_f32acc<E>(BM, D, 0, 1);
 #pragma unroll
   for (int kk = 0; kk < BN / 16; ++kk) {
     const uint32_t poff = (kk / 4) * Cfg<D>::kChunkBytes + (kk % 4) * 32;
@@ -126,7 +127,7 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
   }
 }
 
-template <int D>
+template <int D, Elt E>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const Params p) {
@@ -254,7 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         for (int t = 0; t < 2; ++t) {
           if (nk[t] == 0) continue;
-          issue_s<D>(tmem + C::kTmS0 + t * 128, t ? q_smem1 : q_smem0, k_smem(0));
+          issue_s<D, E>(tmem + C::kTmS0 + t * 128, t ? q_smem1 : q_smem0, k_smem(0));
           tc_commit_e(bar(C::kBarSFull + t));
         }
         tc_commit_e(bar(C::kBarKEmpty + 0));
@@ -272,7 +273,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             have_k = true;
           }
           tc_fence_after();
-          issue_s<D>(tmem + C::kTmS0 + t * 128, t ? q_smem1 : q_smem0, k_smem(j + 1));
+          issue_s<D, E>(tmem + C::kTmS0 + t * 128, t ? q_smem1 : q_smem0, k_smem(j + 1));
           tc_commit_e(bar(C::kBarSFull + t));
         }
         if (!ok) break;
@@ -288,7 +289,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           have_v = true;
         }
         tc_fence_after();
-        issue_pv<D>(tmem + C::kTmO0 + t * D, t ? p_smem1 : p_smem0, v_smem(j), j > 0);
+        issue_pv<D, E>(tmem + C::kTmO0 + t * D, t ? p_smem1 : p_smem0, v_smem(j), j > 0);
         tc_commit_e(bar(C::kBarPVDone + t));
       }
       if (!ok) break;
@@ -384,7 +385,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             pe = make_float2(ex2_approx(x.x), ex2_approx(x.y));
           }
           acc[k & 3] = fadd2(acc[k & 3], pe);
-          pk[k] = pack_bf16x2(pe.x, pe.y);
+          pk[k] = pack2<E>(pe.x, pe.y);
         }
         // keys 32cc..32cc+31 = 16-byte units 4cc..4cc+3 of this row's 256 bytes:
         // chunk (cc / 2), units (cc % 2) * 4 + u, 128-byte swizzle by the row
@@ -419,7 +420,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok && nk[t] > 0) {
       tc_fence_after();
       const float inv_l = (l > 0.0f) ? 1.0f / l : 0.0f;
-      __nv_bfloat16* orow = p.O + (static_cast<size_t>(bh) * p.N + row) * D;
+      uint16_t* orow = p.O + (static_cast<size_t>(bh) * p.N + row) * D;
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t o[32];
@@ -428,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t pk[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k)
-          pk[k] = pack_bf16x2(__uint_as_float(o[2 * k]) * inv_l, __uint_as_float(o[2 * k + 1]) * inv_l);
+          pk[k] = pack2<E>(__uint_as_float(o[2 * k]) * inv_l, __uint_as_float(o[2 * k + 1]) * inv_l);
         if (row < p.N) {
           uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
 #pragma unroll

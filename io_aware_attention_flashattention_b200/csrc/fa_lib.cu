@@ -102,10 +102,14 @@ fa_status prepare_device() {
   if (!st.supported) return FA_ERR_UNSUPPORTED;
   if (!st.attrs_done) {
     cudaError_t e = cudaSuccess;
-    e = e ? e : set_smem(fwd::fa_fwd_kernel<64>, fwd::Cfg<64>::kSmemBytes);
-    e = e ? e : set_smem(fwd::fa_fwd_kernel<128>, fwd::Cfg<128>::kSmemBytes);
-    e = e ? e : set_smem(bwd::fa_bwd_kernel<64>, bwd::Cfg<64>::kSmemBytes);
-    e = e ? e : set_smem(bwd::fa_bwd_kernel<128>, bwd::Cfg<128>::kSmemBytes);
+    e = e ? e : set_smem(fwd::fa_fwd_kernel<64, Elt::BF16>, fwd::Cfg<64>::kSmemBytes);
+    e = e ? e : set_smem(fwd::fa_fwd_kernel<128, Elt::BF16>, fwd::Cfg<128>::kSmemBytes);
+    e = e ? e : set_smem(fwd::fa_fwd_kernel<64, Elt::F16>, fwd::Cfg<64>::kSmemBytes);
+    e = e ? e : set_smem(fwd::fa_fwd_kernel<128, Elt::F16>, fwd::Cfg<128>::kSmemBytes);
+    e = e ? e : set_smem(bwd::fa_bwd_kernel<64, Elt::BF16>, bwd::Cfg<64>::kSmemBytes);
+    e = e ? e : set_smem(bwd::fa_bwd_kernel<128, Elt::BF16>, bwd::Cfg<128>::kSmemBytes);
+    e = e ? e : set_smem(bwd::fa_bwd_kernel<64, Elt::F16>, bwd::Cfg<64>::kSmemBytes);
+    e = e ? e : set_smem(bwd::fa_bwd_kernel<128, Elt::F16>, bwd::Cfg<128>::kSmemBytes);
     e = e ? e : set_smem(f32::fa_f32_bwd_dkdv_kernel<64>, f32::dkdv_smem_bytes<64>());
     e = e ? e : set_smem(f32::fa_f32_bwd_dkdv_kernel<128>, f32::dkdv_smem_bytes<128>());
     e = e ? e : set_smem(f32::fa_f32_bwd_dq_kernel<64>, f32::dq_smem_bytes<64>());
@@ -136,9 +140,11 @@ fa_status check_ptrs(std::initializer_list<const void*> ptrs) {
 
 size_t round256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
 
-// 3-D view [B*H, N, d] of a bf16 tensor with boxes of 64 columns x `box_rows`
-// rows x 1 head, 128-byte swizzle. Rows beyond N read as zero, per head.
-bool make_map_bf16(CUtensorMap* map, const void* ptr, int BH, int N, int d, int box_rows) {
+// 3-D view [B*H, N, d] of a 16-bit tensor (bf16 or f16 by E) with boxes of 64
+// columns x `box_rows` rows x 1 head, 128-byte swizzle. Rows beyond N read as zero,
+// per head.
+template <Elt E>
+bool make_map(CUtensorMap* map, const void* ptr, int BH, int N, int d, int box_rows) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(N),
@@ -147,7 +153,9 @@ bool make_map_bf16(CUtensorMap* map, const void* ptr, int BH, int N, int d, int 
                                  static_cast<cuuint64_t>(N) * d * 2};
   const cuuint32_t box[3] = {64u, static_cast<cuuint32_t>(box_rows), 1u};
   const cuuint32_t estr[3] = {1u, 1u, 1u};
-  return enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+  constexpr CUtensorMapDataType dt =
+      (E == Elt::BF16) ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  return enc(map, dt, 3, const_cast<void*>(ptr), dims, strides, box,
              estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
@@ -161,6 +169,168 @@ fa_status launch_status() {
 }  // namespace fa
 
 using namespace fa;
+
+namespace {
+
+// The bf16 and f16 entry points share these bodies; E picks the kernels' element
+// type and the tensor maps' data type.
+
+template <Elt E>
+fa_status forward_impl(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
+                     int H, int N, int d, float scale, int causal, fa_stream_t stream) {
+  fa_status st = check_shape(B, H, N, d, scale, causal);
+  if (st != FA_OK) return st;
+  if (N == 0) return FA_OK;
+  if ((st = check_ptrs({Q, K, V, O, LSE})) != FA_OK) return st;
+  if ((st = prepare_device()) != FA_OK) return st;
+  const int BH = B * H;
+  CUtensorMap mq, mk, mv;
+  if (!make_map<E>(&mq, Q, BH, N, d, fwd::BM) || !make_map<E>(&mk, K, BH, N, d, fwd::BN) ||
+      !make_map<E>(&mv, V, BH, N, d, fwd::BN))
+    return FA_ERR_CUDA;
+  fwd::Params p;
+  p.O = static_cast<uint16_t*>(O);
+  p.LSE = LSE;
+  p.N = N;
+  p.BH = BH;
+  p.n_qblk = (N + 2 * fwd::BM - 1) / (2 * fwd::BM);
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.causal = causal;
+  p.timeout_ns = watchdog_ns();
+  const dim3 grid(static_cast<unsigned>(p.n_qblk) * BH);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 64)
+    fwd::fa_fwd_kernel<64, E><<<grid, fwd::kThreads, fwd::Cfg<64>::kSmemBytes, s>>>(mq, mk, mv, p);
+  else
+    fwd::fa_fwd_kernel<128, E><<<grid, fwd::kThreads, fwd::Cfg<128>::kSmemBytes, s>>>(mq, mk, mv, p);
+  return launch_status();
+}
+
+// Shared validation and set-up of the three backward stages. Fills the tensor maps
+// only when `maps` is set (the main stage is the only one that needs them).
+struct BwdPlan {
+  int BH, N, Npad, d;
+  float* L2;
+  float* Dv;
+  float* dQacc;
+};
+
+fa_status bwd_plan(const void* const* ptrs, int nptrs, int B, int H, int N, int d,
+                          float scale, int causal, void* workspace, size_t workspace_bytes,
+                          BwdPlan* plan) {
+  fa_status st = check_shape(B, H, N, d, scale, causal);
+  if (st != FA_OK) return st;
+  plan->BH = B * H;
+  plan->N = N;
+  plan->d = d;
+  plan->Npad = (N + 127) / 128 * 128;
+  if (N == 0) return FA_OK;
+  for (int i = 0; i < nptrs; ++i)
+    if (ptrs[i] == nullptr || !aligned16(ptrs[i])) return FA_ERR_INVALID_ARG;
+  if (workspace == nullptr || !aligned16(workspace)) return FA_ERR_INVALID_ARG;
+  if (workspace_bytes < fa_backward_workspace_size(B, H, N, d)) return FA_ERR_INVALID_ARG;
+  if ((st = prepare_device()) != FA_OK) return st;
+  // workspace: L2 [BH, Npad] | D [BH, Npad] | dQ accumulator [BH, N, d] (fp32)
+  char* ws = static_cast<char*>(workspace);
+  const size_t vec_bytes = round256(static_cast<size_t>(plan->BH) * plan->Npad * sizeof(float));
+  plan->L2 = reinterpret_cast<float*>(ws);
+  plan->Dv = reinterpret_cast<float*>(ws + vec_bytes);
+  plan->dQacc = reinterpret_cast<float*>(ws + 2 * vec_bytes);
+  return FA_OK;
+}
+
+template <Elt E>
+fa_status preprocess_impl(const void* O, const void* dO, const float* LSE, int B, int H,
+                                 int N, int d, float scale, int causal, void* workspace,
+                                 size_t workspace_bytes, fa_stream_t stream) {
+  const void* ptrs[] = {O, dO, LSE};
+  BwdPlan pl;
+  fa_status st = bwd_plan(ptrs, 3, B, H, N, d, scale, causal, workspace, workspace_bytes, &pl);
+  if (st != FA_OK || N == 0) return st;
+  const long long rows = static_cast<long long>(pl.BH) * pl.Npad;
+  const unsigned blocks = static_cast<unsigned>((rows + 7) / 8);
+  const auto* O16 = static_cast<const uint16_t*>(O);
+  const auto* dO16 = static_cast<const uint16_t*>(dO);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 64)
+    bwd::fa_bwd_pre_kernel<64, E><<<blocks, 256, 0, s>>>(O16, dO16, LSE, pl.L2, pl.Dv, pl.dQacc, N,
+                                                      pl.Npad, rows);
+  else
+    bwd::fa_bwd_pre_kernel<128, E><<<blocks, 256, 0, s>>>(O16, dO16, LSE, pl.L2, pl.Dv, pl.dQacc, N,
+                                                       pl.Npad, rows);
+  return launch_status();
+}
+
+template <Elt E>
+fa_status main_impl(const void* Q, const void* K, const void* V, const void* dO, void* dK,
+                           void* dV, int B, int H, int N, int d, float scale, int causal,
+                           void* workspace, size_t workspace_bytes, fa_stream_t stream) {
+  const void* ptrs[] = {Q, K, V, dO, dK, dV};
+  BwdPlan pl;
+  fa_status st = bwd_plan(ptrs, 6, B, H, N, d, scale, causal, workspace, workspace_bytes, &pl);
+  if (st != FA_OK || N == 0) return st;
+  CUtensorMap mq, mk, mv, mdo;
+  // Q and dO stream in half tiles of 64 rows; K and V are loaded as 128-row tiles
+  if (!make_map<E>(&mq, Q, pl.BH, N, d, 64) || !make_map<E>(&mk, K, pl.BH, N, d, bwd::BN) ||
+      !make_map<E>(&mv, V, pl.BH, N, d, bwd::BN) || !make_map<E>(&mdo, dO, pl.BH, N, d, 64))
+    return FA_ERR_CUDA;
+  bwd::Params p;
+  p.dK = static_cast<uint16_t*>(dK);
+  p.dV = static_cast<uint16_t*>(dV);
+  p.L2 = pl.L2;
+  p.Dv = pl.Dv;
+  p.dQacc = pl.dQacc;
+  p.N = N;
+  p.Npad = pl.Npad;
+  p.BH = pl.BH;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.causal = causal;
+  p.timeout_ns = watchdog_ns();
+  const dim3 grid(static_cast<unsigned>(pl.Npad / bwd::BN) * pl.BH);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 64)
+    bwd::fa_bwd_kernel<64, E><<<grid, bwd::kThreads, bwd::Cfg<64>::kSmemBytes, s>>>(mq, mk, mv, mdo, p);
+  else
+    bwd::fa_bwd_kernel<128, E><<<grid, bwd::kThreads, bwd::Cfg<128>::kSmemBytes, s>>>(mq, mk, mv, mdo, p);
+  return launch_status();
+}
+
+template <Elt E>
+fa_status dq_convert_impl(void* dQ, int B, int H, int N, int d, float scale, void* workspace,
+                                 size_t workspace_bytes, fa_stream_t stream) {
+  const void* ptrs[] = {dQ};
+  BwdPlan pl;
+  fa_status st = bwd_plan(ptrs, 1, B, H, N, d, scale, 0, workspace, workspace_bytes, &pl);
+  if (st != FA_OK || N == 0) return st;
+  const long long n4 = static_cast<long long>(pl.BH) * N * d / 4;
+  const unsigned blocks = static_cast<unsigned>(std::min<long long>((n4 + 255) / 256, 148 * 16));
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 64)
+    bwd::fa_bwd_dq_kernel<64, E><<<blocks, 256, 0, s>>>(pl.dQacc, static_cast<uint16_t*>(dQ), n4, scale);
+  else
+    bwd::fa_bwd_dq_kernel<128, E><<<blocks, 256, 0, s>>>(pl.dQacc, static_cast<uint16_t*>(dQ), n4, scale);
+  return launch_status();
+}
+
+template <Elt E>
+fa_status backward_impl(const void* Q, const void* K, const void* V, const void* O, const void* dO,
+                      const float* LSE, void* dQ, void* dK, void* dV, int B, int H, int N, int d,
+                      float scale, int causal, void* workspace, size_t workspace_bytes,
+                      fa_stream_t stream) {
+  const void* ptrs[] = {Q, K, V, O, dO, LSE, dQ, dK, dV};
+  BwdPlan pl;
+  fa_status st = bwd_plan(ptrs, 9, B, H, N, d, scale, causal, workspace, workspace_bytes, &pl);
+  if (st != FA_OK || N == 0) return st;
+  st = preprocess_impl<E>(O, dO, LSE, B, H, N, d, scale, causal, workspace, workspace_bytes, stream);
+  if (st != FA_OK) return st;
+  st = main_impl<E>(Q, K, V, dO, dK, dV, B, H, N, d, scale, causal, workspace, workspace_bytes,
+                        stream);
+  if (st != FA_OK) return st;
+  return dq_convert_impl<E>(dQ, B, H, N, d, scale, workspace, workspace_bytes, stream);
+}
+
+}  // namespace
 
 extern "C" {
 
@@ -209,152 +379,47 @@ fa_status fa_watchdog_selftest(int timeout_ms, fa_stream_t stream) {
 
 fa_status fa_forward(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
                      int H, int N, int d, float scale, int causal, fa_stream_t stream) {
-  fa_status st = check_shape(B, H, N, d, scale, causal);
-  if (st != FA_OK) return st;
-  if (N == 0) return FA_OK;
-  if ((st = check_ptrs({Q, K, V, O, LSE})) != FA_OK) return st;
-  if ((st = prepare_device()) != FA_OK) return st;
-  const int BH = B * H;
-  CUtensorMap mq, mk, mv;
-  if (!make_map_bf16(&mq, Q, BH, N, d, fwd::BM) || !make_map_bf16(&mk, K, BH, N, d, fwd::BN) ||
-      !make_map_bf16(&mv, V, BH, N, d, fwd::BN))
-    return FA_ERR_CUDA;
-  fwd::Params p;
-  p.O = static_cast<__nv_bfloat16*>(O);
-  p.LSE = LSE;
-  p.N = N;
-  p.BH = BH;
-  p.n_qblk = (N + 2 * fwd::BM - 1) / (2 * fwd::BM);
-  p.scale_log2 = scale * 1.4426950408889634f;
-  p.causal = causal;
-  p.timeout_ns = watchdog_ns();
-  const dim3 grid(static_cast<unsigned>(p.n_qblk) * BH);
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (d == 64)
-    fwd::fa_fwd_kernel<64><<<grid, fwd::kThreads, fwd::Cfg<64>::kSmemBytes, s>>>(mq, mk, mv, p);
-  else
-    fwd::fa_fwd_kernel<128><<<grid, fwd::kThreads, fwd::Cfg<128>::kSmemBytes, s>>>(mq, mk, mv, p);
-  return launch_status();
+  return forward_impl<Elt::BF16>(Q, K, V, O, LSE, B, H, N, d, scale, causal, stream);
 }
 
-// Shared validation and set-up of the three backward stages. Fills the tensor maps
-// only when `maps` is set (the main stage is the only one that needs them).
-struct BwdPlan {
-  int BH, N, Npad, d;
-  float* L2;
-  float* Dv;
-  float* dQacc;
-};
-
-static fa_status bwd_plan(const void* const* ptrs, int nptrs, int B, int H, int N, int d,
-                          float scale, int causal, void* workspace, size_t workspace_bytes,
-                          BwdPlan* plan) {
-  fa_status st = check_shape(B, H, N, d, scale, causal);
-  if (st != FA_OK) return st;
-  plan->BH = B * H;
-  plan->N = N;
-  plan->d = d;
-  plan->Npad = (N + 127) / 128 * 128;
-  if (N == 0) return FA_OK;
-  for (int i = 0; i < nptrs; ++i)
-    if (ptrs[i] == nullptr || !aligned16(ptrs[i])) return FA_ERR_INVALID_ARG;
-  if (workspace == nullptr || !aligned16(workspace)) return FA_ERR_INVALID_ARG;
-  if (workspace_bytes < fa_backward_workspace_size(B, H, N, d)) return FA_ERR_INVALID_ARG;
-  if ((st = prepare_device()) != FA_OK) return st;
-  // workspace: L2 [BH, Npad] | D [BH, Npad] | dQ accumulator [BH, N, d] (fp32)
-  char* ws = static_cast<char*>(workspace);
-  const size_t vec_bytes = round256(static_cast<size_t>(plan->BH) * plan->Npad * sizeof(float));
-  plan->L2 = reinterpret_cast<float*>(ws);
-  plan->Dv = reinterpret_cast<float*>(ws + vec_bytes);
-  plan->dQacc = reinterpret_cast<float*>(ws + 2 * vec_bytes);
-  return FA_OK;
+fa_status fa_forward_f16(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
+                         int H, int N, int d, float scale, int causal, fa_stream_t stream) {
+  return forward_impl<Elt::F16>(Q, K, V, O, LSE, B, H, N, d, scale, causal, stream);
 }
 
 fa_status fa_backward_preprocess(const void* O, const void* dO, const float* LSE, int B, int H,
                                  int N, int d, float scale, int causal, void* workspace,
                                  size_t workspace_bytes, fa_stream_t stream) {
-  const void* ptrs[] = {O, dO, LSE};
-  BwdPlan pl;
-  fa_status st = bwd_plan(ptrs, 3, B, H, N, d, scale, causal, workspace, workspace_bytes, &pl);
-  if (st != FA_OK || N == 0) return st;
-  const long long rows = static_cast<long long>(pl.BH) * pl.Npad;
-  const unsigned blocks = static_cast<unsigned>((rows + 7) / 8);
-  const auto* O16 = static_cast<const __nv_bfloat16*>(O);
-  const auto* dO16 = static_cast<const __nv_bfloat16*>(dO);
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (d == 64)
-    bwd::fa_bwd_pre_kernel<64><<<blocks, 256, 0, s>>>(O16, dO16, LSE, pl.L2, pl.Dv, pl.dQacc, N,
-                                                      pl.Npad, rows);
-  else
-    bwd::fa_bwd_pre_kernel<128><<<blocks, 256, 0, s>>>(O16, dO16, LSE, pl.L2, pl.Dv, pl.dQacc, N,
-                                                       pl.Npad, rows);
-  return launch_status();
+  return preprocess_impl<Elt::BF16>(O, dO, LSE, B, H, N, d, scale, causal, workspace,
+                                    workspace_bytes, stream);
 }
 
 fa_status fa_backward_main(const void* Q, const void* K, const void* V, const void* dO, void* dK,
                            void* dV, int B, int H, int N, int d, float scale, int causal,
                            void* workspace, size_t workspace_bytes, fa_stream_t stream) {
-  const void* ptrs[] = {Q, K, V, dO, dK, dV};
-  BwdPlan pl;
-  fa_status st = bwd_plan(ptrs, 6, B, H, N, d, scale, causal, workspace, workspace_bytes, &pl);
-  if (st != FA_OK || N == 0) return st;
-  CUtensorMap mq, mk, mv, mdo;
-  // Q and dO stream in half tiles of 64 rows; K and V are loaded as 128-row tiles
-  if (!make_map_bf16(&mq, Q, pl.BH, N, d, 64) || !make_map_bf16(&mk, K, pl.BH, N, d, bwd::BN) ||
-      !make_map_bf16(&mv, V, pl.BH, N, d, bwd::BN) || !make_map_bf16(&mdo, dO, pl.BH, N, d, 64))
-    return FA_ERR_CUDA;
-  bwd::Params p;
-  p.dK = static_cast<__nv_bfloat16*>(dK);
-  p.dV = static_cast<__nv_bfloat16*>(dV);
-  p.L2 = pl.L2;
-  p.Dv = pl.Dv;
-  p.dQacc = pl.dQacc;
-  p.N = N;
-  p.Npad = pl.Npad;
-  p.BH = pl.BH;
-  p.scale = scale;
-  p.scale_log2 = scale * 1.4426950408889634f;
-  p.causal = causal;
-  p.timeout_ns = watchdog_ns();
-  const dim3 grid(static_cast<unsigned>(pl.Npad / bwd::BN) * pl.BH);
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (d == 64)
-    bwd::fa_bwd_kernel<64><<<grid, bwd::kThreads, bwd::Cfg<64>::kSmemBytes, s>>>(mq, mk, mv, mdo, p);
-  else
-    bwd::fa_bwd_kernel<128><<<grid, bwd::kThreads, bwd::Cfg<128>::kSmemBytes, s>>>(mq, mk, mv, mdo, p);
-  return launch_status();
+  return main_impl<Elt::BF16>(Q, K, V, dO, dK, dV, B, H, N, d, scale, causal, workspace,
+                              workspace_bytes, stream);
 }
 
 fa_status fa_backward_dq_convert(void* dQ, int B, int H, int N, int d, float scale, void* workspace,
                                  size_t workspace_bytes, fa_stream_t stream) {
-  const void* ptrs[] = {dQ};
-  BwdPlan pl;
-  fa_status st = bwd_plan(ptrs, 1, B, H, N, d, scale, 0, workspace, workspace_bytes, &pl);
-  if (st != FA_OK || N == 0) return st;
-  const long long n4 = static_cast<long long>(pl.BH) * N * d / 4;
-  const unsigned blocks = static_cast<unsigned>(std::min<long long>((n4 + 255) / 256, 148 * 16));
-  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (d == 64)
-    bwd::fa_bwd_dq_kernel<64><<<blocks, 256, 0, s>>>(pl.dQacc, static_cast<__nv_bfloat16*>(dQ), n4, scale);
-  else
-    bwd::fa_bwd_dq_kernel<128><<<blocks, 256, 0, s>>>(pl.dQacc, static_cast<__nv_bfloat16*>(dQ), n4, scale);
-  return launch_status();
+  return dq_convert_impl<Elt::BF16>(dQ, B, H, N, d, scale, workspace, workspace_bytes, stream);
 }
 
 fa_status fa_backward(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                       const float* LSE, void* dQ, void* dK, void* dV, int B, int H, int N, int d,
                       float scale, int causal, void* workspace, size_t workspace_bytes,
                       fa_stream_t stream) {
-  const void* ptrs[] = {Q, K, V, O, dO, LSE, dQ, dK, dV};
-  BwdPlan pl;
-  fa_status st = bwd_plan(ptrs, 9, B, H, N, d, scale, causal, workspace, workspace_bytes, &pl);
-  if (st != FA_OK || N == 0) return st;
-  st = fa_backward_preprocess(O, dO, LSE, B, H, N, d, scale, causal, workspace, workspace_bytes, stream);
-  if (st != FA_OK) return st;
-  st = fa_backward_main(Q, K, V, dO, dK, dV, B, H, N, d, scale, causal, workspace, workspace_bytes,
-                        stream);
-  if (st != FA_OK) return st;
-  return fa_backward_dq_convert(dQ, B, H, N, d, scale, workspace, workspace_bytes, stream);
+  return backward_impl<Elt::BF16>(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, scale, causal,
+                                  workspace, workspace_bytes, stream);
+}
+
+fa_status fa_backward_f16(const void* Q, const void* K, const void* V, const void* O,
+                          const void* dO, const float* LSE, void* dQ, void* dK, void* dV, int B,
+                          int H, int N, int d, float scale, int causal, void* workspace,
+                          size_t workspace_bytes, fa_stream_t stream) {
+  return backward_impl<Elt::F16>(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, scale, causal,
+                                 workspace, workspace_bytes, stream);
 }
 
 // ---------------------------------------------------------------- backward without allocation

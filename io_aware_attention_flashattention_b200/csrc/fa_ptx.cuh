@@ -5,6 +5,7 @@
 
 #include <cuda.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 namespace fa {
@@ -236,12 +237,17 @@ __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, co
   return __all_sync(0xffffffffu, mbar_wait(bar, parity, wd));
 }
 
-// Instruction descriptor for kind::f16 with bf16 A and B and an fp32 accumulator.
-// a_mn / b_mn: 1 when the operand is MN-major (else K-major).
-__host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, int b_mn) {
+// The 16-bit element types of the tensor-core paths (kind::f16 operands).
+enum class Elt { BF16, F16 };
+
+// Instruction descriptor for kind::f16 with A and B of element type E and an fp32
+// accumulator. a_mn / b_mn: 1 when the operand is MN-major (else K-major).
+template <Elt E>
+__host__ __device__ constexpr uint32_t idesc_f32acc(int M, int N, int a_mn, int b_mn) {
+  constexpr uint32_t fmt = (E == Elt::BF16) ? 1u : 0u;  // A/B format: 1 = bf16, 0 = f16
   return (1u << 4)                               // D format: f32
-         | (1u << 7)                             // A format: bf16
-         | (1u << 10)                            // B format: bf16
+         | (fmt << 7)                            // A format
+         | (fmt << 10)                           // B format
          | (static_cast<uint32_t>(a_mn) << 15)   // A major
          | (static_cast<uint32_t>(b_mn) << 16)   // B major
          | (static_cast<uint32_t>(N >> 3) << 17) // N / 8
@@ -399,12 +405,33 @@ __device__ __forceinline__ float2 exp2_poly2(float2 x) {
                      __uint_as_float(__float_as_uint(q.y) + (__float_as_uint(t.y) << 23)));
 }
 
-// Two fp32 values to a packed bf16x2 word, round-to-nearest-even; `lo` lands in
+// Two fp32 values to a packed 16-bit pair, round-to-nearest-even; `lo` lands in
 // the low half (the element with the smaller index).
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
+}
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+template <Elt E>
+__device__ __forceinline__ uint32_t pack2(float lo, float hi) {
+  if constexpr (E == Elt::BF16) return pack_bf16x2(lo, hi);
+  else return pack_f16x2(lo, hi);
+}
+
+// A packed 16-bit pair back to two fp32 values (exact).
+template <Elt E>
+__device__ __forceinline__ float2 unpack2(uint32_t w) {
+  if constexpr (E == Elt::BF16) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+  } else {
+    __half2 h = *reinterpret_cast<__half2*>(&w);
+    return __half22float2(h);
+  }
 }
 
 }  // namespace fa

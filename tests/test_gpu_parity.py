@@ -4,17 +4,22 @@ same seeded inputs.
 Tolerances (max absolute error against the oracle fed the same rounded inputs):
   bf16 path:  |dO| <= 1e-2, |dLSE| <= 1e-3, each of dQ, dK, dV <= 5e-2 * max|oracle grad|
   fp32 path:  |dO| <= 1e-5, |dLSE| <= 1e-5, each grad <= 1e-5 * max|oracle grad|
-O is stored in bf16: rounding to the output format alone moves a value in
+  f16 path:   |dO| <= 2e-3, |dLSE| <= 1e-3, each grad <= 1e-2 * max|oracle grad|
+The f16 bounds are the bf16 ones scaled by the ratio of the two formats' unit
+roundoffs (2^-11 / 2^-8 = 1/8) and then loosened by about 1.6x, except LSE, which
+is computed from fp32 logits of exactly representable inputs in both formats.
+O is stored in bf16 (f16): rounding to the output format alone moves a value in
 [2^e, 2^(e+1)) by up to 2^(e-8), which exceeds 1e-2 once |O| > 2.56 (near-one-hot
 attention, as with the x8 logits, gives |O| ~ 4). The O bound is therefore read as
-applying to the result before that final rounding: per element, 1e-2 plus half a
-bf16 ulp of the oracle value.
+applying to the result before that final rounding: per element, the bound plus
+half an ulp of the output format at the oracle value.
 Where the oracle's gradient is identically zero (N = 1 gives dQ = dK = 0), the
 relative bound would demand exact zeros from rounded arithmetic; there the bound
 is an absolute floor (1e-3 bf16, 1e-6 fp32), far below
 the gradients' natural scale (|dO| ~ 1).
 Outputs are pre-filled with NaN so that an unwritten element fails the check.
 """
+import dataclasses
 import math
 
 import numpy as np
@@ -29,33 +34,41 @@ pytestmark = pytest.mark.gpu
 
 TOL_BF16 = dict(O=1e-2, L=1e-3, grad=5e-2, floor=1e-3)
 TOL_F32 = dict(O=1e-5, L=1e-5, grad=1e-5, floor=1e-6)
+TOL_F16 = dict(O=2e-3, L=1e-3, grad=1e-2, floor=2e-4)
+TOL = {torch.bfloat16: TOL_BF16, torch.float16: TOL_F16, torch.float32: TOL_F32}
 
 
 def grad_tol(tol, want):
     return max(tol["grad"] * float(np.abs(want).max()) if np.size(want) else 0.0, tol["floor"])
 
 
-def bf16_half_ulp(x):
-    """Half the spacing of the bf16 grid at |x| (8 significant bits)."""
+# significant bits and smallest normal exponent of the 16-bit output formats
+_FORMAT = {torch.bfloat16: (8, -126), torch.float16: (11, -14)}
+
+
+def half_ulp(x, dtype=torch.bfloat16):
+    """Half the spacing of the output format's grid at |x| (fixed below the normals)."""
+    bits, emin = _FORMAT[dtype]
     x = np.abs(np.asarray(x, dtype=np.float64))
-    e = np.floor(np.log2(np.where(x > 0, x, 1.0)))
-    return np.where(x > 0, np.exp2(e - 8), 0.0)
+    e = np.maximum(np.floor(np.log2(np.where(x > 0, x, 1.0))), emin)
+    return np.where(x > 0, np.exp2(e - bits), 0.0)
 
 
-def assert_close_o(name, got, want, tol):
-    """O check: tol plus half a bf16 ulp of the oracle value, element by element."""
+def assert_close_o(name, got, want, tol, dtype=torch.bfloat16):
+    """O check: tol plus half an ulp of the output format at the oracle value,
+    element by element."""
     got = np.asarray(got, dtype=np.float64)
     want = np.asarray(want, dtype=np.float64)
     assert got.shape == want.shape
     assert np.all(np.isfinite(got)), f"{name}: non-finite values (unwritten or overflow)"
     if not got.size:
         return 0.0
-    excess = np.abs(got - want) - (tol + bf16_half_ulp(want))
+    excess = np.abs(got - want) - (tol + half_ulp(want, dtype))
     worst = int(np.argmax(excess))
     err = float(np.abs(got - want).flat[worst])
     assert excess.flat[worst] <= 0, (
         f"{name}: error {err:.3e} at |O|={abs(want.flat[worst]):.3f} exceeds "
-        f"{tol:.1e} + half-ulp {bf16_half_ulp(want.flat[worst]):.2e}")
+        f"{tol:.1e} + half-ulp {half_ulp(want.flat[worst], dtype):.2e}")
     return float(np.max(np.abs(got - want)))
 
 
@@ -71,10 +84,8 @@ def run_forward(q, k, v, scale, causal):
     B, H, N, d = q.shape
     o = _nan_like(q)
     lse = torch.full((B, H, N), float("nan"), dtype=torch.float32, device=q.device)
-    if q.dtype == torch.bfloat16:
-        api.fa_forward(q, k, v, o, lse, scale, causal)
-    else:
-        api.fa_forward_f32(q, k, v, o, lse, scale, causal)
+    {torch.bfloat16: api.fa_forward, torch.float16: api.fa_forward_f16,
+     torch.float32: api.fa_forward_f32}[q.dtype](q, k, v, o, lse, scale, causal)
     torch.cuda.synchronize()
     assert api.fa_get_status() == 0
     return o, lse
@@ -84,10 +95,9 @@ def run_backward(q, k, v, o, lse, do, scale, causal):
     dq, dk, dv = _nan_like(q), _nan_like(k), _nan_like(v)
     ws = api.workspace_for(q)
     ws.fill_(0xFF)  # the workspace's contents on entry must not matter
-    if q.dtype == torch.bfloat16:
-        api.fa_backward(q, k, v, o, do, lse, dq, dk, dv, scale, causal, ws)
-    else:
-        api.fa_backward_f32(q, k, v, o, do, lse, dq, dk, dv, scale, causal, ws)
+    {torch.bfloat16: api.fa_backward, torch.float16: api.fa_backward_f16,
+     torch.float32: api.fa_backward_f32}[q.dtype](q, k, v, o, do, lse, dq, dk, dv, scale,
+                                                  causal, ws)
     torch.cuda.synchronize()
     assert api.fa_get_status() == 0
     return dq, dk, dv
@@ -112,8 +122,8 @@ def check_full(q, k, v, do, scale, causal, tol, backward=True):
     qc, kc, vc, doc = _dev(q, k, v, do)
     o, lse = run_forward(qc, kc, vc, scale, causal)
     O_ref, L_ref = oracle.forward(q, k, v, scale, causal)
-    if q.dtype == torch.bfloat16:
-        assert_close_o("O", _np(o), O_ref, tol["O"])
+    if q.dtype in _FORMAT:
+        assert_close_o("O", _np(o), O_ref, tol["O"], q.dtype)
     else:
         assert_close("O", _np(o), O_ref, tol["O"])
     assert_close("LSE", _np(lse), L_ref, tol["L"])
@@ -157,6 +167,29 @@ def test_f32_small_full_parity(B, H, N, d, causal):
     check_full(q, k, v, do, 1.0 / math.sqrt(d), causal, TOL_F32)
 
 
+F16_SMALL = [
+    (1, 1, 128, 64, False),
+    (1, 1, 256, 128, False),
+    (2, 3, 384, 64, True),
+    (1, 1, 1, 128, True),
+    (2, 1, 200, 128, True),
+    (1, 2, 1000, 64, True),
+    (1, 1, 640, 128, False),
+]
+
+
+@pytest.mark.parametrize("B,H,N,d,causal", F16_SMALL)
+def test_f16_small_full_parity(B, H, N, d, causal):
+    q, k, v, do = make_inputs(B, H, N, d, torch.float16, seed=17 + N + d + int(causal))
+    check_full(q, k, v, do, 1.0 / math.sqrt(d), causal, TOL_F16)
+
+
+def test_f16_large_logits_online_rescale():
+    q, k, v, do = make_inputs(1, 2, 512, 128, torch.float16, seed=98, qk_gain=8.0)
+    check_full(q, k, v, do, 1.0 / math.sqrt(128), True, TOL_F16)
+    check_full(q, k, v, do, 1.0 / math.sqrt(128), False, TOL_F16)
+
+
 def test_bf16_large_logits_online_rescale():
     """Logits spanning +-hundreds force many rescales of the running max."""
     q, k, v, do = make_inputs(1, 2, 512, 128, torch.bfloat16, seed=99, qk_gain=8.0)
@@ -196,6 +229,7 @@ def check_sampled(w, per_head=16, full_heads=(0,), dq_rows=True, dkdv_head=None,
     """Full-size workload on the GPU (the launch the benchmark times); checked
     against the oracle on whole heads and on sampled rows of every head."""
     q, k, v, do = workload_inputs(w)
+    tol = TOL[w.dtype]
     B, H, N, d = q.shape
     BH = B * H
     qc, kc, vc, doc = _dev(q, k, v, do)
@@ -208,8 +242,8 @@ def check_sampled(w, per_head=16, full_heads=(0,), dq_rows=True, dkdv_head=None,
     extra = [(h, list(range(0, 128)) + list(range(N - 128, N))) for h in full_heads]
     heads, rows = _sampled_rows(rng, BH, N, per_head, extra)
     O_ref, L_ref = oracle.forward_rows(q, k, v, w.scale, w.causal, heads, rows)
-    assert_close_o("O rows", o_np[heads, rows], O_ref, TOL_BF16["O"])
-    assert_close("LSE rows", l_np[heads, rows], L_ref, TOL_BF16["L"])
+    assert_close_o("O rows", o_np[heads, rows], O_ref, tol["O"], w.dtype)
+    assert_close("LSE rows", l_np[heads, rows], L_ref, tol["L"])
     if not w.backward:
         return
     dq, dk, dv = run_backward(qc, kc, vc, o, lse, doc, w.scale, w.causal)
@@ -218,7 +252,7 @@ def check_sampled(w, per_head=16, full_heads=(0,), dq_rows=True, dkdv_head=None,
         assert np.all(np.isfinite(g)), f"{name}: non-finite"
     if dq_rows:
         dQ_ref, _ = oracle.backward_dq_rows(q, k, v, do, w.scale, w.causal, heads, rows)
-        assert_close("dQ rows", dq_np[heads, rows], dQ_ref, grad_tol(TOL_BF16, dQ_ref))
+        assert_close("dQ rows", dq_np[heads, rows], dQ_ref, grad_tol(tol, dQ_ref))
     if dkdv_head is not None:
         h = dkdv_head
         all_rows = np.arange(N)
@@ -228,8 +262,8 @@ def check_sampled(w, per_head=16, full_heads=(0,), dq_rows=True, dkdv_head=None,
                                          rng.choice(N, n_keys, replace=False)]))
         dK_ref, dV_ref = oracle.backward_dkdv_rows(q, k, v, do, w.scale, w.causal, h, L_h, D_h,
                                                    keys)
-        assert_close("dK rows", dk_np[h, keys], dK_ref, grad_tol(TOL_BF16, dK_ref))
-        assert_close("dV rows", dv_np[h, keys], dV_ref, grad_tol(TOL_BF16, dV_ref))
+        assert_close("dK rows", dk_np[h, keys], dK_ref, grad_tol(tol, dK_ref))
+        assert_close("dV rows", dv_np[h, keys], dV_ref, grad_tol(tol, dV_ref))
     # properties at full size: sum_j dK_j = 0 and sum_i dV_i = sum_i dO_i per head
     do_np = _np(doc).reshape(BH, N, d)
     sum_dv = dv_np.sum(axis=1)
@@ -264,6 +298,11 @@ def test_workload_mid_b1h8_n4096_d128():
 
 def test_workload_stress_causal_b2h16_n8192_d128_qk8():
     check_sampled(WORKLOADS["stress_causal_b2h16_n8192_d128_qk8"], per_head=16, full_heads=(0, 31))
+
+
+def test_workload_mid_b1h8_n4096_d128_in_f16():
+    w = dataclasses.replace(WORKLOADS["mid_b1h8_n4096_d128"], dtype=torch.float16)
+    check_sampled(w, per_head=32, full_heads=(2,), dkdv_head=6)
 
 
 @pytest.mark.slow
