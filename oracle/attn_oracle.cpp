@@ -20,9 +20,24 @@
 //                              O = PV); the scaling by 1/sqrt(d) is [intelli] section 1
 //                              step 2 and [yunthe] "standard attention" section; the
 //                              scale is an argument here.
-//   S[i][j] = -inf if causal and j > i   [yunthe] "causal mask" troubleshooting item
-//                              (is_causal=True); the key at the query's own position
-//                              is kept.
+//   S[i][j] = -inf where key j is hidden from query i. Three masks, each optional,
+//   combine by AND (a key is seen only if every mask given keeps it):
+//     causal: keeps j <= i     [yunthe] "causal mask" troubleshooting item
+//                              (is_causal=True); the query's own position is kept.
+//     window (left, right): keeps i - left <= j <= i + right; a negative bound is
+//                              no bound on that side. [yunthe] troubleshooting item 3
+//                              (causal mask configuration), its sliding-window example
+//                              (Longformer/Gemma style, a window-size pair such as
+//                              (512, 512) given together with is_causal=True).
+//     block mask M: keeps (i, j) iff M[i / 128][j / 128] != 0, M a row-major
+//                              ceil(N/128) x ceil(N/128) byte matrix, the same for all
+//                              heads. [intelli] section 7 item 2 (block-sparse
+//                              FlashAttention: a sparse pattern over blocks) and [jos]
+//                              p.218 (the algorithm extended to sparse attention); no
+//                              page gives a block size for the mask, so it is the
+//                              tile size 128 of [yunthe] "GPU memory optimisation
+//                              strategy" (Block_Q = Block_K = 128).
+//   A query row that sees no key at all has P = 0, O = 0 and L = -inf.
 //   m_i = max_j S[i][j]        [jsqmd] section 2.1, safe softmax
 //   P[i][j] = exp(S[i][j] - m_i) / sum_j exp(S[i][j] - m_i)
 //   O = P V
@@ -63,16 +78,39 @@ namespace {
 
 const double kNegInf = -std::numeric_limits<double>::infinity();
 
+const int64_t kBlock = 128;  // block-mask granularity (rows and keys)
+
 bool bad_shape(int64_t B, int64_t H, int64_t N, int64_t d) {
   return B < 0 || H < 0 || N < 0 || d <= 0;
 }
 
-// One row of scaled, masked logits: s[j] = scale * <q_i, k_j>, -inf above the
-// diagonal when causal.
+// Which keys a query row sees: the AND of the three masks in the header.
+struct Visibility {
+  int causal;
+  int64_t left, right;    // window bounds; negative = unbounded on that side
+  const uint8_t* blocks;  // [nb x nb] row-major, nonzero = block kept; null = all kept
+  int64_t nb;             // ceil(N / kBlock)
+
+  bool sees(int64_t i, int64_t j) const {
+    if (causal && j > i) return false;
+    if (left >= 0 && j < i - left) return false;
+    if (right >= 0 && j > i + right) return false;
+    if (blocks && !blocks[(i / kBlock) * nb + j / kBlock]) return false;
+    return true;
+  }
+};
+
+Visibility make_vis(int64_t N, int causal, int64_t left, int64_t right,
+                    const uint8_t* blocks) {
+  return Visibility{causal, left, right, blocks, (N + kBlock - 1) / kBlock};
+}
+
+// One row of scaled, masked logits: s[j] = scale * <q_i, k_j>, -inf where the
+// key is hidden.
 void logits_row(const double* q, const double* K, int64_t N, int64_t d, double scale,
-                int causal, int64_t i, double* s) {
+                const Visibility& vis, int64_t i, double* s) {
   for (int64_t j = 0; j < N; ++j) {
-    if (causal && j > i) {
+    if (!vis.sees(i, j)) {
       s[j] = kNegInf;
       continue;
     }
@@ -125,14 +163,16 @@ void oracle_set_num_threads(int n) {
 
 // The row-stochastic matrix P = softmax(S) of one head, N x N, into P.
 int oracle_attention_probs(const double* Q, const double* K, int64_t N, int64_t d,
-                           double scale, int causal, double* P) {
+                           double scale, int causal, int64_t left, int64_t right,
+                           const uint8_t* blocks, double* P) {
   if (bad_shape(1, 1, N, d) || !Q || !K || !P) return 1;
+  const Visibility vis = make_vis(N, causal, left, right, blocks);
 #pragma omp parallel
   {
     std::vector<double> s(N);
 #pragma omp for schedule(static)
     for (int64_t i = 0; i < N; ++i) {
-      logits_row(Q + i * d, K, N, d, scale, causal, i, s.data());
+      logits_row(Q + i * d, K, N, d, scale, vis, i, s.data());
       safe_softmax_row(s.data(), N, P + i * N);
     }
   }
@@ -143,8 +183,10 @@ int oracle_attention_probs(const double* Q, const double* K, int64_t N, int64_t 
 // head at a time.
 int oracle_attention_forward(const double* Q, const double* K, const double* V, int64_t B,
                              int64_t H, int64_t N, int64_t d, double scale, int causal,
-                             double* O, double* L) {
+                             int64_t left, int64_t right, const uint8_t* blocks, double* O,
+                             double* L) {
   if (bad_shape(B, H, N, d) || !Q || !K || !V || !O || !L) return 1;
+  const Visibility vis = make_vis(N, causal, left, right, blocks);
   if (N == 0) return 0;
   std::vector<double> P;
   try {
@@ -162,7 +204,7 @@ int oracle_attention_forward(const double* Q, const double* K, const double* V, 
 #pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < N; ++i) {
       double* row = P.data() + i * N;
-      logits_row(q + i * d, k, N, d, scale, causal, i, row);
+      logits_row(q + i * d, k, N, d, scale, vis, i, row);
       std::vector<double> s(row, row + N);
       l[i] = safe_softmax_row(s.data(), N, row);
     }
@@ -188,9 +230,11 @@ int oracle_attention_forward(const double* Q, const double* K, const double* V, 
 // way of forming D; the two must agree.
 int oracle_attention_backward(const double* Q, const double* K, const double* V,
                               const double* dO, int64_t B, int64_t H, int64_t N, int64_t d,
-                              double scale, int causal, double* dQ, double* dK, double* dV,
+                              double scale, int causal, int64_t left, int64_t right,
+                              const uint8_t* blocks, double* dQ, double* dK, double* dV,
                               double* D, double* Dcheck) {
   if (bad_shape(B, H, N, d) || !Q || !K || !V || !dO || !dQ || !dK || !dV || !D) return 1;
+  const Visibility vis = make_vis(N, causal, left, right, blocks);
   if (N == 0) return 0;
   std::vector<double> P, dS;
   try {
@@ -214,7 +258,7 @@ int oracle_attention_backward(const double* Q, const double* K, const double* V,
       std::vector<double> s(N);
 #pragma omp for schedule(static)
       for (int64_t i = 0; i < N; ++i) {
-        logits_row(q + i * d, k, N, d, scale, causal, i, s.data());
+        logits_row(q + i * d, k, N, d, scale, vis, i, s.data());
         safe_softmax_row(s.data(), N, P.data() + i * N);
       }
     }
@@ -287,10 +331,12 @@ int oracle_attention_backward(const double* Q, const double* K, const double* V,
 // definition as oracle_attention_forward, one materialised row of S and P each.
 int oracle_attention_forward_rows(const double* Q, const double* K, const double* V,
                                   int64_t B, int64_t H, int64_t N, int64_t d, double scale,
-                                  int causal, int64_t R, const int64_t* heads,
+                                  int causal, int64_t left, int64_t right,
+                                  const uint8_t* blocks, int64_t R, const int64_t* heads,
                                   const int64_t* rows, double* O_r, double* L_r) {
   if (bad_shape(B, H, N, d) || R < 0 || (R > 0 && (!heads || !rows || !O_r || !L_r)))
     return 1;
+  const Visibility vis = make_vis(N, causal, left, right, blocks);
   for (int64_t r = 0; r < R; ++r)
     if (heads[r] < 0 || heads[r] >= B * H || rows[r] < 0 || rows[r] >= N) return 1;
 #pragma omp parallel
@@ -301,7 +347,7 @@ int oracle_attention_forward_rows(const double* Q, const double* K, const double
       const int64_t bh = heads[r], i = rows[r];
       const double* k = K + bh * N * d;
       const double* v = V + bh * N * d;
-      logits_row(Q + (bh * N + i) * d, k, N, d, scale, causal, i, s.data());
+      logits_row(Q + (bh * N + i) * d, k, N, d, scale, vis, i, s.data());
       L_r[r] = safe_softmax_row(s.data(), N, p.data());
       double* o = O_r + r * d;
       for (int64_t c = 0; c < d; ++c) o[c] = 0.0;
@@ -317,11 +363,13 @@ int oracle_attention_forward_rows(const double* Q, const double* K, const double
 // D_i = sum_j P_ij dP_ij, dQ_i = scale * sum_j P_ij (dP_ij - D_i) K_j.
 int oracle_attention_backward_dq_rows(const double* Q, const double* K, const double* V,
                                       const double* dO, int64_t B, int64_t H, int64_t N,
-                                      int64_t d, double scale, int causal, int64_t R,
+                                      int64_t d, double scale, int causal, int64_t left,
+                                      int64_t right, const uint8_t* blocks, int64_t R,
                                       const int64_t* heads, const int64_t* rows,
                                       double* dQ_r, double* D_r) {
   if (bad_shape(B, H, N, d) || R < 0 || (R > 0 && (!heads || !rows || !dQ_r || !D_r)))
     return 1;
+  const Visibility vis = make_vis(N, causal, left, right, blocks);
   for (int64_t r = 0; r < R; ++r)
     if (heads[r] < 0 || heads[r] >= B * H || rows[r] < 0 || rows[r] >= N) return 1;
 #pragma omp parallel
@@ -333,7 +381,7 @@ int oracle_attention_backward_dq_rows(const double* Q, const double* K, const do
       const double* k = K + bh * N * d;
       const double* v = V + bh * N * d;
       const double* goi = dO + (bh * N + i) * d;
-      logits_row(Q + (bh * N + i) * d, k, N, d, scale, causal, i, s.data());
+      logits_row(Q + (bh * N + i) * d, k, N, d, scale, vis, i, s.data());
       safe_softmax_row(s.data(), N, p.data());
       double Di = 0.0;
       for (int64_t j = 0; j < N; ++j) {
@@ -363,12 +411,14 @@ int oracle_attention_backward_dq_rows(const double* Q, const double* K, const do
 //   dV_j = sum_i P_ij dO_i,  dK_j = scale * sum_i dS_ij Q_i.
 int oracle_attention_backward_dkdv_rows(const double* Q, const double* K, const double* V,
                                         const double* dO, int64_t B, int64_t H, int64_t N,
-                                        int64_t d, double scale, int causal, int64_t bh,
+                                        int64_t d, double scale, int causal, int64_t left,
+                                        int64_t right, const uint8_t* blocks, int64_t bh,
                                         const double* L, const double* D, int64_t R,
                                         const int64_t* keys, double* dK_r, double* dV_r) {
   if (bad_shape(B, H, N, d) || bh < 0 || bh >= B * H || R < 0 || !L || !D ||
       (R > 0 && (!keys || !dK_r || !dV_r)))
     return 1;
+  const Visibility vis = make_vis(N, causal, left, right, blocks);
   for (int64_t r = 0; r < R; ++r)
     if (keys[r] < 0 || keys[r] >= N) return 1;
   const double* q = Q + bh * N * d;
@@ -387,7 +437,7 @@ int oracle_attention_backward_dkdv_rows(const double* Q, const double* K, const 
       gv[c] = 0.0;
     }
     for (int64_t i = 0; i < N; ++i) {
-      if (causal && j > i) continue;
+      if (!vis.sees(i, j)) continue;
       const double* qi = q + i * d;
       const double* goi = go + i * d;
       double sij = 0.0, dpij = 0.0;

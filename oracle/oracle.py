@@ -20,7 +20,15 @@ Definitions followed (titles of the sources, see the header of attn_oracle.cpp):
     large-model training 3x faster", section 2.1;
   * causal masking (key j visible to query i iff j <= i): "Flash Attention-2:
     acceleration principle and GPU memory optimisation in deployment", causal
-    mask item.
+    mask item;
+  * sliding window (i - left <= j <= i + right) from the sliding-window example
+    of the same item, and a block mask over 128 x 128 blocks (block-sparse
+    FlashAttention, "FlashAttention optimisation: breaking the performance
+    bottleneck of standard attention", section 7). Every entry point takes
+    ``window=(left, right)`` (negative = unbounded side; None = no window) and
+    ``block_mask`` (uint8 [ceil(N/128), ceil(N/128)], shared by all heads; None =
+    every block); they combine with ``causal`` by AND. A row that sees no key has
+    O = 0, L = -inf and zero gradients.
 """
 from __future__ import annotations
 
@@ -38,7 +46,25 @@ _lock = threading.Lock()
 
 _D = ctypes.POINTER(ctypes.c_double)
 _I = ctypes.POINTER(ctypes.c_int64)
+_U8 = ctypes.POINTER(ctypes.c_uint8)
 _i64 = ctypes.c_int64
+_c = ctypes.c_int
+_MASK = [_c, _i64, _i64, _U8]  # causal, window left, window right, block mask
+
+BLOCK = 128  # block-mask granularity
+
+
+def _mask(N: int, causal: bool, window, block_mask):
+    """(ctypes argument list, array to keep alive) for the masks of one call."""
+    left, right = (-1, -1) if window is None else (int(window[0]), int(window[1]))
+    blocks = None
+    if block_mask is not None:
+        nb = (N + BLOCK - 1) // BLOCK
+        blocks = np.ascontiguousarray(np.asarray(block_mask) != 0, dtype=np.uint8)
+        if blocks.shape != (nb, nb):
+            raise ValueError(f"block_mask must be [{nb}, {nb}] for N={N}")
+    ptr = blocks.ctypes.data_as(_U8) if blocks is not None else None
+    return [int(bool(causal)), left, right, ptr], blocks
 
 
 def _compile(src: str, out: str) -> None:
@@ -93,21 +119,19 @@ class Oracle:
         lib = ctypes.CDLL(lib_path)
         lib.oracle_num_threads.restype = ctypes.c_int
         lib.oracle_set_num_threads.argtypes = [ctypes.c_int]
-        lib.oracle_attention_probs.argtypes = [_D, _D, _i64, _i64, ctypes.c_double, ctypes.c_int, _D]
-        lib.oracle_attention_forward.argtypes = [
-            _D, _D, _D, _i64, _i64, _i64, _i64, ctypes.c_double, ctypes.c_int, _D, _D]
-        lib.oracle_attention_backward.argtypes = [
-            _D, _D, _D, _D, _i64, _i64, _i64, _i64, ctypes.c_double, ctypes.c_int,
-            _D, _D, _D, _D, _D]
-        lib.oracle_attention_forward_rows.argtypes = [
-            _D, _D, _D, _i64, _i64, _i64, _i64, ctypes.c_double, ctypes.c_int,
-            _i64, _I, _I, _D, _D]
-        lib.oracle_attention_backward_dq_rows.argtypes = [
-            _D, _D, _D, _D, _i64, _i64, _i64, _i64, ctypes.c_double, ctypes.c_int,
-            _i64, _I, _I, _D, _D]
-        lib.oracle_attention_backward_dkdv_rows.argtypes = [
-            _D, _D, _D, _D, _i64, _i64, _i64, _i64, ctypes.c_double, ctypes.c_int,
-            _i64, _D, _D, _i64, _I, _D, _D]
+        f = ctypes.c_double
+        lib.oracle_attention_probs.argtypes = [_D, _D, _i64, _i64, f] + _MASK + [_D]
+        lib.oracle_attention_forward.argtypes = (
+            [_D, _D, _D, _i64, _i64, _i64, _i64, f] + _MASK + [_D, _D])
+        lib.oracle_attention_backward.argtypes = (
+            [_D, _D, _D, _D, _i64, _i64, _i64, _i64, f] + _MASK + [_D, _D, _D, _D, _D])
+        lib.oracle_attention_forward_rows.argtypes = (
+            [_D, _D, _D, _i64, _i64, _i64, _i64, f] + _MASK + [_i64, _I, _I, _D, _D])
+        lib.oracle_attention_backward_dq_rows.argtypes = (
+            [_D, _D, _D, _D, _i64, _i64, _i64, _i64, f] + _MASK + [_i64, _I, _I, _D, _D])
+        lib.oracle_attention_backward_dkdv_rows.argtypes = (
+            [_D, _D, _D, _D, _i64, _i64, _i64, _i64, f] + _MASK
+            + [_i64, _D, _D, _i64, _I, _D, _D])
         for name in ("oracle_attention_probs", "oracle_attention_forward",
                      "oracle_attention_backward", "oracle_attention_forward_rows",
                      "oracle_attention_backward_dq_rows",
@@ -133,38 +157,44 @@ class Oracle:
     def set_num_threads(self, n: int) -> None:
         self._lib.oracle_set_num_threads(int(n))
 
-    def probs(self, q, k, scale: float, causal: bool) -> np.ndarray:
+    def probs(self, q, k, scale: float, causal: bool, window=None,
+              block_mask=None) -> np.ndarray:
         """P = softmax(scale * q k^T) (masked) of one head; q, k are [N, d]."""
         q, k = _f64(q), _f64(k)
         N, d = q.shape
         P = np.empty((N, N), dtype=np.float64)
-        _check(self._lib.oracle_attention_probs(_p(q), _p(k), N, d, float(scale), int(causal),
-                                                _p(P)), "probs")
+        m, keep = _mask(N, causal, window, block_mask)
+        _check(self._lib.oracle_attention_probs(_p(q), _p(k), N, d, float(scale), *m, _p(P)),
+               "probs")
         return P
 
-    def forward(self, Q, K, V, scale: float, causal: bool):
+    def forward(self, Q, K, V, scale: float, causal: bool, window=None, block_mask=None):
         """(O, L): O [B,H,N,d] fp64, L [B,H,N] fp64 natural-log log-sum-exp."""
         Q, K, V = _f64(Q), _f64(K), _f64(V)
         B, H, N, d = _shape4(Q)
         O = np.empty_like(Q)
         L = np.empty((B, H, N), dtype=np.float64)
+        m, keep = _mask(N, causal, window, block_mask)
         _check(self._lib.oracle_attention_forward(_p(Q), _p(K), _p(V), B, H, N, d, float(scale),
-                                                  int(causal), _p(O), _p(L)), "forward")
+                                                  *m, _p(O), _p(L)), "forward")
         return O, L
 
-    def backward(self, Q, K, V, dO, scale: float, causal: bool, with_check: bool = False):
+    def backward(self, Q, K, V, dO, scale: float, causal: bool, with_check: bool = False,
+                 window=None, block_mask=None):
         """(dQ, dK, dV, D[, Dcheck]) for the loss <dO, O>."""
         Q, K, V, dO = _f64(Q), _f64(K), _f64(V), _f64(dO)
         B, H, N, d = _shape4(Q)
         dQ, dK, dV = np.empty_like(Q), np.empty_like(Q), np.empty_like(Q)
         D = np.empty((B, H, N), dtype=np.float64)
         Dc = np.empty((B, H, N), dtype=np.float64) if with_check else None
+        m, keep = _mask(N, causal, window, block_mask)
         _check(self._lib.oracle_attention_backward(
-            _p(Q), _p(K), _p(V), _p(dO), B, H, N, d, float(scale), int(causal),
+            _p(Q), _p(K), _p(V), _p(dO), B, H, N, d, float(scale), *m,
             _p(dQ), _p(dK), _p(dV), _p(D), _p(Dc) if with_check else None), "backward")
         return (dQ, dK, dV, D, Dc) if with_check else (dQ, dK, dV, D)
 
-    def forward_rows(self, Q, K, V, scale: float, causal: bool, heads, rows):
+    def forward_rows(self, Q, K, V, scale: float, causal: bool, heads, rows, window=None,
+                     block_mask=None):
         """O and L of selected (head, row) pairs, head = b * H + h: ([R, d], [R])."""
         Q, K, V = _f64(Q), _f64(K), _f64(V)
         B, H, N, d = _shape4(Q)
@@ -173,12 +203,14 @@ class Oracle:
         R = heads.shape[0]
         O = np.empty((R, d), dtype=np.float64)
         L = np.empty((R,), dtype=np.float64)
+        m, keep = _mask(N, causal, window, block_mask)
         _check(self._lib.oracle_attention_forward_rows(
-            _p(Q), _p(K), _p(V), B, H, N, d, float(scale), int(causal), R, _pi(heads),
+            _p(Q), _p(K), _p(V), B, H, N, d, float(scale), *m, R, _pi(heads),
             _pi(rows), _p(O), _p(L)), "forward_rows")
         return O, L
 
-    def backward_dq_rows(self, Q, K, V, dO, scale: float, causal: bool, heads, rows):
+    def backward_dq_rows(self, Q, K, V, dO, scale: float, causal: bool, heads, rows,
+                         window=None, block_mask=None):
         """dQ and D of selected (head, row) pairs: ([R, d], [R])."""
         Q, K, V, dO = _f64(Q), _f64(K), _f64(V), _f64(dO)
         B, H, N, d = _shape4(Q)
@@ -187,13 +219,14 @@ class Oracle:
         R = heads.shape[0]
         dQ = np.empty((R, d), dtype=np.float64)
         D = np.empty((R,), dtype=np.float64)
+        m, keep = _mask(N, causal, window, block_mask)
         _check(self._lib.oracle_attention_backward_dq_rows(
-            _p(Q), _p(K), _p(V), _p(dO), B, H, N, d, float(scale), int(causal), R, _pi(heads),
+            _p(Q), _p(K), _p(V), _p(dO), B, H, N, d, float(scale), *m, R, _pi(heads),
             _pi(rows), _p(dQ), _p(D)), "backward_dq_rows")
         return dQ, D
 
     def backward_dkdv_rows(self, Q, K, V, dO, scale: float, causal: bool, head: int, L_head,
-                           D_head, keys):
+                           D_head, keys, window=None, block_mask=None):
         """dK and dV of selected key rows of one head, given that head's L and D as
         computed by this oracle (forward_rows / backward_dq_rows over all rows)."""
         Q, K, V, dO = _f64(Q), _f64(K), _f64(V), _f64(dO)
@@ -205,8 +238,9 @@ class Oracle:
         R = keys.shape[0]
         dK = np.empty((R, d), dtype=np.float64)
         dV = np.empty((R, d), dtype=np.float64)
+        m, keep = _mask(N, causal, window, block_mask)
         _check(self._lib.oracle_attention_backward_dkdv_rows(
-            _p(Q), _p(K), _p(V), _p(dO), B, H, N, d, float(scale), int(causal), int(head),
+            _p(Q), _p(K), _p(V), _p(dO), B, H, N, d, float(scale), *m, int(head),
             _p(L_head), _p(D_head), R, _pi(keys), _p(dK), _p(dV)), "backward_dkdv_rows")
         return dK, dV
 

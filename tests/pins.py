@@ -286,6 +286,141 @@ def pin_gradient_invariants(orc):
         _close(D, np.sum(dO * O, axis=-1), 1e-12 * max(1.0, np.abs(D).max()), "D = rowsum(dO o O)")
 
 
+# --------------------------------------------------------------------------- masks
+#
+# Sliding window (keep i - left <= j <= i + right; "Flash Attention-2: acceleration
+# principle and GPU memory optimisation in deployment", sliding-window example of
+# its causal-mask item) and a block mask over 128 x 128 blocks (block-sparse
+# FlashAttention, "FlashAttention optimisation: breaking the performance bottleneck
+# of standard attention", section 7), both ANDed with the causal mask.
+
+
+def library_mask(N, causal, window, blocks):
+    """The kept (i, j) pairs built with library routines: a band from torch's
+    triu/tril, the block pattern from numpy's Kronecker product."""
+    keep = torch.ones(N, N, dtype=torch.bool)
+    if causal:
+        keep = keep.tril(0)
+    if window is not None:
+        left, right = window
+        if left >= 0:
+            keep = keep.triu(-left)
+        if right >= 0:
+            keep = keep.tril(right)
+    if blocks is not None:
+        full = np.kron(np.asarray(blocks, dtype=np.uint8), np.ones((128, 128), np.uint8))
+        keep = keep & torch.from_numpy(full[:N, :N] != 0)
+    return keep
+
+
+MASK_CASES = [
+    # (N, causal, window, block pattern or None)
+    (40, False, (3, 5), None),
+    (40, True, (7, -1), None),
+    (40, False, (0, 0), None),           # the diagonal only
+    (40, False, (-1, 2), None),          # unbounded on the left
+    (300, False, None, [[1, 0, 1], [0, 1, 0], [1, 1, 0]]),
+    (300, True, (150, -1), [[1, 0, 0], [1, 0, 0], [0, 1, 1]]),
+    (260, False, (20, 20), [[0, 1, 1], [1, 0, 1], [0, 0, 0]]),  # empty rows (last block)
+]
+
+
+def pin_masks_match_library(orc):
+    """Windowed and block-masked attention equals fp64 torch SDPA given the library-
+    built boolean mask (forward, logsumexp, autograd gradients) to 1e-12; rows that
+    see no key have O = 0, L = -inf and zero dQ, and P vanishes exactly where the
+    mask hides a key."""
+    rng = _rng(21)
+    for N, causal, window, blocks in MASK_CASES:
+        B, H, d = 1, 2, 8
+        Q, K, V, dO = (rng.standard_normal((B, H, N, d)) for _ in range(4))
+        scale = 0.4
+        keep = library_mask(N, causal, window, blocks)
+        what = f"N={N} causal={causal} window={window} blocks={blocks}"
+        P = orc.probs(Q[0, 0], K[0, 0], scale, causal, window, blocks)
+        assert np.array_equal(P > 0, keep.numpy()), f"{what}: support of P"
+        O, L = orc.forward(Q, K, V, scale, causal, window, blocks)
+        dQ, dK, dV, _ = orc.backward(Q, K, V, dO, scale, causal, window=window,
+                                     block_mask=blocks)
+        live = keep.any(dim=1).numpy()
+        qt, kt, vt = (torch.tensor(x, requires_grad=True) for x in (Q, K, V))
+        ot = torch.nn.functional.scaled_dot_product_attention(qt, kt, vt, attn_mask=keep,
+                                                              scale=scale)
+        # rows with no visible key are NaN in the library; they are not part of the loss
+        ot_live = ot[:, :, torch.from_numpy(live)]
+        ot_live.backward(torch.tensor(dO[:, :, live]))
+        _close(O[:, :, live], ot_live.detach().numpy(), 1e-12, f"{what}: O")
+        s = torch.einsum("bhid,bhjd->bhij", torch.tensor(Q), torch.tensor(K)) * scale
+        lse = torch.logsumexp(s.masked_fill(~keep, -math.inf), dim=-1).numpy()
+        _close(L[:, :, live], lse[:, :, live], 1e-12, f"{what}: L")
+        _close(dQ[:, :, live], qt.grad.numpy()[:, :, live], 1e-12, f"{what}: dQ")
+        _close(dK, kt.grad.numpy(), 1e-12, f"{what}: dK")
+        _close(dV, vt.grad.numpy(), 1e-12, f"{what}: dV")
+        if not live.all():
+            dead = ~live
+            assert np.all(O[:, :, dead] == 0.0), f"{what}: O of empty rows"
+            assert np.all(L[:, :, dead] == -np.inf), f"{what}: L of empty rows"
+            assert np.all(dQ[:, :, dead] == 0.0), f"{what}: dQ of empty rows"
+
+
+def pin_window_closed_forms(orc):
+    """With every key equal, P is uniform over the visible keys, so O_i is the mean
+    of V over the window max(0, i-left) .. min(N-1, i+right) (causal: .. i) and
+    L_i = s + ln(count); the count of visible keys is the window's length."""
+    rng = _rng(22)
+    N, d = 50, 4
+    for causal, (left, right) in ((False, (4, 9)), (True, (6, -1)), (False, (0, 0)),
+                                  (True, (-1, 3)), (False, (60, 1))):
+        q = rng.standard_normal((N, d))
+        k = np.tile(rng.standard_normal((1, d)), (N, 1))
+        v = rng.standard_normal((N, d))
+        O, L = orc.forward(q[None, None], k[None, None], v[None, None], 0.5, causal,
+                           (left, right))
+        for i in range(N):
+            lo = 0 if left < 0 else max(0, i - left)
+            hi = N - 1 if right < 0 else min(N - 1, i + right)
+            if causal:
+                hi = min(hi, i)
+            s = 0.5 * float(q[i] @ k[0])
+            what = f"row {i} causal={causal} window=({left},{right})"
+            _close(O[0, 0, i], v[lo:hi + 1].mean(axis=0), 1e-13, what + ": O")
+            _close(L[0, 0, i], s + math.log(hi - lo + 1), 1e-12, what + ": L")
+
+
+def pin_masked_finite_differences(orc):
+    """Central differences of <dO, O> through windowed and block-masked attention
+    (a sample of elements at N = 140, all of them at N = 12): error <= 1e-6 of
+    max|grad|."""
+    rng = _rng(23)
+    cases = [(12, 3, False, (2, 1), None, None),
+             (12, 3, True, (4, -1), None, None),
+             (140, 2, False, (30, 5), [[1, 1], [0, 1]], 24)]
+    for N, d, causal, window, blocks, n_sample in cases:
+        Q, K, V, dO = (rng.standard_normal((1, 1, N, d)) for _ in range(4))
+        scale = 0.7
+        grads = orc.backward(Q, K, V, dO, scale, causal, window=window, block_mask=blocks)[:3]
+
+        def loss(q, k, v):
+            O, _ = orc.forward(q, k, v, scale, causal, window, blocks)
+            return float(np.sum(O * dO))
+
+        h = 1e-6
+        for which, grad in enumerate(grads):
+            idxs = list(np.ndindex(*grad.shape))
+            if n_sample is not None:
+                idxs = [idxs[t] for t in rng.choice(len(idxs), n_sample, replace=False)]
+            ref = max(1e-3, float(np.max(np.abs(grad))))
+            for idx in idxs:
+                args_p = [Q.copy(), K.copy(), V.copy()]
+                args_m = [Q.copy(), K.copy(), V.copy()]
+                args_p[which][idx] += h
+                args_m[which][idx] -= h
+                num = (loss(*args_p) - loss(*args_m)) / (2 * h)
+                assert abs(num - grad[idx]) <= 1e-6 * ref, (
+                    f"masked finite differences of {'QKV'[which]}{idx} (N={N}, "
+                    f"window={window}, blocks={blocks}): {num:.6e} vs {grad[idx]:.6e}")
+
+
 # --------------------------------------------------------------------------- golden
 
 
@@ -323,4 +458,7 @@ ALL_PINS = [
     pin_finite_differences,
     pin_gradient_invariants,
     pin_golden_fixtures,
+    pin_masks_match_library,
+    pin_window_closed_forms,
+    pin_masked_finite_differences,
 ]

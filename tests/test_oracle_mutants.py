@@ -12,8 +12,18 @@ import pins
 # (name, original text, replacement); each original occurs in attn_oracle.cpp.
 MUTATIONS = [
     ("logits_without_scale", "s[j] = scale * acc;", "s[j] = acc;"),
-    ("causal_drops_diagonal", "if (causal && j > i) {", "if (causal && j >= i) {"),
-    ("causal_ignored", "if (causal && j > i) {", "if (false) {"),
+    ("causal_drops_diagonal", "if (causal && j > i) return false;",
+     "if (causal && j >= i) return false;"),
+    ("causal_ignored", "if (causal && j > i) return false;", ""),
+    ("window_left_off_by_one", "if (left >= 0 && j < i - left) return false;",
+     "if (left >= 0 && j <= i - left) return false;"),
+    ("window_right_ignored", "if (right >= 0 && j > i + right) return false;", ""),
+    ("window_sides_swapped", "if (left >= 0 && j < i - left) return false;",
+     "if (left >= 0 && j < i - right) return false;"),
+    ("block_mask_transposed", "blocks[(i / kBlock) * nb + j / kBlock]",
+     "blocks[(j / kBlock) * nb + i / kBlock]"),
+    ("block_mask_ignored", "if (blocks && !blocks[(i / kBlock) * nb + j / kBlock]) return false;",
+     ""),
     ("no_max_subtraction", "p[j] = std::exp(s[j] - m);", "p[j] = std::exp(s[j]);"),
     ("no_normalisation", "for (int64_t j = 0; j < N; ++j) p[j] /= sum;", ""),
     ("lse_without_log", "return m + std::log(sum);", "return m + sum;"),

@@ -41,6 +41,36 @@ def test_row_functions_match_full_functions(orc):
         np.testing.assert_allclose(dVr, dV.reshape(B * H, N, d)[head, keys], atol=1e-13)
 
 
+def test_row_functions_match_full_functions_with_masks(orc):
+    """The same agreement under a sliding window and a block mask (one block row
+    empty, so some rows see no key)."""
+    rng = np.random.default_rng(22)
+    B, H, N, d = 1, 2, 260, 4
+    Q, K, V, dO = (rng.standard_normal((B, H, N, d)) for _ in range(4))
+    blocks = [[1, 0, 1], [1, 1, 0], [0, 0, 0]]
+    for causal, window in ((False, (40, 7)), (True, (90, -1))):
+        kw = dict(window=window, block_mask=blocks)
+        O, L = orc.forward(Q, K, V, 0.4, causal, **kw)
+        dQ, dK, dV, D = orc.backward(Q, K, V, dO, 0.4, causal, **kw)
+        heads = rng.integers(0, B * H, 30)
+        rows = rng.integers(0, N, 30)
+        Or, Lr = orc.forward_rows(Q, K, V, 0.4, causal, heads, rows, **kw)
+        np.testing.assert_allclose(Or, O.reshape(B * H, N, d)[heads, rows], atol=1e-13)
+        np.testing.assert_array_equal(np.isinf(Lr), np.isinf(L.reshape(B * H, N)[heads, rows]))
+        fin = np.isfinite(Lr)
+        np.testing.assert_allclose(Lr[fin], L.reshape(B * H, N)[heads, rows][fin], atol=1e-13)
+        dQr, Dr = orc.backward_dq_rows(Q, K, V, dO, 0.4, causal, heads, rows, **kw)
+        np.testing.assert_allclose(dQr, dQ.reshape(B * H, N, d)[heads, rows], atol=1e-13)
+        np.testing.assert_allclose(Dr, D.reshape(B * H, N)[heads, rows], atol=1e-13)
+        head = 1
+        keys = np.array([0, 5, 130, 255, 259, 200])
+        dKr, dVr = orc.backward_dkdv_rows(Q, K, V, dO, 0.4, causal, head,
+                                          L.reshape(B * H, N)[head], D.reshape(B * H, N)[head],
+                                          keys, **kw)
+        np.testing.assert_allclose(dKr, dK.reshape(B * H, N, d)[head, keys], atol=1e-13)
+        np.testing.assert_allclose(dVr, dV.reshape(B * H, N, d)[head, keys], atol=1e-13)
+
+
 def test_bad_arguments_rejected(orc):
     with pytest.raises(RuntimeError):
         orc.forward_rows(np.zeros((1, 1, 4, 2)), np.zeros((1, 1, 4, 2)), np.zeros((1, 1, 4, 2)),
