@@ -42,6 +42,7 @@
 #define FA_B200_FA_H
 
 #include <stddef.h>
+#include <stdint.h>
 
 #ifdef __cplusplus
 extern "C" {
@@ -159,6 +160,37 @@ fa_status fa_backward_f16(const void* Q, const void* K, const void* V, const voi
                           const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
                           int B, int H, int N, int d, float scale, int causal,
                           void* workspace, size_t workspace_bytes, fa_stream_t stream);
+
+/*
+ * Masked attention (bf16): fa_forward and fa_backward with two more masks that
+ * combine with `causal` by AND -- query i sees key j only if every mask keeps it.
+ *   window_left, window_right: a sliding window, key j kept iff
+ *       i - window_left <= j <= i + window_right; a negative value leaves that side
+ *       unbounded (-1, -1 = no window; window_right = 0 is the causal mask). From
+ *       the sliding-window example of "Flash Attention-2: acceleration principle
+ *       and GPU memory optimisation in deployment" (causal-mask item: a window-size
+ *       pair given together with is_causal).
+ *   block_mask: NULL, or DEVICE memory holding a row-major T x T byte matrix,
+ *       T = ceil(N / 128), the same for every batch and head; (i, j) is kept iff
+ *       block_mask[(i / 128) * T + j / 128] != 0. Block-sparse attention,
+ *       "FlashAttention optimisation ...", section 7, at the tile size 128 of the
+ *       "Flash Attention-2 ..." page's block strategy. Tiles the mask drops are
+ *       never loaded or computed. T <= 4096 (N <= 524288), else
+ *       FA_ERR_UNSUPPORTED. Read only; any alignment.
+ * A query row that sees no key gets O = 0 and LSE = -inf, and dQ = 0; a key that
+ * no query sees gets dK = dV = 0. The backward must be given the same masks as
+ * the forward that produced O and LSE. Other arguments as for fa_forward /
+ * fa_backward.
+ */
+fa_status fa_forward_masked(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                            int B, int H, int N, int d, float scale, int causal,
+                            int window_left, int window_right, const uint8_t* block_mask,
+                            fa_stream_t stream);
+fa_status fa_backward_masked(const void* Q, const void* K, const void* V, const void* O,
+                             const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
+                             int B, int H, int N, int d, float scale, int causal,
+                             int window_left, int window_right, const uint8_t* block_mask,
+                             void* workspace, size_t workspace_bytes, fa_stream_t stream);
 
 /*
  * fp32 entry points: the same operation and arguments with fp32 tensors

@@ -24,7 +24,8 @@ from ._lib import FAError, check, lib
 __all__ = [
     "FAError", "fa_forward", "fa_backward", "fa_backward_workspace_size",
     "fa_backward_preprocess", "fa_backward_main", "fa_backward_dq_convert",
-    "fa_backward_noalloc", "fa_forward_f16", "fa_backward_f16", "fa_forward_f32",
+    "fa_backward_noalloc", "fa_forward_f16", "fa_backward_f16", "fa_forward_masked",
+    "fa_backward_masked", "fa_forward_f32",
     "fa_backward_f32", "fa_get_status", "fa_watchdog_selftest", "fa_version",
     "forward", "backward", "attention", "FlashAttentionFunction",
 ]
@@ -82,6 +83,52 @@ def fa_forward_f16(Q, K, V, O, LSE, scale: float, causal: bool, stream=None) -> 
             _need("LSE", LSE, torch.float32, (B, H, N))]
     check("fa_forward_f16", lib().fa_forward_f16(*args, B, H, N, d, float(scale),
                                                  int(bool(causal)), _stream(stream)))
+
+
+def _block_mask(block_mask, N: int):
+    """Device pointer of a [ceil(N/128)]^2 uint8/bool CUDA tensor, or None."""
+    if block_mask is None:
+        return None
+    T = (N + 127) // 128
+    if not isinstance(block_mask, torch.Tensor) or not block_mask.is_cuda:
+        raise ValueError("block_mask must be a CUDA tensor")
+    if block_mask.dtype not in (torch.uint8, torch.bool):
+        raise TypeError("block_mask must be uint8 or bool")
+    if tuple(block_mask.shape) != (T, T) or not block_mask.is_contiguous():
+        raise ValueError(f"block_mask must be a contiguous [{T}, {T}] tensor")
+    return block_mask.data_ptr()
+
+
+def _window(window):
+    if window is None:
+        return -1, -1
+    left, right = window
+    return int(left), int(right)
+
+
+def fa_forward_masked(Q, K, V, O, LSE, scale: float, causal: bool, window=None,
+                      block_mask=None, stream=None) -> None:
+    """fa_forward with a sliding window (left, right) (negative = unbounded side)
+    and/or a 128 x 128 block mask, both ANDed with causal."""
+    B, H, N, d = _shape(Q)
+    bf = torch.bfloat16
+    args = [_need("Q", Q, bf, (B, H, N, d)), _need("K", K, bf, (B, H, N, d)),
+            _need("V", V, bf, (B, H, N, d)), _need("O", O, bf, (B, H, N, d)),
+            _need("LSE", LSE, torch.float32, (B, H, N))]
+    wl, wr = _window(window)
+    check("fa_forward_masked", lib().fa_forward_masked(
+        *args, B, H, N, d, float(scale), int(bool(causal)), wl, wr, _block_mask(block_mask, N),
+        _stream(stream)))
+
+
+def fa_backward_masked(Q, K, V, O, dO, LSE, dQ, dK, dV, scale: float, causal: bool, workspace,
+                       window=None, block_mask=None, stream=None) -> None:
+    ptrs, (B, H, N, d), ws, nbytes = _bwd_args(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace,
+                                               torch.bfloat16)
+    wl, wr = _window(window)
+    check("fa_backward_masked", lib().fa_backward_masked(
+        *ptrs, B, H, N, d, float(scale), int(bool(causal)), wl, wr, _block_mask(block_mask, N),
+        ws, nbytes, _stream(stream)))
 
 
 def fa_forward_f32(Q, K, V, O, LSE, scale: float, causal: bool, stream=None) -> None:
@@ -200,13 +247,22 @@ def _default_scale(d: int, scale):
     return 1.0 / math.sqrt(d) if scale is None else float(scale)
 
 
-def forward(q, k, v, causal: bool = False, scale=None):
-    """(O, LSE) for bf16, f16 or fp32 q, k, v of shape [B, H, N, d] on the GPU."""
+def _masked(window, block_mask) -> bool:
+    return window is not None or block_mask is not None
+
+
+def forward(q, k, v, causal: bool = False, scale=None, window=None, block_mask=None):
+    """(O, LSE) for bf16, f16 or fp32 q, k, v of shape [B, H, N, d] on the GPU.
+    ``window`` / ``block_mask`` (bf16 only) as for fa_forward_masked."""
     B, H, N, d = _shape(q)
     scale = _default_scale(d, scale)
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    if q.dtype == torch.bfloat16:
+    if _masked(window, block_mask):
+        if q.dtype != torch.bfloat16:
+            raise TypeError("window and block_mask are supported for bf16 inputs")
+        fa_forward_masked(q, k, v, o, lse, scale, causal, window, block_mask)
+    elif q.dtype == torch.bfloat16:
         fa_forward(q, k, v, o, lse, scale, causal)
     elif q.dtype == torch.float16:
         fa_forward_f16(q, k, v, o, lse, scale, causal)
@@ -223,13 +279,19 @@ def workspace_for(q) -> torch.Tensor:
     return torch.empty(n, dtype=torch.uint8, device=q.device)
 
 
-def backward(q, k, v, o, lse, do, causal: bool = False, scale=None, workspace=None):
-    """(dQ, dK, dV) of the loss <dO, O>."""
+def backward(q, k, v, o, lse, do, causal: bool = False, scale=None, workspace=None,
+             window=None, block_mask=None):
+    """(dQ, dK, dV) of the loss <dO, O> (same masks as the forward)."""
     B, H, N, d = _shape(q)
     scale = _default_scale(d, scale)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ws = workspace_for(q) if workspace is None else workspace
-    if q.dtype == torch.bfloat16:
+    if _masked(window, block_mask):
+        if q.dtype != torch.bfloat16:
+            raise TypeError("window and block_mask are supported for bf16 inputs")
+        fa_backward_masked(q, k, v, o, do, lse, dq, dk, dv, scale, causal, ws, window,
+                           block_mask)
+    elif q.dtype == torch.bfloat16:
         fa_backward(q, k, v, o, do, lse, dq, dk, dv, scale, causal, ws)
     elif q.dtype == torch.float16:
         fa_backward_f16(q, k, v, o, do, lse, dq, dk, dv, scale, causal, ws)
@@ -244,19 +306,20 @@ class FlashAttentionFunction(torch.autograd.Function):
     """Differentiable exact attention through the library's forward and backward."""
 
     @staticmethod
-    def forward(ctx, q, k, v, causal: bool = False, scale=None):
+    def forward(ctx, q, k, v, causal: bool = False, scale=None, window=None, block_mask=None):
         q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
-        o, lse = forward(q, k, v, causal, scale)
+        o, lse = forward(q, k, v, causal, scale, window, block_mask)
         ctx.save_for_backward(q, k, v, o, lse)
-        ctx.causal, ctx.scale = causal, scale
+        ctx.causal, ctx.scale, ctx.window, ctx.block_mask = causal, scale, window, block_mask
         return o
 
     @staticmethod
     def backward(ctx, do):
         q, k, v, o, lse = ctx.saved_tensors
-        dq, dk, dv = backward(q, k, v, o, lse, do.contiguous(), ctx.causal, ctx.scale)
-        return dq, dk, dv, None, None
+        dq, dk, dv = backward(q, k, v, o, lse, do.contiguous(), ctx.causal, ctx.scale,
+                              window=ctx.window, block_mask=ctx.block_mask)
+        return dq, dk, dv, None, None, None, None
 
 
-def attention(q, k, v, causal: bool = False, scale=None):
-    return FlashAttentionFunction.apply(q, k, v, causal, scale)
+def attention(q, k, v, causal: bool = False, scale=None, window=None, block_mask=None):
+    return FlashAttentionFunction.apply(q, k, v, causal, scale, window, block_mask)

@@ -11,8 +11,8 @@
 //
 // Three launches:
 //   1. fa_bwd_pre_kernel: D_i and L2_i = LSE_i*log2(e) into [B*H, Npad] (padding
-//      rows get D = 0, L2 = +inf so that they contribute nothing), and zero the
-//      fp32 dQ accumulator.
+//      rows, and rows that see no key (LSE = -inf), get L2 = +inf so that they
+//      contribute nothing), and zero the fp32 dQ accumulator.
 //   2. fa_bwd_kernel (one CTA per SM, 512 threads): the CTA owns one tile of 128
 //      keys K_j, V_j and streams the query tiles Q_i, dO_i (128 rows) through a
 //      ring of shared-memory slots with TMA. Each query tile is processed as two
@@ -37,6 +37,10 @@
 //      half h at +64h; P^T_h and dS^T_h (bf16 pairs) alias the first 32 columns of
 //      their half.
 //   3. fa_bwd_dq_kernel: dQ = bf16(scale * accumulator).
+// Masks (the forward's: sliding window wl/wr with causal as wr = 0, and a 128 x 128
+// block mask): a key tile's CTA walks only the query tiles that can see one of its
+// keys, and elements are masked only on steps that cross a window edge. A key tile
+// that no query sees gets dK = dV = 0.
 // No N x N matrix is written to device memory.
 #pragma once
 
@@ -51,6 +55,7 @@ constexpr int kThreads = 512;
 constexpr int kWarpDq = 8;     // first of the 4 dQ warps
 constexpr int kWarpTma = 12;
 constexpr int kWarpMma = 13;
+constexpr int kMaxMaskTiles = 4096;  // largest block mask: 4096 x 4096 tiles (N <= 524288)
 
 template <int D>
 struct Cfg {
@@ -80,9 +85,11 @@ struct Cfg {
   static constexpr int kBarDrain = kBarDKDV + 1;
   static constexpr int kNumBars = kBarDrain + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
-  static constexpr int kSmemBytes = kMiscOff + 16 + 1024;
+  static constexpr int kMaskOff = kMiscOff + 16;  // block-mask column of this key tile, as bits
+  static constexpr int kSmemBytes = kMaskOff + kMaxMaskTiles / 8 + 1024;
   static constexpr uint32_t kTmDK = 0, kTmDV = D, kTmS = 2 * D, kTmDP = 2 * D + 128;
   static constexpr uint32_t kTmDQ64 = 384;  // D = 64 only
+  static_assert(kSmemBytes <= 232448, "exceeds the 227 KB of shared memory a CTA may use");
   static constexpr uint32_t kTmCols = 512;
 };
 
@@ -97,7 +104,9 @@ struct Params {
   int BH;
   float scale;
   float scale_log2;
-  int causal;
+  int wl;                 // keys j >= i - wl are kept; < 0: no left bound
+  int wr;                 // keys j <= i + wr are kept; < 0: no right bound (causal: 0)
+  const uint8_t* blocks;  // [n_kt x n_kt] block mask (nonzero = kept), or null
   unsigned long long timeout_ns;
 };
 
@@ -211,7 +220,8 @@ __global__ void __launch_bounds__(256)
   for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
   if (lane == 0) {
     Dv[r] = s;
-    L2[r] = LSE[row] * 1.4426950408889634f;
+    const float lse = LSE[row];
+    L2[r] = (lse == -INFINITY) ? INFINITY : lse * 1.4426950408889634f;
   }
   float4* z = reinterpret_cast<float4*>(dQacc + row * D);
 #pragma unroll
@@ -261,8 +271,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int j = static_cast<int>(blockIdx.x) % n_kt;
   const int k0 = j * BN;
   const int n_q = (p.N + BM - 1) / BM;
-  const int i_begin = p.causal ? j : 0;  // BM == BN: query tiles i >= j see key tile j
-  const int nsteps = n_q - i_begin;
+  // query tiles [i_lo, i_hi) hold every query that may see a key of this tile
+  const int k1 = min(k0 + BN, p.N) - 1;
+  const int i_lo = (p.wr < 0) ? 0 : max(0, k0 - p.wr) / BM;
+  const int i_hi = (p.wl < 0) ? n_q : min(n_q, (k1 + p.wl) / BM + 1);
+
+  // The block-mask column of this key tile as bits: warp w builds words w, w + 16, ...
+  uint32_t* mask_bits = reinterpret_cast<uint32_t*>(base_ptr + C::kMaskOff);
+  if (p.blocks != nullptr) {
+    for (int wi = warp; wi < (n_q + 31) / 32; wi += kThreads / 32) {
+      const int i = wi * 32 + lane;
+      const bool keep = i < n_q && p.blocks[static_cast<size_t>(i) * n_kt + j] != 0;
+      const uint32_t bits = __ballot_sync(0xffffffffu, keep);
+      if (lane == 0) mask_bits[wi] = bits;
+    }
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(bar(C::kBarKV), 1);
@@ -291,6 +314,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const Watchdog wd{abort_flag, p.timeout_ns};
 
+  // Does some query of query tile i see a key of this tile?
+  auto member = [&](int i) -> bool {
+    if (i < i_lo || i >= i_hi) return false;
+    return p.blocks == nullptr || ((mask_bits[i >> 5] >> (i & 31)) & 1u);
+  };
+  int nsteps = i_hi - i_lo;  // query tiles walked
+  if (p.blocks != nullptr) {
+    nsteps = 0;
+    for (int i = i_lo; i < i_hi; ++i) nsteps += member(i) ? 1 : 0;
+  }
+
   // ring of half tiles: seq = 4*step + 2*h + w, w = 0 for dO (rows 64h.. of query
   // tile i), w = 1 for Q (with L2 and D of those 64 queries)
   auto seq_of = [](int s, int h, int w) { return 4 * s + 2 * h + w; };
@@ -316,8 +350,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     int issued = 0;
     bool ok = true;
+    int i = i_lo - 1;
     for (int s = 0; s < nsteps && ok; ++s) {
-      const int i = i_begin + s;
+      do ++i; while (!member(i));
       for (int hw = 0; hw < 4 && ok; ++hw) {
         const int h = hw >> 1, w = hw & 1;
         const int seq = seq_of(s, h, w);
@@ -417,9 +452,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     uint8_t* ds_row = base_ptr + C::kDSOff + h * C::kChunkBytes + krow * 128;
     const bool ragged_keys = k0 + BN > p.N;
     const int dq_bar = (D == 128) ? C::kBarDQFull + h : C::kBarDQFull;
+    // queries that see this key row: [q_lo, q_hi) (empty for a padding key)
+    const int q_lo = (p.wr < 0) ? 0 : key - p.wr;
+    const int q_hi = (key >= p.N) ? q_lo : ((p.wl < 0) ? p.Npad + BM : key + p.wl + 1);
+    const unsigned q_span = static_cast<unsigned>(q_hi - q_lo);
     bool ok = true;
+    int i = i_lo - 1;
     for (int s = 0; s < nsteps && ok; ++s) {
-      const int i = i_begin + s;
+      do ++i; while (!member(i));
       const int qh0 = i * BM + 64 * h;  // first query of this half
       ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarS + h), s & 1, wd));
       if (ok && s > 0)  // the dQ MMA of the last step has finished reading this dS chunk
@@ -434,9 +474,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float4* Lv = reinterpret_cast<const float4*>(
           base_ptr + C::kVecOff + slot_of(seqQ) * 2 * C::kVecBytes);
       const float4* Dv4 = Lv + 64 / 4;
-      // masking is needed only on the causal diagonal step and on a ragged key tile
-      const bool mask = (p.causal && i == j) || ragged_keys;
-      const int lim = !(key < p.N) ? 1 << 30 : (p.causal ? key - qh0 : -1);  // q index < lim masked
+      // masking is needed only where the half crosses an edge of some key's visible
+      // queries (the causal diagonal, a window edge) and on a ragged key tile
+      const bool mask = ragged_keys || (p.wr >= 0 && k0 + BN - 1 - p.wr > qh0) ||
+                        (p.wl >= 0 && k0 + p.wl < qh0 + 63);
+      const int qoff = qh0 - q_lo;  // query qh0 + x is visible iff qoff + x < q_span (unsigned)
       uint32_t sv[2][16], dv[2][16];
       tmem_ld16(tm_s, sv[0]);
       tmem_ld16(tm_dp, dv[0]);
@@ -460,7 +502,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int e = 0; e < 4; ++e) {
             const int k = 4 * v + e;
             float pe = ex2_approx(fmaf(__uint_as_float(sv[cur][k]), c, -Ls[e]));
-            if (mask && (cc * 16 + k) < lim) pe = 0.f;
+            if (mask && static_cast<unsigned>(qoff + cc * 16 + k) >= q_span) pe = 0.f;
             pv[e] = pe;
             dsv[e] = pe * (__uint_as_float(dv[cur][k]) - Ds[e]);
           }
@@ -484,7 +526,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(C::kBarP + h));
     }
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarDKDV), 0, wd));
+    if (nsteps == 0 && key < p.N) {
+      // no query sees this key: dK = dV = 0 (warps 0-3 dK, warps 4-7 dV)
+      uint4* dst = reinterpret_cast<uint4*>((h == 0 ? p.dK : p.dV) +
+                                            (static_cast<size_t>(bh) * p.N + key) * D);
+#pragma unroll
+      for (int u = 0; u < D / 8; ++u) dst[u] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    if (ok && nsteps > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarDKDV), 0, wd));
     if (ok && nsteps > 0) {
       // warps 0-3 write dK (times scale), warps 4-7 write dV
       tc_fence_after();
@@ -514,8 +563,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const int row = wq * 32 + lane;  // TMEM lane: head-dim element (D = 128) or query (D = 64)
     bool ok = true;
+    int i = i_lo - 1;
     for (int s = 0; s < nsteps && ok; ++s) {
-      const int q0 = (i_begin + s) * BM;
+      do ++i; while (!member(i));
+      const int q0 = i * BM;
       if constexpr (D == 128) {
         for (int h = 0; h < 2 && ok; ++h) {
           ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarDQFull + h), s & 1, wd));

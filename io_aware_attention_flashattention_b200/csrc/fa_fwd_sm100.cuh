@@ -8,7 +8,13 @@
 // with the online-softmax merge of "A survey of key techniques of large language
 // model pre-training systems" (Journal of Software 2026(1), p.218: m = max(m1,
 // m2), l = e^(m1-m) l1 + e^(m2-m) l2). Causal tiles above the diagonal are skipped
-// ("Flash Attention-2: acceleration principle ...", causal-mask item).
+// ("Flash Attention-2: acceleration principle ...", causal-mask item), and so are
+// tiles outside a sliding window (the same item's sliding-window example) or
+// outside a 128 x 128 block mask (block-sparse FlashAttention, "FlashAttention
+// optimisation ...", section 7). Key j is seen by query i iff
+//   j < N, i - wl <= j (wl >= 0), j <= i + wr (wr >= 0; causal is wr = 0), and the
+//   block mask keeps (i / 128, j / 128);
+// the CTA walks only the key tiles that some of its query rows can see.
 //
 // B200 mapping (one CTA per SM, 352 threads):
 //   * CTA = 2 query tiles of 128 rows (256 rows) of one (batch, head); the two tiles
@@ -44,6 +50,8 @@ constexpr int kWarpTmaK = 8;
 constexpr int kWarpMma = 9;
 constexpr int kWarpTmaV = 10;
 constexpr float kRescaleThreshold = 8.0f;  // log2 domain: rescale when max grows > 2^8
+// Largest number of 128-key tiles a block mask may span (N <= 524288).
+constexpr int kMaxMaskTiles = 4096;
 // When kPolyPeriod > 0, one pair of exponentials in every kPolyPeriod goes to the
 // polynomial exp2 on the FMA pipe (exp2_poly2) instead of MUFU.
 constexpr int kPolyPeriod = 0;
@@ -73,8 +81,11 @@ struct Cfg {
   static constexpr int kBarDrain = kBarPVDone + 2;
   static constexpr int kNumBars = kBarDrain + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem base, abort flag
-  static constexpr int kSmemBytes = kMiscOff + 16 + 1024;  // + 1024 for alignment
+  static constexpr int kMaskOff = kMiscOff + 16;            // block-mask bits of both tiles
+  static constexpr int kMaskWords = kMaxMaskTiles / 32;     // per query tile
+  static constexpr int kSmemBytes = kMaskOff + 2 * kMaskWords * 4 + 1024;  // + alignment
   static constexpr uint32_t kTmS0 = 0, kTmO0 = 256;
+  static_assert(kSmemBytes <= 232448, "exceeds the 227 KB of shared memory a CTA may use");
   static constexpr uint32_t kTmCols = 512;
 };
 
@@ -85,7 +96,10 @@ struct Params {
   int BH;
   int n_qblk;        // ceil(N / 256)
   float scale_log2;  // scale * log2(e)
-  int causal;
+  int wl;            // keys j >= i - wl are kept; < 0: no left bound
+  int wr;            // keys j <= i + wr are kept; < 0: no right bound (causal: 0)
+  const uint8_t* blocks;  // [n_kt x n_kt] block mask (nonzero = kept), or null
+  int n_kt;               // ceil(N / 128)
   unsigned long long timeout_ns;
 };
 
@@ -150,15 +164,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int bh = static_cast<int>(blockIdx.x) / p.n_qblk;
   const int qb = (p.n_qblk - 1) - static_cast<int>(blockIdx.x) % p.n_qblk;
   const int q0 = qb * 2 * BM;
-  const int n_kv_total = (p.N + BN - 1) / BN;
-  int nk[2];
+  const int n_kt = p.n_kt;
+  // key tiles [lo[t], hi[t]) hold every key a row of query tile t may see
+  int lo[2], hi[2];
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
-    const int r0 = q0 + t * BM;
-    nk[t] = (r0 < p.N) ? (p.causal ? min(r0 / BN + 1, n_kv_total) : n_kv_total) : 0;
+    const int r0 = q0 + t * BM, r1 = min(r0 + BM, p.N) - 1;
+    lo[t] = (p.wl < 0) ? 0 : max(0, r0 - p.wl) / BN;
+    hi[t] = (p.wr < 0) ? n_kt : min(n_kt, (r1 + p.wr) / BN + 1);
+    if (r0 >= p.N) lo[t] = hi[t] = 0;
   }
-  // Tile 1 never has fewer key tiles than tile 0 unless it is empty.
-  const int nkv = max(nk[0], nk[1]);
+  // The CTA's key tiles: the union of both ranges (contiguous: lo[1] <= hi[0]).
+  const int kt_lo = (hi[0] > lo[0]) ? lo[0] : lo[1];
+  const int kt_hi = max(hi[0], hi[1]);
+
+  // Block mask rows of the two query tiles as bits in shared memory: warp w builds
+  // words w, w + 11, ... with one byte per lane and a ballot.
+  uint32_t* mask_bits = reinterpret_cast<uint32_t*>(base_ptr + C::kMaskOff);
+  if (p.blocks != nullptr) {
+    const int nwords = (n_kt + 31) / 32;
+    for (int w = warp; w < 2 * nwords; w += kThreads / 32) {
+      const int t = w / nwords, wi = w % nwords;
+      const int qt = min(2 * qb + t, n_kt - 1);
+      const int kt = wi * 32 + lane;
+      const bool keep = kt < n_kt && p.blocks[static_cast<size_t>(qt) * n_kt + kt] != 0;
+      const uint32_t bits = __ballot_sync(0xffffffffu, keep);
+      if (lane == 0) mask_bits[t * C::kMaskWords + wi] = bits;
+    }
+  }
 
   if (threadIdx.x == 0) {
     for (int t = 0; t < 2; ++t) {
@@ -190,6 +223,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = *tmem_slot;
   const Watchdog wd{abort_flag, p.timeout_ns};
 
+  // Does query tile t see any key of key tile kt?
+  auto member = [&](int kt, int t) -> bool {
+    if (kt < lo[t] || kt >= hi[t]) return false;
+    return p.blocks == nullptr || ((mask_bits[t * C::kMaskWords + (kt >> 5)] >> (kt & 31)) & 1u);
+  };
+  // first key tile >= kt that either query tile sees (kt_hi if none)
+  auto next_kt = [&](int kt) -> int {
+    while (kt < kt_hi && !(member(kt, 0) || member(kt, 1))) ++kt;
+    return kt;
+  };
+  int nk[2];  // key tiles each query tile sees
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    if (p.blocks == nullptr) {
+      nk[t] = hi[t] - lo[t];
+    } else {
+      nk[t] = 0;
+      for (int kt = lo[t]; kt < hi[t]; ++kt) nk[t] += member(kt, t) ? 1 : 0;
+    }
+  }
+
   auto k_smem = [&](int j) -> uint32_t {
     return base + C::kKOff + (j % C::kKSlots) * C::kTileBytes;
   };
@@ -217,14 +271,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                         q0 + t * BM, bh);
       }
     }
-    int issued = 0;
-    for (int j = 0; j < nkv; ++j) {
+    int issued = 0;  // ring index: the issued-th key tile the CTA walks
+    for (int kt = next_kt(kt_lo); kt < kt_hi; kt = next_kt(kt + 1)) {
+      const int j = issued;
       const int slot = j % nslots, rnd = j / nslots;
       if (rnd > 0 && !mbar_wait_warp(bar(bempty + slot), (rnd - 1) & 1, wd)) break;
       const uint32_t dst = is_k ? k_smem(j) : v_smem(j);
       mbar_arrive_expect_tx_e(bar(bfull + slot), C::kTileBytes);
       for (int c = 0; c < C::kChunks; ++c)
-        tma_load_3d_e(dst + c * C::kChunkBytes, map, bar(bfull + slot), c * 64, j * BN, bh);
+        tma_load_3d_e(dst + c * C::kChunkBytes, map, bar(bfull + slot), c * 64, kt * BN, bh);
       issued = j + 1;
     }
     // Every issued copy must land before the CTA may exit.
@@ -248,52 +303,51 @@ __global__ void __launch_bounds__(kThreads, 1)
     auto wait_v = [&](int j) {
       return mbar_wait_warp(bar(C::kBarVFull + j % C::kVSlots), (j / C::kVSlots) & 1, wd);
     };
-    // prologue: S_t(0)
-    if (ok && nkv > 0) {
-      ok = wait_k(0);
-      if (ok) {
+    // ns[t] / npv[t]: S_t and PV_t products issued so far (their barrier phases)
+    int ns[2] = {0, 0}, npv[2] = {0, 0};
+    // S_t for the key tile at ring index j, for each query tile that sees it, each
+    // as soon as the softmax of that tile has read its previous S out of TMEM
+    auto issue_s_all = [&](int kt, int j) -> bool {
+      bool have_k = false;
+      for (int t = 0; t < 2; ++t) {
+        if (!member(kt, t)) continue;
+        if (ns[t] > 0 && !mbar_wait_warp(bar(C::kBarSFree + t), (ns[t] - 1) & 1, wd))
+          return false;
+        if (!have_k) {
+          if (!wait_k(j)) return false;
+          have_k = true;
+        }
         tc_fence_after();
-        for (int t = 0; t < 2; ++t) {
-          if (nk[t] == 0) continue;
-          issue_s<D, E>(tmem + C::kTmS0 + t * 128, t ? q_smem1 : q_smem0, k_smem(0));
-          tc_commit_e(bar(C::kBarSFull + t));
-        }
-        tc_commit_e(bar(C::kBarKEmpty + 0));
+        issue_s<D, E>(tmem + C::kTmS0 + t * 128, t ? q_smem1 : q_smem0, k_smem(j));
+        tc_commit_e(bar(C::kBarSFull + t));
+        ++ns[t];
       }
-    }
-    for (int j = 0; j < nkv && ok; ++j) {
-      // S_t(j+1) for both tiles, each as soon as S_t(j) has been read out
-      if (j + 1 < nkv) {
-        bool have_k = false;
-        for (int t = 0; t < 2 && ok; ++t) {
-          if (j + 1 >= nk[t]) continue;
-          if (!mbar_wait_warp(bar(C::kBarSFree + t), j & 1, wd)) { ok = false; break; }
-          if (!have_k) {
-            if (!wait_k(j + 1)) { ok = false; break; }
-            have_k = true;
-          }
-          tc_fence_after();
-          issue_s<D, E>(tmem + C::kTmS0 + t * 128, t ? q_smem1 : q_smem0, k_smem(j + 1));
-          tc_commit_e(bar(C::kBarSFull + t));
-        }
-        if (!ok) break;
-        tc_commit_e(bar(C::kBarKEmpty + (j + 1) % C::kKSlots));
-      }
-      // O_t += P_t(j) V_j
+      tc_commit_e(bar(C::kBarKEmpty + j % C::kKSlots));
+      return true;
+    };
+    int cur = next_kt(kt_lo);
+    if (ok && cur < kt_hi) ok = issue_s_all(cur, 0);
+    for (int j = 0; cur < kt_hi && ok; ++j) {
+      // S for the next key tile before PV of this one
+      const int nxt = next_kt(cur + 1);
+      if (nxt < kt_hi && !issue_s_all(nxt, j + 1)) { ok = false; break; }
+      // O_t += P_t V_cur
       bool have_v = false;
       for (int t = 0; t < 2 && ok; ++t) {
-        if (j >= nk[t]) continue;
-        if (!mbar_wait_warp(bar(C::kBarPFull + t), j & 1, wd)) { ok = false; break; }
+        if (!member(cur, t)) continue;
+        if (!mbar_wait_warp(bar(C::kBarPFull + t), npv[t] & 1, wd)) { ok = false; break; }
         if (!have_v) {
           if (!wait_v(j)) { ok = false; break; }
           have_v = true;
         }
         tc_fence_after();
-        issue_pv<D, E>(tmem + C::kTmO0 + t * D, t ? p_smem1 : p_smem0, v_smem(j), j > 0);
+        issue_pv<D, E>(tmem + C::kTmO0 + t * D, t ? p_smem1 : p_smem0, v_smem(j), npv[t] > 0);
         tc_commit_e(bar(C::kBarPVDone + t));
+        ++npv[t];
       }
       if (!ok) break;
       tc_commit_e(bar(C::kBarVEmpty + j % C::kVSlots));
+      cur = nxt;
     }
     // No MMA may be in flight when TMEM is released.
     tc_commit_e(bar(C::kBarDrain));
@@ -313,8 +367,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float c = p.scale_log2;
     float m_ref = -INFINITY;
     float l = 0.0f;
-    bool ok = nk[t] > 0;
-    for (int j = 0; j < nk[t] && ok; ++j) {
+    // this tile's range, count and mask bits as scalars (no per-thread array indexing)
+    const int t_lo = t ? lo[1] : lo[0], t_hi = t ? hi[1] : hi[0];
+    const int t_nk = t ? nk[1] : nk[0];
+    const uint32_t* t_bits = mask_bits + t * C::kMaskWords;
+    auto t_member = [&](int kt) -> bool {
+      if (kt < t_lo || kt >= t_hi) return false;
+      return p.blocks == nullptr || ((t_bits[kt >> 5] >> (kt & 31)) & 1u);
+    };
+    bool ok = t_nk > 0;
+    // visible keys of this row: [k_lo, k_hi)
+    const int k_lo = (p.wl < 0) ? 0 : row - p.wl;
+    const int k_hi = (p.wr < 0) ? p.N : min(p.N, row + p.wr + 1);
+    const int r1 = r0 + BM - 1;
+    int kt = t_lo - 1;
+    for (int j = 0; j < t_nk && ok; ++j) {
+      do ++kt; while (!t_member(kt));
       ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarSFull + t), j & 1, wd));
       if (!ok) break;
       tc_fence_after();
@@ -326,13 +394,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(C::kBarSFree + t));
-      const int kv0 = j * BN;
-      const bool need_mask = (p.causal && kv0 + BN - 1 > r0) || (kv0 + BN > p.N);
+      const int kv0 = kt * BN;
+      // masking only where the tile crosses an edge of some row's visible range
+      const bool need_mask = (kv0 + BN > p.N) || (p.wr >= 0 && kv0 + BN - 1 > r0 + p.wr) ||
+                             (p.wl >= 0 && kv0 < r1 - p.wl);
       if (need_mask) {
-        const int lim = p.causal ? min(row + 1, p.N) : p.N;  // first masked column
+        // key kv0 + k is visible iff 0 <= kv0 + k - k_lo < k_hi - k_lo
+        const int off = kv0 - k_lo;
+        const unsigned span = static_cast<unsigned>(max(k_hi - k_lo, 0));
 #pragma unroll
         for (int k = 0; k < 128; ++k)
-          if (kv0 + k >= lim) s[k / 32][k % 32] = __float_as_uint(-INFINITY);
+          if (static_cast<unsigned>(off + k) >= span) s[k / 32][k % 32] = __float_as_uint(-INFINITY);
       }
       // row max: per 32-column chunk a tree of three-input maxima (short dependency
       // chains, few live temporaries), then across the four chunks
@@ -415,9 +487,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(C::kBarPFull + t));
     }
-    if (ok && nk[t] > 0)
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarPVDone + t), (nk[t] - 1) & 1, wd));
-    if (ok && nk[t] > 0) {
+    if (ok && t_nk > 0)
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarPVDone + t), (t_nk - 1) & 1, wd));
+    if (t_nk == 0 && row < p.N) {
+      // a query tile that sees no key: O = 0, LSE = -inf
+      uint4* dst = reinterpret_cast<uint4*>(p.O + (static_cast<size_t>(bh) * p.N + row) * D);
+#pragma unroll
+      for (int v = 0; v < D / 8; ++v) dst[v] = make_uint4(0u, 0u, 0u, 0u);
+      p.LSE[static_cast<size_t>(bh) * p.N + row] = -INFINITY;
+    }
+    if (ok && t_nk > 0) {
       tc_fence_after();
       const float inv_l = (l > 0.0f) ? 1.0f / l : 0.0f;
       uint16_t* orow = p.O + (static_cast<size_t>(bh) * p.N + row) * D;

@@ -161,6 +161,23 @@ bool make_map(CUtensorMap* map, const void* ptr, int BH, int N, int d, int box_r
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The masks as the kernels take them: window bounds clamped to [-1, N] (-1 = no
+// bound; a bound of N or more keeps every key on that side) and causal folded into
+// the right bound.
+struct MaskSpec {
+  int wl, wr;
+  const uint8_t* blocks;
+};
+
+fa_status make_mask(int N, int causal, int window_left, int window_right,
+                    const uint8_t* block_mask, MaskSpec* m) {
+  m->wl = (window_left < 0 || window_left >= N) ? -1 : window_left;
+  m->wr = causal ? 0 : ((window_right < 0 || window_right >= N) ? -1 : window_right);
+  m->blocks = block_mask;
+  if (block_mask != nullptr && (N + 127) / 128 > fwd::kMaxMaskTiles) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
 fa_status launch_status() {
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -177,7 +194,8 @@ namespace {
 
 template <Elt E>
 fa_status forward_impl(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
-                     int H, int N, int d, float scale, int causal, fa_stream_t stream) {
+                     int H, int N, int d, float scale, int causal, const MaskSpec& mask,
+                     fa_stream_t stream) {
   fa_status st = check_shape(B, H, N, d, scale, causal);
   if (st != FA_OK) return st;
   if (N == 0) return FA_OK;
@@ -195,7 +213,10 @@ fa_status forward_impl(const void* Q, const void* K, const void* V, void* O, flo
   p.BH = BH;
   p.n_qblk = (N + 2 * fwd::BM - 1) / (2 * fwd::BM);
   p.scale_log2 = scale * 1.4426950408889634f;
-  p.causal = causal;
+  p.wl = mask.wl;
+  p.wr = mask.wr;
+  p.blocks = mask.blocks;
+  p.n_kt = (N + fwd::BN - 1) / fwd::BN;
   p.timeout_ns = watchdog_ns();
   const dim3 grid(static_cast<unsigned>(p.n_qblk) * BH);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -264,7 +285,8 @@ fa_status preprocess_impl(const void* O, const void* dO, const float* LSE, int B
 template <Elt E>
 fa_status main_impl(const void* Q, const void* K, const void* V, const void* dO, void* dK,
                            void* dV, int B, int H, int N, int d, float scale, int causal,
-                           void* workspace, size_t workspace_bytes, fa_stream_t stream) {
+                           const MaskSpec& mask, void* workspace, size_t workspace_bytes,
+                           fa_stream_t stream) {
   const void* ptrs[] = {Q, K, V, dO, dK, dV};
   BwdPlan pl;
   fa_status st = bwd_plan(ptrs, 6, B, H, N, d, scale, causal, workspace, workspace_bytes, &pl);
@@ -285,7 +307,9 @@ fa_status main_impl(const void* Q, const void* K, const void* V, const void* dO,
   p.BH = pl.BH;
   p.scale = scale;
   p.scale_log2 = scale * 1.4426950408889634f;
-  p.causal = causal;
+  p.wl = mask.wl;
+  p.wr = mask.wr;
+  p.blocks = mask.blocks;
   p.timeout_ns = watchdog_ns();
   const dim3 grid(static_cast<unsigned>(pl.Npad / bwd::BN) * pl.BH);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -316,16 +340,16 @@ fa_status dq_convert_impl(void* dQ, int B, int H, int N, int d, float scale, voi
 template <Elt E>
 fa_status backward_impl(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                       const float* LSE, void* dQ, void* dK, void* dV, int B, int H, int N, int d,
-                      float scale, int causal, void* workspace, size_t workspace_bytes,
-                      fa_stream_t stream) {
+                      float scale, int causal, const MaskSpec& mask, void* workspace,
+                      size_t workspace_bytes, fa_stream_t stream) {
   const void* ptrs[] = {Q, K, V, O, dO, LSE, dQ, dK, dV};
   BwdPlan pl;
   fa_status st = bwd_plan(ptrs, 9, B, H, N, d, scale, causal, workspace, workspace_bytes, &pl);
   if (st != FA_OK || N == 0) return st;
   st = preprocess_impl<E>(O, dO, LSE, B, H, N, d, scale, causal, workspace, workspace_bytes, stream);
   if (st != FA_OK) return st;
-  st = main_impl<E>(Q, K, V, dO, dK, dV, B, H, N, d, scale, causal, workspace, workspace_bytes,
-                        stream);
+  st = main_impl<E>(Q, K, V, dO, dK, dV, B, H, N, d, scale, causal, mask, workspace,
+                    workspace_bytes, stream);
   if (st != FA_OK) return st;
   return dq_convert_impl<E>(dQ, B, H, N, d, scale, workspace, workspace_bytes, stream);
 }
@@ -379,12 +403,26 @@ fa_status fa_watchdog_selftest(int timeout_ms, fa_stream_t stream) {
 
 fa_status fa_forward(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
                      int H, int N, int d, float scale, int causal, fa_stream_t stream) {
-  return forward_impl<Elt::BF16>(Q, K, V, O, LSE, B, H, N, d, scale, causal, stream);
+  MaskSpec m;
+  make_mask(N, causal, -1, -1, nullptr, &m);
+  return forward_impl<Elt::BF16>(Q, K, V, O, LSE, B, H, N, d, scale, causal, m, stream);
 }
 
 fa_status fa_forward_f16(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
                          int H, int N, int d, float scale, int causal, fa_stream_t stream) {
-  return forward_impl<Elt::F16>(Q, K, V, O, LSE, B, H, N, d, scale, causal, stream);
+  MaskSpec m;
+  make_mask(N, causal, -1, -1, nullptr, &m);
+  return forward_impl<Elt::F16>(Q, K, V, O, LSE, B, H, N, d, scale, causal, m, stream);
+}
+
+fa_status fa_forward_masked(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                            int B, int H, int N, int d, float scale, int causal,
+                            int window_left, int window_right, const uint8_t* block_mask,
+                            fa_stream_t stream) {
+  MaskSpec m;
+  const fa_status st = make_mask(N, causal, window_left, window_right, block_mask, &m);
+  if (st != FA_OK) return st;
+  return forward_impl<Elt::BF16>(Q, K, V, O, LSE, B, H, N, d, scale, causal, m, stream);
 }
 
 fa_status fa_backward_preprocess(const void* O, const void* dO, const float* LSE, int B, int H,
@@ -397,7 +435,9 @@ fa_status fa_backward_preprocess(const void* O, const void* dO, const float* LSE
 fa_status fa_backward_main(const void* Q, const void* K, const void* V, const void* dO, void* dK,
                            void* dV, int B, int H, int N, int d, float scale, int causal,
                            void* workspace, size_t workspace_bytes, fa_stream_t stream) {
-  return main_impl<Elt::BF16>(Q, K, V, dO, dK, dV, B, H, N, d, scale, causal, workspace,
+  MaskSpec m;
+  make_mask(N, causal, -1, -1, nullptr, &m);
+  return main_impl<Elt::BF16>(Q, K, V, dO, dK, dV, B, H, N, d, scale, causal, m, workspace,
                               workspace_bytes, stream);
 }
 
@@ -410,7 +450,21 @@ fa_status fa_backward(const void* Q, const void* K, const void* V, const void* O
                       const float* LSE, void* dQ, void* dK, void* dV, int B, int H, int N, int d,
                       float scale, int causal, void* workspace, size_t workspace_bytes,
                       fa_stream_t stream) {
-  return backward_impl<Elt::BF16>(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, scale, causal,
+  MaskSpec m;
+  make_mask(N, causal, -1, -1, nullptr, &m);
+  return backward_impl<Elt::BF16>(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, scale, causal, m,
+                                  workspace, workspace_bytes, stream);
+}
+
+fa_status fa_backward_masked(const void* Q, const void* K, const void* V, const void* O,
+                             const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
+                             int B, int H, int N, int d, float scale, int causal,
+                             int window_left, int window_right, const uint8_t* block_mask,
+                             void* workspace, size_t workspace_bytes, fa_stream_t stream) {
+  MaskSpec m;
+  const fa_status st = make_mask(N, causal, window_left, window_right, block_mask, &m);
+  if (st != FA_OK) return st;
+  return backward_impl<Elt::BF16>(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, scale, causal, m,
                                   workspace, workspace_bytes, stream);
 }
 
@@ -418,7 +472,9 @@ fa_status fa_backward_f16(const void* Q, const void* K, const void* V, const voi
                           const void* dO, const float* LSE, void* dQ, void* dK, void* dV, int B,
                           int H, int N, int d, float scale, int causal, void* workspace,
                           size_t workspace_bytes, fa_stream_t stream) {
-  return backward_impl<Elt::F16>(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, scale, causal,
+  MaskSpec m;
+  make_mask(N, causal, -1, -1, nullptr, &m);
+  return backward_impl<Elt::F16>(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, scale, causal, m,
                                  workspace, workspace_bytes, stream);
 }
 
