@@ -44,6 +44,8 @@
 // No N x N matrix is written to device memory.
 #pragma once
 
+#include <type_traits>
+
 #include "fa_ptx.cuh"
 
 namespace fa {
@@ -246,7 +248,7 @@ __global__ void __launch_bounds__(256)
 
 // ------------------------------------------------------------------ main kernel
 
-template <int D, Elt E>
+template <int D, Elt E, bool kMasked>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -263,6 +265,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // Without a window's left bound or a block mask (kMasked = false) those are
+  // compile-time constants, so the general tile walk folds to the plain / causal one.
+  const int wl = kMasked ? p.wl : -1;
+  const int wr = p.wr;
+  const uint8_t* const blocks = kMasked ? p.blocks : nullptr;
 
   // Work item: head-major (the resident CTAs share one or two heads' Q, dO and dQ
   // accumulator in L2); within a head, key tile 0 (the heaviest if causal) first.
@@ -273,15 +280,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_q = (p.N + BM - 1) / BM;
   // query tiles [i_lo, i_hi) hold every query that may see a key of this tile
   const int k1 = min(k0 + BN, p.N) - 1;
-  const int i_lo = (p.wr < 0) ? 0 : max(0, k0 - p.wr) / BM;
-  const int i_hi = (p.wl < 0) ? n_q : min(n_q, (k1 + p.wl) / BM + 1);
+  const int i_lo = (wr < 0) ? 0 : max(0, k0 - wr) / BM;
+  const int i_hi = (wl < 0) ? n_q : min(n_q, (k1 + wl) / BM + 1);
 
   // The block-mask column of this key tile as bits: warp w builds words w, w + 16, ...
   uint32_t* mask_bits = reinterpret_cast<uint32_t*>(base_ptr + C::kMaskOff);
-  if (p.blocks != nullptr) {
+  if (blocks != nullptr) {
     for (int wi = warp; wi < (n_q + 31) / 32; wi += kThreads / 32) {
       const int i = wi * 32 + lane;
-      const bool keep = i < n_q && p.blocks[static_cast<size_t>(i) * n_kt + j] != 0;
+      const bool keep = i < n_q && blocks[static_cast<size_t>(i) * n_kt + j] != 0;
       const uint32_t bits = __ballot_sync(0xffffffffu, keep);
       if (lane == 0) mask_bits[wi] = bits;
     }
@@ -317,10 +324,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Does some query of query tile i see a key of this tile?
   auto member = [&](int i) -> bool {
     if (i < i_lo || i >= i_hi) return false;
-    return p.blocks == nullptr || ((mask_bits[i >> 5] >> (i & 31)) & 1u);
+    return blocks == nullptr || ((mask_bits[i >> 5] >> (i & 31)) & 1u);
   };
   int nsteps = i_hi - i_lo;  // query tiles walked
-  if (p.blocks != nullptr) {
+  if (blocks != nullptr) {
     nsteps = 0;
     for (int i = i_lo; i < i_hi; ++i) nsteps += member(i) ? 1 : 0;
   }
@@ -453,8 +460,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool ragged_keys = k0 + BN > p.N;
     const int dq_bar = (D == 128) ? C::kBarDQFull + h : C::kBarDQFull;
     // queries that see this key row: [q_lo, q_hi) (empty for a padding key)
-    const int q_lo = (p.wr < 0) ? 0 : key - p.wr;
-    const int q_hi = (key >= p.N) ? q_lo : ((p.wl < 0) ? p.Npad + BM : key + p.wl + 1);
+    const int q_lo = (wr < 0) ? 0 : key - wr;
+    const int q_hi = (key >= p.N) ? q_lo : ((wl < 0) ? p.Npad + BM : key + wl + 1);
     const unsigned q_span = static_cast<unsigned>(q_hi - q_lo);
     bool ok = true;
     int i = i_lo - 1;
@@ -476,50 +483,59 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float4* Dv4 = Lv + 64 / 4;
       // masking is needed only where the half crosses an edge of some key's visible
       // queries (the causal diagonal, a window edge) and on a ragged key tile
-      const bool mask = ragged_keys || (p.wr >= 0 && k0 + BN - 1 - p.wr > qh0) ||
-                        (p.wl >= 0 && k0 + p.wl < qh0 + 63);
+      const bool mask = ragged_keys || (wr >= 0 && k0 + BN - 1 - wr > qh0) ||
+                        (wl >= 0 && k0 + wl < qh0 + 63);
       const int qoff = qh0 - q_lo;  // query qh0 + x is visible iff qoff + x < q_span (unsigned)
-      uint32_t sv[2][16], dv[2][16];
-      tmem_ld16(tm_s, sv[0]);
-      tmem_ld16(tm_dp, dv[0]);
-      tmem_wait_ld();
+      // The element loop in two compiled forms: with the mask tests only on steps
+      // that cross a mask edge, none on all the others.
+      auto p_ds = [&](auto masked) {
+        constexpr bool kM = decltype(masked)::value;
+        uint32_t sv[2][16], dv[2][16];
+        tmem_ld16(tm_s, sv[0]);
+        tmem_ld16(tm_dp, dv[0]);
+        tmem_wait_ld();
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        const int cur = cc & 1;
-        if (cc + 1 < 4) {  // the next chunk's loads overlap this chunk's arithmetic
-          tmem_ld16(tm_s + 16 * (cc + 1), sv[cur ^ 1]);
-          tmem_ld16(tm_dp + 16 * (cc + 1), dv[cur ^ 1]);
-        }
-        uint32_t pk[8], dk[8];
-#pragma unroll
-        for (int v = 0; v < 4; ++v) {
-          const float4 L4 = Lv[cc * 4 + v];
-          const float4 D4 = Dv4[cc * 4 + v];
-          const float Ls[4] = {L4.x, L4.y, L4.z, L4.w};
-          const float Ds[4] = {D4.x, D4.y, D4.z, D4.w};
-          float pv[4], dsv[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int k = 4 * v + e;
-            float pe = ex2_approx(fmaf(__uint_as_float(sv[cur][k]), c, -Ls[e]));
-            if (mask && static_cast<unsigned>(qoff + cc * 16 + k) >= q_span) pe = 0.f;
-            pv[e] = pe;
-            dsv[e] = pe * (__uint_as_float(dv[cur][k]) - Ds[e]);
+        for (int cc = 0; cc < 4; ++cc) {
+          const int cur = cc & 1;
+          if (cc + 1 < 4) {  // the next chunk's loads overlap this chunk's arithmetic
+            tmem_ld16(tm_s + 16 * (cc + 1), sv[cur ^ 1]);
+            tmem_ld16(tm_dp + 16 * (cc + 1), dv[cur ^ 1]);
           }
-          pk[2 * v] = pack2<E>(pv[0], pv[1]);
-          pk[2 * v + 1] = pack2<E>(pv[2], pv[3]);
-          dk[2 * v] = pack2<E>(dsv[0], dsv[1]);
-          dk[2 * v + 1] = pack2<E>(dsv[2], dsv[3]);
+          uint32_t pk[8], dk[8];
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const float4 L4 = Lv[cc * 4 + v];
+            const float4 D4 = Dv4[cc * 4 + v];
+            const float Ls[4] = {L4.x, L4.y, L4.z, L4.w};
+            const float Ds[4] = {D4.x, D4.y, D4.z, D4.w};
+            float pv[4], dsv[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int k = 4 * v + e;
+              float pe = ex2_approx(fmaf(__uint_as_float(sv[cur][k]), c, -Ls[e]));
+              if (kM && static_cast<unsigned>(qoff + cc * 16 + k) >= q_span) pe = 0.f;
+              pv[e] = pe;
+              dsv[e] = pe * (__uint_as_float(dv[cur][k]) - Ds[e]);
+            }
+            pk[2 * v] = pack2<E>(pv[0], pv[1]);
+            pk[2 * v + 1] = pack2<E>(pv[2], pv[3]);
+            dk[2 * v] = pack2<E>(dsv[0], dsv[1]);
+            dk[2 * v + 1] = pack2<E>(dsv[2], dsv[3]);
+          }
+          tmem_st8(tm_s + 8 * cc, pk);
+          tmem_st8(tm_dp + 8 * cc, dk);
+          // dS into the swizzled shared chunk: 16 queries = 16-byte units 2cc, 2cc+1
+          *reinterpret_cast<uint4*>(ds_row + (((2 * cc) ^ (krow & 7)) * 16)) =
+              make_uint4(dk[0], dk[1], dk[2], dk[3]);
+          *reinterpret_cast<uint4*>(ds_row + (((2 * cc + 1) ^ (krow & 7)) * 16)) =
+              make_uint4(dk[4], dk[5], dk[6], dk[7]);
+          if (cc + 1 < 4) tmem_wait_ld();
         }
-        tmem_st8(tm_s + 8 * cc, pk);
-        tmem_st8(tm_dp + 8 * cc, dk);
-        // dS into the swizzled shared chunk: 16 queries = 16-byte units 2cc, 2cc+1
-        *reinterpret_cast<uint4*>(ds_row + (((2 * cc) ^ (krow & 7)) * 16)) =
-            make_uint4(dk[0], dk[1], dk[2], dk[3]);
-        *reinterpret_cast<uint4*>(ds_row + (((2 * cc + 1) ^ (krow & 7)) * 16)) =
-            make_uint4(dk[4], dk[5], dk[6], dk[7]);
-        if (cc + 1 < 4) tmem_wait_ld();
-      }
+      };
+      if (mask)
+        p_ds(std::true_type{});
+      else
+        p_ds(std::false_type{});
       tmem_wait_st();
       fence_proxy_async_smem();
       tc_fence_before();

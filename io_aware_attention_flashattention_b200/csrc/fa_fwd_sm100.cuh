@@ -86,6 +86,7 @@ struct Cfg {
   static constexpr int kSmemBytes = kMaskOff + 2 * kMaskWords * 4 + 1024;  // + alignment
   static constexpr uint32_t kTmS0 = 0, kTmO0 = 256;
   static_assert(kSmemBytes <= 232448, "exceeds the 227 KB of shared memory a CTA may use");
+  static_assert(kSmemBytes <= 232448, "exceeds the 227 KB of shared memory a CTA may use");
   static constexpr uint32_t kTmCols = 512;
 };
 
@@ -141,7 +142,7 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
   }
 }
 
-template <int D, Elt E>
+template <int D, Elt E, bool kMasked>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const Params p) {
@@ -157,6 +158,11 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  // Without a window's left bound or a block mask (kMasked = false) those are
+  // compile-time constants, so the general tile walk folds to the plain / causal one.
+  const int wl = kMasked ? p.wl : -1;
+  const int wr = p.wr;
+  const uint8_t* const blocks = kMasked ? p.blocks : nullptr;
 
   // Work item: head-major, so that the CTAs resident at any time cover about two
   // heads and their K/V stay in L2; within a head the heaviest query blocks (causal)
@@ -170,8 +176,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
     const int r0 = q0 + t * BM, r1 = min(r0 + BM, p.N) - 1;
-    lo[t] = (p.wl < 0) ? 0 : max(0, r0 - p.wl) / BN;
-    hi[t] = (p.wr < 0) ? n_kt : min(n_kt, (r1 + p.wr) / BN + 1);
+    lo[t] = (wl < 0) ? 0 : max(0, r0 - wl) / BN;
+    hi[t] = (wr < 0) ? n_kt : min(n_kt, (r1 + wr) / BN + 1);
     if (r0 >= p.N) lo[t] = hi[t] = 0;
   }
   // The CTA's key tiles: the union of both ranges (contiguous: lo[1] <= hi[0]).
@@ -181,13 +187,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Block mask rows of the two query tiles as bits in shared memory: warp w builds
   // words w, w + 11, ... with one byte per lane and a ballot.
   uint32_t* mask_bits = reinterpret_cast<uint32_t*>(base_ptr + C::kMaskOff);
-  if (p.blocks != nullptr) {
+  if (blocks != nullptr) {
     const int nwords = (n_kt + 31) / 32;
     for (int w = warp; w < 2 * nwords; w += kThreads / 32) {
       const int t = w / nwords, wi = w % nwords;
       const int qt = min(2 * qb + t, n_kt - 1);
       const int kt = wi * 32 + lane;
-      const bool keep = kt < n_kt && p.blocks[static_cast<size_t>(qt) * n_kt + kt] != 0;
+      const bool keep = kt < n_kt && blocks[static_cast<size_t>(qt) * n_kt + kt] != 0;
       const uint32_t bits = __ballot_sync(0xffffffffu, keep);
       if (lane == 0) mask_bits[t * C::kMaskWords + wi] = bits;
     }
@@ -226,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Does query tile t see any key of key tile kt?
   auto member = [&](int kt, int t) -> bool {
     if (kt < lo[t] || kt >= hi[t]) return false;
-    return p.blocks == nullptr || ((mask_bits[t * C::kMaskWords + (kt >> 5)] >> (kt & 31)) & 1u);
+    return blocks == nullptr || ((mask_bits[t * C::kMaskWords + (kt >> 5)] >> (kt & 31)) & 1u);
   };
   // first key tile >= kt that either query tile sees (kt_hi if none)
   auto next_kt = [&](int kt) -> int {
@@ -236,7 +242,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   int nk[2];  // key tiles each query tile sees
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
-    if (p.blocks == nullptr) {
+    if (blocks == nullptr) {
       nk[t] = hi[t] - lo[t];
     } else {
       nk[t] = 0;
@@ -373,12 +379,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t* t_bits = mask_bits + t * C::kMaskWords;
     auto t_member = [&](int kt) -> bool {
       if (kt < t_lo || kt >= t_hi) return false;
-      return p.blocks == nullptr || ((t_bits[kt >> 5] >> (kt & 31)) & 1u);
+      return blocks == nullptr || ((t_bits[kt >> 5] >> (kt & 31)) & 1u);
     };
     bool ok = t_nk > 0;
     // visible keys of this row: [k_lo, k_hi)
-    const int k_lo = (p.wl < 0) ? 0 : row - p.wl;
-    const int k_hi = (p.wr < 0) ? p.N : min(p.N, row + p.wr + 1);
+    const int k_lo = (wl < 0) ? 0 : row - wl;
+    const int k_hi = (wr < 0) ? p.N : min(p.N, row + wr + 1);
     const int r1 = r0 + BM - 1;
     int kt = t_lo - 1;
     for (int j = 0; j < t_nk && ok; ++j) {
@@ -396,8 +402,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(bar(C::kBarSFree + t));
       const int kv0 = kt * BN;
       // masking only where the tile crosses an edge of some row's visible range
-      const bool need_mask = (kv0 + BN > p.N) || (p.wr >= 0 && kv0 + BN - 1 > r0 + p.wr) ||
-                             (p.wl >= 0 && kv0 < r1 - p.wl);
+      const bool need_mask = (kv0 + BN > p.N) || (wr >= 0 && kv0 + BN - 1 > r0 + wr) ||
+                             (wl >= 0 && kv0 < r1 - wl);
       if (need_mask) {
         // key kv0 + k is visible iff 0 <= kv0 + k - k_lo < k_hi - k_lo
         const int off = kv0 - k_lo;

@@ -84,6 +84,21 @@ cudaError_t set_smem(Kern k, size_t bytes) {
                               static_cast<int>(bytes));
 }
 
+template <int D, Elt E>
+cudaError_t set_smem_d() {
+  cudaError_t e = set_smem(fwd::fa_fwd_kernel<D, E, false>, fwd::Cfg<D>::kSmemBytes);
+  e = e ? e : set_smem(fwd::fa_fwd_kernel<D, E, true>, fwd::Cfg<D>::kSmemBytes);
+  e = e ? e : set_smem(bwd::fa_bwd_kernel<D, E, false>, bwd::Cfg<D>::kSmemBytes);
+  e = e ? e : set_smem(bwd::fa_bwd_kernel<D, E, true>, bwd::Cfg<D>::kSmemBytes);
+  return e;
+}
+
+template <Elt E>
+cudaError_t set_smem_all() {
+  const cudaError_t e = set_smem_d<64, E>();
+  return e ? e : set_smem_d<128, E>();
+}
+
 // Checks that the current device is an sm_100 part and sets the kernels'
 // shared-memory limits once per device.
 fa_status prepare_device() {
@@ -102,14 +117,8 @@ fa_status prepare_device() {
   if (!st.supported) return FA_ERR_UNSUPPORTED;
   if (!st.attrs_done) {
     cudaError_t e = cudaSuccess;
-    e = e ? e : set_smem(fwd::fa_fwd_kernel<64, Elt::BF16>, fwd::Cfg<64>::kSmemBytes);
-    e = e ? e : set_smem(fwd::fa_fwd_kernel<128, Elt::BF16>, fwd::Cfg<128>::kSmemBytes);
-    e = e ? e : set_smem(fwd::fa_fwd_kernel<64, Elt::F16>, fwd::Cfg<64>::kSmemBytes);
-    e = e ? e : set_smem(fwd::fa_fwd_kernel<128, Elt::F16>, fwd::Cfg<128>::kSmemBytes);
-    e = e ? e : set_smem(bwd::fa_bwd_kernel<64, Elt::BF16>, bwd::Cfg<64>::kSmemBytes);
-    e = e ? e : set_smem(bwd::fa_bwd_kernel<128, Elt::BF16>, bwd::Cfg<128>::kSmemBytes);
-    e = e ? e : set_smem(bwd::fa_bwd_kernel<64, Elt::F16>, bwd::Cfg<64>::kSmemBytes);
-    e = e ? e : set_smem(bwd::fa_bwd_kernel<128, Elt::F16>, bwd::Cfg<128>::kSmemBytes);
+    e = e ? e : set_smem_all<Elt::BF16>();
+    e = e ? e : set_smem_all<Elt::F16>();
     e = e ? e : set_smem(f32::fa_f32_bwd_dkdv_kernel<64>, f32::dkdv_smem_bytes<64>());
     e = e ? e : set_smem(f32::fa_f32_bwd_dkdv_kernel<128>, f32::dkdv_smem_bytes<128>());
     e = e ? e : set_smem(f32::fa_f32_bwd_dq_kernel<64>, f32::dq_smem_bytes<64>());
@@ -167,6 +176,9 @@ bool make_map(CUtensorMap* map, const void* ptr, int BH, int N, int d, int box_r
 struct MaskSpec {
   int wl, wr;
   const uint8_t* blocks;
+  // the general kernels are needed only for a left bound or a block mask; a right
+  // bound alone (causal included) is a runtime value of the plain ones
+  bool general() const { return wl >= 0 || blocks != nullptr; }
 };
 
 fa_status make_mask(int N, int causal, int window_left, int window_right,
@@ -220,10 +232,15 @@ fa_status forward_impl(const void* Q, const void* K, const void* V, void* O, flo
   p.timeout_ns = watchdog_ns();
   const dim3 grid(static_cast<unsigned>(p.n_qblk) * BH);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (d == 64)
-    fwd::fa_fwd_kernel<64, E><<<grid, fwd::kThreads, fwd::Cfg<64>::kSmemBytes, s>>>(mq, mk, mv, p);
+  const bool g = mask.general();
+  if (d == 64 && !g)
+    fwd::fa_fwd_kernel<64, E, false><<<grid, fwd::kThreads, fwd::Cfg<64>::kSmemBytes, s>>>(mq, mk, mv, p);
+  else if (d == 64)
+    fwd::fa_fwd_kernel<64, E, true><<<grid, fwd::kThreads, fwd::Cfg<64>::kSmemBytes, s>>>(mq, mk, mv, p);
+  else if (!g)
+    fwd::fa_fwd_kernel<128, E, false><<<grid, fwd::kThreads, fwd::Cfg<128>::kSmemBytes, s>>>(mq, mk, mv, p);
   else
-    fwd::fa_fwd_kernel<128, E><<<grid, fwd::kThreads, fwd::Cfg<128>::kSmemBytes, s>>>(mq, mk, mv, p);
+    fwd::fa_fwd_kernel<128, E, true><<<grid, fwd::kThreads, fwd::Cfg<128>::kSmemBytes, s>>>(mq, mk, mv, p);
   return launch_status();
 }
 
@@ -313,10 +330,16 @@ fa_status main_impl(const void* Q, const void* K, const void* V, const void* dO,
   p.timeout_ns = watchdog_ns();
   const dim3 grid(static_cast<unsigned>(pl.Npad / bwd::BN) * pl.BH);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (d == 64)
-    bwd::fa_bwd_kernel<64, E><<<grid, bwd::kThreads, bwd::Cfg<64>::kSmemBytes, s>>>(mq, mk, mv, mdo, p);
+  const bool g = mask.general();
+  using bwd::Cfg;
+  if (d == 64 && !g)
+    bwd::fa_bwd_kernel<64, E, false><<<grid, bwd::kThreads, Cfg<64>::kSmemBytes, s>>>(mq, mk, mv, mdo, p);
+  else if (d == 64)
+    bwd::fa_bwd_kernel<64, E, true><<<grid, bwd::kThreads, Cfg<64>::kSmemBytes, s>>>(mq, mk, mv, mdo, p);
+  else if (!g)
+    bwd::fa_bwd_kernel<128, E, false><<<grid, bwd::kThreads, Cfg<128>::kSmemBytes, s>>>(mq, mk, mv, mdo, p);
   else
-    bwd::fa_bwd_kernel<128, E><<<grid, bwd::kThreads, bwd::Cfg<128>::kSmemBytes, s>>>(mq, mk, mv, mdo, p);
+    bwd::fa_bwd_kernel<128, E, true><<<grid, bwd::kThreads, Cfg<128>::kSmemBytes, s>>>(mq, mk, mv, mdo, p);
   return launch_status();
 }
 
