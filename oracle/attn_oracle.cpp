@@ -38,6 +38,14 @@
 //                              tile size 128 of [yunthe] "GPU memory optimisation
 //                              strategy" (Block_Q = Block_K = 128).
 //   A query row that sees no key at all has P = 0, O = 0 and L = -inf.
+//   Dropout on P (optional): [jos] p.218 lists dropout among the operations fused into
+//   the attention kernel. With drop probability p, Pd[i][j] = P[i][j] * Z[i][j] / (1 - p)
+//   and O = Pd V; L stays the log-sum-exp of the logits (P is normalised before the
+//   dropout). Z[i][j] = 0 iff the Philox-4x32-10 word for (i, j) is below
+//   t = min(floor(p * 2^32), 2^32 - 1) (an integer decision). The word is element j % 4
+//   of Philox-4x32-10 (Salmon, Moraes, Dror and Shaw, "Parallel random numbers: as easy
+//   as 1, 2, 3", SC 2011) at counter (j / 4, i, bh, offset) under key (seed low 32
+//   bits, seed high 32 bits), bh = b * H + h.
 //   m_i = max_j S[i][j]        [jsqmd] section 2.1, safe softmax
 //   P[i][j] = exp(S[i][j] - m_i) / sum_j exp(S[i][j] - m_i)
 //   O = P V
@@ -51,6 +59,8 @@
 //   dP = dO V^T
 //   D_i = sum_j P[i][j] dP[i][j]   (equal to sum_k dO[i][k] O[i][k])
 //   dS = P o (dP - D)              (softmax Jacobian, row by row)
+//   With dropout: dV = Pd^T dO, dPd = dO V^T, dP = dPd o Z / (1 - p), and
+//   D_i = sum_j P[i][j] dP[i][j] = sum_j Pd[i][j] dPd[i][j] (still rowsum(dO o O)).
 //   dQ = scale * dS K
 //   dK = scale * dS^T Q
 //
@@ -104,6 +114,65 @@ Visibility make_vis(int64_t N, int causal, int64_t left, int64_t right,
                     const uint8_t* blocks) {
   return Visibility{causal, left, right, blocks, (N + kBlock - 1) / kBlock};
 }
+
+// Philox-4x32-10 as published: ten rounds; each multiplies words 0 and 2 by the two
+// round multipliers (high and low halves of the 64-bit products), mixes in words 1
+// and 3 and the round key, and permutes; the key grows by the two Weyl increments
+// between rounds.
+void philox4x32_10(const uint32_t ctr[4], uint32_t k0, uint32_t k1, uint32_t out[4]) {
+  uint32_t x0 = ctr[0], x1 = ctr[1], x2 = ctr[2], x3 = ctr[3];
+  for (int r = 0; r < 10; ++r) {
+    if (r > 0) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+    const uint64_t p0 = static_cast<uint64_t>(0xD2511F53u) * x0;
+    const uint64_t p1 = static_cast<uint64_t>(0xCD9E8D57u) * x2;
+    const uint32_t hi0 = static_cast<uint32_t>(p0 >> 32), lo0 = static_cast<uint32_t>(p0);
+    const uint32_t hi1 = static_cast<uint32_t>(p1 >> 32), lo1 = static_cast<uint32_t>(p1);
+    x0 = hi1 ^ x1 ^ k0;
+    x1 = lo1;
+    x2 = hi0 ^ x3 ^ k1;
+    x3 = lo0;
+  }
+  out[0] = x0;
+  out[1] = x1;
+  out[2] = x2;
+  out[3] = x3;
+}
+
+// Dropout on P (see the header). p = 0 is no dropout.
+struct Dropout {
+  double p;
+  uint64_t seed;
+  uint32_t offset;
+  uint32_t threshold;  // a key is dropped iff its Philox word is below this
+
+  bool on() const { return p > 0.0; }
+  // Z[i][j] of head bh, as 0 or 1
+  bool keep(int64_t bh, int64_t i, int64_t j) const {
+    if (!on()) return true;
+    const uint32_t ctr[4] = {static_cast<uint32_t>(j / 4), static_cast<uint32_t>(i),
+                             static_cast<uint32_t>(bh), offset};
+    uint32_t w[4];
+    philox4x32_10(ctr, static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32), w);
+    return w[j % 4] >= threshold;
+  }
+  // Pd / P for (i, j): Z / (1 - p)
+  double factor(int64_t bh, int64_t i, int64_t j) const {
+    if (!on()) return 1.0;
+    return keep(bh, i, j) ? 1.0 / (1.0 - p) : 0.0;
+  }
+};
+
+Dropout make_dropout(double p, uint64_t seed, uint32_t offset) {
+  double t = std::floor(p * 4294967296.0);
+  if (t > 4294967295.0) t = 4294967295.0;
+  if (!(t > 0.0)) t = 0.0;
+  return Dropout{p, seed, offset, static_cast<uint32_t>(t)};
+}
+
+bool bad_dropout(double p) { return !(p >= 0.0 && p < 1.0); }
 
 // One row of scaled, masked logits: s[j] = scale * <q_i, k_j>, -inf where the
 // key is hidden.
@@ -161,6 +230,11 @@ void oracle_set_num_threads(int n) {
 #endif
 }
 
+// Philox-4x32-10 of one counter under one key (for the generator's own pins).
+void oracle_philox4x32_10(const uint32_t* ctr, uint32_t k0, uint32_t k1, uint32_t* out) {
+  philox4x32_10(ctr, k0, k1, out);
+}
+
 // The row-stochastic matrix P = softmax(S) of one head, N x N, into P.
 int oracle_attention_probs(const double* Q, const double* K, int64_t N, int64_t d,
                            double scale, int causal, int64_t left, int64_t right,
@@ -183,10 +257,11 @@ int oracle_attention_probs(const double* Q, const double* K, int64_t N, int64_t 
 // head at a time.
 int oracle_attention_forward(const double* Q, const double* K, const double* V, int64_t B,
                              int64_t H, int64_t N, int64_t d, double scale, int causal,
-                             int64_t left, int64_t right, const uint8_t* blocks, double* O,
-                             double* L) {
-  if (bad_shape(B, H, N, d) || !Q || !K || !V || !O || !L) return 1;
+                             int64_t left, int64_t right, const uint8_t* blocks, double p_drop,
+                             uint64_t seed, uint32_t offset, double* O, double* L) {
+  if (bad_shape(B, H, N, d) || !Q || !K || !V || !O || !L || bad_dropout(p_drop)) return 1;
   const Visibility vis = make_vis(N, causal, left, right, blocks);
+  const Dropout drop = make_dropout(p_drop, seed, offset);
   if (N == 0) return 0;
   std::vector<double> P;
   try {
@@ -208,14 +283,14 @@ int oracle_attention_forward(const double* Q, const double* K, const double* V, 
       std::vector<double> s(row, row + N);
       l[i] = safe_softmax_row(s.data(), N, row);
     }
-    // O = P V
+    // O = Pd V (Pd = P without dropout)
 #pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < N; ++i) {
       const double* p = P.data() + i * N;
       double* oi = o + i * d;
       for (int64_t c = 0; c < d; ++c) oi[c] = 0.0;
       for (int64_t j = 0; j < N; ++j) {
-        const double pij = p[j];
+        const double pij = p[j] * drop.factor(bh, i, j);
         const double* vj = v + j * d;
         for (int64_t c = 0; c < d; ++c) oi[c] += pij * vj[c];
       }
@@ -231,10 +306,14 @@ int oracle_attention_forward(const double* Q, const double* K, const double* V, 
 int oracle_attention_backward(const double* Q, const double* K, const double* V,
                               const double* dO, int64_t B, int64_t H, int64_t N, int64_t d,
                               double scale, int causal, int64_t left, int64_t right,
-                              const uint8_t* blocks, double* dQ, double* dK, double* dV,
-                              double* D, double* Dcheck) {
-  if (bad_shape(B, H, N, d) || !Q || !K || !V || !dO || !dQ || !dK || !dV || !D) return 1;
+                              const uint8_t* blocks, double p_drop, uint64_t seed,
+                              uint32_t offset, double* dQ, double* dK, double* dV, double* D,
+                              double* Dcheck) {
+  if (bad_shape(B, H, N, d) || !Q || !K || !V || !dO || !dQ || !dK || !dV || !D ||
+      bad_dropout(p_drop))
+    return 1;
   const Visibility vis = make_vis(N, causal, left, right, blocks);
+  const Dropout drop = make_dropout(p_drop, seed, offset);
   if (N == 0) return 0;
   std::vector<double> P, dS;
   try {
@@ -262,7 +341,8 @@ int oracle_attention_backward(const double* Q, const double* K, const double* V,
         safe_softmax_row(s.data(), N, P.data() + i * N);
       }
     }
-    // dP = dO V^T, D_i = sum_j P_ij dP_ij, dS = P o (dP - D); dS holds dP first.
+    // dP = (dO V^T) o Z / (1 - p), D_i = sum_j P_ij dP_ij, dS = P o (dP - D); dS holds
+    // dP first.
 #pragma omp parallel for schedule(static)
     for (int64_t i = 0; i < N; ++i) {
       const double* goi = go + i * d;
@@ -273,17 +353,17 @@ int oracle_attention_backward(const double* Q, const double* K, const double* V,
         const double* vj = v + j * d;
         double acc = 0.0;
         for (int64_t c = 0; c < d; ++c) acc += goi[c] * vj[c];
-        dsi[j] = acc;
-        Di += pi[j] * acc;
+        dsi[j] = acc * drop.factor(bh, i, j);
+        Di += pi[j] * dsi[j];
       }
       Dh[i] = Di;
       for (int64_t j = 0; j < N; ++j) dsi[j] = pi[j] * (dsi[j] - Di);
       if (Dcheck) {
-        // O_i = sum_j P_ij V_j, then sum_k dO_ik O_ik
+        // O_i = sum_j Pd_ij V_j, then sum_k dO_ik O_ik
         double Dc = 0.0;
         for (int64_t c = 0; c < d; ++c) {
           double oic = 0.0;
-          for (int64_t j = 0; j < N; ++j) oic += pi[j] * v[j * d + c];
+          for (int64_t j = 0; j < N; ++j) oic += pi[j] * drop.factor(bh, i, j) * v[j * d + c];
           Dc += goi[c] * oic;
         }
         Dcheck[bh * N + i] = Dc;
@@ -312,7 +392,7 @@ int oracle_attention_backward(const double* Q, const double* K, const double* V,
       }
       for (int64_t i = 0; i < N; ++i) {
         const double ds = dS[i * N + j];
-        const double p = P[i * N + j];
+        const double p = P[i * N + j] * drop.factor(bh, i, j);
         const double* qi = q + i * d;
         const double* goi = go + i * d;
         for (int64_t c = 0; c < d; ++c) {
@@ -332,11 +412,14 @@ int oracle_attention_backward(const double* Q, const double* K, const double* V,
 int oracle_attention_forward_rows(const double* Q, const double* K, const double* V,
                                   int64_t B, int64_t H, int64_t N, int64_t d, double scale,
                                   int causal, int64_t left, int64_t right,
-                                  const uint8_t* blocks, int64_t R, const int64_t* heads,
+                                  const uint8_t* blocks, double p_drop, uint64_t seed,
+                                  uint32_t offset, int64_t R, const int64_t* heads,
                                   const int64_t* rows, double* O_r, double* L_r) {
-  if (bad_shape(B, H, N, d) || R < 0 || (R > 0 && (!heads || !rows || !O_r || !L_r)))
+  if (bad_shape(B, H, N, d) || R < 0 || (R > 0 && (!heads || !rows || !O_r || !L_r)) ||
+      bad_dropout(p_drop))
     return 1;
   const Visibility vis = make_vis(N, causal, left, right, blocks);
+  const Dropout drop = make_dropout(p_drop, seed, offset);
   for (int64_t r = 0; r < R; ++r)
     if (heads[r] < 0 || heads[r] >= B * H || rows[r] < 0 || rows[r] >= N) return 1;
 #pragma omp parallel
@@ -351,8 +434,10 @@ int oracle_attention_forward_rows(const double* Q, const double* K, const double
       L_r[r] = safe_softmax_row(s.data(), N, p.data());
       double* o = O_r + r * d;
       for (int64_t c = 0; c < d; ++c) o[c] = 0.0;
-      for (int64_t j = 0; j < N; ++j)
-        for (int64_t c = 0; c < d; ++c) o[c] += p[j] * v[j * d + c];
+      for (int64_t j = 0; j < N; ++j) {
+        const double pd = p[j] * drop.factor(bh, i, j);
+        for (int64_t c = 0; c < d; ++c) o[c] += pd * v[j * d + c];
+      }
     }
   }
   return 0;
@@ -364,12 +449,15 @@ int oracle_attention_forward_rows(const double* Q, const double* K, const double
 int oracle_attention_backward_dq_rows(const double* Q, const double* K, const double* V,
                                       const double* dO, int64_t B, int64_t H, int64_t N,
                                       int64_t d, double scale, int causal, int64_t left,
-                                      int64_t right, const uint8_t* blocks, int64_t R,
+                                      int64_t right, const uint8_t* blocks, double p_drop,
+                                      uint64_t seed, uint32_t offset, int64_t R,
                                       const int64_t* heads, const int64_t* rows,
                                       double* dQ_r, double* D_r) {
-  if (bad_shape(B, H, N, d) || R < 0 || (R > 0 && (!heads || !rows || !dQ_r || !D_r)))
+  if (bad_shape(B, H, N, d) || R < 0 || (R > 0 && (!heads || !rows || !dQ_r || !D_r)) ||
+      bad_dropout(p_drop))
     return 1;
   const Visibility vis = make_vis(N, causal, left, right, blocks);
+  const Dropout drop = make_dropout(p_drop, seed, offset);
   for (int64_t r = 0; r < R; ++r)
     if (heads[r] < 0 || heads[r] >= B * H || rows[r] < 0 || rows[r] >= N) return 1;
 #pragma omp parallel
@@ -387,8 +475,8 @@ int oracle_attention_backward_dq_rows(const double* Q, const double* K, const do
       for (int64_t j = 0; j < N; ++j) {
         double acc = 0.0;
         for (int64_t c = 0; c < d; ++c) acc += goi[c] * v[j * d + c];
-        dp[j] = acc;
-        Di += p[j] * acc;
+        dp[j] = acc * drop.factor(bh, i, j);
+        Di += p[j] * dp[j];
       }
       D_r[r] = Di;
       double* g = dQ_r + r * d;
@@ -412,13 +500,15 @@ int oracle_attention_backward_dq_rows(const double* Q, const double* K, const do
 int oracle_attention_backward_dkdv_rows(const double* Q, const double* K, const double* V,
                                         const double* dO, int64_t B, int64_t H, int64_t N,
                                         int64_t d, double scale, int causal, int64_t left,
-                                        int64_t right, const uint8_t* blocks, int64_t bh,
+                                        int64_t right, const uint8_t* blocks, double p_drop,
+                                        uint64_t seed, uint32_t offset, int64_t bh,
                                         const double* L, const double* D, int64_t R,
                                         const int64_t* keys, double* dK_r, double* dV_r) {
   if (bad_shape(B, H, N, d) || bh < 0 || bh >= B * H || R < 0 || !L || !D ||
-      (R > 0 && (!keys || !dK_r || !dV_r)))
+      (R > 0 && (!keys || !dK_r || !dV_r)) || bad_dropout(p_drop))
     return 1;
   const Visibility vis = make_vis(N, causal, left, right, blocks);
+  const Dropout drop = make_dropout(p_drop, seed, offset);
   for (int64_t r = 0; r < R; ++r)
     if (keys[r] < 0 || keys[r] >= N) return 1;
   const double* q = Q + bh * N * d;
@@ -446,9 +536,10 @@ int oracle_attention_backward_dkdv_rows(const double* Q, const double* K, const 
         dpij += goi[c] * vj[c];
       }
       const double pij = std::exp(scale * sij - L[i]);
-      const double dsij = pij * (dpij - D[i]);
+      const double f = drop.factor(bh, i, j);
+      const double dsij = pij * (dpij * f - D[i]);
       for (int64_t c = 0; c < d; ++c) {
-        gv[c] += pij * goi[c];
+        gv[c] += pij * f * goi[c];
         gk[c] += dsij * qi[c];
       }
     }

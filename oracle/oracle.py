@@ -28,7 +28,10 @@ Definitions followed (titles of the sources, see the header of attn_oracle.cpp):
     ``window=(left, right)`` (negative = unbounded side; None = no window) and
     ``block_mask`` (uint8 [ceil(N/128), ceil(N/128)], shared by all heads; None =
     every block); they combine with ``causal`` by AND. A row that sees no key has
-    O = 0, L = -inf and zero gradients.
+    O = 0, L = -inf and zero gradients;
+  * dropout on P ([jos] lists it among the fused operations), with the keep/drop
+    decision from Philox-4x32-10 (Salmon et al., "Parallel random numbers: as easy
+    as 1, 2, 3", SC 2011). ``dropout=(p, seed, offset)``; see attn_oracle.cpp.
 """
 from __future__ import annotations
 
@@ -50,6 +53,7 @@ _U8 = ctypes.POINTER(ctypes.c_uint8)
 _i64 = ctypes.c_int64
 _c = ctypes.c_int
 _MASK = [_c, _i64, _i64, _U8]  # causal, window left, window right, block mask
+_DROP = [ctypes.c_double, ctypes.c_uint64, ctypes.c_uint32]  # p, seed, offset
 
 BLOCK = 128  # block-mask granularity
 
@@ -65,6 +69,14 @@ def _mask(N: int, causal: bool, window, block_mask):
             raise ValueError(f"block_mask must be [{nb}, {nb}] for N={N}")
     ptr = blocks.ctypes.data_as(_U8) if blocks is not None else None
     return [int(bool(causal)), left, right, ptr], blocks
+
+
+def _drop(dropout):
+    """ctypes arguments of a dropout spec (p, seed, offset); None = no dropout."""
+    if dropout is None:
+        return [0.0, 0, 0]
+    p, seed, offset = dropout
+    return [float(p), int(seed) & ((1 << 64) - 1), int(offset) & 0xFFFFFFFF]
 
 
 def _compile(src: str, out: str) -> None:
@@ -122,16 +134,20 @@ class Oracle:
         f = ctypes.c_double
         lib.oracle_attention_probs.argtypes = [_D, _D, _i64, _i64, f] + _MASK + [_D]
         lib.oracle_attention_forward.argtypes = (
-            [_D, _D, _D, _i64, _i64, _i64, _i64, f] + _MASK + [_D, _D])
+            [_D, _D, _D, _i64, _i64, _i64, _i64, f] + _MASK + _DROP + [_D, _D])
         lib.oracle_attention_backward.argtypes = (
-            [_D, _D, _D, _D, _i64, _i64, _i64, _i64, f] + _MASK + [_D, _D, _D, _D, _D])
+            [_D, _D, _D, _D, _i64, _i64, _i64, _i64, f] + _MASK + _DROP + [_D, _D, _D, _D, _D])
         lib.oracle_attention_forward_rows.argtypes = (
-            [_D, _D, _D, _i64, _i64, _i64, _i64, f] + _MASK + [_i64, _I, _I, _D, _D])
+            [_D, _D, _D, _i64, _i64, _i64, _i64, f] + _MASK + _DROP + [_i64, _I, _I, _D, _D])
         lib.oracle_attention_backward_dq_rows.argtypes = (
-            [_D, _D, _D, _D, _i64, _i64, _i64, _i64, f] + _MASK + [_i64, _I, _I, _D, _D])
+            [_D, _D, _D, _D, _i64, _i64, _i64, _i64, f] + _MASK + _DROP
+            + [_i64, _I, _I, _D, _D])
         lib.oracle_attention_backward_dkdv_rows.argtypes = (
-            [_D, _D, _D, _D, _i64, _i64, _i64, _i64, f] + _MASK
+            [_D, _D, _D, _D, _i64, _i64, _i64, _i64, f] + _MASK + _DROP
             + [_i64, _D, _D, _i64, _I, _D, _D])
+        _U32 = ctypes.POINTER(ctypes.c_uint32)
+        lib.oracle_philox4x32_10.argtypes = [_U32, ctypes.c_uint32, ctypes.c_uint32, _U32]
+        lib.oracle_philox4x32_10.restype = None
         for name in ("oracle_attention_probs", "oracle_attention_forward",
                      "oracle_attention_backward", "oracle_attention_forward_rows",
                      "oracle_attention_backward_dq_rows",
@@ -168,7 +184,17 @@ class Oracle:
                "probs")
         return P
 
-    def forward(self, Q, K, V, scale: float, causal: bool, window=None, block_mask=None):
+    def philox(self, counter, key):
+        """Philox-4x32-10 of one counter (4 words) under one key (2 words)."""
+        ctr = np.ascontiguousarray(counter, dtype=np.uint32)
+        out = np.zeros(4, dtype=np.uint32)
+        U32 = ctypes.POINTER(ctypes.c_uint32)
+        self._lib.oracle_philox4x32_10(ctr.ctypes.data_as(U32), int(key[0]), int(key[1]),
+                                       out.ctypes.data_as(U32))
+        return out
+
+    def forward(self, Q, K, V, scale: float, causal: bool, window=None, block_mask=None,
+                dropout=None):
         """(O, L): O [B,H,N,d] fp64, L [B,H,N] fp64 natural-log log-sum-exp."""
         Q, K, V = _f64(Q), _f64(K), _f64(V)
         B, H, N, d = _shape4(Q)
@@ -176,11 +202,11 @@ class Oracle:
         L = np.empty((B, H, N), dtype=np.float64)
         m, keep = _mask(N, causal, window, block_mask)
         _check(self._lib.oracle_attention_forward(_p(Q), _p(K), _p(V), B, H, N, d, float(scale),
-                                                  *m, _p(O), _p(L)), "forward")
+                                                  *m, *_drop(dropout), _p(O), _p(L)), "forward")
         return O, L
 
     def backward(self, Q, K, V, dO, scale: float, causal: bool, with_check: bool = False,
-                 window=None, block_mask=None):
+                 window=None, block_mask=None, dropout=None):
         """(dQ, dK, dV, D[, Dcheck]) for the loss <dO, O>."""
         Q, K, V, dO = _f64(Q), _f64(K), _f64(V), _f64(dO)
         B, H, N, d = _shape4(Q)
@@ -189,12 +215,12 @@ class Oracle:
         Dc = np.empty((B, H, N), dtype=np.float64) if with_check else None
         m, keep = _mask(N, causal, window, block_mask)
         _check(self._lib.oracle_attention_backward(
-            _p(Q), _p(K), _p(V), _p(dO), B, H, N, d, float(scale), *m,
+            _p(Q), _p(K), _p(V), _p(dO), B, H, N, d, float(scale), *m, *_drop(dropout),
             _p(dQ), _p(dK), _p(dV), _p(D), _p(Dc) if with_check else None), "backward")
         return (dQ, dK, dV, D, Dc) if with_check else (dQ, dK, dV, D)
 
     def forward_rows(self, Q, K, V, scale: float, causal: bool, heads, rows, window=None,
-                     block_mask=None):
+                     block_mask=None, dropout=None):
         """O and L of selected (head, row) pairs, head = b * H + h: ([R, d], [R])."""
         Q, K, V = _f64(Q), _f64(K), _f64(V)
         B, H, N, d = _shape4(Q)
@@ -205,12 +231,12 @@ class Oracle:
         L = np.empty((R,), dtype=np.float64)
         m, keep = _mask(N, causal, window, block_mask)
         _check(self._lib.oracle_attention_forward_rows(
-            _p(Q), _p(K), _p(V), B, H, N, d, float(scale), *m, R, _pi(heads),
+            _p(Q), _p(K), _p(V), B, H, N, d, float(scale), *m, *_drop(dropout), R, _pi(heads),
             _pi(rows), _p(O), _p(L)), "forward_rows")
         return O, L
 
     def backward_dq_rows(self, Q, K, V, dO, scale: float, causal: bool, heads, rows,
-                         window=None, block_mask=None):
+                         window=None, block_mask=None, dropout=None):
         """dQ and D of selected (head, row) pairs: ([R, d], [R])."""
         Q, K, V, dO = _f64(Q), _f64(K), _f64(V), _f64(dO)
         B, H, N, d = _shape4(Q)
@@ -221,12 +247,12 @@ class Oracle:
         D = np.empty((R,), dtype=np.float64)
         m, keep = _mask(N, causal, window, block_mask)
         _check(self._lib.oracle_attention_backward_dq_rows(
-            _p(Q), _p(K), _p(V), _p(dO), B, H, N, d, float(scale), *m, R, _pi(heads),
-            _pi(rows), _p(dQ), _p(D)), "backward_dq_rows")
+            _p(Q), _p(K), _p(V), _p(dO), B, H, N, d, float(scale), *m, *_drop(dropout), R,
+            _pi(heads), _pi(rows), _p(dQ), _p(D)), "backward_dq_rows")
         return dQ, D
 
     def backward_dkdv_rows(self, Q, K, V, dO, scale: float, causal: bool, head: int, L_head,
-                           D_head, keys, window=None, block_mask=None):
+                           D_head, keys, window=None, block_mask=None, dropout=None):
         """dK and dV of selected key rows of one head, given that head's L and D as
         computed by this oracle (forward_rows / backward_dq_rows over all rows)."""
         Q, K, V, dO = _f64(Q), _f64(K), _f64(V), _f64(dO)
@@ -240,7 +266,7 @@ class Oracle:
         dV = np.empty((R, d), dtype=np.float64)
         m, keep = _mask(N, causal, window, block_mask)
         _check(self._lib.oracle_attention_backward_dkdv_rows(
-            _p(Q), _p(K), _p(V), _p(dO), B, H, N, d, float(scale), *m, int(head),
+            _p(Q), _p(K), _p(V), _p(dO), B, H, N, d, float(scale), *m, *_drop(dropout), int(head),
             _p(L_head), _p(D_head), R, _pi(keys), _p(dK), _p(dV)), "backward_dkdv_rows")
         return dK, dV
 

@@ -421,6 +421,141 @@ def pin_masked_finite_differences(orc):
                     f"window={window}, blocks={blocks}): {num:.6e} vs {grad[idx]:.6e}")
 
 
+# --------------------------------------------------------------------------- dropout
+#
+# Dropout on P ("A survey of key techniques of large language model pre-training
+# systems", p.218, lists it among the operations fused into the attention kernel):
+# Pd = P o Z / (1 - p). Z[i][j] = 0 iff word j % 4 of Philox-4x32-10 at counter
+# (j / 4, i, bh, offset) under key (seed low, seed high) is below floor(p * 2^32).
+
+# Philox-4x32-10 known-answer vectors published with the generator (Salmon, Moraes,
+# Dror and Shaw, "Parallel random numbers: as easy as 1, 2, 3", SC 2011; the Random123
+# distribution's known-answer tests): (counter, key, output).
+PHILOX_KAT = [
+    ((0x00000000, 0x00000000, 0x00000000, 0x00000000), (0x00000000, 0x00000000),
+     (0x6627e8d5, 0xe169c58d, 0xbc57ac4c, 0x9b00dbd8)),
+    ((0xffffffff, 0xffffffff, 0xffffffff, 0xffffffff), (0xffffffff, 0xffffffff),
+     (0x408f276d, 0x41c83b0e, 0xa20bc7c6, 0x6d5451fd)),
+    ((0x243f6a88, 0x85a308d3, 0x13198a2e, 0x03707344), (0xa4093822, 0x299f31d0),
+     (0xd16cfe09, 0x94fdcceb, 0x5001e420, 0x24126ea1)),
+]
+
+
+def philox_py(ctr, key):
+    """Philox-4x32-10 written out from its definition in the paper above."""
+    m = 0xFFFFFFFF
+    x0, x1, x2, x3 = ctr
+    k0, k1 = key
+    for r in range(10):
+        if r:
+            k0, k1 = (k0 + 0x9E3779B9) & m, (k1 + 0xBB67AE85) & m
+        a, b = 0xD2511F53 * x0, 0xCD9E8D57 * x2
+        x0, x1, x2, x3 = (b >> 32) ^ x1 ^ k0, b & m, (a >> 32) ^ x3 ^ k1, a & m
+    return (x0, x1, x2, x3)
+
+
+def dropout_keep(N, bh, p, seed, offset):
+    """Z of one head, [N, N] of 0/1, from philox_py."""
+    t = min(math.floor(p * 4294967296.0), 4294967295)
+    key = (seed & 0xFFFFFFFF, (seed >> 32) & 0xFFFFFFFF)
+    Z = np.zeros((N, N))
+    for i in range(N):
+        for j4 in range((N + 3) // 4):
+            w = philox_py((j4, i, bh, offset), key)
+            for u in range(4):
+                if 4 * j4 + u < N:
+                    Z[i, 4 * j4 + u] = 1.0 if w[u] >= t else 0.0
+    return Z
+
+
+def pin_philox_known_answers(orc):
+    """The oracle's Philox-4x32-10 reproduces the published known-answer vectors and
+    agrees with the definition written out here on random counters and keys."""
+    for ctr, key, want in PHILOX_KAT:
+        assert tuple(int(x) for x in orc.philox(ctr, key)) == want, f"Philox KAT {ctr}"
+        assert philox_py(ctr, key) == want
+    rng = _rng(31)
+    for _ in range(64):
+        ctr = tuple(int(x) for x in rng.integers(0, 2**32, 4))
+        key = tuple(int(x) for x in rng.integers(0, 2**32, 2))
+        assert tuple(int(x) for x in orc.philox(ctr, key)) == philox_py(ctr, key)
+
+
+def pin_dropout_reduces_to_softmax_and_generator(orc):
+    """With dropout, O = (P o Z / (1 - p)) V with P from the (pinned) softmax and Z from
+    the generator above, L is the logits' log-sum-exp without dropout, and p = 0 is
+    exactly no dropout."""
+    rng = _rng(32)
+    B, H, N, d = 1, 2, 37, 6
+    Q, K, V = (rng.standard_normal((B, H, N, d)) for _ in range(3))
+    for causal, p, seed, offset in ((False, 0.3, 0x1234_5678_9ABC_DEF0, 7),
+                                    (True, 0.75, 42, 0), (False, 0.05, 2**63 + 5, 2**31)):
+        O, L = orc.forward(Q, K, V, 0.6, causal, dropout=(p, seed, offset))
+        O0, L0 = orc.forward(Q, K, V, 0.6, causal)
+        _close(L, L0, 0.0, "L does not depend on dropout")
+        for bh in range(B * H):
+            P = orc.probs(Q[0, bh], K[0, bh], 0.6, causal)
+            Z = dropout_keep(N, bh, p, seed, offset)
+            _close(O[0, bh], (P * Z / (1.0 - p)) @ V[0, bh], 1e-13,
+                   f"dropout O (p={p}, head {bh})")
+    Op, Lp = orc.forward(Q, K, V, 0.6, True, dropout=(0.0, 99, 3))
+    Oz, Lz = orc.forward(Q, K, V, 0.6, True)
+    assert np.array_equal(Op, Oz) and np.array_equal(Lp, Lz), "p = 0 must be no dropout"
+
+
+def pin_dropout_keep_rate(orc):
+    """The kept fraction matches 1 - p within 5 binomial standard deviations, and
+    different offsets give different masks."""
+    N = 160
+    for p in (0.1, 0.5, 0.9):
+        Z = dropout_keep(N, 3, p, 2024, 11)
+        n = Z.size
+        sigma = math.sqrt(n * p * (1 - p))
+        assert abs(Z.sum() - n * (1 - p)) <= 5 * sigma, f"keep rate at p={p}"
+    # the oracle's masks: rows of P o Z are zero exactly where Z is
+    rng = _rng(33)
+    q = rng.standard_normal((1, 1, N, N)) * 0.1  # one head width d = N for Q, K and V
+    k = rng.standard_normal((1, 1, N, N)) * 0.1
+    eye = np.eye(N)[None, None]  # V = I exposes Pd itself as O
+    O1, _ = orc.forward(q, k, eye, 0.5, False, dropout=(0.5, 2024, 11))
+    O2, _ = orc.forward(q, k, eye, 0.5, False, dropout=(0.5, 2024, 12))
+    Z = dropout_keep(N, 0, 0.5, 2024, 11)
+    assert np.array_equal(O1[0, 0] != 0, Z != 0), "zeros of Pd are the dropped keys"
+    assert not np.array_equal(O1 != 0, O2 != 0), "offsets must change the mask"
+
+
+def pin_dropout_finite_differences(orc):
+    """Central differences of <dO, O> through dropout (Z fixed by the seed) at N <= 12,
+    and D = rowsum(dO o O) computed both ways."""
+    rng = _rng(34)
+    for N, d, causal, p in ((12, 3, False, 0.4), (9, 4, True, 0.2)):
+        Q, K, V, dO = (rng.standard_normal((1, 2, N, d)) for _ in range(4))
+        drop = (p, 77, 5)
+        dQ, dK, dV, D, Dc = orc.backward(Q, K, V, dO, 0.5, causal, with_check=True,
+                                         dropout=drop)
+        O, _ = orc.forward(Q, K, V, 0.5, causal, dropout=drop)
+        _close(D, np.sum(dO * O, axis=-1), 1e-12, "D = rowsum(dO o O) with dropout")
+        _close(D, Dc, 1e-12, "D two ways with dropout")
+
+        def loss(q, k, v):
+            o, _ = orc.forward(q, k, v, 0.5, causal, dropout=drop)
+            return float(np.sum(o * dO))
+
+        h = 1e-6
+        for which, grad in ((0, dQ), (1, dK), (2, dV)):
+            num = np.zeros_like(grad)
+            for idx in np.ndindex(*grad.shape):
+                ap = [Q.copy(), K.copy(), V.copy()]
+                am = [Q.copy(), K.copy(), V.copy()]
+                ap[which][idx] += h
+                am[which][idx] -= h
+                num[idx] = (loss(*ap) - loss(*am)) / (2 * h)
+            ref = max(1e-3, float(np.max(np.abs(num))))
+            err = float(np.max(np.abs(num - grad)))
+            assert err <= 1e-6 * ref, (
+                f"dropout finite differences of {'QKV'[which]} (N={N}, p={p}): {err:.3e}")
+
+
 # --------------------------------------------------------------------------- golden
 
 
@@ -461,4 +596,8 @@ ALL_PINS = [
     pin_masks_match_library,
     pin_window_closed_forms,
     pin_masked_finite_differences,
+    pin_philox_known_answers,
+    pin_dropout_reduces_to_softmax_and_generator,
+    pin_dropout_keep_rate,
+    pin_dropout_finite_differences,
 ]

@@ -22,6 +22,17 @@ MUTATIONS = [
      "if (left >= 0 && j < i - right) return false;"),
     ("block_mask_transposed", "blocks[(i / kBlock) * nb + j / kBlock]",
      "blocks[(j / kBlock) * nb + i / kBlock]"),
+    ("philox_wrong_multiplier", "static_cast<uint64_t>(0xD2511F53u) * x0",
+     "static_cast<uint64_t>(0xD2511F55u) * x0"),
+    ("philox_no_key_bump", "k0 += 0x9E3779B9u;", ""),
+    ("dropout_no_rescale", "return keep(bh, i, j) ? 1.0 / (1.0 - p) : 0.0;",
+     "return keep(bh, i, j) ? 1.0 : 0.0;"),
+    ("dropout_word_index", "return w[j % 4] >= threshold;", "return w[0] >= threshold;"),
+    ("dropout_counter_swapped", "static_cast<uint32_t>(j / 4), static_cast<uint32_t>(i),",
+     "static_cast<uint32_t>(i), static_cast<uint32_t>(j / 4),"),
+    ("dropout_dP_without_Z", "dsi[j] = acc * drop.factor(bh, i, j);", "dsi[j] = acc;"),
+    ("dropout_dV_without_Z", "const double p = P[i * N + j] * drop.factor(bh, i, j);",
+     "const double p = P[i * N + j];"),
     ("block_mask_ignored", "if (blocks && !blocks[(i / kBlock) * nb + j / kBlock]) return false;",
      ""),
     ("no_max_subtraction", "p[j] = std::exp(s[j] - m);", "p[j] = std::exp(s[j]);"),
@@ -36,7 +47,8 @@ MUTATIONS = [
     ("dK_without_scale", "for (int64_t c = 0; c < d; ++c) gkj[c] *= scale;", ""),
     ("dK_transposed_dS", "const double ds = dS[i * N + j];", "const double ds = dS[j * N + i];"),
     ("dV_from_dS", "gvj[c] += p * goi[c];", "gvj[c] += ds * goi[c];"),
-    ("dV_not_transposed", "const double p = P[i * N + j];", "const double p = P[j * N + i];"),
+    ("dV_not_transposed", "const double p = P[i * N + j] * drop.factor(bh, i, j);",
+     "const double p = P[j * N + i] * drop.factor(bh, i, j);"),
     ("dQ_uses_Q", "gqi[c] += dsi[j] * kj[c];", "gqi[c] += dsi[j] * q[j * d + c];"),
 ]
 

@@ -43,13 +43,14 @@ def test_row_functions_match_full_functions(orc):
 
 def test_row_functions_match_full_functions_with_masks(orc):
     """The same agreement under a sliding window and a block mask (one block row
-    empty, so some rows see no key)."""
+    empty, so some rows see no key), with and without dropout."""
     rng = np.random.default_rng(22)
     B, H, N, d = 1, 2, 260, 4
     Q, K, V, dO = (rng.standard_normal((B, H, N, d)) for _ in range(4))
     blocks = [[1, 0, 1], [1, 1, 0], [0, 0, 0]]
-    for causal, window in ((False, (40, 7)), (True, (90, -1))):
-        kw = dict(window=window, block_mask=blocks)
+    for causal, window, dropout in ((False, (40, 7), None), (True, (90, -1), None),
+                                    (False, (40, 7), (0.3, 1234, 9))):
+        kw = dict(window=window, block_mask=blocks, dropout=dropout)
         O, L = orc.forward(Q, K, V, 0.4, causal, **kw)
         dQ, dK, dV, D = orc.backward(Q, K, V, dO, 0.4, causal, **kw)
         heads = rng.integers(0, B * H, 30)
