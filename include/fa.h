@@ -193,6 +193,32 @@ fa_status fa_backward_masked(const void* Q, const void* K, const void* V, const 
                              void* workspace, size_t workspace_bytes, fa_stream_t stream);
 
 /*
+ * Masked attention with dropout on P (bf16): fa_forward_masked / fa_backward_masked
+ * plus dropout, one of the operations "A survey of key techniques of large language
+ * model pre-training systems" (Journal of Software 2026(1), p.218) lists as fused
+ * into the attention kernel. With drop probability p_drop in [0, 1):
+ *   Pd = P o Z / (1 - p_drop),  O = Pd V,  LSE = the log-sum-exp of the logits
+ *   (unchanged by dropout); the backward regenerates Z, so nothing N x N is stored.
+ * Z[i][j] = 0 iff word (j mod 4) of Philox-4x32-10 (Salmon, Moraes, Dror and Shaw,
+ * "Parallel random numbers: as easy as 1, 2, 3", SC 2011) at counter
+ * (j / 4, i, b * H + h, offset) under key (seed & 0xffffffff, seed >> 32) is below
+ * min(floor(p_drop * 2^32), 2^32 - 1). `offset` lets successive calls draw
+ * independent masks under one seed. The backward must be given the same seed,
+ * offset, p_drop and masks as the forward. p_drop = 0 is no dropout; p_drop outside
+ * [0, 1) (or NaN) is FA_ERR_INVALID_ARG.
+ */
+fa_status fa_forward_dropout(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                             int B, int H, int N, int d, float scale, int causal,
+                             int window_left, int window_right, const uint8_t* block_mask,
+                             float p_drop, uint64_t seed, uint32_t offset, fa_stream_t stream);
+fa_status fa_backward_dropout(const void* Q, const void* K, const void* V, const void* O,
+                              const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
+                              int B, int H, int N, int d, float scale, int causal,
+                              int window_left, int window_right, const uint8_t* block_mask,
+                              float p_drop, uint64_t seed, uint32_t offset, void* workspace,
+                              size_t workspace_bytes, fa_stream_t stream);
+
+/*
  * fp32 entry points: the same operation and arguments with fp32 tensors
  * (float [B,H,N,d]), computed in fp32 on the CUDA cores (FFMA), for callers that
  * need fp32 accuracy; tensor-core fp32 (tf32) cannot reach it. The backward is

@@ -16,6 +16,7 @@ FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = ran
 
 # name -> (restype, argtypes), exactly the declarations of include/fa.h
 _vp, _i, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+_u32, _u64 = ctypes.c_uint32, ctypes.c_uint64
 SIGNATURES = {
     "fa_forward": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp]),
     "fa_backward_workspace_size": (_sz, [_i, _i, _i, _i]),
@@ -34,6 +35,11 @@ SIGNATURES = {
                                _vp]),
     "fa_backward_masked": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                 _i, _i, _i, _i, _f, _i, _i, _i, _vp, _vp, _sz, _vp]),
+    "fa_forward_dropout": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _i, _i, _vp,
+                                _f, _u64, _u32, _vp]),
+    "fa_backward_dropout": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                 _i, _i, _i, _i, _f, _i, _i, _i, _vp, _f, _u64, _u32,
+                                 _vp, _sz, _vp]),
     "fa_forward_f32": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp]),
     "fa_backward_f32": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                              _i, _i, _i, _i, _f, _i, _vp, _sz, _vp]),

@@ -25,7 +25,7 @@ __all__ = [
     "FAError", "fa_forward", "fa_backward", "fa_backward_workspace_size",
     "fa_backward_preprocess", "fa_backward_main", "fa_backward_dq_convert",
     "fa_backward_noalloc", "fa_forward_f16", "fa_backward_f16", "fa_forward_masked",
-    "fa_backward_masked", "fa_forward_f32",
+    "fa_backward_masked", "fa_forward_dropout", "fa_backward_dropout", "fa_forward_f32",
     "fa_backward_f32", "fa_get_status", "fa_watchdog_selftest", "fa_version",
     "forward", "backward", "attention", "FlashAttentionFunction",
 ]
@@ -129,6 +129,37 @@ def fa_backward_masked(Q, K, V, O, dO, LSE, dQ, dK, dV, scale: float, causal: bo
     check("fa_backward_masked", lib().fa_backward_masked(
         *ptrs, B, H, N, d, float(scale), int(bool(causal)), wl, wr, _block_mask(block_mask, N),
         ws, nbytes, _stream(stream)))
+
+
+def _dropout(dropout):
+    if dropout is None:
+        return 0.0, 0, 0
+    p, seed, offset = dropout
+    return float(p), int(seed) & ((1 << 64) - 1), int(offset) & 0xFFFFFFFF
+
+
+def fa_forward_dropout(Q, K, V, O, LSE, scale: float, causal: bool, dropout, window=None,
+                       block_mask=None, stream=None) -> None:
+    """fa_forward_masked with dropout=(p, seed, offset) on P (Philox-4x32-10 mask)."""
+    B, H, N, d = _shape(Q)
+    bf = torch.bfloat16
+    args = [_need("Q", Q, bf, (B, H, N, d)), _need("K", K, bf, (B, H, N, d)),
+            _need("V", V, bf, (B, H, N, d)), _need("O", O, bf, (B, H, N, d)),
+            _need("LSE", LSE, torch.float32, (B, H, N))]
+    wl, wr = _window(window)
+    check("fa_forward_dropout", lib().fa_forward_dropout(
+        *args, B, H, N, d, float(scale), int(bool(causal)), wl, wr, _block_mask(block_mask, N),
+        *_dropout(dropout), _stream(stream)))
+
+
+def fa_backward_dropout(Q, K, V, O, dO, LSE, dQ, dK, dV, scale: float, causal: bool, workspace,
+                        dropout, window=None, block_mask=None, stream=None) -> None:
+    ptrs, (B, H, N, d), ws, nbytes = _bwd_args(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace,
+                                               torch.bfloat16)
+    wl, wr = _window(window)
+    check("fa_backward_dropout", lib().fa_backward_dropout(
+        *ptrs, B, H, N, d, float(scale), int(bool(causal)), wl, wr, _block_mask(block_mask, N),
+        *_dropout(dropout), ws, nbytes, _stream(stream)))
 
 
 def fa_forward_f32(Q, K, V, O, LSE, scale: float, causal: bool, stream=None) -> None:

@@ -109,6 +109,7 @@ struct Params {
   int wl;                 // keys j >= i - wl are kept; < 0: no left bound
   int wr;                 // keys j <= i + wr are kept; < 0: no right bound (causal: 0)
   const uint8_t* blocks;  // [n_kt x n_kt] block mask (nonzero = kept), or null
+  DropoutParams drop;     // used by the kDropout instances only
   unsigned long long timeout_ns;
 };
 
@@ -248,7 +249,7 @@ __global__ void __launch_bounds__(256)
 
 // ------------------------------------------------------------------ main kernel
 
-template <int D, Elt E, bool kMasked>
+template <int D, Elt E, bool kMasked, bool kDropout = false>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -514,8 +515,24 @@ __global__ void __launch_bounds__(kThreads, 1)
               const int k = 4 * v + e;
               float pe = ex2_approx(fmaf(__uint_as_float(sv[cur][k]), c, -Ls[e]));
               if (kM && static_cast<unsigned>(qoff + cc * 16 + k) >= q_span) pe = 0.f;
-              pv[e] = pe;
-              dsv[e] = pe * (__uint_as_float(dv[cur][k]) - Ds[e]);
+              if constexpr (kDropout) {
+                // Z for (query qh0 + 16cc + k, this key): word (key mod 4) of the counter
+                // (key / 4, query, bh, offset); dV takes P o Z / (1 - p) and
+                // dS = P o (dP o Z / (1 - p) - D)
+                const uint4 w = philox4x32_10(
+                    make_uint4(static_cast<uint32_t>(key >> 2),
+                               static_cast<uint32_t>(qh0 + cc * 16 + k), static_cast<uint32_t>(bh),
+                               p.drop.offset),
+                    p.drop.seed_lo, p.drop.seed_hi);
+                const int wsel = key & 3;
+                const uint32_t word = wsel == 0 ? w.x : wsel == 1 ? w.y : wsel == 2 ? w.z : w.w;
+                const float zs = (word >= p.drop.threshold) ? p.drop.scale : 0.0f;
+                pv[e] = pe * zs;
+                dsv[e] = pe * (__uint_as_float(dv[cur][k]) * zs - Ds[e]);
+              } else {
+                pv[e] = pe;
+                dsv[e] = pe * (__uint_as_float(dv[cur][k]) - Ds[e]);
+              }
             }
             pk[2 * v] = pack2<E>(pv[0], pv[1]);
             pk[2 * v + 1] = pack2<E>(pv[2], pv[3]);

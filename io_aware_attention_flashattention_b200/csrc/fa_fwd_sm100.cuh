@@ -101,6 +101,7 @@ struct Params {
   int wr;            // keys j <= i + wr are kept; < 0: no right bound (causal: 0)
   const uint8_t* blocks;  // [n_kt x n_kt] block mask (nonzero = kept), or null
   int n_kt;               // ceil(N / 128)
+  DropoutParams drop;     // used by the kDropout instances only
   unsigned long long timeout_ns;
 };
 
@@ -142,7 +143,7 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
   }
 }
 
-template <int D, Elt E, bool kMasked>
+template <int D, Elt E, bool kMasked, bool kDropout = false>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const Params p) {
@@ -449,6 +450,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float2 c2 = make_float2(c, c), nm2 = make_float2(-m_use, -m_use);
       float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                        make_float2(0.f, 0.f)};
+      uint4 rnd = make_uint4(0u, 0u, 0u, 0u);  // Philox words of the current 4 keys (dropout)
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         uint32_t pk[16];
@@ -462,7 +464,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             pe = make_float2(ex2_approx(x.x), ex2_approx(x.y));
           }
-          acc[k & 3] = fadd2(acc[k & 3], pe);
+          acc[k & 3] = fadd2(acc[k & 3], pe);  // l is the sum before dropout
+          if constexpr (kDropout) {
+            // keys kv0 + 32cc + 2k, +1: words (2k mod 4), +1 of the counter for the four
+            // keys starting at kv0 + 32cc + 4(k / 2)
+            if ((k & 1) == 0)
+              rnd = philox4x32_10(make_uint4(static_cast<uint32_t>((kv0 + 32 * cc + 2 * k) >> 2),
+                                             static_cast<uint32_t>(row), static_cast<uint32_t>(bh),
+                                             p.drop.offset),
+                                  p.drop.seed_lo, p.drop.seed_hi);
+            const uint32_t wa = (k & 1) ? rnd.z : rnd.x, wb = (k & 1) ? rnd.w : rnd.y;
+            pe.x = (wa >= p.drop.threshold) ? pe.x * p.drop.scale : 0.0f;
+            pe.y = (wb >= p.drop.threshold) ? pe.y * p.drop.scale : 0.0f;
+          }
           pk[k] = pack2<E>(pe.x, pe.y);
         }
         // keys 32cc..32cc+31 = 16-byte units 4cc..4cc+3 of this row's 256 bytes:

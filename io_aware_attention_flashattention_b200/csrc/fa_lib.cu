@@ -95,8 +95,15 @@ cudaError_t set_smem_d() {
 
 template <Elt E>
 cudaError_t set_smem_all() {
-  const cudaError_t e = set_smem_d<64, E>();
-  return e ? e : set_smem_d<128, E>();
+  cudaError_t e = set_smem_d<64, E>();
+  e = e ? e : set_smem_d<128, E>();
+  if constexpr (E == Elt::BF16) {  // dropout instances (bf16, general masks)
+    e = e ? e : set_smem(fwd::fa_fwd_kernel<64, E, true, true>, fwd::Cfg<64>::kSmemBytes);
+    e = e ? e : set_smem(fwd::fa_fwd_kernel<128, E, true, true>, fwd::Cfg<128>::kSmemBytes);
+    e = e ? e : set_smem(bwd::fa_bwd_kernel<64, E, true, true>, bwd::Cfg<64>::kSmemBytes);
+    e = e ? e : set_smem(bwd::fa_bwd_kernel<128, E, true, true>, bwd::Cfg<128>::kSmemBytes);
+  }
+  return e;
 }
 
 // Checks that the current device is an sm_100 part and sets the kernels'
@@ -190,6 +197,26 @@ fa_status make_mask(int N, int causal, int window_left, int window_right,
   return FA_OK;
 }
 
+// Dropout as the kernels take it: keep iff the Philox word >= threshold, where
+// threshold = min(floor(p * 2^32), 2^32 - 1); kept values scaled by 1 / (1 - p).
+struct DropSpec {
+  bool on = false;
+  DropoutParams params{};
+};
+
+fa_status make_drop(float p_drop, uint64_t seed, uint32_t offset, DropSpec* d) {
+  if (!(p_drop >= 0.0f && p_drop < 1.0f)) return FA_ERR_INVALID_ARG;
+  d->on = p_drop > 0.0f;
+  double t = std::floor(static_cast<double>(p_drop) * 4294967296.0);
+  if (t > 4294967295.0) t = 4294967295.0;
+  d->params.threshold = static_cast<uint32_t>(t);
+  d->params.scale = static_cast<float>(1.0 / (1.0 - static_cast<double>(p_drop)));
+  d->params.seed_lo = static_cast<uint32_t>(seed);
+  d->params.seed_hi = static_cast<uint32_t>(seed >> 32);
+  d->params.offset = offset;
+  return FA_OK;
+}
+
 fa_status launch_status() {
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -207,7 +234,7 @@ namespace {
 template <Elt E>
 fa_status forward_impl(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
                      int H, int N, int d, float scale, int causal, const MaskSpec& mask,
-                     fa_stream_t stream) {
+                     const DropSpec& drop, fa_stream_t stream) {
   fa_status st = check_shape(B, H, N, d, scale, causal);
   if (st != FA_OK) return st;
   if (N == 0) return FA_OK;
@@ -229,10 +256,24 @@ fa_status forward_impl(const void* Q, const void* K, const void* V, void* O, flo
   p.wr = mask.wr;
   p.blocks = mask.blocks;
   p.n_kt = (N + fwd::BN - 1) / fwd::BN;
+  p.drop = drop.params;
   p.timeout_ns = watchdog_ns();
   const dim3 grid(static_cast<unsigned>(p.n_qblk) * BH);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool g = mask.general();
+  if constexpr (E == Elt::BF16) {
+    if (drop.on) {
+      if (d == 64)
+        fwd::fa_fwd_kernel<64, E, true, true><<<grid, fwd::kThreads, fwd::Cfg<64>::kSmemBytes, s>>>(
+            mq, mk, mv, p);
+      else
+        fwd::fa_fwd_kernel<128, E, true, true><<<grid, fwd::kThreads, fwd::Cfg<128>::kSmemBytes, s>>>(
+            mq, mk, mv, p);
+      return launch_status();
+    }
+  } else if (drop.on) {
+    return FA_ERR_UNSUPPORTED;
+  }
   if (d == 64 && !g)
     fwd::fa_fwd_kernel<64, E, false><<<grid, fwd::kThreads, fwd::Cfg<64>::kSmemBytes, s>>>(mq, mk, mv, p);
   else if (d == 64)
@@ -302,8 +343,8 @@ fa_status preprocess_impl(const void* O, const void* dO, const float* LSE, int B
 template <Elt E>
 fa_status main_impl(const void* Q, const void* K, const void* V, const void* dO, void* dK,
                            void* dV, int B, int H, int N, int d, float scale, int causal,
-                           const MaskSpec& mask, void* workspace, size_t workspace_bytes,
-                           fa_stream_t stream) {
+                           const MaskSpec& mask, const DropSpec& drop, void* workspace,
+                           size_t workspace_bytes, fa_stream_t stream) {
   const void* ptrs[] = {Q, K, V, dO, dK, dV};
   BwdPlan pl;
   fa_status st = bwd_plan(ptrs, 6, B, H, N, d, scale, causal, workspace, workspace_bytes, &pl);
@@ -327,11 +368,25 @@ fa_status main_impl(const void* Q, const void* K, const void* V, const void* dO,
   p.wl = mask.wl;
   p.wr = mask.wr;
   p.blocks = mask.blocks;
+  p.drop = drop.params;
   p.timeout_ns = watchdog_ns();
   const dim3 grid(static_cast<unsigned>(pl.Npad / bwd::BN) * pl.BH);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool g = mask.general();
   using bwd::Cfg;
+  if constexpr (E == Elt::BF16) {
+    if (drop.on) {
+      if (d == 64)
+        bwd::fa_bwd_kernel<64, E, true, true><<<grid, bwd::kThreads, Cfg<64>::kSmemBytes, s>>>(
+            mq, mk, mv, mdo, p);
+      else
+        bwd::fa_bwd_kernel<128, E, true, true><<<grid, bwd::kThreads, Cfg<128>::kSmemBytes, s>>>(
+            mq, mk, mv, mdo, p);
+      return launch_status();
+    }
+  } else if (drop.on) {
+    return FA_ERR_UNSUPPORTED;
+  }
   if (d == 64 && !g)
     bwd::fa_bwd_kernel<64, E, false><<<grid, bwd::kThreads, Cfg<64>::kSmemBytes, s>>>(mq, mk, mv, mdo, p);
   else if (d == 64)
@@ -363,15 +418,15 @@ fa_status dq_convert_impl(void* dQ, int B, int H, int N, int d, float scale, voi
 template <Elt E>
 fa_status backward_impl(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                       const float* LSE, void* dQ, void* dK, void* dV, int B, int H, int N, int d,
-                      float scale, int causal, const MaskSpec& mask, void* workspace,
-                      size_t workspace_bytes, fa_stream_t stream) {
+                      float scale, int causal, const MaskSpec& mask, const DropSpec& drop,
+                      void* workspace, size_t workspace_bytes, fa_stream_t stream) {
   const void* ptrs[] = {Q, K, V, O, dO, LSE, dQ, dK, dV};
   BwdPlan pl;
   fa_status st = bwd_plan(ptrs, 9, B, H, N, d, scale, causal, workspace, workspace_bytes, &pl);
   if (st != FA_OK || N == 0) return st;
   st = preprocess_impl<E>(O, dO, LSE, B, H, N, d, scale, causal, workspace, workspace_bytes, stream);
   if (st != FA_OK) return st;
-  st = main_impl<E>(Q, K, V, dO, dK, dV, B, H, N, d, scale, causal, mask, workspace,
+  st = main_impl<E>(Q, K, V, dO, dK, dV, B, H, N, d, scale, causal, mask, drop, workspace,
                     workspace_bytes, stream);
   if (st != FA_OK) return st;
   return dq_convert_impl<E>(dQ, B, H, N, d, scale, workspace, workspace_bytes, stream);
@@ -428,14 +483,14 @@ fa_status fa_forward(const void* Q, const void* K, const void* V, void* O, float
                      int H, int N, int d, float scale, int causal, fa_stream_t stream) {
   MaskSpec m;
   make_mask(N, causal, -1, -1, nullptr, &m);
-  return forward_impl<Elt::BF16>(Q, K, V, O, LSE, B, H, N, d, scale, causal, m, stream);
+  return forward_impl<Elt::BF16>(Q, K, V, O, LSE, B, H, N, d, scale, causal, m, DropSpec{}, stream);
 }
 
 fa_status fa_forward_f16(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
                          int H, int N, int d, float scale, int causal, fa_stream_t stream) {
   MaskSpec m;
   make_mask(N, causal, -1, -1, nullptr, &m);
-  return forward_impl<Elt::F16>(Q, K, V, O, LSE, B, H, N, d, scale, causal, m, stream);
+  return forward_impl<Elt::F16>(Q, K, V, O, LSE, B, H, N, d, scale, causal, m, DropSpec{}, stream);
 }
 
 fa_status fa_forward_masked(const void* Q, const void* K, const void* V, void* O, float* LSE,
@@ -445,7 +500,7 @@ fa_status fa_forward_masked(const void* Q, const void* K, const void* V, void* O
   MaskSpec m;
   const fa_status st = make_mask(N, causal, window_left, window_right, block_mask, &m);
   if (st != FA_OK) return st;
-  return forward_impl<Elt::BF16>(Q, K, V, O, LSE, B, H, N, d, scale, causal, m, stream);
+  return forward_impl<Elt::BF16>(Q, K, V, O, LSE, B, H, N, d, scale, causal, m, DropSpec{}, stream);
 }
 
 fa_status fa_backward_preprocess(const void* O, const void* dO, const float* LSE, int B, int H,
@@ -460,8 +515,8 @@ fa_status fa_backward_main(const void* Q, const void* K, const void* V, const vo
                            void* workspace, size_t workspace_bytes, fa_stream_t stream) {
   MaskSpec m;
   make_mask(N, causal, -1, -1, nullptr, &m);
-  return main_impl<Elt::BF16>(Q, K, V, dO, dK, dV, B, H, N, d, scale, causal, m, workspace,
-                              workspace_bytes, stream);
+  return main_impl<Elt::BF16>(Q, K, V, dO, dK, dV, B, H, N, d, scale, causal, m, DropSpec{},
+                              workspace, workspace_bytes, stream);
 }
 
 fa_status fa_backward_dq_convert(void* dQ, int B, int H, int N, int d, float scale, void* workspace,
@@ -476,7 +531,7 @@ fa_status fa_backward(const void* Q, const void* K, const void* V, const void* O
   MaskSpec m;
   make_mask(N, causal, -1, -1, nullptr, &m);
   return backward_impl<Elt::BF16>(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, scale, causal, m,
-                                  workspace, workspace_bytes, stream);
+                                  DropSpec{}, workspace, workspace_bytes, stream);
 }
 
 fa_status fa_backward_masked(const void* Q, const void* K, const void* V, const void* O,
@@ -488,7 +543,7 @@ fa_status fa_backward_masked(const void* Q, const void* K, const void* V, const 
   const fa_status st = make_mask(N, causal, window_left, window_right, block_mask, &m);
   if (st != FA_OK) return st;
   return backward_impl<Elt::BF16>(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, scale, causal, m,
-                                  workspace, workspace_bytes, stream);
+                                  DropSpec{}, workspace, workspace_bytes, stream);
 }
 
 fa_status fa_backward_f16(const void* Q, const void* K, const void* V, const void* O,
@@ -498,7 +553,7 @@ fa_status fa_backward_f16(const void* Q, const void* K, const void* V, const voi
   MaskSpec m;
   make_mask(N, causal, -1, -1, nullptr, &m);
   return backward_impl<Elt::F16>(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, scale, causal, m,
-                                 workspace, workspace_bytes, stream);
+                                 DropSpec{}, workspace, workspace_bytes, stream);
 }
 
 // ---------------------------------------------------------------- backward without allocation
@@ -545,6 +600,33 @@ fa_status fa_backward_noalloc(const void* Q, const void* K, const void* V, const
   // left in the array does not matter.
   return fa_backward(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, scale, causal, scratch,
                      kNoAllocScratchBytes, stream);
+}
+
+fa_status fa_forward_dropout(const void* Q, const void* K, const void* V, void* O, float* LSE,
+                             int B, int H, int N, int d, float scale, int causal,
+                             int window_left, int window_right, const uint8_t* block_mask,
+                             float p_drop, uint64_t seed, uint32_t offset, fa_stream_t stream) {
+  MaskSpec m;
+  DropSpec dr;
+  fa_status st = make_drop(p_drop, seed, offset, &dr);
+  if (st != FA_OK) return st;
+  if ((st = make_mask(N, causal, window_left, window_right, block_mask, &m)) != FA_OK) return st;
+  return forward_impl<Elt::BF16>(Q, K, V, O, LSE, B, H, N, d, scale, causal, m, dr, stream);
+}
+
+fa_status fa_backward_dropout(const void* Q, const void* K, const void* V, const void* O,
+                              const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
+                              int B, int H, int N, int d, float scale, int causal,
+                              int window_left, int window_right, const uint8_t* block_mask,
+                              float p_drop, uint64_t seed, uint32_t offset, void* workspace,
+                              size_t workspace_bytes, fa_stream_t stream) {
+  MaskSpec m;
+  DropSpec dr;
+  fa_status st = make_drop(p_drop, seed, offset, &dr);
+  if (st != FA_OK) return st;
+  if ((st = make_mask(N, causal, window_left, window_right, block_mask, &m)) != FA_OK) return st;
+  return backward_impl<Elt::BF16>(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, scale, causal, m,
+                                  dr, workspace, workspace_bytes, stream);
 }
 
 fa_status fa_forward_f32(const float* Q, const float* K, const float* V, float* O, float* LSE,

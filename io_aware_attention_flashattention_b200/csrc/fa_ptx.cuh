@@ -434,4 +434,32 @@ __device__ __forceinline__ float2 unpack2(uint32_t w) {
   }
 }
 
+// ---------------------------------------------------------------- dropout RNG
+
+// Philox-4x32-10, the counter-based generator of Salmon, Moraes, Dror and Shaw
+// ("Parallel random numbers: as easy as 1, 2, 3", SC 2011): in each of ten rounds the
+// words 0 and 2 are multiplied by the two round constants, the high halves of the
+// products are mixed with words 1 and 3 and the round key, and the words are
+// permuted; the key advances by the two Weyl constants between rounds.
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    const uint32_t lo0 = 0xD2511F53u * c.x, hi0 = __umulhi(0xD2511F53u, c.x);
+    const uint32_t lo1 = 0xCD9E8D57u * c.z, hi1 = __umulhi(0xCD9E8D57u, c.z);
+    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+    k0 += 0x9E3779B9u;
+    k1 += 0xBB67AE85u;
+  }
+  return c;
+}
+
+// Dropout on P: key j of query row i in head bh is kept iff word (j mod 4) of
+// philox4x32_10((j / 4, i, bh, offset), seed) is at least `threshold`
+// (= floor(p * 2^32)); kept values are scaled by 1 / (1 - p).
+struct DropoutParams {
+  uint32_t threshold;
+  float scale;
+  uint32_t seed_lo, seed_hi, offset;
+};
+
 }  // namespace fa
