@@ -95,7 +95,13 @@ struct Params {
   float* LSE;
   int N;
   int BH;
-  int n_qblk;        // ceil(N / 256)
+  // Work split: per head, pairs_ph CTAs own two consecutive query tiles each (tiles
+  // [singles_ph, n_qt)) and singles_ph CTAs own one (tiles [0, singles_ph)). All pair
+  // CTAs (n_pair_ctas = BH * pairs_ph) come first in the grid, so the single-tile
+  // CTAs (half the work) fill the last, partial wave.
+  int pairs_ph;
+  int singles_ph;
+  int n_pair_ctas;
   float scale_log2;  // scale * log2(e)
   int wl;            // keys j >= i - wl are kept; < 0: no left bound
   int wr;            // keys j <= i + wr are kept; < 0: no right bound (causal: 0)
@@ -166,11 +172,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint8_t* const blocks = kMasked ? p.blocks : nullptr;
 
   // Work item: head-major, so that the CTAs resident at any time cover about two
-  // heads and their K/V stay in L2; within a head the heaviest query blocks (causal)
-  // go first.
-  const int bh = static_cast<int>(blockIdx.x) / p.n_qblk;
-  const int qb = (p.n_qblk - 1) - static_cast<int>(blockIdx.x) % p.n_qblk;
-  const int q0 = qb * 2 * BM;
+  // heads and their K/V stay in L2; within a head the heaviest query tiles (causal)
+  // go first. Single-tile CTAs, on the lightest tiles, come after all pairs.
+  int bh, qt0;
+  bool own1;  // does this CTA own query tile 1 (qt0 + 1)?
+  if (static_cast<int>(blockIdx.x) < p.n_pair_ctas) {
+    const int c = static_cast<int>(blockIdx.x);
+    bh = c / p.pairs_ph;
+    qt0 = p.singles_ph + 2 * (p.pairs_ph - 1 - c % p.pairs_ph);
+    own1 = true;
+  } else {
+    const int c = static_cast<int>(blockIdx.x) - p.n_pair_ctas;
+    bh = c / p.singles_ph;
+    qt0 = p.singles_ph - 1 - c % p.singles_ph;
+    own1 = false;
+  }
+  const int q0 = qt0 * BM;
   const int n_kt = p.n_kt;
   // key tiles [lo[t], hi[t]) hold every key a row of query tile t may see
   int lo[2], hi[2];
@@ -179,7 +196,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r0 = q0 + t * BM, r1 = min(r0 + BM, p.N) - 1;
     lo[t] = (wl < 0) ? 0 : max(0, r0 - wl) / BN;
     hi[t] = (wr < 0) ? n_kt : min(n_kt, (r1 + wr) / BN + 1);
-    if (r0 >= p.N) lo[t] = hi[t] = 0;
+    if (r0 >= p.N || (t == 1 && !own1)) lo[t] = hi[t] = 0;
   }
   // The CTA's key tiles: the union of both ranges (contiguous: lo[1] <= hi[0]).
   const int kt_lo = (hi[0] > lo[0]) ? lo[0] : lo[1];
@@ -192,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nwords = (n_kt + 31) / 32;
     for (int w = warp; w < 2 * nwords; w += kThreads / 32) {
       const int t = w / nwords, wi = w % nwords;
-      const int qt = min(2 * qb + t, n_kt - 1);
+      const int qt = min(qt0 + t, n_kt - 1);
       const int kt = wi * 32 + lane;
       const bool keep = kt < n_kt && blocks[static_cast<size_t>(qt) * n_kt + kt] != 0;
       const uint32_t bits = __ballot_sync(0xffffffffu, keep);
@@ -509,7 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok && t_nk > 0)
       ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarPVDone + t), (t_nk - 1) & 1, wd));
-    if (t_nk == 0 && row < p.N) {
+    if (t_nk == 0 && row < p.N && (t == 0 || own1)) {
       // a query tile that sees no key: O = 0, LSE = -inf
       uint4* dst = reinterpret_cast<uint4*>(p.O + (static_cast<size_t>(bh) * p.N + row) * D);
 #pragma unroll

@@ -12,7 +12,11 @@
 #include <cstdint>
 #include <algorithm>
 #include <cstdlib>
+#include <map>
 #include <mutex>
+#include <queue>
+#include <tuple>
+#include <vector>
 
 #include "fa_ptx.cuh"
 #include "fa_fwd_sm100.cuh"
@@ -74,6 +78,7 @@ struct DeviceState {
   bool checked = false;
   bool supported = false;
   bool attrs_done = false;
+  int sms = 0;  // streaming multiprocessors
 };
 DeviceState g_devices[kMaxDevices];
 std::mutex g_mutex;
@@ -119,6 +124,8 @@ fa_status prepare_device() {
         cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
       return FA_ERR_CUDA;
     st.supported = (major == 10 && minor == 0);
+    if (cudaDeviceGetAttribute(&st.sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      return FA_ERR_CUDA;
     st.checked = true;
   }
   if (!st.supported) return FA_ERR_UNSUPPORTED;
@@ -217,6 +224,86 @@ fa_status make_drop(float p_drop, uint64_t seed, uint32_t offset, DropSpec* d) {
   return FA_OK;
 }
 
+// ---------------------------------------------------------------- forward work split
+//
+// The forward CTA owns two query tiles (they share every K/V tile it loads). With
+// one CTA per SM, B*H*ceil(N/256) such CTAs often leave the last wave of the grid
+// mostly empty (B1 H8 N16384: 512 CTAs on 148 SMs = 3.46 waves). So per head the
+// lightest `singles` query tiles get a CTA of their own, launched after all pair
+// CTAs, where they fill that last wave at about half the cost of a pair. The split
+// is chosen by simulating the launch: CTAs start in grid order on the first free SM;
+// a pair costs the larger key-tile count of its two tiles, a single 0.74 of its own
+// (measured on B1 H8 N16384 d128: 1024 single-tile CTAs run at 0.77x the rate of
+// 512 pair CTAs). Cached per shape.
+struct FwdSplit {
+  int pairs_ph, singles_ph;
+};
+
+double split_makespan(int BH, int n_qt, int singles, int sms,
+                      const std::vector<int>& key_tiles) {
+  std::priority_queue<double, std::vector<double>, std::greater<double>> free_at;
+  for (int i = 0; i < sms; ++i) free_at.push(0.0);
+  double end = 0.0;
+  auto run = [&](double cost) {
+    const double t = free_at.top() + cost;
+    free_at.pop();
+    free_at.push(t);
+    end = std::max(end, t);
+  };
+  const int pairs = (n_qt - singles) / 2;
+  for (int h = 0; h < BH; ++h)
+    for (int k = pairs - 1; k >= 0; --k) {
+      const int t0 = singles + 2 * k;
+      run(std::max(key_tiles[t0], key_tiles[t0 + 1]));
+    }
+  for (int h = 0; h < BH; ++h)
+    for (int t = singles - 1; t >= 0; --t) run(0.74 * key_tiles[t]);
+  return end;
+}
+
+FwdSplit fwd_split(int BH, int N, int wl, int wr, int sms) {
+  const int n_qt = (N + fwd::BM - 1) / fwd::BM;
+  const int n_kt = (N + fwd::BN - 1) / fwd::BN;
+  const int min_singles = n_qt % 2;
+  FwdSplit plain{(n_qt - min_singles) / 2, min_singles};
+  if (sms <= 0 || static_cast<long long>(BH) * n_qt > 65536) return plain;
+  static std::mutex mu;
+  static std::map<std::tuple<int, int, int, int, int>, FwdSplit> cache;
+  const auto key = std::make_tuple(BH, N, wl, wr, sms);
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+  }
+  // key tiles each query tile walks (window and causal; a block mask is ignored here)
+  std::vector<int> key_tiles(n_qt);
+  for (int t = 0; t < n_qt; ++t) {
+    const int r0 = t * fwd::BM, r1 = std::min(r0 + fwd::BM, N) - 1;
+    const int lo = (wl < 0) ? 0 : std::max(0, r0 - wl) / fwd::BN;
+    const int hi = (wr < 0) ? n_kt : std::min(n_kt, (r1 + wr) / fwd::BN + 1);
+    key_tiles[t] = std::max(hi - lo, 1);
+  }
+  FwdSplit best = plain;
+  double best_t = split_makespan(BH, n_qt, min_singles, sms, key_tiles);
+  for (int sg = min_singles + 2; sg <= n_qt; sg += 2) {
+    const double t = split_makespan(BH, n_qt, sg, sms, key_tiles);
+    if (t < best_t * 0.999) {
+      best_t = t;
+      best = FwdSplit{(n_qt - sg) / 2, sg};
+    }
+  }
+  std::lock_guard<std::mutex> lock(mu);
+  cache[key] = best;
+  return best;
+}
+
+int device_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
+  std::lock_guard<std::mutex> lock(g_mutex);
+  return g_devices[dev].sms;
+}
+
 fa_status launch_status() {
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -250,7 +337,10 @@ fa_status forward_impl(const void* Q, const void* K, const void* V, void* O, flo
   p.LSE = LSE;
   p.N = N;
   p.BH = BH;
-  p.n_qblk = (N + 2 * fwd::BM - 1) / (2 * fwd::BM);
+  const FwdSplit split = fwd_split(BH, N, mask.wl, mask.wr, device_sms());
+  p.pairs_ph = split.pairs_ph;
+  p.singles_ph = split.singles_ph;
+  p.n_pair_ctas = BH * split.pairs_ph;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wl = mask.wl;
   p.wr = mask.wr;
@@ -258,7 +348,7 @@ fa_status forward_impl(const void* Q, const void* K, const void* V, void* O, flo
   p.n_kt = (N + fwd::BN - 1) / fwd::BN;
   p.drop = drop.params;
   p.timeout_ns = watchdog_ns();
-  const dim3 grid(static_cast<unsigned>(p.n_qblk) * BH);
+  const dim3 grid(static_cast<unsigned>(BH) * (split.pairs_ph + split.singles_ph));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool g = mask.general();
   if constexpr (E == Elt::BF16) {
