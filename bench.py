@@ -206,10 +206,15 @@ def oracle_sample(w, seconds: float, rng_seed: int = 0, inputs=None):
         return float(np.sum(visible)) * w.d * 10.0, dt
 
     r0 = max(32, 4 * oracle.num_threads())
+    run(r0)  # warm-up: thread pool start-up and cold caches, not timed
     _, t0 = run(r0)  # calibration: enough rows to occupy every thread
     per_row = t0 / r0
     R = int(max(1, seconds / max(per_row, 1e-9)))
     flops, dt = run(R)
+    if dt < 0.6 * seconds:  # calibration overestimated the row cost: top up once
+        R2 = int(max(1, (seconds - dt) * R / max(dt, 1e-9)))
+        f2, dt2 = run(R2)
+        flops, dt, R = flops + f2, dt + dt2, R + R2
     return flops, dt, R, oracle.num_threads()
 
 
