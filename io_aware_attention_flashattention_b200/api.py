@@ -282,14 +282,20 @@ def _masked(window, block_mask) -> bool:
     return window is not None or block_mask is not None
 
 
-def forward(q, k, v, causal: bool = False, scale=None, window=None, block_mask=None):
+def forward(q, k, v, causal: bool = False, scale=None, window=None, block_mask=None,
+            dropout=None):
     """(O, LSE) for bf16, f16 or fp32 q, k, v of shape [B, H, N, d] on the GPU.
-    ``window`` / ``block_mask`` (bf16 only) as for fa_forward_masked."""
+    ``window`` / ``block_mask`` as for fa_forward_masked and ``dropout`` = (p, seed,
+    offset) as for fa_forward_dropout (bf16 only)."""
     B, H, N, d = _shape(q)
     scale = _default_scale(d, scale)
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    if _masked(window, block_mask):
+    if dropout is not None:
+        if q.dtype != torch.bfloat16:
+            raise TypeError("dropout is supported for bf16 inputs")
+        fa_forward_dropout(q, k, v, o, lse, scale, causal, dropout, window, block_mask)
+    elif _masked(window, block_mask):
         if q.dtype != torch.bfloat16:
             raise TypeError("window and block_mask are supported for bf16 inputs")
         fa_forward_masked(q, k, v, o, lse, scale, causal, window, block_mask)
@@ -311,13 +317,18 @@ def workspace_for(q) -> torch.Tensor:
 
 
 def backward(q, k, v, o, lse, do, causal: bool = False, scale=None, workspace=None,
-             window=None, block_mask=None):
-    """(dQ, dK, dV) of the loss <dO, O> (same masks as the forward)."""
+             window=None, block_mask=None, dropout=None):
+    """(dQ, dK, dV) of the loss <dO, O> (same masks and dropout as the forward)."""
     B, H, N, d = _shape(q)
     scale = _default_scale(d, scale)
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ws = workspace_for(q) if workspace is None else workspace
-    if _masked(window, block_mask):
+    if dropout is not None:
+        if q.dtype != torch.bfloat16:
+            raise TypeError("dropout is supported for bf16 inputs")
+        fa_backward_dropout(q, k, v, o, do, lse, dq, dk, dv, scale, causal, ws, dropout, window,
+                            block_mask)
+    elif _masked(window, block_mask):
         if q.dtype != torch.bfloat16:
             raise TypeError("window and block_mask are supported for bf16 inputs")
         fa_backward_masked(q, k, v, o, do, lse, dq, dk, dv, scale, causal, ws, window,
@@ -337,20 +348,26 @@ class FlashAttentionFunction(torch.autograd.Function):
     """Differentiable exact attention through the library's forward and backward."""
 
     @staticmethod
-    def forward(ctx, q, k, v, causal: bool = False, scale=None, window=None, block_mask=None):
+    def forward(ctx, q, k, v, causal: bool = False, scale=None, window=None, block_mask=None,
+                dropout=None):
         q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
-        o, lse = forward(q, k, v, causal, scale, window, block_mask)
+        o, lse = forward(q, k, v, causal, scale, window, block_mask, dropout)
         ctx.save_for_backward(q, k, v, o, lse)
         ctx.causal, ctx.scale, ctx.window, ctx.block_mask = causal, scale, window, block_mask
+        ctx.dropout = dropout  # the backward regenerates the same keep mask
         return o
 
     @staticmethod
     def backward(ctx, do):
         q, k, v, o, lse = ctx.saved_tensors
         dq, dk, dv = backward(q, k, v, o, lse, do.contiguous(), ctx.causal, ctx.scale,
-                              window=ctx.window, block_mask=ctx.block_mask)
-        return dq, dk, dv, None, None, None, None
+                              window=ctx.window, block_mask=ctx.block_mask,
+                              dropout=ctx.dropout)
+        return dq, dk, dv, None, None, None, None, None
 
 
-def attention(q, k, v, causal: bool = False, scale=None, window=None, block_mask=None):
-    return FlashAttentionFunction.apply(q, k, v, causal, scale, window, block_mask)
+def attention(q, k, v, causal: bool = False, scale=None, window=None, block_mask=None,
+              dropout=None):
+    """Differentiable attention; ``dropout`` = (p, seed, offset): pass a new offset (or
+    seed) per call to draw a new mask."""
+    return FlashAttentionFunction.apply(q, k, v, causal, scale, window, block_mask, dropout)

@@ -510,23 +510,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float Ls[4] = {L4.x, L4.y, L4.z, L4.w};
             const float Ds[4] = {D4.x, D4.y, D4.z, D4.w};
             float pv[4], dsv[4];
+            // Dropout words for this key and queries qh0 + 16cc + 4v + e: the counter
+            // (key / 4, query, bh, offset) is shared by the four lanes holding keys
+            // 4g..4g+3 (key mod 4 = lane mod 4), so lane u draws the block of query
+            // 4v + u and a transpose across the four lanes hands each its own word.
+            uint32_t zw[4] = {0u, 0u, 0u, 0u};
+            if constexpr (kDropout) {
+              const int u = lane & 3;
+              const uint4 w = philox4x32_10(
+                  make_uint4(static_cast<uint32_t>(key >> 2),
+                             static_cast<uint32_t>(qh0 + cc * 16 + 4 * v + u),
+                             static_cast<uint32_t>(bh), p.drop.offset),
+                  p.drop.seed_lo, p.drop.seed_hi);
+              zw[0] = w.x;
+              zw[1] = w.y;
+              zw[2] = w.z;
+              zw[3] = w.w;
+              transpose4_lanes(zw, u);
+            }
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int k = 4 * v + e;
               float pe = ex2_approx(fmaf(__uint_as_float(sv[cur][k]), c, -Ls[e]));
               if (kM && static_cast<unsigned>(qoff + cc * 16 + k) >= q_span) pe = 0.f;
               if constexpr (kDropout) {
-                // Z for (query qh0 + 16cc + k, this key): word (key mod 4) of the counter
-                // (key / 4, query, bh, offset); dV takes P o Z / (1 - p) and
-                // dS = P o (dP o Z / (1 - p) - D)
-                const uint4 w = philox4x32_10(
-                    make_uint4(static_cast<uint32_t>(key >> 2),
-                               static_cast<uint32_t>(qh0 + cc * 16 + k), static_cast<uint32_t>(bh),
-                               p.drop.offset),
-                    p.drop.seed_lo, p.drop.seed_hi);
-                const int wsel = key & 3;
-                const uint32_t word = wsel == 0 ? w.x : wsel == 1 ? w.y : wsel == 2 ? w.z : w.w;
-                const float zs = (word >= p.drop.threshold) ? p.drop.scale : 0.0f;
+                // dV takes P o Z / (1 - p) and dS = P o (dP o Z / (1 - p) - D)
+                const float zs = (zw[e] >= p.drop.threshold) ? p.drop.scale : 0.0f;
                 pv[e] = pe * zs;
                 dsv[e] = pe * (__uint_as_float(dv[cur][k]) * zs - Ds[e]);
               } else {

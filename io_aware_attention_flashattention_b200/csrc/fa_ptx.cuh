@@ -453,6 +453,25 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1
   return c;
 }
 
+// Lanes 4g..4g+3 of a warp each hold one row of a 4 x 4 matrix (lane 4g+r: a[] = row
+// r); afterwards lane 4g+c holds column c (a[r] = element (r, c)). Two butterfly
+// rounds; in each, paired lanes swap the two elements the other one needs.
+__device__ __forceinline__ void transpose4_lanes(uint32_t (&a)[4], int u) {
+#pragma unroll
+  for (int d = 1; d <= 2; d <<= 1) {
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      if (j & d) continue;  // the pair (j, j + d)
+      const bool hi = (u & d) != 0;
+      const uint32_t recv = __shfl_xor_sync(0xffffffffu, hi ? a[j] : a[j | d], d);
+      if (hi)
+        a[j] = recv;
+      else
+        a[j | d] = recv;
+    }
+  }
+}
+
 // Dropout on P: key j of query row i in head bh is kept iff word (j mod 4) of
 // philox4x32_10((j / 4, i, bh, offset), seed) is at least `threshold`
 // (= floor(p * 2^32)); kept values are scaled by 1 / (1 - p).

@@ -143,3 +143,20 @@ def test_dropout_argument_errors():
         assert lib.fa_forward_dropout(p, p, p, p, lse.data_ptr(), 1, 1, 128, 64, 0.1, 0, -1, -1,
                                       None, bad, 1, 0, s) == 1
     assert api.fa_get_status() == 0
+
+
+def test_autograd_with_window_and_dropout_matches_oracle():
+    """The differentiable wrapper carries the window and the dropout spec into its
+    backward."""
+    q, k, v, do = make_inputs(1, 2, 300, 128, torch.bfloat16, seed=77)
+    drop, window = (0.2, 31337, 4), (100, -1)
+    qc, kc, vc = (t.cuda().requires_grad_() for t in (q, k, v))
+    out = api.attention(qc, kc, vc, causal=True, window=window, dropout=drop)
+    out.backward(do.cuda())
+    scale = 1 / math.sqrt(128)
+    kw = dict(window=window, dropout=drop)
+    O_ref, _ = oracle.forward(q, k, v, scale, True, **kw)
+    dQ, dK, dV, _ = oracle.backward(q, k, v, do, scale, True, **kw)
+    assert_close_o("O", _np(out), O_ref, TOL_BF16["O"])
+    for name, got, want in (("dQ", qc.grad, dQ), ("dK", kc.grad, dK), ("dV", vc.grad, dV)):
+        assert_close(name, _np(got), want, grad_tol(TOL_BF16, want))
