@@ -514,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             // (key / 4, query, bh, offset) is shared by the four lanes holding keys
             // 4g..4g+3 (key mod 4 = lane mod 4), so lane u draws the block of query
             // 4v + u and a transpose across the four lanes hands each its own word.
-            uint32_t zw[4] = {0u, 0u, 0u, 0u};
+            [[maybe_unused]] uint32_t zw[4] = {0u, 0u, 0u, 0u};
             if constexpr (kDropout) {
               const int u = lane & 3;
               const uint4 w = philox4x32_10(
