@@ -469,14 +469,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < nsteps && ok; ++s) {
       do ++i; while (!member(i));
       const int qh0 = i * BM + 64 * h;  // first query of this half
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarS + h), s & 1, wd));
-      if (ok && s > 0)  // the dQ MMA of the last step has finished reading this dS chunk
+      // The two barriers that completed long ago are observed first, so that the work
+      // starts as soon as S^T and dP^T are in TMEM: the dQ MMA of the last step has
+      // finished reading this dS chunk, and L2 and D of this half arrived with its Q rows.
+      if (s > 0)
         ok = __all_sync(0xffffffffu, mbar_wait(bar(dq_bar), (s - 1) & 1, wd));
-      // L2 and D of this half arrived with its Q rows: observe that copy's barrier
       const int seqQ = seq_of(s, h, 1);
       if (ok)
         ok = __all_sync(0xffffffffu,
                         mbar_wait(bar(C::kBarFull + slot_of(seqQ)), round_of(seqQ) & 1, wd));
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarS + h), s & 1, wd));
       if (!ok) break;
       tc_fence_after();
       const float4* Lv = reinterpret_cast<const float4*>(
