@@ -24,8 +24,10 @@
  *     in DEVICE memory, base addresses 16-byte aligned. Q, K and V share one N
  *     (self-attention shape).
  *   - The caller owns every buffer, including the backward workspace; the
- *     library allocates no device memory. It holds one device status word per
- *     GPU and a host-side cache of nothing that outlives a call.
+ *     library allocates no device memory at run time. Its state: one device
+ *     status word per GPU, the fixed scratch array of fa_backward_noalloc (part
+ *     of the module image), and on the host each GPU's SM count and a cache of
+ *     the forward's work split per shape (thread-safe).
  *   - Calls are asynchronous on `stream` (0 = the legacy default stream).
  *     Argument errors are returned synchronously and launch nothing. A failed
  *     launch returns FA_ERR_CUDA.
