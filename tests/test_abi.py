@@ -71,3 +71,47 @@ def test_no_cpu_fallback_in_product_path():
             if f.endswith(".py"):
                 src = open(os.path.join(root, f)).read()
                 assert "import oracle" not in src and "from oracle" not in src, f
+
+
+def _fn(libfa, name):
+    f = getattr(libfa, name)
+    f.restype, f.argtypes = _lib.SIGNATURES[name]
+    return f
+
+
+def test_host_validation_of_every_entry_point(libfa):
+    """Each entry point rejects bad arguments on the host, before any CUDA call, with
+    the documented status (1 invalid argument, 2 unsupported); no GPU is needed."""
+    P = 0x10000  # a 16-byte-aligned stand-in address; a rejected call never touches it
+    fwd = _fn(libfa, "fa_forward")
+    assert fwd(P, P, P, P, P, 1, 1, 1 << 24, 128, 0.1, 0, None) == 2  # B*H*N*d = 2^31
+    assert fwd(P, P, P, P, P, 1, 1, 128, 64, float("nan"), 0, None) == 1
+    assert fwd(P, P, P, P, P, 1, 1, 128, 64, 0.0, 0, None) == 1
+    assert fwd(P, P, P, P, P, 1, 1, 128, 64, 0.1, 2, None) == 1
+    assert fwd(P, P, P, P, P, 0, 1, 128, 64, 0.1, 0, None) == 1
+    assert fwd(P, P, P, P, P, 1, 1, -1, 64, 0.1, 0, None) == 1
+    assert fwd(P + 8, P, P, P, P, 1, 1, 128, 64, 0.1, 0, None) == 1  # misaligned
+    f16 = _fn(libfa, "fa_forward_f16")
+    assert f16(P, P, P, P, P, 1, 1, 128, 32, 0.1, 0, None) == 2
+    masked = _fn(libfa, "fa_forward_masked")
+    big_n = 4097 * 128  # a block mask of more than 4096 x 4096 tiles
+    assert masked(P, P, P, P, P, 1, 1, big_n, 64, 0.1, 0, -1, -1, P, None) == 2
+    assert masked(P, P, P, P, P, 1, 1, 256, 64, 0.1, 3, 4, 4, None, None) == 1
+    drop = _fn(libfa, "fa_forward_dropout")
+    for p in (1.0, -0.25, float("nan"), float("inf")):
+        assert drop(P, P, P, P, P, 1, 1, 256, 64, 0.1, 0, -1, -1, None, p, 7, 0, None) == 1
+    ws = _fn(libfa, "fa_backward_workspace_size")(1, 2, 384, 64)
+    bwd = _fn(libfa, "fa_backward")
+    assert bwd(P, P, P, P, P, P, P, P, P, 1, 2, 384, 64, 0.1, 0, P, ws - 1, None) == 1
+    assert bwd(P, P, P, P, P, P, P, P, P, 1, 2, 384, 64, 0.1, 0, None, ws, None) == 1
+    assert bwd(P, P, P, P, P, None, P, P, P, 1, 2, 384, 64, 0.1, 0, P, ws, None) == 1
+    bwd16 = _fn(libfa, "fa_backward_f16")
+    assert bwd16(P, P, P, P, P, P, P, P, P, 1, 2, 384, 96, 0.1, 0, P, ws, None) == 2
+    noalloc = _fn(libfa, "fa_backward_noalloc")
+    # B1 H8 N16384 d128 needs 68 MB of workspace, more than the 32 MiB built in
+    assert noalloc(P, P, P, P, P, P, P, P, P, 1, 8, 16384, 128, 0.1, 0, None) == 2
+    bdrop = _fn(libfa, "fa_backward_dropout")
+    assert bdrop(P, P, P, P, P, P, P, P, P, 1, 2, 384, 64, 0.1, 0, -1, -1, None, 1.5, 1, 0,
+                 P, ws, None) == 1
+    f32 = _fn(libfa, "fa_backward_f32")
+    assert f32(P, P, P, P, P, P, P, P, P, 1, 2, 384, 64, 0.1, 0, P, ws - 1, None) == 1
