@@ -56,7 +56,7 @@ typedef struct CUstream_st* fa_stream_t;
 typedef enum {
   FA_OK = 0,
   FA_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad shape, bad scale */
-  FA_ERR_UNSUPPORTED = 2, /* valid arguments outside what this build implements */
+  FA_ERR_UNSUPPORTED = 2, /* valid arguments outside what this library implements */
   FA_ERR_CUDA = 3,        /* a CUDA call or launch failed (no device, bad context) */
   FA_ERR_TIMEOUT = 4      /* a kernel's bounded wait ran out (see fa_get_status) */
 } fa_status;

@@ -442,7 +442,7 @@ PHILOX_KAT = [
 
 
 def philox_py(ctr, key):
-    """Philox-4x32-10 written out from its definition in the paper above."""
+    """Philox-4x32-10 written out from its definition (Salmon et al., SC 2011, cited above)."""
     m = 0xFFFFFFFF
     x0, x1, x2, x3 = ctr
     k0, k1 = key
