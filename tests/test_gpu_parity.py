@@ -306,6 +306,20 @@ def test_workload_mid_b1h8_n4096_d128_in_f16():
 
 
 @pytest.mark.slow
+def test_workload_long_b1h8_n16384_d128_causal():
+    """The long workload's shape with the causal mask (tiles above the diagonal never
+    loaded; the forward's pair/single split differs from the non-causal one)."""
+    w = dataclasses.replace(WORKLOADS["long_b1h8_n16384_d128"], causal=True)
+    check_sampled(w, per_head=24, full_heads=(1,), dkdv_head=6, n_keys=32)
+
+
+def test_workload_stress_causal_b2h16_n8192_d128_qk8_in_f16():
+    """The x8-logit causal stress shape with f16 inputs (forward only)."""
+    w = dataclasses.replace(WORKLOADS["stress_causal_b2h16_n8192_d128_qk8"], dtype=torch.float16)
+    check_sampled(w, per_head=12, full_heads=(3,))
+
+
+@pytest.mark.slow
 def test_workload_long_b1h8_n16384_d128():
     check_sampled(WORKLOADS["long_b1h8_n16384_d128"], per_head=32, full_heads=(0, 7),
                   dkdv_head=5, n_keys=32)
