@@ -556,6 +556,37 @@ def pin_dropout_finite_differences(orc):
                 f"dropout finite differences of {'QKV'[which]} (N={N}, p={p}): {err:.3e}")
 
 
+# --------------------------------------------------------------------------- row functions
+
+
+def pin_row_functions_agree(orc):
+    """The row-restricted entry points (used where whole heads are too slow) equal the
+    full ones, which the pins above tie down: plain, causal with a window and a block
+    mask, and with dropout."""
+    rng = _rng(41)
+    B, H, N, d = 1, 2, 140, 4
+    Q, K, V, dO = (rng.standard_normal((B, H, N, d)) for _ in range(4))
+    blocks = [[1, 0], [1, 1]]
+    cases = [dict(), dict(window=(50, -1), block_mask=blocks), dict(dropout=(0.3, 99, 2))]
+    for causal, kw in zip((False, True, False), cases):
+        O, L = orc.forward(Q, K, V, 0.5, causal, **kw)
+        dQ, dK, dV, D = orc.backward(Q, K, V, dO, 0.5, causal, **kw)
+        heads = rng.integers(0, B * H, 24)
+        rows = rng.integers(0, N, 24)
+        Or, Lr = orc.forward_rows(Q, K, V, 0.5, causal, heads, rows, **kw)
+        _close(Or, O.reshape(B * H, N, d)[heads, rows], 1e-13, f"forward_rows O {kw}")
+        _close(Lr, L.reshape(B * H, N)[heads, rows], 1e-13, f"forward_rows L {kw}")
+        dQr, Dr = orc.backward_dq_rows(Q, K, V, dO, 0.5, causal, heads, rows, **kw)
+        _close(dQr, dQ.reshape(B * H, N, d)[heads, rows], 1e-13, f"backward_dq_rows dQ {kw}")
+        _close(Dr, D.reshape(B * H, N)[heads, rows], 1e-13, f"backward_dq_rows D {kw}")
+        head, keys = 1, np.array([0, 3, 64, 127, 128, 139])
+        dKr, dVr = orc.backward_dkdv_rows(Q, K, V, dO, 0.5, causal, head,
+                                          L.reshape(B * H, N)[head], D.reshape(B * H, N)[head],
+                                          keys, **kw)
+        _close(dKr, dK.reshape(B * H, N, d)[head, keys], 1e-13, f"backward_dkdv_rows dK {kw}")
+        _close(dVr, dV.reshape(B * H, N, d)[head, keys], 1e-13, f"backward_dkdv_rows dV {kw}")
+
+
 # --------------------------------------------------------------------------- golden
 
 
@@ -600,4 +631,5 @@ ALL_PINS = [
     pin_dropout_reduces_to_softmax_and_generator,
     pin_dropout_keep_rate,
     pin_dropout_finite_differences,
+    pin_row_functions_agree,
 ]

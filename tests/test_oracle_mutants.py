@@ -33,6 +33,14 @@ MUTATIONS = [
     ("dropout_dP_without_Z", "dsi[j] = acc * drop.factor(bh, i, j);", "dsi[j] = acc;"),
     ("dropout_dV_without_Z", "const double p = P[i * N + j] * drop.factor(bh, i, j);",
      "const double p = P[i * N + j];"),
+    ("dkdv_rows_ignore_masks", "if (!vis.sees(i, j)) continue;", ""),
+    ("dkdv_rows_wrong_sign", "const double dsij = pij * (dpij * f - D[i]);",
+     "const double dsij = pij * (dpij * f + D[i]);"),
+    ("dkdv_rows_dV_without_Z", "gv[c] += pij * f * goi[c];", "gv[c] += pij * goi[c];"),
+    ("dq_rows_without_scale", "for (int64_t c = 0; c < d; ++c) g[c] *= scale;", ""),
+    ("dq_rows_dP_without_Z", "dp[j] = acc * drop.factor(bh, i, j);", "dp[j] = acc;"),
+    ("forward_rows_without_Z", "const double pd = p[j] * drop.factor(bh, i, j);",
+     "const double pd = p[j];"),
     ("block_mask_ignored", "if (blocks && !blocks[(i / kBlock) * nb + j / kBlock]) return false;",
      ""),
     ("no_max_subtraction", "p[j] = std::exp(s[j] - m);", "p[j] = std::exp(s[j]);"),
