@@ -12,7 +12,9 @@ stream around every kernel of every step; L2 is flushed (a 256 MiB write) before
 each timed step, outside the events; W untimed warm-up steps; a barrier and a
 device synchronise on both sides of the K timed steps; max over ranks. With N > 1
 each rank runs its own replica of the workload (independent heads; no collective
-on the data path), so the scaling is weak.
+on the data path), so the scaling is weak. nvidia-smi samples the clocks during
+the timed region; a hardware or thermal slowdown, or SM clocks held far below
+their maximum with no reason active, takes the measurement again, once.
 
 Prints one JSON line (rank 0).
 """
@@ -126,24 +128,52 @@ class ClockSampler:
             self.proc.kill()
         if self.thread:
             self.thread.join(timeout=2)
-        sm, smax, power, reasons = [], [], [], set()
-        for line in self.lines:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax.append(float(parts[2]))
-                power.append(float(parts[3]))
-            except ValueError:
-                continue
-            for name, val in zip(self.NAMES, parts[5:9]):
-                if val.lower() == "active":
-                    reasons.add(name)
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None,
-                "power_w_max": max(power) if power else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        return summarise_clock_lines(self.lines)
+
+
+def summarise_clock_lines(lines):
+    """Median SM clock, the highest max clock and power, and the throttle reasons seen
+    active, from `nvidia-smi --format=csv,noheader,nounits` lines of the fields in
+    ClockSampler.FIELDS. Lines that do not parse (a header, a cut-off last line) are
+    skipped."""
+    sm, smax, power, reasons = [], [], [], set()
+    for line in lines:
+        parts = [p.strip() for p in line.split(",")]
+        if len(parts) < 9:
+            continue
+        try:
+            sm.append(float(parts[1]))
+            smax.append(float(parts[2]))
+            power.append(float(parts[3]))
+        except ValueError:
+            continue
+        for name, val in zip(ClockSampler.NAMES, parts[5:9]):
+            if val.lower() == "active":
+                reasons.add(name)
+    return {"sm_mhz": statistics.median(sm) if sm else None,
+            "sm_max_mhz": max(smax) if smax else None,
+            "power_w_max": max(power) if power else None,
+            "reasons": sorted(reasons), "samples": len(sm)}
+
+
+REJECTING_REASONS = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown")
+PINNED_LOW_FRACTION = 0.75
+
+
+def clock_verdict(clocks):
+    """Why a timed region's clock record rejects its number, or None if it stands.
+
+    A hardware or thermal slowdown rejects it. So does a median SM clock below
+    PINNED_LOW_FRACTION of the maximum with no reason active (a clock lock left behind
+    by someone else). sw_power_cap alone is normal under a dense load and is kept. No
+    samples (no nvidia-smi) gives no verdict."""
+    bad = [r for r in clocks.get("reasons", []) if r in REJECTING_REASONS]
+    if bad:
+        return "throttled: " + ",".join(bad)
+    sm, smax = clocks.get("sm_mhz"), clocks.get("sm_max_mhz")
+    if sm is not None and smax and not clocks.get("reasons") and sm < PINNED_LOW_FRACTION * smax:
+        return f"SM clock {sm:.0f} MHz of {smax:.0f} MHz with no reason active"
+    return None
 
 
 # ---------------------------------------------------------------- ranks
@@ -331,20 +361,32 @@ def main():
     if api.fa_get_status() != 0:
         raise SystemExit("kernel watchdog fired during warm-up")
 
-    events = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)] for _ in range(args.steps)]
-    sampler = ClockSampler(torch.cuda.current_device())
-    barrier()
-    torch.cuda.synchronize()
-    sampler.start()
-    time.sleep(0.2)  # let the sampler start before the timed region
-    wall0 = time.perf_counter()
-    for s in range(args.steps):
-        flush.zero_()
-        step(events[s])
-    torch.cuda.synchronize()
-    wall = time.perf_counter() - wall0
-    barrier()
-    clocks = sampler.stop()
+    def timed_region():
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(nev)]
+               for _ in range(args.steps)]
+        sampler = ClockSampler(torch.cuda.current_device())
+        barrier()
+        torch.cuda.synchronize()
+        sampler.start()
+        time.sleep(0.2)  # let the sampler start before the timed region
+        t0 = time.perf_counter()
+        for s in range(args.steps):
+            flush.zero_()
+            step(evs[s])
+        torch.cuda.synchronize()
+        t1 = time.perf_counter() - t0
+        barrier()
+        return evs, sampler.stop(), t1
+
+    events, clocks, wall = timed_region()
+    # a number taken under a hardware or thermal slowdown, or under a clock lock, is
+    # taken again once; every rank takes the same decision (max of the flags)
+    rejected = clock_verdict(clocks)
+    if max_over_ranks(1.0 if rejected else 0.0, world, dev) > 0:
+        first = dict(clocks, rejected=rejected or "another rank's clocks")
+        events, clocks, wall = timed_region()
+        clocks = dict(clocks, remeasured=True, first_run=first)
+    clocks["verdict"] = clock_verdict(clocks) or "ok"
     status = api.fa_get_status()
     per_kernel = [[events[s][i].elapsed_time(events[s][i + 1]) for s in range(args.steps)]
                   for i in range(len(names))]
