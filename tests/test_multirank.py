@@ -46,7 +46,7 @@ def _worker(rank, world, port, out):
 def test_two_ranks_gloo():
     world = 2
     port = _free_port()
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:
         out = mgr.dict()
         mp.start_processes(_worker, args=(world, port, out), nprocs=world, join=True,
                            start_method="spawn")
