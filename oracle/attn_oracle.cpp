@@ -41,11 +41,14 @@
 //   Dropout on P (optional): [jos] p.218 lists dropout among the operations fused into
 //   the attention kernel. With drop probability p, Pd[i][j] = P[i][j] * Z[i][j] / (1 - p)
 //   and O = Pd V; L stays the log-sum-exp of the logits (P is normalised before the
-//   dropout). Z[i][j] = 0 iff the Philox-4x32-10 word for (i, j) is below
-//   t = min(floor(p * 2^32), 2^32 - 1) (an integer decision). The word is element j % 4
-//   of Philox-4x32-10 (Salmon, Moraes, Dror and Shaw, "Parallel random numbers: as easy
-//   as 1, 2, 3", SC 2011) at counter (j / 4, i, bh, offset) under key (seed low 32
-//   bits, seed high 32 bits), bh = b * H + h.
+//   dropout). One Philox-4x32-10 block (Salmon, Moraes, Dror and Shaw, "Parallel
+//   random numbers: as easy as 1, 2, 3", SC 2011) covers 4 queries x 4 keys: the block
+//   at counter (j / 4, i / 4, bh, offset) under key (seed low 32 bits, seed high 32
+//   bits), bh = b * H + h, gives query i its word i % 4 and key j byte j % 4 of that
+//   word (byte 0 the least significant). Z[i][j] = 0 iff that byte is below
+//   t = floor(256 p) (an integer decision), so the drop probability is t / 256: p
+//   rounded down to a multiple of 1/256, and the factor 1/(1 - p) above is taken with
+//   that rounded p, 256 / (256 - t).
 //   m_i = max_j S[i][j]        [jsqmd] section 2.1, safe softmax
 //   P[i][j] = exp(S[i][j] - m_i) / sum_j exp(S[i][j] - m_i)
 //   O = P V
@@ -146,28 +149,29 @@ struct Dropout {
   double p;
   uint64_t seed;
   uint32_t offset;
-  uint32_t threshold;  // a key is dropped iff its Philox word is below this
+  uint32_t threshold;  // a key is dropped iff its Philox byte is below this (0..255)
 
   bool on() const { return p > 0.0; }
   // Z[i][j] of head bh, as 0 or 1
   bool keep(int64_t bh, int64_t i, int64_t j) const {
     if (!on()) return true;
-    const uint32_t ctr[4] = {static_cast<uint32_t>(j / 4), static_cast<uint32_t>(i),
+    const uint32_t ctr[4] = {static_cast<uint32_t>(j / 4), static_cast<uint32_t>(i / 4),
                              static_cast<uint32_t>(bh), offset};
     uint32_t w[4];
     philox4x32_10(ctr, static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32), w);
-    return w[j % 4] >= threshold;
+    const uint32_t byte = (w[i % 4] >> (8 * (j % 4))) & 0xffu;
+    return byte >= threshold;
   }
-  // Pd / P for (i, j): Z / (1 - p)
+  // Pd / P for (i, j): Z / (1 - t/256)
   double factor(int64_t bh, int64_t i, int64_t j) const {
     if (!on()) return 1.0;
-    return keep(bh, i, j) ? 1.0 / (1.0 - p) : 0.0;
+    return keep(bh, i, j) ? 256.0 / (256.0 - threshold) : 0.0;
   }
 };
 
 Dropout make_dropout(double p, uint64_t seed, uint32_t offset) {
-  double t = std::floor(p * 4294967296.0);
-  if (t > 4294967295.0) t = 4294967295.0;
+  double t = std::floor(p * 256.0);
+  if (t > 255.0) t = 255.0;
   if (!(t > 0.0)) t = 0.0;
   return Dropout{p, seed, offset, static_cast<uint32_t>(t)};
 }

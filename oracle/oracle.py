@@ -30,8 +30,9 @@ Definitions followed (titles of the sources, see the header of attn_oracle.cpp):
     every block); they combine with ``causal`` by AND. A row that sees no key has
     O = 0, L = -inf and zero gradients;
   * dropout on P ([jos] lists it among the fused operations), with the keep/drop
-    decision from Philox-4x32-10 (Salmon et al., "Parallel random numbers: as easy
-    as 1, 2, 3", SC 2011). ``dropout=(p, seed, offset)``; see attn_oracle.cpp.
+    decision from a byte of Philox-4x32-10 (Salmon et al., "Parallel random numbers:
+    as easy as 1, 2, 3", SC 2011) against floor(256 p), so p acts rounded down to a
+    multiple of 1/256. ``dropout=(p, seed, offset)``; see attn_oracle.cpp.
 """
 from __future__ import annotations
 

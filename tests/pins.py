@@ -425,8 +425,9 @@ def pin_masked_finite_differences(orc):
 #
 # Dropout on P ("A survey of key techniques of large language model pre-training
 # systems", p.218, lists it among the operations fused into the attention kernel):
-# Pd = P o Z / (1 - p). Z[i][j] = 0 iff word j % 4 of Philox-4x32-10 at counter
-# (j / 4, i, bh, offset) under key (seed low, seed high) is below floor(p * 2^32).
+# Pd = P o Z / (1 - t/256) with t = floor(256 p). Z[i][j] = 0 iff byte j % 4 of word
+# i % 4 of Philox-4x32-10 at counter (j / 4, i / 4, bh, offset) under key (seed low,
+# seed high) is below t.
 
 # Philox-4x32-10 known-answer vectors published with the generator (Salmon, Moraes,
 # Dror and Shaw, "Parallel random numbers: as easy as 1, 2, 3", SC 2011; the Random123
@@ -454,18 +455,32 @@ def philox_py(ctr, key):
     return (x0, x1, x2, x3)
 
 
+def dropout_threshold(p):
+    """The byte threshold t = floor(256 p); the drop probability is t / 256."""
+    return min(math.floor(p * 256.0), 255)
+
+
 def dropout_keep(N, bh, p, seed, offset):
-    """Z of one head, [N, N] of 0/1, from philox_py."""
-    t = min(math.floor(p * 4294967296.0), 4294967295)
+    """Z of one head, [N, N] of 0/1, from philox_py: the block at counter
+    (j // 4, i // 4, bh, offset) gives query i its word i % 4 and key j byte j % 4 of
+    it; a byte below floor(256 p) drops the pair."""
+    t = dropout_threshold(p)
     key = (seed & 0xFFFFFFFF, (seed >> 32) & 0xFFFFFFFF)
     Z = np.zeros((N, N))
-    for i in range(N):
+    for i4 in range((N + 3) // 4):
         for j4 in range((N + 3) // 4):
-            w = philox_py((j4, i, bh, offset), key)
-            for u in range(4):
-                if 4 * j4 + u < N:
-                    Z[i, 4 * j4 + u] = 1.0 if w[u] >= t else 0.0
+            w = philox_py((j4, i4, bh, offset), key)
+            for r in range(4):
+                for b in range(4):
+                    i, j = 4 * i4 + r, 4 * j4 + b
+                    if i < N and j < N:
+                        Z[i, j] = 1.0 if (w[r] >> (8 * b)) & 0xFF >= t else 0.0
     return Z
+
+
+def dropout_scale(p):
+    """1 / (1 - t/256): the kept values' factor for the rounded drop probability."""
+    return 256.0 / (256.0 - dropout_threshold(p))
 
 
 def pin_philox_known_answers(orc):
@@ -482,9 +497,9 @@ def pin_philox_known_answers(orc):
 
 
 def pin_dropout_reduces_to_softmax_and_generator(orc):
-    """With dropout, O = (P o Z / (1 - p)) V with P from the (pinned) softmax and Z from
-    the generator above, L is the logits' log-sum-exp without dropout, and p = 0 is
-    exactly no dropout."""
+    """With dropout, O = (P o Z / (1 - t/256)) V with P from the (pinned) softmax, Z
+    from the generator above and t = floor(256 p), L is the logits' log-sum-exp
+    without dropout, and p = 0 is exactly no dropout."""
     rng = _rng(32)
     B, H, N, d = 1, 2, 37, 6
     Q, K, V = (rng.standard_normal((B, H, N, d)) for _ in range(3))
@@ -496,7 +511,7 @@ def pin_dropout_reduces_to_softmax_and_generator(orc):
         for bh in range(B * H):
             P = orc.probs(Q[0, bh], K[0, bh], 0.6, causal)
             Z = dropout_keep(N, bh, p, seed, offset)
-            _close(O[0, bh], (P * Z / (1.0 - p)) @ V[0, bh], 1e-13,
+            _close(O[0, bh], (P * Z * dropout_scale(p)) @ V[0, bh], 1e-13,
                    f"dropout O (p={p}, head {bh})")
     Op, Lp = orc.forward(Q, K, V, 0.6, True, dropout=(0.0, 99, 3))
     Oz, Lz = orc.forward(Q, K, V, 0.6, True)
@@ -504,14 +519,22 @@ def pin_dropout_reduces_to_softmax_and_generator(orc):
 
 
 def pin_dropout_keep_rate(orc):
-    """The kept fraction matches 1 - p within 5 binomial standard deviations, and
+    """The kept fraction matches 1 - t/256 within 5 binomial standard deviations, and
     different offsets give different masks."""
     N = 160
+    assert [dropout_threshold(p) for p in (0.0, 0.1, 0.5, 0.9, 0.999)] == [0, 25, 128, 230, 255]
     for p in (0.1, 0.5, 0.9):
         Z = dropout_keep(N, 3, p, 2024, 11)
-        n = Z.size
-        sigma = math.sqrt(n * p * (1 - p))
-        assert abs(Z.sum() - n * (1 - p)) <= 5 * sigma, f"keep rate at p={p}"
+        n, pe = Z.size, dropout_threshold(p) / 256.0
+        sigma = math.sqrt(n * pe * (1 - pe))
+        assert abs(Z.sum() - n * (1 - pe)) <= 5 * sigma, f"keep rate at p={p}"
+    # the keep rate of every byte position of every word is the same
+    Z = dropout_keep(N, 1, 0.5, 7, 0)
+    for r in range(4):
+        for b in range(4):
+            sub = Z[r::4, b::4]
+            sigma = math.sqrt(sub.size * 0.25)
+            assert abs(sub.sum() - sub.size * 0.5) <= 5 * sigma, f"word {r} byte {b}"
     # the oracle's masks: rows of P o Z are zero exactly where Z is
     rng = _rng(33)
     q = rng.standard_normal((1, 1, N, N)) * 0.1  # one head width d = N for Q, K and V

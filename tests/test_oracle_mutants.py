@@ -25,11 +25,14 @@ MUTATIONS = [
     ("philox_wrong_multiplier", "static_cast<uint64_t>(0xD2511F53u) * x0",
      "static_cast<uint64_t>(0xD2511F55u) * x0"),
     ("philox_no_key_bump", "k0 += 0x9E3779B9u;", ""),
-    ("dropout_no_rescale", "return keep(bh, i, j) ? 1.0 / (1.0 - p) : 0.0;",
+    ("dropout_no_rescale", "return keep(bh, i, j) ? 256.0 / (256.0 - threshold) : 0.0;",
      "return keep(bh, i, j) ? 1.0 : 0.0;"),
-    ("dropout_word_index", "return w[j % 4] >= threshold;", "return w[0] >= threshold;"),
-    ("dropout_counter_swapped", "static_cast<uint32_t>(j / 4), static_cast<uint32_t>(i),",
-     "static_cast<uint32_t>(i), static_cast<uint32_t>(j / 4),"),
+    ("dropout_rescale_unrounded_p", "return keep(bh, i, j) ? 256.0 / (256.0 - threshold) : 0.0;",
+     "return keep(bh, i, j) ? 1.0 / (1.0 - p) : 0.0;"),
+    ("dropout_word_index", "(w[i % 4] >> (8 * (j % 4)))", "(w[j % 4] >> (8 * (j % 4)))"),
+    ("dropout_byte_index", "(w[i % 4] >> (8 * (j % 4)))", "(w[i % 4] >> (8 * (i % 4)))"),
+    ("dropout_counter_swapped", "static_cast<uint32_t>(j / 4), static_cast<uint32_t>(i / 4),",
+     "static_cast<uint32_t>(i / 4), static_cast<uint32_t>(j / 4),"),
     ("dropout_dP_without_Z", "dsi[j] = acc * drop.factor(bh, i, j);", "dsi[j] = acc;"),
     ("dropout_dV_without_Z", "const double p = P[i * N + j] * drop.factor(bh, i, j);",
      "const double p = P[i * N + j];"),
