@@ -198,14 +198,16 @@ fa_status fa_backward_masked(const void* Q, const void* K, const void* V, const 
  * Masked attention with dropout on P (bf16): fa_forward_masked / fa_backward_masked
  * plus dropout, one of the operations "A survey of key techniques of large language
  * model pre-training systems" (Journal of Software 2026(1), p.218) lists as fused
- * into the attention kernel. With drop probability p_drop in [0, 1):
- *   Pd = P o Z / (1 - p_drop),  O = Pd V,  LSE = the log-sum-exp of the logits
+ * into the attention kernel. With p_drop in [0, 1), t = floor(256 p_drop) and the drop
+ * probability t / 256 (p_drop rounded down to a multiple of 1/256):
+ *   Pd = P o Z * 256 / (256 - t),  O = Pd V,  LSE = the log-sum-exp of the logits
  *   (unchanged by dropout); the backward regenerates Z, so nothing N x N is stored.
- * Z[i][j] = 0 iff word (j mod 4) of Philox-4x32-10 (Salmon, Moraes, Dror and Shaw,
- * "Parallel random numbers: as easy as 1, 2, 3", SC 2011) at counter
- * (j / 4, i, b * H + h, offset) under key (seed & 0xffffffff, seed >> 32) is below
- * min(floor(p_drop * 2^32), 2^32 - 1). `offset` lets successive calls draw
- * independent masks under one seed. The backward must be given the same seed,
+ * One Philox-4x32-10 block (Salmon, Moraes, Dror and Shaw, "Parallel random numbers:
+ * as easy as 1, 2, 3", SC 2011) covers 4 queries x 4 keys: the block at counter
+ * (j / 4, i / 4, b * H + h, offset) under key (seed & 0xffffffff, seed >> 32) gives
+ * query i its word i mod 4 and key j byte j mod 4 of that word (byte 0 the least
+ * significant); Z[i][j] = 0 iff that byte is below t. `offset` lets successive calls
+ * draw independent masks under one seed. The backward must be given the same seed,
  * offset, p_drop and masks as the forward. p_drop = 0 is no dropout; p_drop outside
  * [0, 1) (or NaN) is FA_ERR_INVALID_ARG.
  */

@@ -140,7 +140,8 @@ def _dropout(dropout):
 
 def fa_forward_dropout(Q, K, V, O, LSE, scale: float, causal: bool, dropout, window=None,
                        block_mask=None, stream=None) -> None:
-    """fa_forward_masked with dropout=(p, seed, offset) on P (Philox-4x32-10 mask)."""
+    """fa_forward_masked with dropout=(p, seed, offset) on P (Philox-4x32-10 mask, one
+    byte per element; the drop rate is p rounded down to a multiple of 1/256)."""
     B, H, N, d = _shape(Q)
     bf = torch.bfloat16
     args = [_need("Q", Q, bf, (B, H, N, d)), _need("K", K, bf, (B, H, N, d)),

@@ -504,6 +504,28 @@ __global__ void __launch_bounds__(kThreads, 1)
             tmem_ld16(tm_s + 16 * (cc + 1), sv[cur ^ 1]);
             tmem_ld16(tm_dp + 16 * (cc + 1), dv[cur ^ 1]);
           }
+          // Dropout bytes of this key for the chunk's 16 queries: byte e of zq[v] is
+          // query 16cc + 4v + e of the half. One block covers 4 queries x 4 keys, and
+          // the lanes of keys 4g..4g+3 share its counter: lane u draws the block of the
+          // query group (qh0 + 16cc) / 4 + u, regroups its bytes by key (zq[b] = byte b
+          // of words 0..3) and a 4 x 4 transpose across the four lanes hands each lane
+          // its own key's bytes of all four blocks.
+          [[maybe_unused]] uint32_t zq[4] = {0u, 0u, 0u, 0u};
+          if constexpr (kDropout) {
+            const int u = lane & 3;
+            const uint4 w = philox4x32_10(
+                make_uint4(static_cast<uint32_t>(key >> 2),
+                           static_cast<uint32_t>(((qh0 + cc * 16) >> 2) + u),
+                           static_cast<uint32_t>(bh), p.drop.offset),
+                p.drop.seed_lo, p.drop.seed_hi);
+            const uint32_t t0 = __byte_perm(w.x, w.y, 0x5140), t1 = __byte_perm(w.x, w.y, 0x7362);
+            const uint32_t t2 = __byte_perm(w.z, w.w, 0x5140), t3 = __byte_perm(w.z, w.w, 0x7362);
+            zq[0] = __byte_perm(t0, t2, 0x5410);
+            zq[1] = __byte_perm(t0, t2, 0x7632);
+            zq[2] = __byte_perm(t1, t3, 0x5410);
+            zq[3] = __byte_perm(t1, t3, 0x7632);
+            transpose4_lanes(zq, u);
+          }
           uint32_t pk[8], dk[8];
 #pragma unroll
           for (int v = 0; v < 4; ++v) {
@@ -512,32 +534,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float Ls[4] = {L4.x, L4.y, L4.z, L4.w};
             const float Ds[4] = {D4.x, D4.y, D4.z, D4.w};
             float pv[4], dsv[4];
-            // Dropout words for this key and queries qh0 + 16cc + 4v + e: the counter
-            // (key / 4, query, bh, offset) is shared by the four lanes holding keys
-            // 4g..4g+3 (key mod 4 = lane mod 4), so lane u draws the block of query
-            // 4v + u and a transpose across the four lanes hands each its own word.
-            [[maybe_unused]] uint32_t zw[4] = {0u, 0u, 0u, 0u};
-            if constexpr (kDropout) {
-              const int u = lane & 3;
-              const uint4 w = philox4x32_10(
-                  make_uint4(static_cast<uint32_t>(key >> 2),
-                             static_cast<uint32_t>(qh0 + cc * 16 + 4 * v + u),
-                             static_cast<uint32_t>(bh), p.drop.offset),
-                  p.drop.seed_lo, p.drop.seed_hi);
-              zw[0] = w.x;
-              zw[1] = w.y;
-              zw[2] = w.z;
-              zw[3] = w.w;
-              transpose4_lanes(zw, u);
-            }
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const int k = 4 * v + e;
               float pe = ex2_approx(fmaf(__uint_as_float(sv[cur][k]), c, -Ls[e]));
               if (kM && static_cast<unsigned>(qoff + cc * 16 + k) >= q_span) pe = 0.f;
               if constexpr (kDropout) {
-                // dV takes P o Z / (1 - p) and dS = P o (dP o Z / (1 - p) - D)
-                const float zs = (zw[e] >= p.drop.threshold) ? p.drop.scale : 0.0f;
+                // dV takes P o Z * scale and dS = P o (dP o Z * scale - D), with
+                // scale = 1 / (1 - threshold / 256)
+                const float zs =
+                    (((zq[v] >> (8 * e)) & 0xffu) >= p.drop.threshold) ? p.drop.scale : 0.0f;
                 pv[e] = pe * zs;
                 dsv[e] = pe * (__uint_as_float(dv[cur][k]) * zs - Ds[e]);
               } else {

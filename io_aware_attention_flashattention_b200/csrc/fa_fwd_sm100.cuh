@@ -467,7 +467,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float2 c2 = make_float2(c, c), nm2 = make_float2(-m_use, -m_use);
       float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                        make_float2(0.f, 0.f)};
-      uint4 rnd = make_uint4(0u, 0u, 0u, 0u);  // Philox words of the current 4 keys (dropout)
+      // dropout: this row's four words for the current 16 keys (byte b of word m is key
+      // 4m + b of the group)
+      [[maybe_unused]] uint32_t zw[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
         uint32_t pk[16];
@@ -483,16 +485,28 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           acc[k & 3] = fadd2(acc[k & 3], pe);  // l is the sum before dropout
           if constexpr (kDropout) {
-            // keys kv0 + 32cc + 2k, +1: words (2k mod 4), +1 of the counter for the four
-            // keys starting at kv0 + 32cc + 4(k / 2)
-            if ((k & 1) == 0)
-              rnd = philox4x32_10(make_uint4(static_cast<uint32_t>((kv0 + 32 * cc + 2 * k) >> 2),
-                                             static_cast<uint32_t>(row), static_cast<uint32_t>(bh),
-                                             p.drop.offset),
-                                  p.drop.seed_lo, p.drop.seed_hi);
-            const uint32_t wa = (k & 1) ? rnd.z : rnd.x, wb = (k & 1) ? rnd.w : rnd.y;
-            pe.x = (wa >= p.drop.threshold) ? pe.x * p.drop.scale : 0.0f;
-            pe.y = (wb >= p.drop.threshold) ? pe.y * p.drop.scale : 0.0f;
+            // One block covers 4 rows x 4 keys; the lanes of rows 4g..4g+3 share its
+            // counter. Every 16 keys, lane u (row mod 4) draws the block of keys
+            // 4u..4u+3 of the 16, and a 4 x 4 transpose across the four lanes hands
+            // each lane its own row's word of all four blocks.
+            if ((k & 7) == 0) {
+              const int u = lane & 3;
+              const uint4 w = philox4x32_10(
+                  make_uint4(static_cast<uint32_t>(((kv0 + 32 * cc + 2 * k) >> 2) + u),
+                             static_cast<uint32_t>(row >> 2), static_cast<uint32_t>(bh),
+                             p.drop.offset),
+                  p.drop.seed_lo, p.drop.seed_hi);
+              zw[0] = w.x;
+              zw[1] = w.y;
+              zw[2] = w.z;
+              zw[3] = w.w;
+              transpose4_lanes(zw, u);
+            }
+            // keys 2k, 2k + 1 of the chunk = keys 2(k mod 8), +1 of the group: word
+            // (k mod 8) / 2, bytes 2(k mod 2) and 2(k mod 2) + 1
+            const uint32_t wd = zw[(k & 7) >> 1] >> (16 * (k & 1));
+            pe.x = ((wd & 0xffu) >= p.drop.threshold) ? pe.x * p.drop.scale : 0.0f;
+            pe.y = (((wd >> 8) & 0xffu) >= p.drop.threshold) ? pe.y * p.drop.scale : 0.0f;
           }
           pk[k] = pack2<E>(pe.x, pe.y);
         }

@@ -204,8 +204,9 @@ fa_status make_mask(int N, int causal, int window_left, int window_right,
   return FA_OK;
 }
 
-// Dropout as the kernels take it: keep iff the Philox word >= threshold, where
-// threshold = min(floor(p * 2^32), 2^32 - 1); kept values scaled by 1 / (1 - p).
+// Dropout as the kernels take it: keep iff the element's Philox byte >= threshold,
+// where threshold = floor(256 p) (the drop probability is threshold / 256); kept
+// values are scaled by 256 / (256 - threshold).
 struct DropSpec {
   bool on = false;
   DropoutParams params{};
@@ -214,10 +215,11 @@ struct DropSpec {
 fa_status make_drop(float p_drop, uint64_t seed, uint32_t offset, DropSpec* d) {
   if (!(p_drop >= 0.0f && p_drop < 1.0f)) return FA_ERR_INVALID_ARG;
   d->on = p_drop > 0.0f;
-  double t = std::floor(static_cast<double>(p_drop) * 4294967296.0);
-  if (t > 4294967295.0) t = 4294967295.0;
+  // one byte per element: the drop probability is floor(256 p) / 256
+  double t = std::floor(static_cast<double>(p_drop) * 256.0);
+  if (t > 255.0) t = 255.0;
   d->params.threshold = static_cast<uint32_t>(t);
-  d->params.scale = static_cast<float>(1.0 / (1.0 - static_cast<double>(p_drop)));
+  d->params.scale = static_cast<float>(256.0 / (256.0 - t));
   d->params.seed_lo = static_cast<uint32_t>(seed);
   d->params.seed_hi = static_cast<uint32_t>(seed >> 32);
   d->params.offset = offset;

@@ -474,9 +474,10 @@ __device__ __forceinline__ void transpose4_lanes(uint32_t (&a)[4], int u) {
   }
 }
 
-// Dropout on P: key j of query row i in head bh is kept iff word (j mod 4) of
-// philox4x32_10((j / 4, i, bh, offset), seed) is at least `threshold`
-// (= floor(p * 2^32)); kept values are scaled by 1 / (1 - p).
+// Dropout on P: key j of query row i in head bh is kept iff byte (j mod 4) of word
+// (i mod 4) of philox4x32_10((j / 4, i / 4, bh, offset), seed) is at least
+// `threshold` (= floor(256 p), so the drop probability is threshold / 256); kept
+// values are scaled by `scale` = 256 / (256 - threshold).
 struct DropoutParams {
   uint32_t threshold;
   float scale;
