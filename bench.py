@@ -53,6 +53,9 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle sample")
+    ap.add_argument("--reference-seconds", type=float, default=150.0,
+                    help="--impl reference: CPU time of the whole run (warm-up and timed "
+                         "steps), split evenly over the steps")
     return ap.parse_args()
 
 
@@ -256,7 +259,7 @@ def reference_arm(args, w):
     from io_aware_attention_flashattention_b200.inputs import workload_inputs
 
     inputs = workload_inputs(w)
-    budget = 150.0 / max(1, args.steps + args.warmup)
+    budget = args.reference_seconds / max(1, args.steps + args.warmup)
     for i in range(args.warmup):
         oracle_sample(w, budget, rng_seed=i, inputs=inputs)
     flops = secs = 0.0

@@ -109,3 +109,42 @@ def test_oracle_sample_is_bounded_and_counts_visible_pairs():
     per_row = flops / rows / (10.0 * w.d)
     assert 1.0 <= per_row <= w.N
     assert per_row == pytest.approx((w.N + 1) / 2, rel=0.5)
+
+
+def test_reference_arm_prints_the_contract_line():
+    """`bench.py --impl reference` runs the oracle alone on the host cores (no GPU)
+    and prints one JSON line with the reference arm's keys."""
+    import subprocess
+    import sys
+
+    out = subprocess.run(
+        [sys.executable, os.path.join(bench.ROOT, "bench.py"), "--impl", "reference",
+         "--workload", "gpt2_causal_b8h12_n1024_d64", "--steps", "2", "--warmup", "1",
+         "--reference-seconds", "1.5"],
+        capture_output=True, text=True, timeout=120, cwd=bench.ROOT)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC
+    assert d["unit"] == "TFLOP/s" and d["higher_is_better"] is True
+    assert d["steps"] == 2 and d["warmup"] == 1 and d["value"] > 0
+    assert d["config"]["workload"] == "gpt2_causal_b8h12_n1024_d64"
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["cpu_baseline"]["cores"] >= 1
+    assert d["e2e"] == {"value": d["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    """Under torchrun only rank 0 runs the oracle; the other ranks exit 0 at once."""
+    import subprocess
+    import sys
+
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    out = subprocess.run(
+        [sys.executable, os.path.join(bench.ROOT, "bench.py"), "--impl", "reference",
+         "--gpus", "2", "--steps", "3", "--warmup", "3"],
+        capture_output=True, text=True, timeout=60, cwd=bench.ROOT, env=env)
+    assert out.returncode == 0, out.stderr[-2000:]
+    assert not [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
