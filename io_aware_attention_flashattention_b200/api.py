@@ -15,6 +15,8 @@ LSE = natural-log log-sum-exp per query row, for [B, H, N, d] tensors, d in
 """
 from __future__ import annotations
 
+import contextlib
+import functools
 import math
 
 import torch
@@ -29,6 +31,29 @@ __all__ = [
     "fa_backward_f32", "fa_get_status", "fa_watchdog_selftest", "fa_version",
     "forward", "backward", "attention", "FlashAttentionFunction",
 ]
+
+
+def _one_device(*args):
+    """A context that makes current the one CUDA device of a call's tensors (and
+    stream): the library launches on the current device, and a stream left as None
+    is that device's current stream. Arguments on two different GPUs raise."""
+    devs = set()
+    for a in args:
+        dev = getattr(a, "device", None)
+        if isinstance(dev, torch.device) and dev.type == "cuda" and dev.index is not None:
+            devs.add(dev)
+    if len(devs) > 1:
+        raise ValueError("the tensors of one call must be on one GPU, got "
+                         + ", ".join(sorted(str(x) for x in devs)))
+    return torch.cuda.device(devs.pop()) if devs else contextlib.nullcontext()
+
+
+def _on_one_device(fn):
+    @functools.wraps(fn)
+    def call(*args, **kwargs):
+        with _one_device(*args, *kwargs.values()):
+            return fn(*args, **kwargs)
+    return call
 
 
 def _stream(stream) -> int:
@@ -65,6 +90,7 @@ def fa_backward_workspace_size(B: int, H: int, N: int, d: int) -> int:
     return int(lib().fa_backward_workspace_size(B, H, N, d))
 
 
+@_on_one_device
 def fa_forward(Q, K, V, O, LSE, scale: float, causal: bool, stream=None) -> None:
     B, H, N, d = _shape(Q)
     bf = torch.bfloat16
@@ -75,6 +101,7 @@ def fa_forward(Q, K, V, O, LSE, scale: float, causal: bool, stream=None) -> None
                                          _stream(stream)))
 
 
+@_on_one_device
 def fa_forward_f16(Q, K, V, O, LSE, scale: float, causal: bool, stream=None) -> None:
     B, H, N, d = _shape(Q)
     h = torch.float16
@@ -106,6 +133,7 @@ def _window(window):
     return int(left), int(right)
 
 
+@_on_one_device
 def fa_forward_masked(Q, K, V, O, LSE, scale: float, causal: bool, window=None,
                       block_mask=None, stream=None) -> None:
     """fa_forward with a sliding window (left, right) (negative = unbounded side)
@@ -121,6 +149,7 @@ def fa_forward_masked(Q, K, V, O, LSE, scale: float, causal: bool, window=None,
         _stream(stream)))
 
 
+@_on_one_device
 def fa_backward_masked(Q, K, V, O, dO, LSE, dQ, dK, dV, scale: float, causal: bool, workspace,
                        window=None, block_mask=None, stream=None) -> None:
     ptrs, (B, H, N, d), ws, nbytes = _bwd_args(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace,
@@ -138,6 +167,7 @@ def _dropout(dropout):
     return float(p), int(seed) & ((1 << 64) - 1), int(offset) & 0xFFFFFFFF
 
 
+@_on_one_device
 def fa_forward_dropout(Q, K, V, O, LSE, scale: float, causal: bool, dropout, window=None,
                        block_mask=None, stream=None) -> None:
     """fa_forward_masked with dropout=(p, seed, offset) on P (Philox-4x32-10 mask, one
@@ -153,6 +183,7 @@ def fa_forward_dropout(Q, K, V, O, LSE, scale: float, causal: bool, dropout, win
         *_dropout(dropout), _stream(stream)))
 
 
+@_on_one_device
 def fa_backward_dropout(Q, K, V, O, dO, LSE, dQ, dK, dV, scale: float, causal: bool, workspace,
                         dropout, window=None, block_mask=None, stream=None) -> None:
     ptrs, (B, H, N, d), ws, nbytes = _bwd_args(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace,
@@ -163,6 +194,7 @@ def fa_backward_dropout(Q, K, V, O, dO, LSE, dQ, dK, dV, scale: float, causal: b
         *_dropout(dropout), ws, nbytes, _stream(stream)))
 
 
+@_on_one_device
 def fa_forward_f32(Q, K, V, O, LSE, scale: float, causal: bool, stream=None) -> None:
     B, H, N, d = _shape(Q)
     f = torch.float32
@@ -185,6 +217,7 @@ def _bwd_args(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace, dtype):
     return ptrs, (B, H, N, d), workspace.data_ptr(), workspace.numel() * workspace.element_size()
 
 
+@_on_one_device
 def fa_backward(Q, K, V, O, dO, LSE, dQ, dK, dV, scale: float, causal: bool, workspace,
                 stream=None) -> None:
     ptrs, (B, H, N, d), ws, nbytes = _bwd_args(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace,
@@ -199,6 +232,7 @@ def _ws(workspace):
     return workspace.data_ptr(), workspace.numel() * workspace.element_size()
 
 
+@_on_one_device
 def fa_backward_preprocess(O, dO, LSE, scale: float, causal: bool, workspace, stream=None):
     B, H, N, d = _shape(O)
     bf = torch.bfloat16
@@ -209,6 +243,7 @@ def fa_backward_preprocess(O, dO, LSE, scale: float, causal: bool, workspace, st
         int(bool(causal)), ws, nbytes, _stream(stream)))
 
 
+@_on_one_device
 def fa_backward_main(Q, K, V, dO, dK, dV, scale: float, causal: bool, workspace, stream=None):
     B, H, N, d = _shape(Q)
     s4, bf = (B, H, N, d), torch.bfloat16
@@ -219,6 +254,7 @@ def fa_backward_main(Q, K, V, dO, dK, dV, scale: float, causal: bool, workspace,
         B, H, N, d, float(scale), int(bool(causal)), ws, nbytes, _stream(stream)))
 
 
+@_on_one_device
 def fa_backward_dq_convert(dQ, scale: float, workspace, stream=None):
     B, H, N, d = _shape(dQ)
     ws, nbytes = _ws(workspace)
@@ -227,6 +263,7 @@ def fa_backward_dq_convert(dQ, scale: float, workspace, stream=None):
         _stream(stream)))
 
 
+@_on_one_device
 def fa_backward_noalloc(Q, K, V, O, dO, LSE, dQ, dK, dV, scale: float, causal: bool,
                         stream=None) -> None:
     """fa_backward for callers that cannot allocate device memory: the workspace
@@ -244,6 +281,7 @@ def fa_backward_noalloc(Q, K, V, O, dO, LSE, dQ, dK, dV, scale: float, causal: b
         *ptrs, B, H, N, d, float(scale), int(bool(causal)), _stream(stream)))
 
 
+@_on_one_device
 def fa_backward_f16(Q, K, V, O, dO, LSE, dQ, dK, dV, scale: float, causal: bool, workspace,
                     stream=None) -> None:
     ptrs, (B, H, N, d), ws, nbytes = _bwd_args(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace,
@@ -253,6 +291,7 @@ def fa_backward_f16(Q, K, V, O, dO, LSE, dQ, dK, dV, scale: float, causal: bool,
                                                    _stream(stream)))
 
 
+@_on_one_device
 def fa_backward_f32(Q, K, V, O, dO, LSE, dQ, dK, dV, scale: float, causal: bool, workspace,
                     stream=None) -> None:
     ptrs, (B, H, N, d), ws, nbytes = _bwd_args(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace,
@@ -262,12 +301,14 @@ def fa_backward_f32(Q, K, V, O, dO, LSE, dQ, dK, dV, scale: float, causal: bool,
                                                    _stream(stream)))
 
 
+@_on_one_device
 def fa_get_status(stream=None) -> int:
     """Synchronises the stream; returns the library status code (0 = ok, 4 = a
     kernel's bounded wait ran out since the last call)."""
     return int(lib().fa_get_status(_stream(stream)))
 
 
+@_on_one_device
 def fa_watchdog_selftest(timeout_ms: int, stream=None) -> None:
     check("fa_watchdog_selftest", lib().fa_watchdog_selftest(int(timeout_ms), _stream(stream)))
 

@@ -115,3 +115,25 @@ def test_host_validation_of_every_entry_point(libfa):
                  P, ws, None) == 1
     f32 = _fn(libfa, "fa_backward_f32")
     assert f32(P, P, P, P, P, P, P, P, P, 1, 2, 384, 64, 0.1, 0, P, ws - 1, None) == 1
+
+
+def test_binding_runs_each_call_on_its_tensors_gpu():
+    """Every entry point of the binding makes its tensors' GPU current (the library
+    launches on the current device) and refuses tensors spread over two GPUs."""
+    import types
+
+    import torch
+
+    from io_aware_attention_flashattention_b200 import api
+
+    on = lambda i: types.SimpleNamespace(device=torch.device("cuda", i))  # noqa: E731
+    with pytest.raises(ValueError, match="one GPU"):
+        api._one_device(on(0), on(1))
+    ctx = api._one_device(on(1), on(1), torch.zeros(1), 7, None)
+    assert isinstance(ctx, torch.cuda.device) and ctx.idx == 1
+    assert not isinstance(api._one_device(torch.zeros(1), 3.0), torch.cuda.device)
+    for name in api.__all__:
+        fn = getattr(api, name)
+        if name.startswith("fa_") and callable(fn) and name not in (
+                "fa_version", "fa_backward_workspace_size"):
+            assert getattr(fn, "__wrapped__", None) is not None, f"{name} is not device-guarded"
