@@ -37,7 +37,10 @@
  *     return early, leaving its outputs undefined; fa_get_status() reports it as
  *     FA_ERR_TIMEOUT.
  *   - Supported: B, H >= 1; N >= 0 (N = 0 is a no-op); d in {64, 128};
- *     causal in {0, 1}; scale finite and > 0; B*H*N*d < 2^31.
+ *     causal in {0, 1}; scale finite and > 0; N <= 2^30 and
+ *     B*H*ceil(N/128) < 2^27 (a bound on the launch grids; tensor offsets are
+ *     64-bit, so one tensor may exceed 2^31 elements). Larger shapes return
+ *     FA_ERR_UNSUPPORTED.
  *   - Outputs are overwritten, never accumulated into.
  */
 #ifndef FA_B200_FA_H
@@ -135,7 +138,8 @@ fa_status fa_backward_dq_convert(void* dQ, int B, int H, int N, int d, float sca
  *     bytes) return FA_ERR_UNSUPPORTED and launch nothing.
  *   Set-up: the first call on a GPU looks up the array's device address with
  *     that GPU current (and may load the library's module there); make that first
- *     call before any stream capture.
+ *     call before any stream capture. If the GPU's context is destroyed and
+ *     created again (cudaDeviceReset), the next call looks the address up again.
  *   Sharing: every call on a GPU uses the same array. Each call rewrites all of
  *     it that it reads (the dQ accumulator is zeroed by the call itself), but two
  *     calls whose kernels can overlap on the GPU (different streams without an
@@ -209,12 +213,20 @@ fa_status fa_backward_masked(const void* Q, const void* K, const void* V, const 
  * significant); Z[i][j] = 0 iff that byte is below t. `offset` lets successive calls
  * draw independent masks under one seed. The backward must be given the same seed,
  * offset, p_drop and masks as the forward. p_drop = 0 is no dropout; p_drop outside
- * [0, 1) (or NaN) is FA_ERR_INVALID_ARG.
+ * [0, 1) (or NaN) is FA_ERR_INVALID_ARG; p_drop in (0, 1/256), which would round
+ * down to no dropout, is FA_ERR_UNSUPPORTED. fa_dropout_rate(p_drop) returns the
+ * rate actually applied.
  */
 fa_status fa_forward_dropout(const void* Q, const void* K, const void* V, void* O, float* LSE,
                              int B, int H, int N, int d, float scale, int causal,
                              int window_left, int window_right, const uint8_t* block_mask,
                              float p_drop, uint64_t seed, uint32_t offset, fa_stream_t stream);
+/*
+ * The drop probability the dropout calls apply for `p_drop`: floor(256 p_drop) / 256
+ * (for example 0.1 gives 25/256 = 0.09765625). Returns -1 for a p_drop those calls
+ * refuse (outside [0, 1), NaN, or in (0, 1/256)). Host only; no CUDA call.
+ */
+float fa_dropout_rate(float p_drop);
 fa_status fa_backward_dropout(const void* Q, const void* K, const void* V, const void* O,
                               const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
                               int B, int H, int N, int d, float scale, int causal,

@@ -35,6 +35,7 @@ SIGNATURES = {
                                _vp]),
     "fa_backward_masked": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                 _i, _i, _i, _i, _f, _i, _i, _i, _vp, _vp, _sz, _vp]),
+    "fa_dropout_rate": (_f, [_f]),
     "fa_forward_dropout": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _i, _i, _vp,
                                 _f, _u64, _u32, _vp]),
     "fa_backward_dropout": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,

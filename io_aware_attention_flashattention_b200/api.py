@@ -28,7 +28,7 @@ __all__ = [
     "fa_backward_preprocess", "fa_backward_main", "fa_backward_dq_convert",
     "fa_backward_noalloc", "fa_forward_f16", "fa_backward_f16", "fa_forward_masked",
     "fa_backward_masked", "fa_forward_dropout", "fa_backward_dropout", "fa_forward_f32",
-    "fa_backward_f32", "fa_get_status", "fa_watchdog_selftest", "fa_version",
+    "fa_backward_f32", "fa_get_status", "fa_watchdog_selftest", "fa_version", "fa_dropout_rate",
     "forward", "backward", "attention", "FlashAttentionFunction",
 ]
 
@@ -158,6 +158,16 @@ def fa_backward_masked(Q, K, V, O, dO, LSE, dQ, dK, dV, scale: float, causal: bo
     check("fa_backward_masked", lib().fa_backward_masked(
         *ptrs, B, H, N, d, float(scale), int(bool(causal)), wl, wr, _block_mask(block_mask, N),
         ws, nbytes, _stream(stream)))
+
+
+def fa_dropout_rate(p: float) -> float:
+    """The drop probability the dropout calls apply for ``p``: p rounded down to a
+    multiple of 1/256. Raises ValueError for a rate they refuse (outside [0, 1), or
+    in (0, 1/256), which would round down to no dropout)."""
+    r = float(lib().fa_dropout_rate(float(p)))
+    if r < 0:
+        raise ValueError(f"dropout rate {p} is outside [0, 1) or below 1/256")
+    return r
 
 
 def _dropout(dropout):

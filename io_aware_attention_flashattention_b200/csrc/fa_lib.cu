@@ -16,6 +16,7 @@
 #include <mutex>
 #include <queue>
 #include <tuple>
+#include <utility>
 #include <vector>
 
 #include "fa_ptx.cuh"
@@ -73,15 +74,69 @@ unsigned long long watchdog_ns() {
   return v;
 }
 
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+
+// Unique id of the calling thread's current CUDA context, or 0 if it cannot be
+// had. A context that is destroyed and created again (cudaDeviceReset, or the
+// primary context released and retained) gets a new id, so per-context state
+// cached under the old id is never used with the new context. The runtime makes
+// the device's primary context current first (cudaSetDevice initialises it).
+unsigned long long current_ctx_id() {
+  static CtxGetCurrentFn get_current = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<CtxGetCurrentFn>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  if (!get_current || !get_id) return 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaSetDevice(dev) != cudaSuccess) return 0;
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
 constexpr int kMaxDevices = 64;
 struct DeviceState {
   bool checked = false;
   bool supported = false;
-  bool attrs_done = false;
   int sms = 0;  // streaming multiprocessors
+  // The kernels' shared-memory limits are attributes of the context: they are
+  // set again whenever the current context's id differs from the one they were
+  // set in (0 = never set).
+  unsigned long long attrs_ctx = 0;
 };
 DeviceState g_devices[kMaxDevices];
 std::mutex g_mutex;
+
+// Launches `kernel` and returns the status of this launch alone: an error left
+// pending by earlier, unrelated CUDA work is neither reported nor cleared. A
+// failed launch's own error is cleared, so that it does not surface later in the
+// caller's error checks.
+template <typename... KArgs, typename... Args>
+fa_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                 Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+  if (e == cudaSuccess) return FA_OK;
+  (void)cudaGetLastError();
+  return FA_ERR_CUDA;
+}
 
 template <typename Kern>
 cudaError_t set_smem(Kern k, size_t bytes) {
@@ -129,7 +184,8 @@ fa_status prepare_device() {
     st.checked = true;
   }
   if (!st.supported) return FA_ERR_UNSUPPORTED;
-  if (!st.attrs_done) {
+  const unsigned long long ctx = current_ctx_id();
+  if (ctx == 0 || st.attrs_ctx != ctx) {
     cudaError_t e = cudaSuccess;
     e = e ? e : set_smem_all<Elt::BF16>();
     e = e ? e : set_smem_all<Elt::F16>();
@@ -138,7 +194,7 @@ fa_status prepare_device() {
     e = e ? e : set_smem(f32::fa_f32_bwd_dq_kernel<64>, f32::dq_smem_bytes<64>());
     e = e ? e : set_smem(f32::fa_f32_bwd_dq_kernel<128>, f32::dq_smem_bytes<128>());
     if (e != cudaSuccess) return FA_ERR_CUDA;
-    st.attrs_done = true;
+    st.attrs_ctx = ctx;
   }
   return FA_OK;
 }
@@ -150,8 +206,14 @@ fa_status check_shape(int B, int H, int N, int d, float scale, int causal) {
   if (!(std::isfinite(scale) && scale > 0.0f)) return FA_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
-  const long long total = static_cast<long long>(B) * H * N * d;
-  if (total >= (1ll << 31)) return FA_ERR_UNSUPPORTED;
+  // Offsets into the tensors are 64-bit. The bound is on the grids: one grid
+  // dimension holds every (batch, head) x row block, and the smallest blocks (8 rows
+  // of the backward preprocess, 16 of the fp32 kernels) number at most
+  // 16 * B * H * ceil(N / 128).
+  const long long tiles = static_cast<long long>(B) * H * ((static_cast<long long>(N) + 127) / 128);
+  // Row indices stay 32-bit: N <= 2^30 keeps every row + window sum below 2^31.
+  if (N > (1 << 30) || static_cast<long long>(B) * H >= (1ll << 31) || 16 * tiles >= (1ll << 31))
+    return FA_ERR_UNSUPPORTED;
   return FA_OK;
 }
 
@@ -212,12 +274,21 @@ struct DropSpec {
   DropoutParams params{};
 };
 
+// floor(256 p) for p in [0, 1), the byte threshold; -1 for p outside [0, 1).
+int drop_threshold(float p_drop) {
+  if (!(p_drop >= 0.0f && p_drop < 1.0f)) return -1;
+  const double t = std::floor(static_cast<double>(p_drop) * 256.0);
+  return static_cast<int>(std::min(t, 255.0));
+}
+
 fa_status make_drop(float p_drop, uint64_t seed, uint32_t offset, DropSpec* d) {
-  if (!(p_drop >= 0.0f && p_drop < 1.0f)) return FA_ERR_INVALID_ARG;
-  d->on = p_drop > 0.0f;
+  const int ti = drop_threshold(p_drop);
+  if (ti < 0) return FA_ERR_INVALID_ARG;
+  // A rate in (0, 1/256) has threshold 0: it would silently drop nothing.
+  if (ti == 0 && p_drop > 0.0f) return FA_ERR_UNSUPPORTED;
+  d->on = ti > 0;
   // one byte per element: the drop probability is floor(256 p) / 256
-  double t = std::floor(static_cast<double>(p_drop) * 256.0);
-  if (t > 255.0) t = 255.0;
+  const double t = ti;
   d->params.threshold = static_cast<uint32_t>(t);
   d->params.scale = static_cast<float>(256.0 / (256.0 - t));
   d->params.seed_lo = static_cast<uint32_t>(seed);
@@ -268,9 +339,15 @@ FwdSplit fwd_split(int BH, int N, int wl, int wr, int sms) {
   const int n_kt = (N + fwd::BN - 1) / fwd::BN;
   const int min_singles = n_qt % 2;
   FwdSplit plain{(n_qt - min_singles) / 2, min_singles};
-  if (sms <= 0 || static_cast<long long>(BH) * n_qt > 65536) return plain;
+  if (sms <= 0) return plain;
+  // Singles only help while they fit in the last wave: at most about sms / BH per
+  // head are tried. The simulation replays every CTA per candidate, so the total
+  // (candidates x CTAs) is bounded too; beyond it the plain split is used.
+  const int max_singles = std::min(n_qt, 2 * ((sms + BH - 1) / BH) + 1);
+  const long long candidates = (max_singles - min_singles) / 2 + 1;
+  if (candidates * BH * n_qt > (1ll << 22)) return plain;
   static std::mutex mu;
-  static std::map<std::tuple<int, int, int, int, int>, FwdSplit> cache;
+  static std::map<std::tuple<int, int, int, int, int>, FwdSplit> cache;  // at most 1024 shapes
   const auto key = std::make_tuple(BH, N, wl, wr, sms);
   {
     std::lock_guard<std::mutex> lock(mu);
@@ -287,7 +364,7 @@ FwdSplit fwd_split(int BH, int N, int wl, int wr, int sms) {
   }
   FwdSplit best = plain;
   double best_t = split_makespan(BH, n_qt, min_singles, sms, key_tiles);
-  for (int sg = min_singles + 2; sg <= n_qt; sg += 2) {
+  for (int sg = min_singles + 2; sg <= max_singles; sg += 2) {
     const double t = split_makespan(BH, n_qt, sg, sms, key_tiles);
     if (t < best_t * 0.999) {
       best_t = t;
@@ -295,6 +372,7 @@ FwdSplit fwd_split(int BH, int N, int wl, int wr, int sms) {
     }
   }
   std::lock_guard<std::mutex> lock(mu);
+  if (cache.size() >= 1024) cache.clear();
   cache[key] = best;
   return best;
 }
@@ -306,9 +384,6 @@ int device_sms() {
   return g_devices[dev].sms;
 }
 
-fa_status launch_status() {
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
-}
 
 }  // namespace
 }  // namespace fa
@@ -353,28 +428,20 @@ fa_status forward_impl(const void* Q, const void* K, const void* V, void* O, flo
   const dim3 grid(static_cast<unsigned>(BH) * (split.pairs_ph + split.singles_ph));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool g = mask.general();
+  constexpr int T = fwd::kThreads;
+  constexpr size_t S64 = fwd::Cfg<64>::kSmemBytes, S128 = fwd::Cfg<128>::kSmemBytes;
   if constexpr (E == Elt::BF16) {
     if (drop.on) {
-      if (d == 64)
-        fwd::fa_fwd_kernel<64, E, true, true><<<grid, fwd::kThreads, fwd::Cfg<64>::kSmemBytes, s>>>(
-            mq, mk, mv, p);
-      else
-        fwd::fa_fwd_kernel<128, E, true, true><<<grid, fwd::kThreads, fwd::Cfg<128>::kSmemBytes, s>>>(
-            mq, mk, mv, p);
-      return launch_status();
+      if (d == 64) return launch(fwd::fa_fwd_kernel<64, E, true, true>, grid, T, S64, s, mq, mk, mv, p);
+      return launch(fwd::fa_fwd_kernel<128, E, true, true>, grid, T, S128, s, mq, mk, mv, p);
     }
   } else if (drop.on) {
     return FA_ERR_UNSUPPORTED;
   }
-  if (d == 64 && !g)
-    fwd::fa_fwd_kernel<64, E, false><<<grid, fwd::kThreads, fwd::Cfg<64>::kSmemBytes, s>>>(mq, mk, mv, p);
-  else if (d == 64)
-    fwd::fa_fwd_kernel<64, E, true><<<grid, fwd::kThreads, fwd::Cfg<64>::kSmemBytes, s>>>(mq, mk, mv, p);
-  else if (!g)
-    fwd::fa_fwd_kernel<128, E, false><<<grid, fwd::kThreads, fwd::Cfg<128>::kSmemBytes, s>>>(mq, mk, mv, p);
-  else
-    fwd::fa_fwd_kernel<128, E, true><<<grid, fwd::kThreads, fwd::Cfg<128>::kSmemBytes, s>>>(mq, mk, mv, p);
-  return launch_status();
+  if (d == 64 && !g) return launch(fwd::fa_fwd_kernel<64, E, false>, grid, T, S64, s, mq, mk, mv, p);
+  if (d == 64) return launch(fwd::fa_fwd_kernel<64, E, true>, grid, T, S64, s, mq, mk, mv, p);
+  if (!g) return launch(fwd::fa_fwd_kernel<128, E, false>, grid, T, S128, s, mq, mk, mv, p);
+  return launch(fwd::fa_fwd_kernel<128, E, true>, grid, T, S128, s, mq, mk, mv, p);
 }
 
 // Shared validation and set-up of the three backward stages. Fills the tensor maps
@@ -424,12 +491,10 @@ fa_status preprocess_impl(const void* O, const void* dO, const float* LSE, int B
   const auto* dO16 = static_cast<const uint16_t*>(dO);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (d == 64)
-    bwd::fa_bwd_pre_kernel<64, E><<<blocks, 256, 0, s>>>(O16, dO16, LSE, pl.L2, pl.Dv, pl.dQacc, N,
-                                                      pl.Npad, rows);
-  else
-    bwd::fa_bwd_pre_kernel<128, E><<<blocks, 256, 0, s>>>(O16, dO16, LSE, pl.L2, pl.Dv, pl.dQacc, N,
-                                                       pl.Npad, rows);
-  return launch_status();
+    return launch(bwd::fa_bwd_pre_kernel<64, E>, blocks, 256, 0, s, O16, dO16, LSE, pl.L2, pl.Dv,
+                  pl.dQacc, N, pl.Npad, rows);
+  return launch(bwd::fa_bwd_pre_kernel<128, E>, blocks, 256, 0, s, O16, dO16, LSE, pl.L2, pl.Dv,
+                pl.dQacc, N, pl.Npad, rows);
 }
 
 template <Elt E>
@@ -466,28 +531,21 @@ fa_status main_impl(const void* Q, const void* K, const void* V, const void* dO,
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool g = mask.general();
   using bwd::Cfg;
+  constexpr int T = bwd::kThreads;
+  constexpr size_t S64 = Cfg<64>::kSmemBytes, S128 = Cfg<128>::kSmemBytes;
   if constexpr (E == Elt::BF16) {
     if (drop.on) {
       if (d == 64)
-        bwd::fa_bwd_kernel<64, E, true, true><<<grid, bwd::kThreads, Cfg<64>::kSmemBytes, s>>>(
-            mq, mk, mv, mdo, p);
-      else
-        bwd::fa_bwd_kernel<128, E, true, true><<<grid, bwd::kThreads, Cfg<128>::kSmemBytes, s>>>(
-            mq, mk, mv, mdo, p);
-      return launch_status();
+        return launch(bwd::fa_bwd_kernel<64, E, true, true>, grid, T, S64, s, mq, mk, mv, mdo, p);
+      return launch(bwd::fa_bwd_kernel<128, E, true, true>, grid, T, S128, s, mq, mk, mv, mdo, p);
     }
   } else if (drop.on) {
     return FA_ERR_UNSUPPORTED;
   }
-  if (d == 64 && !g)
-    bwd::fa_bwd_kernel<64, E, false><<<grid, bwd::kThreads, Cfg<64>::kSmemBytes, s>>>(mq, mk, mv, mdo, p);
-  else if (d == 64)
-    bwd::fa_bwd_kernel<64, E, true><<<grid, bwd::kThreads, Cfg<64>::kSmemBytes, s>>>(mq, mk, mv, mdo, p);
-  else if (!g)
-    bwd::fa_bwd_kernel<128, E, false><<<grid, bwd::kThreads, Cfg<128>::kSmemBytes, s>>>(mq, mk, mv, mdo, p);
-  else
-    bwd::fa_bwd_kernel<128, E, true><<<grid, bwd::kThreads, Cfg<128>::kSmemBytes, s>>>(mq, mk, mv, mdo, p);
-  return launch_status();
+  if (d == 64 && !g) return launch(bwd::fa_bwd_kernel<64, E, false>, grid, T, S64, s, mq, mk, mv, mdo, p);
+  if (d == 64) return launch(bwd::fa_bwd_kernel<64, E, true>, grid, T, S64, s, mq, mk, mv, mdo, p);
+  if (!g) return launch(bwd::fa_bwd_kernel<128, E, false>, grid, T, S128, s, mq, mk, mv, mdo, p);
+  return launch(bwd::fa_bwd_kernel<128, E, true>, grid, T, S128, s, mq, mk, mv, mdo, p);
 }
 
 template <Elt E>
@@ -500,11 +558,9 @@ fa_status dq_convert_impl(void* dQ, int B, int H, int N, int d, float scale, voi
   const long long n4 = static_cast<long long>(pl.BH) * N * d / 4;
   const unsigned blocks = static_cast<unsigned>(std::min<long long>((n4 + 255) / 256, 148 * 16));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (d == 64)
-    bwd::fa_bwd_dq_kernel<64, E><<<blocks, 256, 0, s>>>(pl.dQacc, static_cast<uint16_t*>(dQ), n4, scale);
-  else
-    bwd::fa_bwd_dq_kernel<128, E><<<blocks, 256, 0, s>>>(pl.dQacc, static_cast<uint16_t*>(dQ), n4, scale);
-  return launch_status();
+  uint16_t* dQ16 = static_cast<uint16_t*>(dQ);
+  if (d == 64) return launch(bwd::fa_bwd_dq_kernel<64, E>, blocks, 256, 0, s, pl.dQacc, dQ16, n4, scale);
+  return launch(bwd::fa_bwd_dq_kernel<128, E>, blocks, 256, 0, s, pl.dQacc, dQ16, n4, scale);
 }
 
 template <Elt E>
@@ -548,6 +604,12 @@ size_t fa_backward_workspace_size(int B, int H, int N, int d) {
   return 2 * round256(bh * npad * sizeof(float)) + round256(bh * N * d * sizeof(float));
 }
 
+float fa_dropout_rate(float p_drop) {
+  const int t = drop_threshold(p_drop);
+  if (t < 0 || (t == 0 && p_drop > 0.0f)) return -1.0f;
+  return static_cast<float>(t) / 256.0f;
+}
+
 fa_status fa_get_status(fa_stream_t stream) {
   if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return FA_ERR_CUDA;
@@ -566,9 +628,8 @@ fa_status fa_watchdog_selftest(int timeout_ms, fa_stream_t stream) {
   if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
     return FA_ERR_CUDA;
   if (major != 10) return FA_ERR_UNSUPPORTED;
-  watchdog_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      static_cast<unsigned long long>(timeout_ms) * 1000000ull);
-  return launch_status();
+  return launch(watchdog_selftest_kernel, 1, 32, 0, reinterpret_cast<cudaStream_t>(stream),
+                static_cast<unsigned long long>(timeout_ms) * 1000000ull);
 }
 
 fa_status fa_forward(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
@@ -661,10 +722,17 @@ fa_status fa_backward_f16(const void* Q, const void* K, const void* V, const voi
 constexpr size_t kNoAllocScratchBytes = 32ull << 20;  // 32 MiB per GPU
 static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
 
-// Device address of g_noalloc_scratch on each GPU. In host code the array's name
-// only stands in for the symbol; the address a kernel may use comes from
-// cudaGetSymbolAddress with that GPU current.
-static void* g_noalloc_ptr[kMaxDevices];
+// Device address of g_noalloc_scratch on each GPU, with the id of the context it
+// was looked up in. In host code the array's name only stands in for the symbol;
+// the address a kernel may use comes from cudaGetSymbolAddress with that GPU
+// current. If the context is destroyed and created again (cudaDeviceReset), the
+// module is loaded anew and the array may move: a changed context id makes the
+// next call look the address up again.
+struct NoAllocScratch {
+  unsigned long long ctx = 0;
+  void* ptr = nullptr;
+};
+static NoAllocScratch g_noalloc[kMaxDevices];
 
 fa_status fa_backward_noalloc(const void* Q, const void* K, const void* V, const void* O,
                               const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
@@ -678,14 +746,17 @@ fa_status fa_backward_noalloc(const void* Q, const void* K, const void* V, const
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
   void* scratch = nullptr;
   {
+    const unsigned long long ctx = current_ctx_id();  // 0: unknown, look up every call
     std::lock_guard<std::mutex> lock(g_mutex);
-    if (g_noalloc_ptr[dev] == nullptr) {
+    NoAllocScratch& e = g_noalloc[dev];
+    if (ctx == 0 || e.ctx != ctx || e.ptr == nullptr) {
       void* p = nullptr;
       if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || p == nullptr)
         return FA_ERR_CUDA;
-      g_noalloc_ptr[dev] = p;
+      e.ptr = p;
+      e.ctx = ctx;
     }
-    scratch = g_noalloc_ptr[dev];
+    scratch = e.ptr;
   }
   // The preprocess stage rewrites every byte of scratch the later stages read
   // (LSE*log2e, D, and the dQ accumulator it zeroes), so whatever an earlier call
@@ -729,13 +800,13 @@ fa_status fa_forward_f32(const float* Q, const float* K, const float* V, float* 
   if (N == 0) return FA_OK;
   if ((st = check_ptrs({Q, K, V, O, LSE})) != FA_OK) return st;
   if ((st = prepare_device()) != FA_OK) return st;
-  const dim3 grid((N + f32::kRowsPerBlock - 1) / f32::kRowsPerBlock, B * H);
+  // grid.x = (batch, head) x row blocks (check_shape bounds it below 2^31)
+  const dim3 grid(static_cast<unsigned>(static_cast<long long>(B) * H *
+                                        ((N + f32::kRowsPerBlock - 1) / f32::kRowsPerBlock)));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  if (d == 64)
-    f32::fa_f32_fwd_kernel<64><<<grid, f32::kWarps * 32, 0, s>>>(Q, K, V, O, LSE, N, scale, causal);
-  else
-    f32::fa_f32_fwd_kernel<128><<<grid, f32::kWarps * 32, 0, s>>>(Q, K, V, O, LSE, N, scale, causal);
-  return launch_status();
+  constexpr int T = f32::kWarps * 32;
+  if (d == 64) return launch(f32::fa_f32_fwd_kernel<64>, grid, T, 0, s, Q, K, V, O, LSE, N, scale, causal);
+  return launch(f32::fa_f32_fwd_kernel<128>, grid, T, 0, s, Q, K, V, O, LSE, N, scale, causal);
 }
 
 fa_status fa_backward_f32(const float* Q, const float* K, const float* V, const float* O,
@@ -752,21 +823,49 @@ fa_status fa_backward_f32(const float* Q, const float* K, const float* V, const 
   float* Dvec = static_cast<float*>(workspace);
   const long long rows = static_cast<long long>(B) * H * N;
   const unsigned dot_blocks = static_cast<unsigned>((rows + f32::kWarps - 1) / f32::kWarps);
-  const dim3 grid((N + f32::kRowsPerBlock - 1) / f32::kRowsPerBlock, B * H);
+  const dim3 grid(static_cast<unsigned>(static_cast<long long>(B) * H *
+                                        ((N + f32::kRowsPerBlock - 1) / f32::kRowsPerBlock)));
+  constexpr int T = f32::kWarps * 32;
   if (d == 64) {
-    f32::fa_f32_bwd_dot_kernel<64><<<dot_blocks, f32::kWarps * 32, 0, s>>>(O, dO, Dvec, rows);
-    f32::fa_f32_bwd_dkdv_kernel<64><<<grid, f32::kWarps * 32, f32::dkdv_smem_bytes<64>(), s>>>(
-        Q, K, V, dO, LSE, Dvec, dK, dV, N, scale, causal);
-    f32::fa_f32_bwd_dq_kernel<64><<<grid, f32::kWarps * 32, f32::dq_smem_bytes<64>(), s>>>(
-        Q, K, V, dO, LSE, Dvec, dQ, N, scale, causal);
+    st = launch(f32::fa_f32_bwd_dot_kernel<64>, dot_blocks, T, 0, s, O, dO, Dvec, rows);
+    if (st == FA_OK)
+      st = launch(f32::fa_f32_bwd_dkdv_kernel<64>, grid, T, f32::dkdv_smem_bytes<64>(), s, Q, K, V,
+                  dO, LSE, Dvec, dK, dV, N, scale, causal);
+    if (st == FA_OK)
+      st = launch(f32::fa_f32_bwd_dq_kernel<64>, grid, T, f32::dq_smem_bytes<64>(), s, Q, K, V, dO,
+                  LSE, Dvec, dQ, N, scale, causal);
   } else {
-    f32::fa_f32_bwd_dot_kernel<128><<<dot_blocks, f32::kWarps * 32, 0, s>>>(O, dO, Dvec, rows);
-    f32::fa_f32_bwd_dkdv_kernel<128><<<grid, f32::kWarps * 32, f32::dkdv_smem_bytes<128>(), s>>>(
-        Q, K, V, dO, LSE, Dvec, dK, dV, N, scale, causal);
-    f32::fa_f32_bwd_dq_kernel<128><<<grid, f32::kWarps * 32, f32::dq_smem_bytes<128>(), s>>>(
-        Q, K, V, dO, LSE, Dvec, dQ, N, scale, causal);
+    st = launch(f32::fa_f32_bwd_dot_kernel<128>, dot_blocks, T, 0, s, O, dO, Dvec, rows);
+    if (st == FA_OK)
+      st = launch(f32::fa_f32_bwd_dkdv_kernel<128>, grid, T, f32::dkdv_smem_bytes<128>(), s, Q, K,
+                  V, dO, LSE, Dvec, dK, dV, N, scale, causal);
+    if (st == FA_OK)
+      st = launch(f32::fa_f32_bwd_dq_kernel<128>, grid, T, f32::dq_smem_bytes<128>(), s, Q, K, V, dO,
+                  LSE, Dvec, dQ, N, scale, causal);
   }
-  return launch_status();
+  return st;
 }
+
+
+#ifdef FA_TRACE
+// Profiling aid (built only with -DFA_TRACE): arm the timeline trace for one CTA
+// of the next launches (clearing it), and read back the slots and the two global
+// timer stamps.
+int fa_trace_arm(int cta) {
+  static std::vector<uint32_t> zeros(kTraceCap, 0u);
+  if (cudaMemcpyToSymbol(g_trace, zeros.data(), kTraceCap * sizeof(uint32_t)) != cudaSuccess)
+    return -1;
+  if (cudaMemcpyToSymbol(g_trace_cta, &cta, sizeof(cta)) != cudaSuccess) return -1;
+  return 0;
+}
+int fa_trace_read(uint32_t* slots, unsigned long long* ns) {
+  if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+  if (cudaMemcpyFromSymbol(slots, g_trace, kTraceCap * sizeof(uint32_t)) != cudaSuccess)
+    return -1;
+  if (cudaMemcpyFromSymbol(ns, g_trace_ns, 2 * sizeof(unsigned long long)) != cudaSuccess)
+    return -1;
+  return static_cast<int>(kTraceCap);
+}
+#endif
 
 }  // extern "C"

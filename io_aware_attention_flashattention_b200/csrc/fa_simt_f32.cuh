@@ -63,8 +63,11 @@ __global__ void __launch_bounds__(kWarps * 32)
   __shared__ __align__(16) float sK[kTile * P];
   __shared__ __align__(16) float sV[kTile * P];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const size_t head = static_cast<size_t>(blockIdx.y) * N * D;
-  const int row0 = blockIdx.x * kRowsPerBlock;
+  // grid.x = (batch, head) x row blocks, head-major (grid.y is capped at 65535)
+  const int rblocks = (N + kRowsPerBlock - 1) / kRowsPerBlock;
+  const size_t bh = blockIdx.x / rblocks;
+  const size_t head = bh * N * D;
+  const int row0 = static_cast<int>(blockIdx.x % rblocks) * kRowsPerBlock;
   load_rows<D>(sQ, Q + head + static_cast<size_t>(row0) * D, kRowsPerBlock, N - row0);
 
   float m[kRowsPerWarp], l[kRowsPerWarp], acc[kRowsPerWarp][CPL];
@@ -127,7 +130,7 @@ __global__ void __launch_bounds__(kWarps * 32)
 #pragma unroll
     for (int c = 0; c < CPL; ++c) O[head + static_cast<size_t>(row) * D + lane + 32 * c] = acc[r][c] * inv;
     if (lane == 0)
-      LSE[static_cast<size_t>(blockIdx.y) * N + row] = l[r] > 0.f ? m[r] + logf(l[r]) : -INFINITY;
+      LSE[bh * N + row] = l[r] > 0.f ? m[r] + logf(l[r]) : -INFINITY;
   }
 }
 
@@ -174,9 +177,11 @@ __global__ void __launch_bounds__(kWarps * 32)
   float* sL = sdO + kTile * P;
   float* sD = sL + kTile;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const size_t head = static_cast<size_t>(blockIdx.y) * N * D;
-  const size_t hrow = static_cast<size_t>(blockIdx.y) * N;
-  const int key0 = blockIdx.x * kRowsPerBlock;
+  const int rblocks = (N + kRowsPerBlock - 1) / kRowsPerBlock;  // grid.x = heads x blocks
+  const size_t bh = blockIdx.x / rblocks;
+  const size_t head = bh * N * D;
+  const size_t hrow = bh * N;
+  const int key0 = static_cast<int>(blockIdx.x % rblocks) * kRowsPerBlock;
   load_rows<D>(sK, K + head + static_cast<size_t>(key0) * D, kRowsPerBlock, N - key0);
   load_rows<D>(sV, V + head + static_cast<size_t>(key0) * D, kRowsPerBlock, N - key0);
   float gk[kRowsPerWarp][CPL], gv[kRowsPerWarp][CPL];
@@ -258,9 +263,11 @@ __global__ void __launch_bounds__(kWarps * 32)
   float* sK = sdO + kRowsPerBlock * P;
   float* sV = sK + kTile * P;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const size_t head = static_cast<size_t>(blockIdx.y) * N * D;
-  const size_t hrow = static_cast<size_t>(blockIdx.y) * N;
-  const int row0 = blockIdx.x * kRowsPerBlock;
+  const int rblocks = (N + kRowsPerBlock - 1) / kRowsPerBlock;  // grid.x = heads x blocks
+  const size_t bh = blockIdx.x / rblocks;
+  const size_t head = bh * N * D;
+  const size_t hrow = bh * N;
+  const int row0 = static_cast<int>(blockIdx.x % rblocks) * kRowsPerBlock;
   load_rows<D>(sQ, Q + head + static_cast<size_t>(row0) * D, kRowsPerBlock, N - row0);
   load_rows<D>(sdO, dO + head + static_cast<size_t>(row0) * D, kRowsPerBlock, N - row0);
   float Lr[kRowsPerWarp], Dr[kRowsPerWarp], gq[kRowsPerWarp][CPL];

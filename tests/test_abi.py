@@ -84,7 +84,9 @@ def test_host_validation_of_every_entry_point(libfa):
     the documented status (1 invalid argument, 2 unsupported); no GPU is needed."""
     P = 0x10000  # a 16-byte-aligned stand-in address; a rejected call never touches it
     fwd = _fn(libfa, "fa_forward")
-    assert fwd(P, P, P, P, P, 1, 1, 1 << 24, 128, 0.1, 0, None) == 2  # B*H*N*d = 2^31
+    assert fwd(P, P, P, P, P, 1, 1, (1 << 30) + 1, 128, 0.1, 0, None) == 2  # N > 2^30
+    assert fwd(P, P, P, P, P, 1 << 14, 1 << 13, 128, 128, 0.1, 0, None) == 2  # B*H = 2^27 tiles
+    assert fwd(P, P, P, P, P, 1 << 16, 1 << 16, 0, 64, 0.1, 0, None) == 2  # B*H = 2^32
     assert fwd(P, P, P, P, P, 1, 1, 128, 64, float("nan"), 0, None) == 1
     assert fwd(P, P, P, P, P, 1, 1, 128, 64, 0.0, 0, None) == 1
     assert fwd(P, P, P, P, P, 1, 1, 128, 64, 0.1, 2, None) == 1
@@ -100,6 +102,8 @@ def test_host_validation_of_every_entry_point(libfa):
     drop = _fn(libfa, "fa_forward_dropout")
     for p in (1.0, -0.25, float("nan"), float("inf")):
         assert drop(P, P, P, P, P, 1, 1, 256, 64, 0.1, 0, -1, -1, None, p, 7, 0, None) == 1
+    # a rate below 1/256 would round down to no dropout at all: refused
+    assert drop(P, P, P, P, P, 1, 1, 256, 64, 0.1, 0, -1, -1, None, 0.003, 7, 0, None) == 2
     ws = _fn(libfa, "fa_backward_workspace_size")(1, 2, 384, 64)
     bwd = _fn(libfa, "fa_backward")
     assert bwd(P, P, P, P, P, P, P, P, P, 1, 2, 384, 64, 0.1, 0, P, ws - 1, None) == 1
@@ -115,6 +119,21 @@ def test_host_validation_of_every_entry_point(libfa):
                  P, ws, None) == 1
     f32 = _fn(libfa, "fa_backward_f32")
     assert f32(P, P, P, P, P, P, P, P, P, 1, 2, 384, 64, 0.1, 0, P, ws - 1, None) == 1
+    bdrop_ok = bdrop(P, P, P, P, P, P, P, P, P, 1, 2, 384, 64, 0.1, 0, -1, -1, None, 0.001, 1, 0,
+                     P, ws, None)
+    assert bdrop_ok == 2
+
+
+def test_dropout_rate_is_the_byte_threshold(libfa):
+    """fa_dropout_rate returns the drop probability the kernels apply: p rounded down
+    to a multiple of 1/256; -1 for a rate the dropout calls refuse."""
+    rate = _fn(libfa, "fa_dropout_rate")
+    assert rate(0.0) == 0.0
+    assert rate(0.1) == 25 / 256
+    assert rate(0.5) == 0.5
+    assert rate(255.9 / 256) == 255 / 256
+    for p in (0.001, 1.0, -0.5, float("nan")):
+        assert rate(p) == -1.0
 
 
 def test_binding_runs_each_call_on_its_tensors_gpu():
@@ -135,5 +154,5 @@ def test_binding_runs_each_call_on_its_tensors_gpu():
     for name in api.__all__:
         fn = getattr(api, name)
         if name.startswith("fa_") and callable(fn) and name not in (
-                "fa_version", "fa_backward_workspace_size"):
+                "fa_version", "fa_backward_workspace_size", "fa_dropout_rate"):
             assert getattr(fn, "__wrapped__", None) is not None, f"{name} is not device-guarded"
