@@ -321,6 +321,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Watchdog wd{abort_flag, p.timeout_ns};
+  if (warp == kWarpMma) FA_TRACE_POINT(0, 0, 0);
 
   // Does some query of query tile i see a key of this tile?
   auto member = [&](int i) -> bool {
@@ -366,10 +367,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int seq = seq_of(s, h, w);
         const int slot = slot_of(seq);
         const int rnd = round_of(seq);
+        FA_TRACE_POINT(30, seq, 0);
         if (rnd > 0 && !mbar_wait_warp(bar(C::kBarEmpty + slot), (rnd - 1) & 1, wd)) {
           ok = false;
           break;
         }
+        FA_TRACE_POINT(31, seq, 0);
         const uint32_t full = bar(C::kBarFull + slot);
         const uint32_t dst = slot_smem(seq);
         const int row0 = i * BM + 64 * h;
@@ -384,6 +387,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         for (int c = 0; c < C::kChunks; ++c)
           tma_load_3d_e(dst + c * C::kHalfChunkBytes, w ? &tmQ : &tmdO, full, c * 64, row0, bh);
+        FA_TRACE_POINT(32, seq, 0);
         issued = seq + 1;
       }
     }
@@ -406,14 +410,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int h = 0; h < 2; ++h) {
         const int seqO = seq_of(s, h, 0), seqQ = seq_of(s, h, 1);
         if (!(wait_full(seqO) && wait_full(seqQ))) return false;
+        FA_TRACE_POINT(5, s, h);
         tc_fence_after();
         issue_xyT_half<D, E>(tm_dp + 64 * h, v_smem, slot_smem(seqO));
         if (D == 128 && s > 0) {  // S^T_h shares columns with dQ^T_h of the last step
           if (!mbar_wait_warp(bar(C::kBarDQEmpty + h), (s - 1) & 1, wd)) return false;
+          FA_TRACE_POINT(7, s, h);
           tc_fence_after();
         }
         issue_xyT_half<D, E>(tm_s + 64 * h, k_smem, slot_smem(seqQ));
         tc_commit_e(bar(C::kBarS + h));
+        FA_TRACE_POINT(8, s, h);
       }
       return true;
     };
@@ -421,7 +428,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int s = 0; s < nsteps && ok; ++s) {
       for (int h = 0; h < 2 && ok; ++h) {
         const int seqO = seq_of(s, h, 0), seqQ = seq_of(s, h, 1);
+        FA_TRACE_POINT(1, s, h);
         if (!mbar_wait_warp(bar(C::kBarP + h), s & 1, wd)) { ok = false; break; }
+        FA_TRACE_POINT(2, s, h);
         tc_fence_after();
         const bool acc = (s > 0) || (h > 0);
         issue_acc_half<D, E>(tmem + C::kTmDV, tm_s + 64 * h, slot_smem(seqO), acc);   // dV
@@ -432,6 +441,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_commit_e(bar(C::kBarEmpty + slot_of(seqO)));
         tc_commit_e(bar(C::kBarEmpty + slot_of(seqQ)));
+        FA_TRACE_POINT(3, s, h);
       }
       if (!ok) break;
       if constexpr (D == 64) {
@@ -448,6 +458,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_commit_e(bar(C::kBarDrain));
     drain_wait(bar(C::kBarDrain), 0, p.timeout_ns);
     __syncwarp();
+    FA_TRACE_POINT(99, 0, 0);
   } else if (warp < 8) {
     // ------------------------------------------------------------ P^T, dS^T (key rows)
     const int h = warp >> 2;                  // query half
@@ -474,11 +485,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       // finished reading this dS chunk, and L2 and D of this half arrived with its Q rows.
       if (s > 0)
         ok = __all_sync(0xffffffffu, mbar_wait(bar(dq_bar), (s - 1) & 1, wd));
+      if ((warp & 3) == 0) FA_TRACE_POINT(10, s, h);
       const int seqQ = seq_of(s, h, 1);
       if (ok)
         ok = __all_sync(0xffffffffu,
                         mbar_wait(bar(C::kBarFull + slot_of(seqQ)), round_of(seqQ) & 1, wd));
+      if ((warp & 3) == 0) FA_TRACE_POINT(12, s, h);
       if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarS + h), s & 1, wd));
+      if ((warp & 3) == 0) FA_TRACE_POINT(14, s, h);
       if (!ok) break;
       tc_fence_after();
       const float4* Lv = reinterpret_cast<const float4*>(
@@ -575,6 +589,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(C::kBarP + h));
+      if ((warp & 3) == 0) FA_TRACE_POINT(16, s, h);
     }
     if (nsteps == 0 && key < p.N) {
       // no query sees this key: dK = dV = 0 (warps 0-3 dK, warps 4-7 dV)
@@ -621,6 +636,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int h = 0; h < 2 && ok; ++h) {
           ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarDQFull + h), s & 1, wd));
           if (!ok) break;
+          if (warp == kWarpDq) FA_TRACE_POINT(20, s, h);
           tc_fence_after();
           uint32_t v[2][32];
           tmem_ld32(tmem + lane_off + C::kTmS + 64 * h, v[0]);
@@ -629,6 +645,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(bar(C::kBarDQEmpty + h));
+          if (warp == kWarpDq) FA_TRACE_POINT(22, s, h);
           // element `row` of the head dimension for 64 queries: a warp covers 32
           // consecutive elements of one query row (128 contiguous bytes) per add
           float* dst = p.dQacc + (static_cast<size_t>(bh) * p.N + q0 + 64 * h) * D + row;
@@ -636,6 +653,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int qq = 0; qq < 64; ++qq)
             if (qq < nq) red_add(dst + static_cast<size_t>(qq) * D, __uint_as_float(v[qq / 32][qq % 32]));
+          if (warp == kWarpDq) FA_TRACE_POINT(24, s, h);
         }
       } else {
         ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarDQFull), s & 1, wd));

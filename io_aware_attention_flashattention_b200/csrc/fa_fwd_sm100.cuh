@@ -52,9 +52,15 @@ constexpr int kWarpTmaV = 10;
 constexpr float kRescaleThreshold = 8.0f;  // log2 domain: rescale when max grows > 2^8
 // Largest number of 128-key tiles a block mask may span (N <= 524288).
 constexpr int kMaxMaskTiles = 4096;
-// When kPolyPeriod > 0, one pair of exponentials in every kPolyPeriod goes to the
-// polynomial exp2 on the FMA pipe (exp2_poly2) instead of MUFU.
-constexpr int kPolyPeriod = 0;
+// When Cfg<D>::kPolyPeriod > 0, one pair of exponentials in every kPolyPeriod goes
+// to the polynomial exp2 on the FMA pipe (exp2_poly2) instead of MUFU. The build
+// may set the periods with -DFA_FWD_POLY_PERIOD_D64=... / _D128=... (0 = off).
+#ifndef FA_FWD_POLY_PERIOD_D64
+#define FA_FWD_POLY_PERIOD_D64 0
+#endif
+#ifndef FA_FWD_POLY_PERIOD_D128
+#define FA_FWD_POLY_PERIOD_D128 0
+#endif
 
 template <int D>
 struct Cfg {
@@ -86,8 +92,8 @@ struct Cfg {
   static constexpr int kSmemBytes = kMaskOff + 2 * kMaskWords * 4 + 1024;  // + alignment
   static constexpr uint32_t kTmS0 = 0, kTmO0 = 256;
   static_assert(kSmemBytes <= 232448, "exceeds the 227 KB of shared memory a CTA may use");
-  static_assert(kSmemBytes <= 232448, "exceeds the 227 KB of shared memory a CTA may use");
   static constexpr uint32_t kTmCols = 512;
+  static constexpr int kPolyPeriod = (D == 64) ? FA_FWD_POLY_PERIOD_D64 : FA_FWD_POLY_PERIOD_D128;
 };
 
 struct Params {
@@ -478,7 +484,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float2 x = ffma2(make_float2(__uint_as_float(s[cc][2 * k]),
                                              __uint_as_float(s[cc][2 * k + 1])), c2, nm2);
           float2 pe;
-          if (kPolyPeriod > 0 && k % (kPolyPeriod > 0 ? kPolyPeriod : 1) == kPolyPeriod - 1) {
+          constexpr int kPoly = C::kPolyPeriod;
+          if (kPoly > 0 && k % (kPoly > 0 ? kPoly : 1) == kPoly - 1) {
             pe = exp2_poly2(x);  // a share of the exponentials on the FMA pipe
           } else {
             pe = make_float2(ex2_approx(x.x), ex2_approx(x.y));

@@ -27,6 +27,33 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
 
 __device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31; }
 
+// Timeline trace, a profiling aid compiled only with -DFA_TRACE (never in the
+// library build): lane 0 of the calling warp, in the one CTA g_trace_cta names,
+// stores the SM clock of event (code < 128, a < 1024, b < 2) into its own slot of
+// g_trace (plain stores, no atomics, so the trace barely perturbs the timeline),
+// and the global timer into g_trace_ns for codes 0 and 99 (start and end). The
+// host reads both back with cudaMemcpyFromSymbol.
+#ifdef FA_TRACE
+constexpr unsigned kTraceCap = 128u * 1024u * 2u;
+__device__ uint32_t g_trace[kTraceCap];
+__device__ unsigned long long g_trace_ns[2];
+__device__ int g_trace_cta;
+__device__ __forceinline__ void trace_point(uint32_t code, uint32_t a, uint32_t b) {
+  if (static_cast<int>(blockIdx.x) == g_trace_cta && (threadIdx.x & 31) == 0) {
+    g_trace[((code & 127u) * 1024u + (a & 1023u)) * 2u + (b & 1u)] =
+        static_cast<uint32_t>(clock64());
+    if (code == 0u || code == 99u) {
+      unsigned long long t;
+      asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+      g_trace_ns[code == 0u ? 0 : 1] = t;
+    }
+  }
+}
+#define FA_TRACE_POINT(code, a, b) ::fa::trace_point((code), (a), (b))
+#else
+#define FA_TRACE_POINT(code, a, b) ((void)0)
+#endif
+
 // ---------------------------------------------------------------- mbarrier
 
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
