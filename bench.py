@@ -51,6 +51,8 @@ def parse():
                     help="override the workload's N (same B, H, d, dtype, mask and scale)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the secondary configurations (rank 0, one GPU only)")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle sample")
     ap.add_argument("--reference-seconds", type=float, default=150.0,
@@ -200,6 +202,42 @@ def max_over_ranks(value_ms: float, world: int, device=None) -> float:
     return float(t.item())
 
 
+def workload_config(w, world: int) -> dict:
+    """The ``config`` object of the JSON line; both arms print the same one."""
+    return {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d, "causal": w.causal,
+            "scale": w.scale, "parallelism": f"replicas{world}",
+            "l2": "flushed (256 MiB write) before every timed step"}
+
+
+def visible_pairs(N: int, causal: bool, window=None, block_mask=None) -> int:
+    """Number of (query, key) pairs the masks keep, for one head: causal keeps j <= i,
+    a window (left, right) keeps i - left <= j <= i + right (negative = unbounded), a
+    block mask over 128 x 128 blocks keeps (i, j) iff mask[i // 128][j // 128]."""
+    import numpy as np
+
+    i = np.arange(N, dtype=np.int64)
+    lo = np.zeros(N, dtype=np.int64)
+    hi = np.full(N, N - 1, dtype=np.int64)
+    if causal:
+        hi = np.minimum(hi, i)
+    if window is not None:
+        left, right = window
+        if left >= 0:
+            lo = np.maximum(lo, i - left)
+        if right >= 0:
+            hi = np.minimum(hi, i + right)
+    if block_mask is None:
+        return int(np.maximum(hi - lo + 1, 0).sum())
+    m = np.asarray(block_mask) != 0
+    T = m.shape[0]
+    total = 0
+    for kb in range(T):  # keys of block kb visible to each row: [max(lo, kb*128), min(hi, ...)]
+        k0, k1 = kb * 128, min(N, kb * 128 + 128) - 1
+        cnt = np.maximum(np.minimum(hi, k1) - np.maximum(lo, k0) + 1, 0)
+        total += int((cnt * m[i // 128, kb]).sum())
+    return total
+
+
 def job_throughput(flops_per_step: float, world: int, steps: int, job_ms: float) -> float:
     """Whole-job TFLOP/s: the work of all ranks divided by the slowest rank's time."""
     return flops_per_step * world * steps / (job_ms * 1e-3) / 1e12
@@ -277,8 +315,7 @@ def reference_arm(args, w):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": secs / args.steps * 1e3, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
-                   "causal": w.causal, "scale": w.scale},
+        "config": workload_config(w, int(os.environ.get("WORLD_SIZE", "1"))),
         "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": threads,
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -286,6 +323,129 @@ def reference_arm(args, w):
     }
     print(json.dumps(out))
     return 0
+
+
+# ---------------------------------------------------------------- secondary configurations
+
+# (label, workload, field overrides, window, block-mask density, dropout p). Masked and
+# dropout cases use the long workload's shape; a block mask keeps each 128 x 128 block
+# with the given probability (numpy seed 77) and always keeps the diagonal blocks.
+SECONDARY = [
+    ("gpt2_causal_b8h12_n1024_d64", "gpt2_causal_b8h12_n1024_d64", {}, None, None, None),
+    ("mid_b1h8_n4096_d128", "mid_b1h8_n4096_d128", {}, None, None, None),
+    ("mid_b1h8_n4096_d128_f16", "mid_b1h8_n4096_d128", {"dtype": "f16"}, None, None, None),
+    ("stress_causal_b2h16_n8192_d128_qk8", "stress_causal_b2h16_n8192_d128_qk8", {}, None, None,
+     None),
+    ("long_b1h8_n16384_d128", "long_b1h8_n16384_d128", {}, None, None, None),
+    ("long_b1h8_n16384_d128_causal", "long_b1h8_n16384_d128", {"causal": True}, None, None, None),
+    ("long_causal_window512", "long_b1h8_n16384_d128", {"causal": True}, (512, 512), None, None),
+    ("long_causal_blocks25", "long_b1h8_n16384_d128", {"causal": True}, None, 0.25, None),
+    ("long_dropout0.1", "long_b1h8_n16384_d128", {}, None, None, 0.1),
+]
+
+
+def secondary_configs(dev, peak: float, steps: int = 10, warmup: int = 3):
+    """Forward and backward TFLOP/s of every SECONDARY case, timed like the main line:
+    CUDA events on the launching stream around the forward and around the three
+    backward kernels, L2 flushed before each step, median of ``steps`` steps. FLOPs
+    count only the (query, key) pairs the masks keep; the backward is 2.5x the
+    forward. Inputs are seeded draws on the device (timing only; the parity tests use
+    the host generator)."""
+    import dataclasses
+    import statistics
+
+    import numpy as np
+    import torch
+
+    from io_aware_attention_flashattention_b200 import api
+    from io_aware_attention_flashattention_b200.inputs import WORKLOADS, make_inputs_device
+
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    out = {}
+    for label, wname, over, window, density, p_drop in SECONDARY:
+        over = dict(over)
+        if over.get("dtype") == "f16":
+            over["dtype"] = torch.float16
+        w = dataclasses.replace(WORKLOADS[wname], **over)
+        q, k, v, do = make_inputs_device(w.B, w.H, w.N, w.d, w.dtype, w.seed, device=dev)
+        if w.qk_gain != 1.0:
+            q.mul_(w.qk_gain)
+            k.mul_(w.qk_gain)
+        blocks = None
+        if density is not None:
+            T = (w.N + 127) // 128
+            m = (np.random.default_rng(77).random((T, T)) < density).astype(np.uint8)
+            np.fill_diagonal(m, 1)
+            blocks = m
+        bm = torch.from_numpy(blocks).to(dev) if blocks is not None else None
+        drop = (p_drop, 1234, 0) if p_drop is not None else None
+        pairs = visible_pairs(w.N, w.causal, window, blocks)
+        fwd_f = 4.0 * w.B * w.H * w.d * pairs
+        bwd_f = 2.5 * fwd_f
+        o = torch.empty_like(q)
+        lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+        dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+        ws = api.workspace_for(q)
+
+        def fwd():
+            if drop is not None:
+                api.fa_forward_dropout(q, k, v, o, lse, w.scale, w.causal, drop, window, bm)
+            elif window is not None or bm is not None:
+                api.fa_forward_masked(q, k, v, o, lse, w.scale, w.causal, window, bm)
+            elif w.dtype == torch.float16:
+                api.fa_forward_f16(q, k, v, o, lse, w.scale, w.causal)
+            else:
+                api.fa_forward(q, k, v, o, lse, w.scale, w.causal)
+
+        def bwd():
+            if drop is not None:
+                api.fa_backward_dropout(q, k, v, o, do, lse, dq, dk, dv, w.scale, w.causal, ws,
+                                        drop, window, bm)
+            elif window is not None or bm is not None:
+                api.fa_backward_masked(q, k, v, o, do, lse, dq, dk, dv, w.scale, w.causal, ws,
+                                       window, bm)
+            elif w.dtype == torch.float16:
+                api.fa_backward_f16(q, k, v, o, do, lse, dq, dk, dv, w.scale, w.causal, ws)
+            else:
+                api.fa_backward(q, k, v, o, do, lse, dq, dk, dv, w.scale, w.causal, ws)
+
+        tf, tb = [], []
+        for it in range(warmup + steps):
+            flush.zero_()
+            e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
+            e[0].record(stream)
+            fwd()
+            e[1].record(stream)
+            if w.backward:
+                flush.zero_()  # the backward starts from a cold L2 too (outside its events)
+                e[2].record(stream)
+                bwd()
+                e[3].record(stream)
+            torch.cuda.synchronize()
+            if it >= warmup:
+                tf.append(e[0].elapsed_time(e[1]))
+                if w.backward:
+                    tb.append(e[2].elapsed_time(e[3]))
+        if api.fa_get_status() != 0:
+            raise SystemExit(f"kernel watchdog fired in {label}")
+        ent = {"B": w.B, "H": w.H, "N": w.N, "d": w.d, "dtype": str(w.dtype).split(".")[-1],
+               "causal": w.causal, "window": list(window) if window else None,
+               "block_density": density, "dropout": p_drop,
+               "visible_pairs_per_head": pairs}
+        fm = statistics.median(tf)
+        ent["fwd_ms"] = fm
+        ent["fwd_tflops"] = fwd_f / (fm * 1e-3) / 1e12
+        ent["fwd_frac"] = ent["fwd_tflops"] / peak
+        if w.backward:
+            bm_ms = statistics.median(tb)
+            ent["bwd_ms"] = bm_ms
+            ent["bwd_tflops"] = bwd_f / (bm_ms * 1e-3) / 1e12
+            ent["bwd_frac"] = ent["bwd_tflops"] / peak
+        out[label] = ent
+        del q, k, v, do, o, lse, dq, dk, dv, ws, bm
+    del flush
+    return out
 
 
 # ---------------------------------------------------------------- our arm
@@ -503,6 +663,11 @@ def main():
                "ms_per_step": e_ms / n_e2e,
                "mode": "two buffer sets, copy-in / kernels / copy-out on three streams"}
 
+    per_config = None
+    if world == 1 and not args.no_per_config:
+        peaks, _ = load_peaks()
+        per_config = secondary_configs(dev, float(peaks["bf16_tflops"]))
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         f, t, R, threads = oracle_sample(w, args.cpu_seconds)
@@ -520,9 +685,7 @@ def main():
         "steps": args.steps, "warmup": max(3, args.warmup),
         "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d,
-                   "causal": w.causal, "scale": w.scale, "parallelism": f"replicas{world}",
-                   "l2": "flushed (256 MiB write) before every timed step"},
+        "config": workload_config(w, world),
         "fwd_tflops": fwd_f / (kernels["fa_fwd_kernel"]["avg_ms"] * 1e-3) / 1e12,
         "bwd_tflops": bwd_f / (sum(kernels[n]["avg_ms"] for n in names[1:]) * 1e-3) / 1e12,
         "frac_of_peak": {"fwd": None, "bwd": None, "peak_tflops": float(peaks["bf16_tflops"])},
@@ -531,6 +694,7 @@ def main():
         "gpu_launches": len(names) * args.steps,
         "clocks": clocks,
         "e2e": e2e,
+        "per_config": per_config,
         "cpu_baseline": cpu,
         "watchdog_status": status,
         "wall_s_timed_region": wall,

@@ -130,6 +130,9 @@ def test_reference_arm_prints_the_contract_line():
     assert d["unit"] == "TFLOP/s" and d["higher_is_better"] is True
     assert d["steps"] == 2 and d["warmup"] == 1 and d["value"] > 0
     assert d["config"]["workload"] == "gpt2_causal_b8h12_n1024_d64"
+    # the same config object our arm prints, so the two lines compare as one workload
+    from io_aware_attention_flashattention_b200.inputs import WORKLOADS
+    assert d["config"] == bench.workload_config(WORKLOADS["gpt2_causal_b8h12_n1024_d64"], 1)
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["cpu_baseline"]["cores"] >= 1
     assert d["e2e"] == {"value": d["value"], "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -148,3 +151,30 @@ def test_reference_arm_runs_on_rank_zero_only():
         capture_output=True, text=True, timeout=60, cwd=bench.ROOT, env=env)
     assert out.returncode == 0, out.stderr[-2000:]
     assert not [ln for ln in out.stdout.splitlines() if ln.startswith("{")]
+
+
+def test_visible_pairs_match_brute_force():
+    """The masked FLOP count of the secondary configurations: pairs kept by causal, a
+    window and a block mask, against an N x N boolean matrix."""
+    import numpy as np
+
+    rng = np.random.default_rng(3)
+    for N in (1, 77, 128, 300, 1000):
+        T = (N + 127) // 128
+        for causal in (False, True):
+            for window in (None, (5, 7), (-1, 3), (10, -1), (512, 512)):
+                for bm in (None, (rng.random((T, T)) < 0.5).astype(np.uint8)):
+                    i = np.arange(N)[:, None]
+                    j = np.arange(N)[None, :]
+                    vis = np.ones((N, N), bool)
+                    if causal:
+                        vis &= j <= i
+                    if window:
+                        left, right = window
+                        if left >= 0:
+                            vis &= j >= i - left
+                        if right >= 0:
+                            vis &= j <= i + right
+                    if bm is not None:
+                        vis &= bm[i // 128, j // 128] != 0
+                    assert bench.visible_pairs(N, causal, window, bm) == int(vis.sum())
