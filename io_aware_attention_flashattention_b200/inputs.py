@@ -80,5 +80,16 @@ def make_inputs(B: int, H: int, N: int, d: int, dtype: torch.dtype, seed: int,
     return q.to(dtype), k.to(dtype), v.to(dtype), do.to(dtype)
 
 
+def make_inputs_device(B: int, H: int, N: int, d: int, dtype: torch.dtype, seed: int,
+                       device="cuda"):
+    """(Q, K, V, dO) drawn directly on a CUDA device, for shapes too large to stage
+    in host memory: ``torch.Generator(device).manual_seed(seed)`` and four ``randn``
+    draws of [B, H, N, d] in ``dtype``, in the order Q, K, V, dO. The oracle reads
+    back whichever slices it checks, so both sides still see the same bits."""
+    g = torch.Generator(device=device).manual_seed(int(seed))
+    shape = (B, H, N, d)
+    return tuple(torch.randn(shape, generator=g, dtype=dtype, device=device) for _ in range(4))
+
+
 def workload_inputs(w: Workload):
     return make_inputs(w.B, w.H, w.N, w.d, w.dtype, w.seed, w.qk_gain)

@@ -28,7 +28,8 @@ import torch
 
 import oracle
 from io_aware_attention_flashattention_b200 import api
-from io_aware_attention_flashattention_b200.inputs import WORKLOADS, make_inputs, workload_inputs
+from io_aware_attention_flashattention_b200.inputs import (WORKLOADS, make_inputs,
+                                                         make_inputs_device, workload_inputs)
 
 pytestmark = pytest.mark.gpu
 
@@ -226,8 +227,12 @@ def _sampled_rows(rng, BH, N, per_head, extra_head_rows=()):
 
 
 def check_sampled(w, per_head=16, full_heads=(0,), dq_rows=True, dkdv_head=None, n_keys=64):
-    """Full-size workload on the GPU (the launch the benchmark times); checked
-    against the oracle on whole heads and on sampled rows of every head."""
+    """Full-size workload on the GPU (the launch the benchmark times), checked
+    against the oracle on sampled elements: ``per_head`` random rows of every head,
+    plus the first and last 128 rows of each head in ``full_heads`` (O, LSE, dQ),
+    and dK/dV of ``n_keys`` random keys plus the first and last 32 keys of head
+    ``dkdv_head``. A fast pre-check; test_gpu_full_parity.py compares every element
+    of the same launches."""
     q, k, v, do = workload_inputs(w)
     tol = TOL[w.dtype]
     B, H, N, d = q.shape
@@ -325,6 +330,32 @@ def test_workload_long_b1h8_n16384_d128():
                   dkdv_head=5, n_keys=32)
 
 
+def test_tensors_beyond_2p31_elements():
+    """Offsets are 64-bit: B1 H1040 N16384 d128 puts 2.18e9 elements in each tensor
+    (4.4 GB of bf16), so the last head starts past element 2^31. Its O, LSE, dQ, dK
+    and dV are compared with the oracle on that head's inputs (the definition is per
+    head, so one head is a [1, 1, N, d] problem)."""
+    B, H, N, d = 1, 1040, 16384, 128
+    if torch.cuda.mem_get_info()[0] < (64 << 30):
+        pytest.skip("needs about 50 GB of free device memory")
+    assert (H - 1) * N * d > 2 ** 31
+    scale = 1.0 / math.sqrt(d)
+    q, k, v, do = make_inputs_device(B, H, N, d, torch.bfloat16, seed=2031)
+    o, lse = run_forward(q, k, v, scale, False)
+    dq, dk, dv = run_backward(q, k, v, o, lse, do, scale, False)
+    sl = (slice(0, 1), slice(H - 1, H))
+    qh, kh, vh, doh = (t[sl].cpu() for t in (q, k, v, do))
+    O_ref, L_ref = oracle.forward(qh, kh, vh, scale, False)
+    assert_close_o("O", _np(o[sl]), O_ref, TOL_BF16["O"])
+    assert_close("LSE", _np(lse[sl]), L_ref, TOL_BF16["L"])
+    dQ, dK, dV, _ = oracle.backward(qh, kh, vh, doh, scale, False)
+    for name, got, want in (("dQ", dq, dQ), ("dK", dk, dK), ("dV", dv, dV)):
+        assert_close(name, _np(got[sl]), want, grad_tol(TOL_BF16, want))
+    # every head was written (NaN-prefilled outputs)
+    for t in (o, lse, dq, dk, dv):
+        assert not torch.isnan(t).any()
+
+
 # ------------------------------------------------------------------ behaviour
 
 
@@ -354,6 +385,29 @@ def test_argument_errors_launch_nothing():
     assert lib.fa_backward(p, p, p, p, p, lse.data_ptr(), p, p, p, 1, 1, 128, 64, 0.1, 0,
                            p, ws_need - 1, s) == 1
     assert api.fa_get_status() == 0
+
+
+def test_call_on_a_second_gpu_while_the_first_is_current():
+    """The binding makes the tensors' GPU current for the call, so the library's
+    per-GPU state (status word, SM count, shared-memory attributes, work split) is
+    that GPU's. Needs two GPUs."""
+    if torch.cuda.device_count() < 2:
+        pytest.skip("needs two GPUs")
+    q, k, v, do = make_inputs(1, 2, 384, 128, torch.bfloat16, seed=31)
+    with torch.cuda.device(0):
+        qc, kc, vc, doc = (t.to("cuda:1") for t in (q, k, v, do))
+        o, lse = api.forward(qc, kc, vc, causal=True)
+        dq, dk, dv = api.backward(qc, kc, vc, o, lse, doc, causal=True)
+        assert torch.cuda.current_device() == 0
+        torch.cuda.synchronize(1)
+        assert api.fa_get_status(torch.cuda.current_stream(1)) == 0
+    scale = 1.0 / math.sqrt(128)
+    O_ref, L_ref = oracle.forward(q, k, v, scale, True)
+    dQ, dK, dV, _ = oracle.backward(q, k, v, do, scale, True)
+    assert_close_o("O", _np(o), O_ref, TOL_BF16["O"])
+    assert_close("LSE", _np(lse), L_ref, TOL_BF16["L"])
+    for name, got, want in (("dQ", dq, dQ), ("dK", dk, dK), ("dV", dv, dV)):
+        assert_close(name, _np(got), want, grad_tol(TOL_BF16, want))
 
 
 def test_watchdog_timeout_is_reported_and_context_survives():

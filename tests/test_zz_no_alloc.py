@@ -5,7 +5,8 @@ their own pool). Its workspace is a fixed 32 MiB array inside the library.
 
 Checked through the C ABI against fa_backward (caller-provided workspace) on the
 same inputs, for two calls in a row with different shapes, so that the second
-call runs on whatever the first left in the shared array. This file is collected
+call runs on whatever the first left in the shared array: dK and dV must match bit
+for bit, dQ (fp32 atomic adds) within two bf16 ulps. This file is collected
 last and also passes when run alone in a fresh process (the first call on the GPU
 does the one-time address look-up).
 """
@@ -71,13 +72,23 @@ def test_noalloc_matches_workspace_backward_twice(first, second):
         assert st == 0, api.lib().fa_status_string(st)
         torch.cuda.synchronize()
         assert api.fa_get_status() == 0
-        for name, g, w in zip(("dQ", "dK", "dV"), got, want):
-            g = g.double().cpu().numpy()
-            w = w.double().cpu().numpy()
-            assert np.all(np.isfinite(g)), f"call {call}: {name} not fully written"
-            tol = max(5e-2 * float(np.abs(w).max()), 1e-3)
-            err = float(np.max(np.abs(g - w)))
-            assert err <= tol, f"call {call}: {name} differs by {err:.3e} > {tol:.3e}"
+        # Same kernels, same inputs: dK and dV are deterministic, so they must be
+        # identical bit for bit. dQ is summed with fp32 atomic adds in whatever order
+        # the key tiles finish, which moves the fp32 sum by about 1e-6 of its size;
+        # after rounding to bf16 an element may land one ulp away. Allowed: 2 bf16
+        # ulps at the element's magnitude plus 1e-5 of the largest |dQ|.
+        for name, g, w in zip(("dK", "dV"), got[1:], want[1:]):
+            assert torch.equal(g, w), f"call {call}: {name} differs from fa_backward's"
+        g = got[0].double().cpu().numpy()
+        w = want[0].double().cpu().numpy()
+        assert np.all(np.isfinite(g)), f"call {call}: dQ not fully written"
+        mag = np.maximum(np.abs(g), np.abs(w))
+        ulp = np.exp2(np.floor(np.log2(np.where(mag > 0, mag, 1.0))) - 7)
+        excess = np.abs(g - w) - (2 * ulp + 1e-5 * float(np.abs(w).max()))
+        worst = int(np.argmax(excess))
+        assert excess.flat[worst] <= 0, (
+            f"call {call}: dQ differs by {abs(g.flat[worst] - w.flat[worst]):.3e} at "
+            f"|dQ| = {abs(w.flat[worst]):.3e}")
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
