@@ -305,7 +305,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int kt = next_kt(kt_lo); kt < kt_hi; kt = next_kt(kt + 1)) {
       const int j = issued;
       const int slot = j % nslots, rnd = j / nslots;
+      FA_TRACE_POINT(40, j, is_k ? 0 : 1);
       if (rnd > 0 && !mbar_wait_warp(bar(bempty + slot), (rnd - 1) & 1, wd)) break;
+      FA_TRACE_POINT(41, j, is_k ? 0 : 1);
       const uint32_t dst = is_k ? k_smem(j) : v_smem(j);
       mbar_arrive_expect_tx_e(bar(bfull + slot), C::kTileBytes);
       for (int c = 0; c < C::kChunks; ++c)
@@ -322,6 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
     // (the whole warp runs the loop; one elected lane issues each MMA and commit)
+    FA_TRACE_POINT(0, 0, 0);
     bool ok = true;
     for (int t = 0; t < 2 && ok; ++t)
       if (nk[t] > 0) ok = mbar_wait_warp(bar(C::kBarQFull + t), 0, wd);
@@ -341,15 +344,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool have_k = false;
       for (int t = 0; t < 2; ++t) {
         if (!member(kt, t)) continue;
+        FA_TRACE_POINT(42, ns[t], t);
         if (ns[t] > 0 && !mbar_wait_warp(bar(C::kBarSFree + t), (ns[t] - 1) & 1, wd))
           return false;
+        FA_TRACE_POINT(43, ns[t], t);
         if (!have_k) {
           if (!wait_k(j)) return false;
+          FA_TRACE_POINT(44, j, 0);
           have_k = true;
         }
         tc_fence_after();
         issue_s<D, E>(tmem + C::kTmS0 + t * 128, t ? q_smem1 : q_smem0, k_smem(j));
         tc_commit_e(bar(C::kBarSFull + t));
+        FA_TRACE_POINT(45, ns[t], t);
         ++ns[t];
       }
       tc_commit_e(bar(C::kBarKEmpty + j % C::kKSlots));
@@ -365,14 +372,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool have_v = false;
       for (int t = 0; t < 2 && ok; ++t) {
         if (!member(cur, t)) continue;
+        FA_TRACE_POINT(46, npv[t], t);
         if (!mbar_wait_warp(bar(C::kBarPFull + t), npv[t] & 1, wd)) { ok = false; break; }
+        FA_TRACE_POINT(47, npv[t], t);
         if (!have_v) {
           if (!wait_v(j)) { ok = false; break; }
+          FA_TRACE_POINT(48, j, 0);
           have_v = true;
         }
         tc_fence_after();
         issue_pv<D, E>(tmem + C::kTmO0 + t * D, t ? p_smem1 : p_smem0, v_smem(j), npv[t] > 0);
         tc_commit_e(bar(C::kBarPVDone + t));
+        FA_TRACE_POINT(49, npv[t], t);
         ++npv[t];
       }
       if (!ok) break;
@@ -383,6 +394,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_commit_e(bar(C::kBarDrain));
     drain_wait(bar(C::kBarDrain), 0, p.timeout_ns);
     __syncwarp();
+    FA_TRACE_POINT(99, 0, 0);
   } else {
     // ------------------------------------------------------------ softmax
     const int t = warp >> 2;
@@ -397,6 +409,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const float c = p.scale_log2;
     float m_ref = -INFINITY;
     float l = 0.0f;
+    // lr: the same sum over P as rounded for the PV product. O is divided by lr, so
+    // the weights it applies to V sum to exactly 1: the rounding of the largest
+    // p (up to 2^8 under the lagging reference max, so up to 2^-8 relative) then
+    // cancels instead of showing in O. LSE keeps the unrounded l. With dropout the
+    // rounded values carry the keep mask, so there O is divided by l.
+    float lr = 0.0f;
     // this tile's range, count and mask bits as scalars (no per-thread array indexing)
     const int t_lo = t ? lo[1] : lo[0], t_hi = t ? hi[1] : hi[0];
     const int t_nk = t ? nk[1] : nk[0];
@@ -413,7 +431,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     int kt = t_lo - 1;
     for (int j = 0; j < t_nk && ok; ++j) {
       do ++kt; while (!t_member(kt));
+      if (wq == 0) FA_TRACE_POINT(50, j, t);
       ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarSFull + t), j & 1, wd));
+      if (wq == 0) FA_TRACE_POINT(51, j, t);
       if (!ok) break;
       tc_fence_after();
       uint32_t s[4][32];
@@ -424,6 +444,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(C::kBarSFree + t));
+      if (wq == 0) FA_TRACE_POINT(52, j, t);
       const int kv0 = kt * BN;
       // masking only where the tile crosses an edge of some row's visible range
       const bool need_mask = (kv0 + BN > p.N) || (wr >= 0 && kv0 + BN - 1 > r0 + wr) ||
@@ -462,15 +483,19 @@ __global__ void __launch_bounds__(kThreads, 1)
         alpha = (m_ref == -INFINITY) ? 0.0f : ex2_approx(m_ref - m_new);
         m_ref = m_new;
         l *= alpha;
+        lr *= alpha;
       }
       // PV_t(j-1) must be complete before P_t is overwritten and O_t rescaled.
       if (j > 0) {
+        if (wq == 0) FA_TRACE_POINT(53, j, t);
         ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarPVDone + t), (j - 1) & 1, wd));
+        if (wq == 0) FA_TRACE_POINT(54, j, t);
         if (!ok) break;
         tc_fence_after();
       }
       const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
       const float2 c2 = make_float2(c, c), nm2 = make_float2(-m_use, -m_use);
+      float2 accr[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
       float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                        make_float2(0.f, 0.f)};
       // dropout: this row's four words for the current 16 keys (byte b of word m is key
@@ -516,6 +541,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             pe.y = (((wd >> 8) & 0xffu) >= p.drop.threshold) ? pe.y * p.drop.scale : 0.0f;
           }
           pk[k] = pack2<E>(pe.x, pe.y);
+          if constexpr (!kDropout) accr[k & 1] = fadd2(accr[k & 1], unpack2<E>(pk[k]));
         }
         // keys 32cc..32cc+31 = 16-byte units 4cc..4cc+3 of this row's 256 bytes:
         // chunk (cc / 2), units (cc % 2) * 4 + u, 128-byte swizzle by the row
@@ -527,6 +553,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       l += (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y) + (acc[2].x + acc[2].y) +
            (acc[3].x + acc[3].y);
+      lr += (accr[0].x + accr[0].y) + (accr[1].x + accr[1].y);
       if (move && j > 0) {
         // bring the sum up to key tile j-1 to the new reference max before PV_t(j)
 #pragma unroll
@@ -544,6 +571,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(bar(C::kBarPFull + t));
+      if (wq == 0) FA_TRACE_POINT(55, j, t);
     }
     if (ok && t_nk > 0)
       ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarPVDone + t), (t_nk - 1) & 1, wd));
@@ -556,7 +584,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok && t_nk > 0) {
       tc_fence_after();
-      const float inv_l = (l > 0.0f) ? 1.0f / l : 0.0f;
+      const float norm = kDropout ? l : lr;
+      const float inv_l = (norm > 0.0f) ? 1.0f / norm : 0.0f;
       uint16_t* orow = p.O + (static_cast<size_t>(bh) * p.N + row) * D;
 #pragma unroll
       for (int cc = 0; cc < D / 32; ++cc) {
