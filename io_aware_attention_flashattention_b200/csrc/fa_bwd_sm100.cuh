@@ -58,10 +58,6 @@ constexpr int kWarpDq = 8;     // first of the 4 dQ warps
 constexpr int kWarpTma = 12;
 constexpr int kWarpMma = 13;
 constexpr int kMaxMaskTiles = 4096;  // largest block mask: 4096 x 4096 tiles (N <= 524288)
-// Slots of the Q/dO half-tile ring at D = 128 (16.5 KB each; 7 fit beside K, V and dS).
-#ifndef FA_BWD_SLOTS_D128
-#define FA_BWD_SLOTS_D128 6
-#endif
 
 template <int D>
 struct Cfg {
@@ -71,7 +67,7 @@ struct Cfg {
   // Q and dO stream in half tiles (64 rows x D): 64-row chunks of 8 KB
   static constexpr int kHalfChunkBytes = 64 * 128;
   static constexpr int kHalfBytes = kChunks * kHalfChunkBytes;
-  static constexpr int kSlots = (D == 128) ? FA_BWD_SLOTS_D128 : 12;  // half-tile ring
+  static constexpr int kSlots = (D == 128) ? 7 : 12;  // half-tile ring (7 x 16.5 KB fit at D = 128)
   static constexpr int kVecBytes = 64 * 4;             // 64 fp32 (L2 or D of a half)
   static constexpr int kKOff = 0;
   static constexpr int kVOff = kTileBytes;
@@ -87,15 +83,12 @@ struct Cfg {
   static constexpr int kBarP = kBarS + 2;       // [2]
   static constexpr int kBarDQFull = kBarP + 2;  // [2]
   static constexpr int kBarDQEmpty = kBarDQFull + 2;  // [2]
-  static constexpr int kBarDKDV = kBarDQEmpty + 2;      // dK, dV of a segment complete
-  static constexpr int kBarDKDVFree = kBarDKDV + 1;     // ... and read out of TMEM (8 warps)
-  static constexpr int kBarKVEmpty = kBarDKDVFree + 1;  // last MMA reading K_j, V_j done
-  static constexpr int kBarSplitWritten = kBarKVEmpty + 1;   // split tile: 8 warps' slot rows
-  static constexpr int kBarSplitDecided = kBarSplitWritten + 1;  // ... arrival counted
-  static constexpr int kBarDrain = kBarSplitDecided + 1;
+  static constexpr int kBarDKDV = kBarDQEmpty + 2;
+  static constexpr int kBarDrain = kBarDKDV + 1;
   static constexpr int kNumBars = kBarDrain + 1;
-  static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem base, abort flag, arrivals
-  static constexpr int kSmemBytes = kMiscOff + 16 + 1024;
+  static constexpr int kMiscOff = kBarOff + kNumBars * 8;
+  static constexpr int kMaskOff = kMiscOff + 16;  // block-mask column of this key tile, as bits
+  static constexpr int kSmemBytes = kMaskOff + kMaxMaskTiles / 8 + 1024;
   static constexpr uint32_t kTmDK = 0, kTmDV = D, kTmS = 2 * D, kTmDP = 2 * D + 128;
   static constexpr uint32_t kTmDQ64 = 384;  // D = 64 only
   static_assert(kSmemBytes <= 232448, "exceeds the 227 KB of shared memory a CTA may use");
@@ -118,170 +111,6 @@ struct Params {
   const uint8_t* blocks;  // [n_kt x n_kt] block mask (nonzero = kept), or null
   DropoutParams drop;     // used by the kDropout instances only
   unsigned long long timeout_ns;
-  // Work schedule (see Schedule below): gridDim.x persistent CTAs.
-  int n_kt;        // key tiles per head, Npad / 128
-  int n_tiles;     // BH * n_kt, head-major
-  int rounds;      // whole units each CTA takes round robin before the tail
-  int tail_split;  // 1: the tail's steps are split evenly over all CTAs
-  int pair_units;  // 1: a unit is the key tiles j, n_kt - 1 - j of a head; 0: one tile
-  float* part;     // [gridDim.x][2 slots][dK, dV][128][D] fp32 partial sums of split tiles
-  unsigned* arrivals;  // [gridDim.x] arrival counts of split tiles (zeroed by the preprocess)
-};
-
-// ------------------------------------------------------------------ work schedule
-//
-// The main kernel is persistent: gridDim.x = G CTAs, about one per SM. Its work is
-// the B*H*n_kt key tiles; key tile j of a head walks the query tiles that can see
-// one of its keys, one "step" each. The tiles are grouped into units of two per head
-// -- j and n_kt - 1 - j -- whose step counts add up to about the same number even
-// when causal (n_q - j and j + 1), and the units are numbered head-major. CTA c first
-// takes whole units round robin: c, c + G, c + 2G, ... for p.rounds rounds, so the
-// CTAs running at any time hold units of two or three consecutive heads, whose Q, dO
-// and dQ accumulator stay in L2. The units left over (fewer than G) are the tail.
-// With p.tail_split the tail's tiles are laid end to end, T' steps in all, and CTA c
-// takes steps [c T'/G, (c+1) T'/G): every CTA then ends at about the same time instead
-// of a last, partly empty wave. A tile whose steps fall to several CTAs is "split":
-// each of them writes its partial dK, dV (fp32) to a slot of its own, counts itself
-// in with an atomic add, and the one that arrives last adds the slots up in CTA order
-// and writes dK, dV. The order of that sum does not depend on which CTA arrives last,
-// so dK and dV stay deterministic. Without p.tail_split (block masks, whose step
-// counts are device data) the round robin also covers the tail.
-
-struct Seg {
-  int tile;     // key tile, head-major: bh = tile / n_kt, j = tile % n_kt
-  int s0, s1;   // this CTA's steps of the tile, [s0, s1) of its walk
-  int slot;     // -1: the whole tile; 0 / 1: the CTA's first / last partial slot
-  int c0, c1;   // the CTAs that share a split tile (c0 == c1 when whole)
-  long long a;  // tail: the tile's first step in the tail's sequence
-};
-
-// Query tiles [lo, hi) that can see a key of key tile j (window and causal bounds;
-// a block mask may drop some of them).
-struct TileRange {
-  int lo, hi;
-};
-__host__ __device__ __forceinline__ TileRange query_range(int j, int N, int n_q, int wl,
-                                                          int wr) {
-  const int k0 = j * BN, k1 = (k0 + BN < N ? k0 + BN : N) - 1;
-  TileRange r;
-  r.lo = (wr < 0) ? 0 : (k0 - wr > 0 ? k0 - wr : 0) / BM;
-  r.hi = (wl < 0) ? n_q : ((k1 + wl) / BM + 1 < n_q ? (k1 + wl) / BM + 1 : n_q);
-  if (r.hi < r.lo) r.hi = r.lo;
-  return r;
-}
-
-// Iterates one CTA's segments in order; every warp role of the CTA walks its own
-// copy and sees the same sequence. `steps(j)` is the step count of key tile j.
-struct Schedule {
-  int c, G, n_kt, n_units, units_ph, rounds, tail_split, pair;
-  int k;             // round robin: units handed out so far
-  int part;          // round robin: next tile (0, 1) of the current unit
-  int u;             // tail: current unit
-  int up;            // tail: next tile (0, 1) of unit u
-  long long Tt;      // tail: first step of the next tile in the tail's sequence
-  long long total;   // tail: all its steps
-  long long lo, hi;  // tail: this CTA's steps [lo, hi)
-
-  // tile `which` (0, 1) of unit uu, or -1 if the unit has only one
-  __host__ __device__ int unit_tile(int uu, int which) const {
-    const int bh = uu / units_ph, q = uu % units_ph;
-    if (!pair) return which == 0 ? bh * n_kt + q : -1;
-    const int pos = 2 * q + which;
-    if (pos >= n_kt) return -1;
-    const int j = (pos & 1) ? n_kt - 1 - (pos >> 1) : (pos >> 1);
-    return bh * n_kt + j;
-  }
-  __host__ __device__ long long start(int cc) const { return (static_cast<long long>(cc) * total) / G; }
-  // The slot CTA cc uses for the split tile starting at tail step a: 0 when its range
-  // starts inside the tile (the tile is its first), 1 when the tile starts inside its
-  // range (the tile is its last).
-  __host__ __device__ int slot_of(int cc, long long a) const { return start(cc) > a ? 0 : 1; }
-  // the CTA whose tail range holds step x
-  __host__ __device__ int cta_of(long long x) const {
-    int g = static_cast<int>((x * G) / (total > 0 ? total : 1));
-    g = g < 0 ? 0 : (g > G - 1 ? G - 1 : g);
-    while (g + 1 < G && start(g + 1) <= x) ++g;
-    while (g > 0 && start(g) > x) --g;
-    return g;
-  }
-
-  template <typename StepsFn>
-  __host__ __device__ void init(const Params& p, int cta, int ctas, StepsFn steps) {
-    c = cta;
-    G = ctas;
-    n_kt = p.n_kt;
-    pair = p.pair_units;
-    units_ph = pair ? (n_kt + 1) / 2 : n_kt;
-    n_units = (p.n_tiles / n_kt) * units_ph;
-    rounds = p.rounds;
-    tail_split = p.tail_split;
-    k = 0;
-    part = 0;
-    u = rounds * G;
-    up = 0;
-    Tt = 0;
-    total = 0;
-    if (tail_split)
-      for (int uu = rounds * G; uu < n_units; ++uu)
-        for (int w = 0; w < 2; ++w) {
-          const int t = unit_tile(uu, w);
-          if (t >= 0) total += steps(t % n_kt);
-        }
-    lo = start(c);
-    hi = start(c + 1);
-  }
-
-  template <typename StepsFn>
-  __host__ __device__ bool next(Seg& s, StepsFn steps) {
-    // round robin: whole units c + k G
-    while (k < rounds || (!tail_split && c + k * G < n_units)) {
-      const int uu = c + k * G;
-      const int t = unit_tile(uu, part);
-      if (part == 1 || unit_tile(uu, 1) < 0) {
-        part = 0;
-        ++k;
-      } else {
-        part = 1;
-      }
-      if (t < 0) continue;
-      s.tile = t;
-      s.s0 = 0;
-      s.s1 = steps(t % n_kt);
-      s.slot = -1;
-      s.c0 = s.c1 = c;
-      s.a = 0;
-      return true;
-    }
-    if (!tail_split) return false;
-    // tail: the next tile holding some of this CTA's steps [lo, hi)
-    while (u < n_units) {
-      const int t = unit_tile(u, up);
-      if (up == 1 || unit_tile(u, 1) < 0) {
-        up = 0;
-        ++u;
-      } else {
-        up = 1;
-      }
-      if (t < 0) continue;
-      const int n = steps(t % n_kt);
-      const long long a = Tt, b = Tt + n;
-      Tt = b;
-      if (b <= lo || n == 0) continue;
-      if (a >= hi) {
-        u = n_units;
-        return false;
-      }
-      s.tile = t;
-      s.s0 = static_cast<int>((a > lo ? a : lo) - a);
-      s.s1 = static_cast<int>((b < hi ? b : hi) - a);
-      s.c0 = cta_of(a);
-      s.c1 = cta_of(b - 1);
-      s.a = a;
-      s.slot = (s.c0 == s.c1) ? -1 : slot_of(c, a);
-      return true;
-    }
-    return false;
-  }
 };
 
 __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
@@ -362,9 +191,7 @@ __global__ void __launch_bounds__(256)
     fa_bwd_pre_kernel(const uint16_t* __restrict__ O, const uint16_t* __restrict__ dO,
                       const float* __restrict__ LSE, float* __restrict__ L2,
                       float* __restrict__ Dv, float* __restrict__ dQacc, int N, int Npad,
-                      long long total_rows, unsigned* __restrict__ arrivals, int n_arrivals) {
-  if (blockIdx.x == 0)  // the main kernel's arrival counters of split tiles
-    for (int k = threadIdx.x; k < n_arrivals; k += blockDim.x) arrivals[k] = 0u;
+                      long long total_rows) {
   const long long r = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (r >= total_rows) return;  // total_rows = BH * Npad
@@ -436,7 +263,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar = [&](int i) -> uint32_t { return bars + 8u * static_cast<uint32_t>(i); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + C::kMiscOff + 4);
-  volatile unsigned* arrived = reinterpret_cast<volatile unsigned*>(base_ptr + C::kMiscOff + 8);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -445,39 +271,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int wl = kMasked ? p.wl : -1;
   const int wr = p.wr;
   const uint8_t* const blocks = kMasked ? p.blocks : nullptr;
-  const int n_kt = p.n_kt;
-  const int n_q = (p.N + BM - 1) / BM;
 
-  // Does some query of query tile i see a key of key tile j (block mask only; the
-  // window and causal bounds are the tile range)?
-  auto kept = [&](int i, int j) -> bool {
-    return blocks == nullptr || blocks[static_cast<size_t>(i) * n_kt + j] != 0;
-  };
-  // Steps (query tiles walked) of key tile j.
-  auto steps = [&](int j) -> int {
-    const TileRange r = query_range(j, p.N, n_q, wl, wr);
-    if (blocks == nullptr) return r.hi - r.lo;
-    int n = 0;
-    for (int i = r.lo; i < r.hi; ++i) n += kept(i, j) ? 1 : 0;
-    return n;
-  };
-  // The query tile of step s0 of key tile j (a segment starts mid-tile only without
-  // a block mask), and the query tile after i.
-  auto first_qt = [&](int j, int s0) -> int {
-    const TileRange r = query_range(j, p.N, n_q, wl, wr);
-    if (blocks == nullptr) return r.lo + s0;
-    int i = r.lo;
-    while (i < r.hi && !kept(i, j)) ++i;
-    return i;
-  };
-  auto next_qt = [&](int i, int j) -> int {
-    do ++i; while (blocks != nullptr && i < n_q && !kept(i, j));
-    return i;
-  };
-  // query tile of step s (0-based within the segment) given the previous one
-  auto step_qt = [&](int s, int i_prev, const Seg& sg) -> int {
-    return (s == 0) ? first_qt(sg.tile % n_kt, sg.s0) : next_qt(i_prev, sg.tile % n_kt);
-  };
+  // Work item: head-major (the resident CTAs share one or two heads' Q, dO and dQ
+  // accumulator in L2); within a head, key tile 0 (the heaviest if causal) first.
+  const int n_kt = p.Npad / BN;
+  const int bh = static_cast<int>(blockIdx.x) / n_kt;
+  const int j = static_cast<int>(blockIdx.x) % n_kt;
+  const int k0 = j * BN;
+  const int n_q = (p.N + BM - 1) / BM;
+  // query tiles [i_lo, i_hi) hold every query that may see a key of this tile
+  const int k1 = min(k0 + BN, p.N) - 1;
+  const int i_lo = (wr < 0) ? 0 : max(0, k0 - wr) / BM;
+  const int i_hi = (wl < 0) ? n_q : min(n_q, (k1 + wl) / BM + 1);
+
+  // The block-mask column of this key tile as bits: warp w builds words w, w + 16, ...
+  uint32_t* mask_bits = reinterpret_cast<uint32_t*>(base_ptr + C::kMaskOff);
+  if (blocks != nullptr) {
+    for (int wi = warp; wi < (n_q + 31) / 32; wi += kThreads / 32) {
+      const int i = wi * 32 + lane;
+      const bool keep = i < n_q && blocks[static_cast<size_t>(i) * n_kt + j] != 0;
+      const uint32_t bits = __ballot_sync(0xffffffffu, keep);
+      if (lane == 0) mask_bits[wi] = bits;
+    }
+  }
 
   if (threadIdx.x == 0) {
     mbar_init(bar(C::kBarKV), 1);
@@ -492,10 +308,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(C::kBarDQEmpty + h), 4);  // the 4 dQ warps
     }
     mbar_init(bar(C::kBarDKDV), 1);
-    mbar_init(bar(C::kBarDKDVFree), 8);  // the 8 P/dS warps
-    mbar_init(bar(C::kBarKVEmpty), 1);
-    mbar_init(bar(C::kBarSplitWritten), 8);  // the 8 P/dS warps
-    mbar_init(bar(C::kBarSplitDecided), 1);
     mbar_init(bar(C::kBarDrain), 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -511,13 +323,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   const Watchdog wd{abort_flag, p.timeout_ns};
   if (warp == kWarpMma) FA_TRACE_POINT(0, 0, 0);
 
-  Schedule sched;
-  sched.init(p, static_cast<int>(blockIdx.x), static_cast<int>(gridDim.x), steps);
+  // Does some query of query tile i see a key of this tile?
+  auto member = [&](int i) -> bool {
+    if (i < i_lo || i >= i_hi) return false;
+    return blocks == nullptr || ((mask_bits[i >> 5] >> (i & 31)) & 1u);
+  };
+  int nsteps = i_hi - i_lo;  // query tiles walked
+  if (blocks != nullptr) {
+    nsteps = 0;
+    for (int i = i_lo; i < i_hi; ++i) nsteps += member(i) ? 1 : 0;
+  }
 
-  // ring of half tiles: seq = 4*gs + 2*h + w over the CTA's steps gs = 0, 1, ... of all
-  // its segments, w = 0 for dO (rows 64h.. of the step's query tile), w = 1 for Q
-  // (with L2 and D of those 64 queries)
-  auto seq_of = [](int gs, int h, int w) { return 4 * gs + 2 * h + w; };
+  // ring of half tiles: seq = 4*step + 2*h + w, w = 0 for dO (rows 64h.. of query
+  // tile i), w = 1 for Q (with L2 and D of those 64 queries)
+  auto seq_of = [](int s, int h, int w) { return 4 * s + 2 * h + w; };
   auto slot_of = [&](int seq) { return seq % C::kSlots; };
   auto round_of = [&](int seq) { return seq / C::kSlots; };
   auto slot_smem = [&](int seq) -> uint32_t {
@@ -533,57 +352,48 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmdO);
     }
-    int issued = 0, gs = 0, kvn = 0;
+    mbar_arrive_expect_tx_e(bar(C::kBarKV), 2 * C::kTileBytes);
+    for (int c = 0; c < C::kChunks; ++c) {
+      tma_load_3d_e(base + C::kKOff + c * C::kChunkBytes, &tmK, bar(C::kBarKV), c * 64, k0, bh);
+      tma_load_3d_e(base + C::kVOff + c * C::kChunkBytes, &tmV, bar(C::kBarKV), c * 64, k0, bh);
+    }
+    int issued = 0;
     bool ok = true;
-    Seg sg;
-    while (ok && sched.next(sg, steps)) {
-      if (sg.s1 <= sg.s0) continue;
-      const int bh = sg.tile / n_kt, j = sg.tile % n_kt;
-      // K_j, V_j replace the last segment's once its MMAs have read them
-      if (kvn > 0 && !mbar_wait_warp(bar(C::kBarKVEmpty), (kvn - 1) & 1, wd)) break;
-      mbar_arrive_expect_tx_e(bar(C::kBarKV), 2 * C::kTileBytes);
-      for (int c = 0; c < C::kChunks; ++c) {
-        tma_load_3d_e(base + C::kKOff + c * C::kChunkBytes, &tmK, bar(C::kBarKV), c * 64, j * BN, bh);
-        tma_load_3d_e(base + C::kVOff + c * C::kChunkBytes, &tmV, bar(C::kBarKV), c * 64, j * BN, bh);
-      }
-      ++kvn;
-      int i = -1;
-      for (int s = 0; s < sg.s1 - sg.s0 && ok; ++s, ++gs) {
-        i = step_qt(s, i, sg);
-        for (int hw = 0; hw < 4 && ok; ++hw) {
-          const int h = hw >> 1, w = hw & 1;
-          const int seq = seq_of(gs, h, w);
-          const int slot = slot_of(seq);
-          const int rnd = round_of(seq);
-          FA_TRACE_POINT(30, seq, 0);
-          if (rnd > 0 && !mbar_wait_warp(bar(C::kBarEmpty + slot), (rnd - 1) & 1, wd)) {
-            ok = false;
-            break;
-          }
-          FA_TRACE_POINT(31, seq, 0);
-          const uint32_t full = bar(C::kBarFull + slot);
-          const uint32_t dst = slot_smem(seq);
-          const int row0 = i * BM + 64 * h;
-          if (w == 1) {
-            mbar_arrive_expect_tx_e(full, C::kHalfBytes + 2 * C::kVecBytes);
-            const uint32_t vec = base + C::kVecOff + slot * 2 * C::kVecBytes;
-            const size_t off = static_cast<size_t>(bh) * p.Npad + static_cast<size_t>(row0);
-            bulk_load_e(vec, p.L2 + off, C::kVecBytes, full);
-            bulk_load_e(vec + C::kVecBytes, p.Dv + off, C::kVecBytes, full);
-          } else {
-            mbar_arrive_expect_tx_e(full, C::kHalfBytes);
-          }
-          for (int c = 0; c < C::kChunks; ++c)
-            tma_load_3d_e(dst + c * C::kHalfChunkBytes, w ? &tmQ : &tmdO, full, c * 64, row0, bh);
-          FA_TRACE_POINT(32, seq, 0);
-          issued = seq + 1;
+    int i = i_lo - 1;
+    for (int s = 0; s < nsteps && ok; ++s) {
+      do ++i; while (!member(i));
+      for (int hw = 0; hw < 4 && ok; ++hw) {
+        const int h = hw >> 1, w = hw & 1;
+        const int seq = seq_of(s, h, w);
+        const int slot = slot_of(seq);
+        const int rnd = round_of(seq);
+        FA_TRACE_POINT(30, seq, 0);
+        if (rnd > 0 && !mbar_wait_warp(bar(C::kBarEmpty + slot), (rnd - 1) & 1, wd)) {
+          ok = false;
+          break;
         }
+        FA_TRACE_POINT(31, seq, 0);
+        const uint32_t full = bar(C::kBarFull + slot);
+        const uint32_t dst = slot_smem(seq);
+        const int row0 = i * BM + 64 * h;
+        if (w == 1) {
+          mbar_arrive_expect_tx_e(full, C::kHalfBytes + 2 * C::kVecBytes);
+          const uint32_t vec = base + C::kVecOff + slot * 2 * C::kVecBytes;
+          const size_t off = static_cast<size_t>(bh) * p.Npad + static_cast<size_t>(row0);
+          bulk_load_e(vec, p.L2 + off, C::kVecBytes, full);
+          bulk_load_e(vec + C::kVecBytes, p.Dv + off, C::kVecBytes, full);
+        } else {
+          mbar_arrive_expect_tx_e(full, C::kHalfBytes);
+        }
+        for (int c = 0; c < C::kChunks; ++c)
+          tma_load_3d_e(dst + c * C::kHalfChunkBytes, w ? &tmQ : &tmdO, full, c * 64, row0, bh);
+        FA_TRACE_POINT(32, seq, 0);
+        issued = seq + 1;
       }
     }
-    // Every issued copy must land before the CTA may exit.
     for (int seq = max(0, issued - C::kSlots); seq < issued; ++seq)
       drain_wait(bar(C::kBarFull + slot_of(seq)), round_of(seq) & 1, p.timeout_ns);
-    if (kvn > 0) drain_wait(bar(C::kBarKV), (kvn - 1) & 1, p.timeout_ns);
+    drain_wait(bar(C::kBarKV), 0, p.timeout_ns);
     __syncwarp();
   } else if (warp == kWarpMma) {
     // ------------------------------------------------------------ MMA issuer
@@ -591,77 +401,62 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t k_smem = base + C::kKOff, v_smem = base + C::kVOff;
     const uint32_t ds_smem = base + C::kDSOff;
     const uint32_t tm_s = tmem + C::kTmS, tm_dp = tmem + C::kTmDP;
-    bool ok = true;
+    bool ok = mbar_wait_warp(bar(C::kBarKV), 0, wd);
     auto wait_full = [&](int seq) -> bool {
       return mbar_wait_warp(bar(C::kBarFull + slot_of(seq)), round_of(seq) & 1, wd);
     };
-    // S^T and dP^T of both halves of global step gs (dP^T first: its columns free up
-    // earlier)
-    auto issue_sdp = [&](int gs) -> bool {
+    // S^T and dP^T of both halves of step s (dP^T first: its columns free up earlier)
+    auto issue_sdp = [&](int s) -> bool {
       for (int h = 0; h < 2; ++h) {
-        const int seqO = seq_of(gs, h, 0), seqQ = seq_of(gs, h, 1);
+        const int seqO = seq_of(s, h, 0), seqQ = seq_of(s, h, 1);
         if (!(wait_full(seqO) && wait_full(seqQ))) return false;
-        FA_TRACE_POINT(5, gs, h);
+        FA_TRACE_POINT(5, s, h);
         tc_fence_after();
         issue_xyT_half<D, E>(tm_dp + 64 * h, v_smem, slot_smem(seqO));
-        if (D == 128 && gs > 0) {  // S^T_h shares columns with dQ^T_h of the last step
-          if (!mbar_wait_warp(bar(C::kBarDQEmpty + h), (gs - 1) & 1, wd)) return false;
-          FA_TRACE_POINT(7, gs, h);
+        if (D == 128 && s > 0) {  // S^T_h shares columns with dQ^T_h of the last step
+          if (!mbar_wait_warp(bar(C::kBarDQEmpty + h), (s - 1) & 1, wd)) return false;
+          FA_TRACE_POINT(7, s, h);
           tc_fence_after();
         }
         issue_xyT_half<D, E>(tm_s + 64 * h, k_smem, slot_smem(seqQ));
         tc_commit_e(bar(C::kBarS + h));
-        FA_TRACE_POINT(8, gs, h);
+        FA_TRACE_POINT(8, s, h);
       }
       return true;
     };
-    int gs = 0, kvn = 0;
-    Seg sg;
-    while (ok && sched.next(sg, steps)) {
-      const int nsteps = sg.s1 - sg.s0;
-      if (nsteps <= 0) continue;
-      ok = mbar_wait_warp(bar(C::kBarKV), kvn & 1, wd);
-      if (ok) ok = issue_sdp(gs);
-      for (int s = 0; s < nsteps && ok; ++s, ++gs) {
-        for (int h = 0; h < 2 && ok; ++h) {
-          const int seqO = seq_of(gs, h, 0), seqQ = seq_of(gs, h, 1);
-          FA_TRACE_POINT(1, gs, h);
-          if (!mbar_wait_warp(bar(C::kBarP + h), gs & 1, wd)) { ok = false; break; }
-          FA_TRACE_POINT(2, gs, h);
-          const bool first = (s == 0) && (h == 0);
-          if (first && kvn > 0) {
-            // dK, dV of the last segment must be read out before they are overwritten
-            if (!mbar_wait_warp(bar(C::kBarDKDVFree), (kvn - 1) & 1, wd)) { ok = false; break; }
-          }
-          tc_fence_after();
-          issue_acc_half<D, E>(tmem + C::kTmDV, tm_s + 64 * h, slot_smem(seqO), !first);   // dV
-          issue_acc_half<D, E>(tmem + C::kTmDK, tm_dp + 64 * h, slot_smem(seqQ), !first);  // dK
-          // dV and dK are the last readers of this half's dO and Q: free their slots
-          // before the dQ product, so the next loads start a product earlier
-          tc_commit_e(bar(C::kBarEmpty + slot_of(seqO)));
-          tc_commit_e(bar(C::kBarEmpty + slot_of(seqQ)));
-          if constexpr (D == 128) {
-            issue_dqT_half<E>(tm_s + 64 * h, k_smem, ds_smem + h * C::kChunkBytes);
-            tc_commit_e(bar(C::kBarDQFull + h));
-          }
-          FA_TRACE_POINT(3, gs, h);
+    if (ok && nsteps > 0) ok = issue_sdp(0);
+    for (int s = 0; s < nsteps && ok; ++s) {
+      for (int h = 0; h < 2 && ok; ++h) {
+        const int seqO = seq_of(s, h, 0), seqQ = seq_of(s, h, 1);
+        FA_TRACE_POINT(1, s, h);
+        if (!mbar_wait_warp(bar(C::kBarP + h), s & 1, wd)) { ok = false; break; }
+        FA_TRACE_POINT(2, s, h);
+        tc_fence_after();
+        const bool acc = (s > 0) || (h > 0);
+        issue_acc_half<D, E>(tmem + C::kTmDV, tm_s + 64 * h, slot_smem(seqO), acc);   // dV
+        issue_acc_half<D, E>(tmem + C::kTmDK, tm_dp + 64 * h, slot_smem(seqQ), acc);  // dK
+        // dV and dK are the last readers of this half's dO and Q: free their slots
+        // before the dQ product, so that the next loads start a product earlier
+        tc_commit_e(bar(C::kBarEmpty + slot_of(seqO)));
+        tc_commit_e(bar(C::kBarEmpty + slot_of(seqQ)));
+        if constexpr (D == 128) {
+          issue_dqT_half<E>(tm_s + 64 * h, k_smem, ds_smem + h * C::kChunkBytes);
+          tc_commit_e(bar(C::kBarDQFull + h));
         }
-        if (!ok) break;
-        if constexpr (D == 64) {
-          if (gs > 0) {  // the dQ columns are reused: the previous dQ must have been read
-            if (!mbar_wait_warp(bar(C::kBarDQEmpty), (gs - 1) & 1, wd)) { ok = false; break; }
-            tc_fence_after();
-          }
-          issue_dq64<E>(tmem + C::kTmDQ64, ds_smem, k_smem);
-          tc_commit_e(bar(C::kBarDQFull));
-        }
-        if (s + 1 < nsteps) ok = issue_sdp(gs + 1);
+        FA_TRACE_POINT(3, s, h);
       }
       if (!ok) break;
-      tc_commit_e(bar(C::kBarDKDV));     // dK, dV of this segment
-      tc_commit_e(bar(C::kBarKVEmpty));  // every MMA reading K_j, V_j
-      ++kvn;
+      if constexpr (D == 64) {
+        if (s > 0) {  // the dQ columns are reused: the previous dQ must have been read
+          if (!mbar_wait_warp(bar(C::kBarDQEmpty), (s - 1) & 1, wd)) { ok = false; break; }
+          tc_fence_after();
+        }
+        issue_dq64<E>(tmem + C::kTmDQ64, ds_smem, k_smem);
+        tc_commit_e(bar(C::kBarDQFull));
+      }
+      if (s + 1 < nsteps) ok = issue_sdp(s + 1);
     }
+    if (ok) tc_commit_e(bar(C::kBarDKDV));
     tc_commit_e(bar(C::kBarDrain));
     drain_wait(bar(C::kBarDrain), 0, p.timeout_ns);
     __syncwarp();
@@ -670,262 +465,162 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ P^T, dS^T (key rows)
     const int h = warp >> 2;                  // query half
     const int krow = (warp & 3) * 32 + lane;  // key row within the tile = TMEM lane
+    const int key = k0 + krow;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t tm_s = tmem + lane_off + C::kTmS + 64 * h;
     const uint32_t tm_dp = tmem + lane_off + C::kTmDP + 64 * h;
     const float c = p.scale_log2;
     uint8_t* ds_row = base_ptr + C::kDSOff + h * C::kChunkBytes + krow * 128;
+    const bool ragged_keys = k0 + BN > p.N;
     const int dq_bar = (D == 128) ? C::kBarDQFull + h : C::kBarDQFull;
+    // queries that see this key row: [q_lo, q_hi) (empty for a padding key)
+    const int q_lo = (wr < 0) ? 0 : key - wr;
+    const int q_hi = (key >= p.N) ? q_lo : ((wl < 0) ? p.Npad + BM : key + wl + 1);
+    const unsigned q_span = static_cast<unsigned>(q_hi - q_lo);
     bool ok = true;
-    int gs = 0, kvn = 0, nsplit = 0;
-    Seg sg;
-    while (ok && sched.next(sg, steps)) {
-      const int bh = sg.tile / n_kt, j = sg.tile % n_kt;
-      const int k0 = j * BN;
-      const int key = k0 + krow;
-      const int nsteps = sg.s1 - sg.s0;
-      // warps 0-3 own dK, warps 4-7 dV (rows of this tile)
-      uint16_t* out = (h == 0 ? p.dK : p.dV) + (static_cast<size_t>(bh) * p.N + key) * D;
-      if (nsteps <= 0) {
-        // no query sees this tile: dK = dV = 0 (only whole tiles can be empty)
-        if (key < p.N) {
-          uint4* dst = reinterpret_cast<uint4*>(out);
+    int i = i_lo - 1;
+    for (int s = 0; s < nsteps && ok; ++s) {
+      do ++i; while (!member(i));
+      const int qh0 = i * BM + 64 * h;  // first query of this half
+      // The two barriers that completed long ago are observed first, so that the work
+      // starts as soon as S^T and dP^T are in TMEM: the dQ MMA of the last step has
+      // finished reading this dS chunk, and L2 and D of this half arrived with its Q rows.
+      if (s > 0)
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(dq_bar), (s - 1) & 1, wd));
+      if ((warp & 3) == 0) FA_TRACE_POINT(10, s, h);
+      const int seqQ = seq_of(s, h, 1);
+      if (ok)
+        ok = __all_sync(0xffffffffu,
+                        mbar_wait(bar(C::kBarFull + slot_of(seqQ)), round_of(seqQ) & 1, wd));
+      if ((warp & 3) == 0) FA_TRACE_POINT(12, s, h);
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarS + h), s & 1, wd));
+      if ((warp & 3) == 0) FA_TRACE_POINT(14, s, h);
+      if (!ok) break;
+      tc_fence_after();
+      const float4* Lv = reinterpret_cast<const float4*>(
+          base_ptr + C::kVecOff + slot_of(seqQ) * 2 * C::kVecBytes);
+      const float4* Dv4 = Lv + 64 / 4;
+      // masking is needed only where the half crosses an edge of some key's visible
+      // queries (the causal diagonal, a window edge) and on a ragged key tile
+      const bool mask = ragged_keys || (wr >= 0 && k0 + BN - 1 - wr > qh0) ||
+                        (wl >= 0 && k0 + wl < qh0 + 63);
+      const int qoff = qh0 - q_lo;  // query qh0 + x is visible iff qoff + x < q_span (unsigned)
+      // The element loop in two compiled forms: with the mask tests only on steps
+      // that cross a mask edge, none on all the others.
+      auto p_ds = [&](auto masked) {
+        constexpr bool kM = decltype(masked)::value;
+        uint32_t sv[2][16], dv[2][16];
+        tmem_ld16(tm_s, sv[0]);
+        tmem_ld16(tm_dp, dv[0]);
+        tmem_wait_ld();
 #pragma unroll
-          for (int u = 0; u < D / 8; ++u) dst[u] = make_uint4(0u, 0u, 0u, 0u);
-        }
-        continue;
-      }
-      const bool ragged_keys = k0 + BN > p.N;
-      // queries that see this key row: [q_lo, q_hi) (empty for a padding key)
-      const int q_lo = (wr < 0) ? 0 : key - wr;
-      const int q_hi = (key >= p.N) ? q_lo : ((wl < 0) ? p.Npad + BM : key + wl + 1);
-      const unsigned q_span = static_cast<unsigned>(q_hi - q_lo);
-      int i = -1;
-      for (int s = 0; s < nsteps && ok; ++s, ++gs) {
-        i = step_qt(s, i, sg);
-        const int qh0 = i * BM + 64 * h;  // first query of this half
-        // The two barriers that completed long ago are observed first, so that the work
-        // starts as soon as S^T and dP^T are in TMEM: the dQ MMA of the last step has
-        // finished reading this dS chunk, and L2 and D of this half arrived with its Q rows.
-        if (gs > 0)
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(dq_bar), (gs - 1) & 1, wd));
-        if ((warp & 3) == 0) FA_TRACE_POINT(10, gs, h);
-        const int seqQ = seq_of(gs, h, 1);
-        if (ok)
-          ok = __all_sync(0xffffffffu,
-                          mbar_wait(bar(C::kBarFull + slot_of(seqQ)), round_of(seqQ) & 1, wd));
-        if ((warp & 3) == 0) FA_TRACE_POINT(12, gs, h);
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarS + h), gs & 1, wd));
-        if ((warp & 3) == 0) FA_TRACE_POINT(14, gs, h);
-        if (!ok) break;
-        tc_fence_after();
-        const float4* Lv = reinterpret_cast<const float4*>(
-            base_ptr + C::kVecOff + slot_of(seqQ) * 2 * C::kVecBytes);
-        const float4* Dv4 = Lv + 64 / 4;
-        // masking is needed only where the half crosses an edge of some key's visible
-        // queries (the causal diagonal, a window edge) and on a ragged key tile
-        const bool mask = ragged_keys || (wr >= 0 && k0 + BN - 1 - wr > qh0) ||
-                          (wl >= 0 && k0 + wl < qh0 + 63);
-        const int qoff = qh0 - q_lo;  // query qh0 + x is visible iff qoff + x < q_span (unsigned)
-        // The element loop in two compiled forms: with the mask tests only on steps
-        // that cross a mask edge, none on all the others.
-        auto p_ds = [&](auto masked) {
-          constexpr bool kM = decltype(masked)::value;
-          uint32_t sv[2][16], dv[2][16];
-          tmem_ld16(tm_s, sv[0]);
-          tmem_ld16(tm_dp, dv[0]);
-          tmem_wait_ld();
-          if ((warp & 3) == 0) FA_TRACE_POINT(60, gs, h);
-#pragma unroll
-          for (int cc = 0; cc < 4; ++cc) {
-            const int cur = cc & 1;
-            if (cc + 1 < 4) {  // the next chunk's loads overlap this chunk's arithmetic
-              tmem_ld16(tm_s + 16 * (cc + 1), sv[cur ^ 1]);
-              tmem_ld16(tm_dp + 16 * (cc + 1), dv[cur ^ 1]);
-            }
-            // Dropout bytes of this key for the chunk's 16 queries: byte e of zq[v] is
-            // query 16cc + 4v + e of the half. One block covers 4 queries x 4 keys, and
-            // the lanes of keys 4g..4g+3 share its counter: lane u draws the block of the
-            // query group (qh0 + 16cc) / 4 + u, regroups its bytes by key (zq[b] = byte b
-            // of words 0..3) and a 4 x 4 transpose across the four lanes hands each lane
-            // its own key's bytes of all four blocks.
-            [[maybe_unused]] uint32_t zq[4] = {0u, 0u, 0u, 0u};
-            if constexpr (kDropout) {
-              const int u = lane & 3;
-              const uint4 w = philox4x32_10(
-                  make_uint4(static_cast<uint32_t>(key >> 2),
-                             static_cast<uint32_t>(((qh0 + cc * 16) >> 2) + u),
-                             static_cast<uint32_t>(bh), p.drop.offset),
-                  p.drop.seed_lo, p.drop.seed_hi);
-              const uint32_t t0 = __byte_perm(w.x, w.y, 0x5140), t1 = __byte_perm(w.x, w.y, 0x7362);
-              const uint32_t t2 = __byte_perm(w.z, w.w, 0x5140), t3 = __byte_perm(w.z, w.w, 0x7362);
-              zq[0] = __byte_perm(t0, t2, 0x5410);
-              zq[1] = __byte_perm(t0, t2, 0x7632);
-              zq[2] = __byte_perm(t1, t3, 0x5410);
-              zq[3] = __byte_perm(t1, t3, 0x7632);
-              transpose4_lanes(zq, u);
-            }
-            uint32_t pk[8], dk[8];
-#pragma unroll
-            for (int v = 0; v < 4; ++v) {
-              const float4 L4 = Lv[cc * 4 + v];
-              const float4 D4 = Dv4[cc * 4 + v];
-              const float Ls[4] = {L4.x, L4.y, L4.z, L4.w};
-              const float Ds[4] = {D4.x, D4.y, D4.z, D4.w};
-              float pv[4], dsv[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int k = 4 * v + e;
-                float pe = ex2_approx(fmaf(__uint_as_float(sv[cur][k]), c, -Ls[e]));
-                if (kM && static_cast<unsigned>(qoff + cc * 16 + k) >= q_span) pe = 0.f;
-                if constexpr (kDropout) {
-                  // dV takes P o Z * scale and dS = P o (dP o Z * scale - D), with
-                  // scale = 1 / (1 - threshold / 256)
-                  const float zs =
-                      (((zq[v] >> (8 * e)) & 0xffu) >= p.drop.threshold) ? p.drop.scale : 0.0f;
-                  pv[e] = pe * zs;
-                  dsv[e] = pe * (__uint_as_float(dv[cur][k]) * zs - Ds[e]);
-                } else {
-                  pv[e] = pe;
-                  dsv[e] = pe * (__uint_as_float(dv[cur][k]) - Ds[e]);
-                }
-              }
-              pk[2 * v] = pack2<E>(pv[0], pv[1]);
-              pk[2 * v + 1] = pack2<E>(pv[2], pv[3]);
-              dk[2 * v] = pack2<E>(dsv[0], dsv[1]);
-              dk[2 * v + 1] = pack2<E>(dsv[2], dsv[3]);
-            }
-            tmem_st8(tm_s + 8 * cc, pk);
-            tmem_st8(tm_dp + 8 * cc, dk);
-            // dS into the swizzled shared chunk: 16 queries = 16-byte units 2cc, 2cc+1
-            *reinterpret_cast<uint4*>(ds_row + (((2 * cc) ^ (krow & 7)) * 16)) =
-                make_uint4(dk[0], dk[1], dk[2], dk[3]);
-            *reinterpret_cast<uint4*>(ds_row + (((2 * cc + 1) ^ (krow & 7)) * 16)) =
-                make_uint4(dk[4], dk[5], dk[6], dk[7]);
-            if (cc + 1 < 4) tmem_wait_ld();
+        for (int cc = 0; cc < 4; ++cc) {
+          const int cur = cc & 1;
+          if (cc + 1 < 4) {  // the next chunk's loads overlap this chunk's arithmetic
+            tmem_ld16(tm_s + 16 * (cc + 1), sv[cur ^ 1]);
+            tmem_ld16(tm_dp + 16 * (cc + 1), dv[cur ^ 1]);
           }
-        };
-        if (mask)
-          p_ds(std::true_type{});
-        else
-          p_ds(std::false_type{});
-        if ((warp & 3) == 0) FA_TRACE_POINT(61, gs, h);
-        tmem_wait_st();
-        if ((warp & 3) == 0) FA_TRACE_POINT(62, gs, h);
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(C::kBarP + h));
-        if ((warp & 3) == 0) FA_TRACE_POINT(16, gs, h);
-      }
-      if (!ok) break;
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarDKDV), kvn & 1, wd));
-      if (!ok) break;
-      // Read dK (warps 0-3, times scale) or dV (warps 4-7) out of TMEM: to the output
-      // for a whole tile, else to this CTA's partial slot (fp32, unscaled).
+          // Dropout bytes of this key for the chunk's 16 queries: byte e of zq[v] is
+          // query 16cc + 4v + e of the half. One block covers 4 queries x 4 keys, and
+          // the lanes of keys 4g..4g+3 share its counter: lane u draws the block of the
+          // query group (qh0 + 16cc) / 4 + u, regroups its bytes by key (zq[b] = byte b
+          // of words 0..3) and a 4 x 4 transpose across the four lanes hands each lane
+          // its own key's bytes of all four blocks.
+          [[maybe_unused]] uint32_t zq[4] = {0u, 0u, 0u, 0u};
+          if constexpr (kDropout) {
+            const int u = lane & 3;
+            const uint4 w = philox4x32_10(
+                make_uint4(static_cast<uint32_t>(key >> 2),
+                           static_cast<uint32_t>(((qh0 + cc * 16) >> 2) + u),
+                           static_cast<uint32_t>(bh), p.drop.offset),
+                p.drop.seed_lo, p.drop.seed_hi);
+            const uint32_t t0 = __byte_perm(w.x, w.y, 0x5140), t1 = __byte_perm(w.x, w.y, 0x7362);
+            const uint32_t t2 = __byte_perm(w.z, w.w, 0x5140), t3 = __byte_perm(w.z, w.w, 0x7362);
+            zq[0] = __byte_perm(t0, t2, 0x5410);
+            zq[1] = __byte_perm(t0, t2, 0x7632);
+            zq[2] = __byte_perm(t1, t3, 0x5410);
+            zq[3] = __byte_perm(t1, t3, 0x7632);
+            transpose4_lanes(zq, u);
+          }
+          uint32_t pk[8], dk[8];
+#pragma unroll
+          for (int v = 0; v < 4; ++v) {
+            const float4 L4 = Lv[cc * 4 + v];
+            const float4 D4 = Dv4[cc * 4 + v];
+            const float Ls[4] = {L4.x, L4.y, L4.z, L4.w};
+            const float Ds[4] = {D4.x, D4.y, D4.z, D4.w};
+            float pv[4], dsv[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int k = 4 * v + e;
+              float pe = ex2_approx(fmaf(__uint_as_float(sv[cur][k]), c, -Ls[e]));
+              if (kM && static_cast<unsigned>(qoff + cc * 16 + k) >= q_span) pe = 0.f;
+              if constexpr (kDropout) {
+                // dV takes P o Z * scale and dS = P o (dP o Z * scale - D), with
+                // scale = 1 / (1 - threshold / 256)
+                const float zs =
+                    (((zq[v] >> (8 * e)) & 0xffu) >= p.drop.threshold) ? p.drop.scale : 0.0f;
+                pv[e] = pe * zs;
+                dsv[e] = pe * (__uint_as_float(dv[cur][k]) * zs - Ds[e]);
+              } else {
+                pv[e] = pe;
+                dsv[e] = pe * (__uint_as_float(dv[cur][k]) - Ds[e]);
+              }
+            }
+            pk[2 * v] = pack2<E>(pv[0], pv[1]);
+            pk[2 * v + 1] = pack2<E>(pv[2], pv[3]);
+            dk[2 * v] = pack2<E>(dsv[0], dsv[1]);
+            dk[2 * v + 1] = pack2<E>(dsv[2], dsv[3]);
+          }
+          tmem_st8(tm_s + 8 * cc, pk);
+          tmem_st8(tm_dp + 8 * cc, dk);
+          // dS into the swizzled shared chunk: 16 queries = 16-byte units 2cc, 2cc+1
+          *reinterpret_cast<uint4*>(ds_row + (((2 * cc) ^ (krow & 7)) * 16)) =
+              make_uint4(dk[0], dk[1], dk[2], dk[3]);
+          *reinterpret_cast<uint4*>(ds_row + (((2 * cc + 1) ^ (krow & 7)) * 16)) =
+              make_uint4(dk[4], dk[5], dk[6], dk[7]);
+          if (cc + 1 < 4) tmem_wait_ld();
+        }
+      };
+      if (mask)
+        p_ds(std::true_type{});
+      else
+        p_ds(std::false_type{});
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::kBarP + h));
+      if ((warp & 3) == 0) FA_TRACE_POINT(16, s, h);
+    }
+    if (nsteps == 0 && key < p.N) {
+      // no query sees this key: dK = dV = 0 (warps 0-3 dK, warps 4-7 dV)
+      uint4* dst = reinterpret_cast<uint4*>((h == 0 ? p.dK : p.dV) +
+                                            (static_cast<size_t>(bh) * p.N + key) * D);
+#pragma unroll
+      for (int u = 0; u < D / 8; ++u) dst[u] = make_uint4(0u, 0u, 0u, 0u);
+    }
+    if (ok && nsteps > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarDKDV), 0, wd));
+    if (ok && nsteps > 0) {
+      // warps 0-3 write dK (times scale), warps 4-7 write dV
       tc_fence_after();
       const uint32_t tm_acc = tmem + lane_off + (h == 0 ? C::kTmDK : C::kTmDV);
+      uint16_t* out = (h == 0 ? p.dK : p.dV) + (static_cast<size_t>(bh) * p.N + key) * D;
       const float mul = (h == 0) ? p.scale : 1.0f;
-      // slot layout: [CTA][slot 0/1][dK, dV][128 key rows][D]
-      auto slot_row = [&](int cta, int slot) -> float* {
-        return p.part + ((static_cast<size_t>(cta) * 2 + slot) * 2 + h) * (BN * D) +
-               static_cast<size_t>(krow) * D;
-      };
-      float* part = (sg.slot < 0) ? nullptr : slot_row(static_cast<int>(blockIdx.x), sg.slot);
 #pragma unroll 1
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t v[32];
         tmem_ld32(tm_acc + cc * 32, v);
         tmem_wait_ld();
-        if (part != nullptr) {
-          float4* dst = reinterpret_cast<float4*>(part + cc * 32);
+        uint32_t pk[16];
 #pragma unroll
-          for (int u = 0; u < 8; ++u)
-            dst[u] = make_float4(__uint_as_float(v[4 * u]), __uint_as_float(v[4 * u + 1]),
-                                 __uint_as_float(v[4 * u + 2]), __uint_as_float(v[4 * u + 3]));
-        } else {
-          uint32_t pk[16];
+        for (int k = 0; k < 16; ++k)
+          pk[k] = pack2<E>(__uint_as_float(v[2 * k]) * mul, __uint_as_float(v[2 * k + 1]) * mul);
+        if (key < p.N) {
+          uint4* dst = reinterpret_cast<uint4*>(out + cc * 32);
 #pragma unroll
-          for (int k = 0; k < 16; ++k)
-            pk[k] = pack2<E>(__uint_as_float(v[2 * k]) * mul, __uint_as_float(v[2 * k + 1]) * mul);
-          if (key < p.N) {
-            uint4* dst = reinterpret_cast<uint4*>(out + cc * 32);
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-              dst[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-          }
-        }
-      }
-      if (part != nullptr) __threadfence();  // the slot rows before this CTA's arrival
-      // the accumulators may be overwritten by the next segment now
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(C::kBarDKDVFree));
-      ++kvn;
-      if (sg.slot >= 0) {
-        // Split tile: count this CTA in; the last of the c1 - c0 + 1 CTAs adds the
-        // slots up in CTA order and writes dK, dV. Warp 0 counts the CTA in once all
-        // 8 warps' slot rows are written (bounded waits: a warp that gave up on an
-        // earlier wait never strands the others).
-        if (lane == 0) mbar_arrive(bar(C::kBarSplitWritten));
-        if (warp == 0) {
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarSplitWritten), nsplit & 1, wd));
-          if (ok && lane == 0) {
-            __threadfence();
-            *arrived = atomicAdd(p.arrivals + sg.c1, 1u);
-            mbar_arrive(bar(C::kBarSplitDecided));
-          }
-        }
-        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarSplitDecided), nsplit & 1, wd));
-        ++nsplit;
-        if (!ok) break;
-        if (*arrived == static_cast<unsigned>(sg.c1 - sg.c0)) {
-          __threadfence();
-          float acc[32];
-#pragma unroll 1
-          for (int cc = 0; cc < D / 32; ++cc) {
-#pragma unroll
-            for (int k = 0; k < 32; ++k) acc[k] = 0.0f;
-            // two slots' loads in flight at a time; the sum stays in CTA order
-            for (int cta = sg.c0; cta <= sg.c1; cta += 2) {
-              const bool two = cta + 1 <= sg.c1;
-              const float4* a4 =
-                  reinterpret_cast<const float4*>(slot_row(cta, sched.slot_of(cta, sg.a)) + cc * 32);
-              const float4* b4 = reinterpret_cast<const float4*>(
-                  slot_row(two ? cta + 1 : cta, sched.slot_of(two ? cta + 1 : cta, sg.a)) + cc * 32);
-              float4 xa[8], xb[8];
-#pragma unroll
-              for (int u = 0; u < 8; ++u) {
-                xa[u] = __ldcg(a4 + u);
-                xb[u] = two ? __ldcg(b4 + u) : make_float4(0.f, 0.f, 0.f, 0.f);
-              }
-#pragma unroll
-              for (int u = 0; u < 8; ++u) {
-                acc[4 * u] += xa[u].x;
-                acc[4 * u + 1] += xa[u].y;
-                acc[4 * u + 2] += xa[u].z;
-                acc[4 * u + 3] += xa[u].w;
-              }
-              if (two) {
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                  acc[4 * u] += xb[u].x;
-                  acc[4 * u + 1] += xb[u].y;
-                  acc[4 * u + 2] += xb[u].z;
-                  acc[4 * u + 3] += xb[u].w;
-                }
-              }
-            }
-            uint32_t pk[16];
-#pragma unroll
-            for (int k = 0; k < 16; ++k) pk[k] = pack2<E>(acc[2 * k] * mul, acc[2 * k + 1] * mul);
-            if (key < p.N) {
-              uint4* dst = reinterpret_cast<uint4*>(out + cc * 32);
-#pragma unroll
-              for (int u = 0; u < 4; ++u)
-                dst[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-            }
-          }
+          for (int u = 0; u < 4; ++u)
+            dst[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
         }
       }
     }
@@ -935,59 +630,53 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
     const int row = wq * 32 + lane;  // TMEM lane: head-dim element (D = 128) or query (D = 64)
     bool ok = true;
-    int gs = 0;
-    Seg sg;
-    while (ok && sched.next(sg, steps)) {
-      const int bh = sg.tile / n_kt;
-      const int nsteps = sg.s1 - sg.s0;
-      int i = -1;
-      for (int s = 0; s < nsteps && ok; ++s, ++gs) {
-        i = step_qt(s, i, sg);
-        const int q0 = i * BM;
-        if constexpr (D == 128) {
-          for (int h = 0; h < 2 && ok; ++h) {
-            ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarDQFull + h), gs & 1, wd));
-            if (!ok) break;
-            if (warp == kWarpDq) FA_TRACE_POINT(20, gs, h);
-            tc_fence_after();
-            uint32_t v[2][32];
-            tmem_ld32(tmem + lane_off + C::kTmS + 64 * h, v[0]);
-            tmem_ld32(tmem + lane_off + C::kTmS + 64 * h + 32, v[1]);
-            tmem_wait_ld();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(bar(C::kBarDQEmpty + h));
-            if (warp == kWarpDq) FA_TRACE_POINT(22, gs, h);
-            // element `row` of the head dimension for 64 queries: a warp covers 32
-            // consecutive elements of one query row (128 contiguous bytes) per add
-            float* dst = p.dQacc + (static_cast<size_t>(bh) * p.N + q0 + 64 * h) * D + row;
-            const int nq = min(64, p.N - (q0 + 64 * h));
-#pragma unroll
-            for (int qq = 0; qq < 64; ++qq)
-              if (qq < nq) red_add(dst + static_cast<size_t>(qq) * D, __uint_as_float(v[qq / 32][qq % 32]));
-            if (warp == kWarpDq) FA_TRACE_POINT(24, gs, h);
-          }
-        } else {
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarDQFull), gs & 1, wd));
+    int i = i_lo - 1;
+    for (int s = 0; s < nsteps && ok; ++s) {
+      do ++i; while (!member(i));
+      const int q0 = i * BM;
+      if constexpr (D == 128) {
+        for (int h = 0; h < 2 && ok; ++h) {
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarDQFull + h), s & 1, wd));
           if (!ok) break;
+          if (warp == kWarpDq) FA_TRACE_POINT(20, s, h);
           tc_fence_after();
           uint32_t v[2][32];
-          tmem_ld32(tmem + lane_off + C::kTmDQ64, v[0]);
-          tmem_ld32(tmem + lane_off + C::kTmDQ64 + 32, v[1]);
+          tmem_ld32(tmem + lane_off + C::kTmS + 64 * h, v[0]);
+          tmem_ld32(tmem + lane_off + C::kTmS + 64 * h + 32, v[1]);
           tmem_wait_ld();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(bar(C::kBarDQEmpty));
-          const int q = q0 + row;
-          if (q < p.N) {
-            float* dst = p.dQacc + (static_cast<size_t>(bh) * p.N + q) * D;
+          if (lane == 0) mbar_arrive(bar(C::kBarDQEmpty + h));
+          if (warp == kWarpDq) FA_TRACE_POINT(22, s, h);
+          // element `row` of the head dimension for 64 queries: a warp covers 32
+          // consecutive elements of one query row (128 contiguous bytes) per add
+          float* dst = p.dQacc + (static_cast<size_t>(bh) * p.N + q0 + 64 * h) * D + row;
+          const int nq = min(64, p.N - (q0 + 64 * h));
 #pragma unroll
-            for (int k = 0; k < 16; ++k)
-              red_add_v4(dst + 4 * k, __uint_as_float(v[k / 8][(4 * k) % 32]),
-                         __uint_as_float(v[k / 8][(4 * k + 1) % 32]),
-                         __uint_as_float(v[k / 8][(4 * k + 2) % 32]),
-                         __uint_as_float(v[k / 8][(4 * k + 3) % 32]));
-          }
+          for (int qq = 0; qq < 64; ++qq)
+            if (qq < nq) red_add(dst + static_cast<size_t>(qq) * D, __uint_as_float(v[qq / 32][qq % 32]));
+          if (warp == kWarpDq) FA_TRACE_POINT(24, s, h);
+        }
+      } else {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarDQFull), s & 1, wd));
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t v[2][32];
+        tmem_ld32(tmem + lane_off + C::kTmDQ64, v[0]);
+        tmem_ld32(tmem + lane_off + C::kTmDQ64 + 32, v[1]);
+        tmem_wait_ld();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(C::kBarDQEmpty));
+        const int q = q0 + row;
+        if (q < p.N) {
+          float* dst = p.dQacc + (static_cast<size_t>(bh) * p.N + q) * D;
+#pragma unroll
+          for (int k = 0; k < 16; ++k)
+            red_add_v4(dst + 4 * k, __uint_as_float(v[k / 8][(4 * k) % 32]),
+                       __uint_as_float(v[k / 8][(4 * k + 1) % 32]),
+                       __uint_as_float(v[k / 8][(4 * k + 2) % 32]),
+                       __uint_as_float(v[k / 8][(4 * k + 3) % 32]));
         }
       }
     }

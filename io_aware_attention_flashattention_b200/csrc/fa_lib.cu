@@ -377,78 +377,6 @@ FwdSplit fwd_split(int BH, int N, int wl, int wr, int sms) {
   return best;
 }
 
-// ---------------------------------------------------------------- backward schedule
-//
-// The backward main kernel is persistent (see the schedule in fa_bwd_sm100.cuh): G
-// CTAs, at most one per SM and at most kMaxBwdCtas, and no more than one per
-// kMinBwdSteps steps of work. Whole key tiles go round robin; the tail (fewer than G
-// tiles) is split by steps over all CTAs, except with a block mask, whose per-tile
-// step counts are device data: there the round robin covers the tail too.
-constexpr int kMaxBwdCtas = 160;
-constexpr long long kMinBwdSteps = 4;
-
-struct BwdSched {
-  int G, rounds, tail_split, pair_units;
-};
-
-// The schedule the backward uses: 0 = one CTA per key tile (the grid is the tiles);
-// 1 = persistent CTAs over units of two tiles, round robin only; 2 = as 1, with the
-// tail split by steps over all CTAs.
-#ifndef FA_BWD_SCHED
-#define FA_BWD_SCHED 2
-#endif
-
-// Query tiles walked by key tile j without a block mask (the kernel's query_range).
-long long bwd_tile_steps(int j, int N, int wl, int wr) {
-  const int n_q = (N + 127) / 128;
-  const int k0 = j * 128, k1 = std::min(k0 + 128, N) - 1;
-  const int lo = (wr < 0) ? 0 : std::max(0, k0 - wr) / 128;
-  const int hi = (wl < 0) ? n_q : std::min(n_q, (k1 + wl) / 128 + 1);
-  return std::max(hi - lo, 0);
-}
-
-BwdSched bwd_schedule(int BH, int N, int wl, int wr, bool block_mask, int sms) {
-  const int n_kt = (N + 127) / 128;
-  long long G = std::min<long long>(sms > 0 ? sms : 148, kMaxBwdCtas);
-  BwdSched sc{};
-  sc.pair_units = 1;
-  if (FA_BWD_SCHED == 0) {  // one CTA per tile: units of one tile, G = all of them
-    sc.pair_units = 0;
-    sc.G = static_cast<int>(std::min<long long>(static_cast<long long>(BH) * n_kt, 1ll << 30));
-    sc.rounds = 1;
-    sc.tail_split = 0;
-    return sc;
-  }
-  if (block_mask) {
-    const long long n_units = static_cast<long long>(BH) * ((n_kt + 1) / 2);
-    G = std::max<long long>(1, std::min(G, n_units));
-    sc.G = static_cast<int>(G);
-    sc.rounds = static_cast<int>(n_units / G);
-    sc.tail_split = 0;
-    return sc;
-  }
-  long long per_head = 0;
-  for (int j = 0; j < n_kt; ++j) per_head += bwd_tile_steps(j, N, wl, wr);
-  const long long total = per_head * BH;
-  G = std::max<long long>(1, std::min(G, total / kMinBwdSteps));
-  // units of two key tiles (j, n_kt - 1 - j) per head
-  const long long n_units = static_cast<long long>(BH) * ((n_kt + 1) / 2);
-  sc.G = static_cast<int>(G);
-  sc.rounds = static_cast<int>(n_units / G);
-  sc.tail_split = (FA_BWD_SCHED == 2 && (n_units % G) != 0) ? 1 : 0;
-  return sc;
-}
-
-// Upper bound of G for a shape, known without the device: the workspace holds the
-// partial-sum slots of that many CTAs.
-long long bwd_max_ctas(long long BH, int N) {
-  const long long n_kt = (static_cast<long long>(N) + 127) / 128;
-  const long long steps = BH * n_kt * n_kt;  // every tile walking every query tile
-  const long long units = BH * ((n_kt + 1) / 2);
-  return std::max<long long>(1, std::min<long long>(kMaxBwdCtas,
-                                                    std::max(units, steps / kMinBwdSteps)));
-}
-
 int device_sms() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
@@ -523,9 +451,6 @@ struct BwdPlan {
   float* L2;
   float* Dv;
   float* dQacc;
-  float* part;          // partial dK/dV slots of split tiles
-  unsigned* arrivals;   // their arrival counters
-  int n_arrivals;
 };
 
 fa_status bwd_plan(const void* const* ptrs, int nptrs, int B, int H, int N, int d,
@@ -543,19 +468,12 @@ fa_status bwd_plan(const void* const* ptrs, int nptrs, int B, int H, int N, int 
   if (workspace == nullptr || !aligned16(workspace)) return FA_ERR_INVALID_ARG;
   if (workspace_bytes < fa_backward_workspace_size(B, H, N, d)) return FA_ERR_INVALID_ARG;
   if ((st = prepare_device()) != FA_OK) return st;
-  // workspace: L2 [BH, Npad] | D [BH, Npad] | dQ accumulator [BH, N, d] (fp32) |
-  // partial slots [Gmax][2][2][128][d] (fp32) | arrival counters [Gmax]
+  // workspace: L2 [BH, Npad] | D [BH, Npad] | dQ accumulator [BH, N, d] (fp32)
   char* ws = static_cast<char*>(workspace);
   const size_t vec_bytes = round256(static_cast<size_t>(plan->BH) * plan->Npad * sizeof(float));
-  const size_t acc_bytes = round256(static_cast<size_t>(plan->BH) * N * d * sizeof(float));
-  const long long gmax = bwd_max_ctas(plan->BH, N);
-  const size_t part_bytes = round256(static_cast<size_t>(gmax) * 4 * 128 * d * sizeof(float));
   plan->L2 = reinterpret_cast<float*>(ws);
   plan->Dv = reinterpret_cast<float*>(ws + vec_bytes);
   plan->dQacc = reinterpret_cast<float*>(ws + 2 * vec_bytes);
-  plan->part = reinterpret_cast<float*>(ws + 2 * vec_bytes + acc_bytes);
-  plan->arrivals = reinterpret_cast<unsigned*>(ws + 2 * vec_bytes + acc_bytes + part_bytes);
-  plan->n_arrivals = static_cast<int>(gmax);
   return FA_OK;
 }
 
@@ -574,9 +492,9 @@ fa_status preprocess_impl(const void* O, const void* dO, const float* LSE, int B
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (d == 64)
     return launch(bwd::fa_bwd_pre_kernel<64, E>, blocks, 256, 0, s, O16, dO16, LSE, pl.L2, pl.Dv,
-                  pl.dQacc, N, pl.Npad, rows, pl.arrivals, pl.n_arrivals);
+                  pl.dQacc, N, pl.Npad, rows);
   return launch(bwd::fa_bwd_pre_kernel<128, E>, blocks, 256, 0, s, O16, dO16, LSE, pl.L2, pl.Dv,
-                pl.dQacc, N, pl.Npad, rows, pl.arrivals, pl.n_arrivals);
+                pl.dQacc, N, pl.Npad, rows);
 }
 
 template <Elt E>
@@ -609,17 +527,7 @@ fa_status main_impl(const void* Q, const void* K, const void* V, const void* dO,
   p.blocks = mask.blocks;
   p.drop = drop.params;
   p.timeout_ns = watchdog_ns();
-  const BwdSched sc = bwd_schedule(pl.BH, N, mask.wl, mask.wr, mask.blocks != nullptr,
-                                   device_sms());
-  p.n_kt = pl.Npad / bwd::BN;
-  p.n_tiles = pl.BH * p.n_kt;
-  p.rounds = sc.rounds;
-  p.tail_split = sc.tail_split;
-  p.pair_units = sc.pair_units;
-  p.part = pl.part;
-  p.arrivals = pl.arrivals;
-  if (sc.tail_split && sc.G > pl.n_arrivals) return FA_ERR_UNSUPPORTED;  // G <= the bound
-  const dim3 grid(static_cast<unsigned>(sc.G));
+  const dim3 grid(static_cast<unsigned>(pl.Npad / bwd::BN) * pl.BH);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool g = mask.general();
   using bwd::Cfg;
@@ -693,9 +601,7 @@ size_t fa_backward_workspace_size(int B, int H, int N, int d) {
   if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
   const size_t bh = static_cast<size_t>(B) * H;
   const size_t npad = (static_cast<size_t>(N) + 127) / 128 * 128;
-  const size_t gmax = static_cast<size_t>(bwd_max_ctas(static_cast<long long>(B) * H, N));
-  return 2 * round256(bh * npad * sizeof(float)) + round256(bh * N * d * sizeof(float)) +
-         round256(gmax * 4 * 128 * d * sizeof(float)) + round256(gmax * sizeof(unsigned));
+  return 2 * round256(bh * npad * sizeof(float)) + round256(bh * N * d * sizeof(float));
 }
 
 float fa_dropout_rate(float p_drop) {
