@@ -9,7 +9,8 @@ of seeded synthetic inputs already resident in HBM.
 Metric: attention fwd+bwd TFLOP/s, counting 4*B*H*N^2*d for the forward (halved
 when causal) and 2.5x that for the backward. Timing: CUDA events on the launching
 stream around every kernel of every step; L2 is flushed (a 256 MiB write) before
-each timed step, outside the events; W untimed warm-up steps; a barrier and a
+each timed step, and the step's launches are queued ahead (a short GPU-side spin),
+both outside the events; W untimed warm-up steps; a barrier and a
 device synchronise on both sides of the K timed steps; max over ranks. With N > 1
 each rank runs its own replica of the workload (independent heads; no collective
 on the data path), so the scaling is weak. nvidia-smi samples the clocks during
@@ -38,6 +39,10 @@ METRIC = "attention fwd/bwd TFLOP/s (bf16, d=128) and % of B200 dense BF16 peak"
 DEFAULT_WORKLOAD = "long_b1h8_n16384_d128"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0}
 L2_FLUSH_BYTES = 256 << 20
+# A GPU-side spin of this many clocks (about 100 us) before each timed region, outside its
+# events: the host has then queued every launch of the region before the GPU reaches the
+# first event, so the events time the kernels and not the Python call overhead between them.
+QUEUE_AHEAD_CYCLES = 200_000
 
 
 def parse():
@@ -347,7 +352,8 @@ SECONDARY = [
 def secondary_configs(dev, peak: float, steps: int = 10, warmup: int = 3):
     """Forward and backward TFLOP/s of every SECONDARY case, timed like the main line:
     CUDA events on the launching stream around the forward and around the three
-    backward kernels, L2 flushed before each step, median of ``steps`` steps. FLOPs
+    backward kernels, L2 flushed and the launches queued ahead before each, median of
+    ``steps`` steps. FLOPs
     count only the (query, key) pairs the masks keep; the backward is 2.5x the
     forward. Inputs are seeded draws on the device (timing only; the parity tests use
     the host generator)."""
@@ -413,12 +419,14 @@ def secondary_configs(dev, peak: float, steps: int = 10, warmup: int = 3):
         tf, tb = [], []
         for it in range(warmup + steps):
             flush.zero_()
+            torch.cuda._sleep(QUEUE_AHEAD_CYCLES)
             e = [torch.cuda.Event(enable_timing=True) for _ in range(4)]
             e[0].record(stream)
             fwd()
             e[1].record(stream)
             if w.backward:
                 flush.zero_()  # the backward starts from a cold L2 too (outside its events)
+                torch.cuda._sleep(QUEUE_AHEAD_CYCLES)
                 e[2].record(stream)
                 bwd()
                 e[3].record(stream)
@@ -535,6 +543,7 @@ def main():
         t0 = time.perf_counter()
         for s in range(args.steps):
             flush.zero_()
+            torch.cuda._sleep(QUEUE_AHEAD_CYCLES)
             step(evs[s])
         torch.cuda.synchronize()
         t1 = time.perf_counter() - t0
