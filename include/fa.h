@@ -77,9 +77,13 @@ fa_status fa_forward(const void* Q, const void* K, const void* V, void* O, float
 
 /*
  * Workspace bytes fa_backward and fa_backward_f32 need for this shape, with
- * Npad = N rounded up to a multiple of 128:
+ * Npad = N rounded up to a multiple of 128 and T = B*H*Npad/128 key tiles:
  *   LSE*log2(e) (fp32 [B*H, Npad]) + D (fp32 [B*H, Npad]) + dQ accumulator
- *   (fp32 [B,H,N,d]), each region rounded up to 256 bytes.
+ *   (fp32 [B,H,N,d]) + room for S split key tiles: fp32 dK and dV partials of
+ *   both halves (fp32 [S,2,2,128,d]) and an arrival counter each (u32 [S]);
+ *   each region rounded up to 256 bytes. S = min(T, 160) when T <= 592 and
+ *   Npad >= 4096 (32 query tiles per key tile), else 0. (A launch of few key tiles runs some of them as two CTAs, one per
+ *   half of the query tiles, to fill the SMs' last wave.)
  * Returns 0 for a shape that is invalid or empty.
  */
 size_t fa_backward_workspace_size(int B, int H, int N, int d);
@@ -134,8 +138,11 @@ fa_status fa_backward_dq_convert(void* dQ, int B, int H, int N, int d, float sca
  *   Scratch: a 32 MiB array built into the library, one per GPU, placed in device
  *     memory when the library's module is loaded on that GPU and held until the
  *     process exits. The call allocates nothing.
- *   Limit: shapes whose fa_backward_workspace_size exceeds 32 MiB (33554432
- *     bytes) return FA_ERR_UNSUPPORTED and launch nothing.
+ *   Limit: shapes whose LSE*log2(e), D and dQ accumulator regions (the workspace size
+ *     with S = 0, see fa_backward_workspace_size) exceed 32 MiB (33554432 bytes)
+ *     return FA_ERR_UNSUPPORTED and launch nothing. The array holds no room for
+ *     split key tiles: every key tile runs whole, so where fa_backward would
+ *     split tiles dK and dV may differ from its result in the last bits.
  *   Set-up: the first call on a GPU looks up the array's device address with
  *     that GPU current (and may load the library's module there); make that first
  *     call before any stream capture. If the GPU's context is destroyed and

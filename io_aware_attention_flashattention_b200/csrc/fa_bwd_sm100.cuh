@@ -84,7 +84,9 @@ struct Cfg {
   static constexpr int kBarDQFull = kBarP + 2;  // [2]
   static constexpr int kBarDQEmpty = kBarDQFull + 2;  // [2]
   static constexpr int kBarDKDV = kBarDQEmpty + 2;
-  static constexpr int kBarDrain = kBarDKDV + 1;
+  static constexpr int kBarSplitWritten = kBarDKDV + 1;        // split tile: 8 warps' rows written
+  static constexpr int kBarSplitDecided = kBarSplitWritten + 1;  // ... and the arrival counted
+  static constexpr int kBarDrain = kBarSplitDecided + 1;
   static constexpr int kNumBars = kBarDrain + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kMaskOff = kMiscOff + 16;  // block-mask column of this key tile, as bits
@@ -111,7 +113,25 @@ struct Params {
   const uint8_t* blocks;  // [n_kt x n_kt] block mask (nonzero = kept), or null
   DropoutParams drop;     // used by the kDropout instances only
   unsigned long long timeout_ns;
+  // Split key tiles (no block mask): the last n_split tiles (head-major) have their
+  // query steps cut in two segments, [0, a) and [a, steps) with a = steps * split_num /
+  // 16 rounded and kept within [1, steps - 1], each run by a CTA of its own. The grid
+  // is the whole tiles first, then the larger segments, then the smaller ones. A
+  // segment's CTA writes its fp32 dK, dV partial to its slot, counts itself in, and
+  // the second to arrive adds the two slots (segment 0 first) and writes dK, dV.
+  int n_split;
+  int split_num;
+  float* part;         // [n_split][2 segments][dK, dV][128 key rows][D] fp32
+  unsigned* arrivals;  // [n_split] (zeroed by the preprocess)
 };
+
+// The first segment's step count for a tile of `steps` steps.
+__host__ __device__ __forceinline__ int split_point(int steps, int split_num) {
+  int a = (steps * split_num + 8) / 16;
+  if (a < 1) a = 1;
+  if (a > steps - 1) a = steps - 1;
+  return a;
+}
 
 __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b),
@@ -191,7 +211,9 @@ __global__ void __launch_bounds__(256)
     fa_bwd_pre_kernel(const uint16_t* __restrict__ O, const uint16_t* __restrict__ dO,
                       const float* __restrict__ LSE, float* __restrict__ L2,
                       float* __restrict__ Dv, float* __restrict__ dQacc, int N, int Npad,
-                      long long total_rows) {
+                      long long total_rows, unsigned* __restrict__ arrivals, int n_arrivals) {
+  if (blockIdx.x == 0)  // the main kernel's arrival counters of split tiles
+    for (int k = threadIdx.x; k < n_arrivals; k += blockDim.x) arrivals[k] = 0u;
   const long long r = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (r >= total_rows) return;  // total_rows = BH * Npad
@@ -263,6 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   auto bar = [&](int i) -> uint32_t { return bars + 8u * static_cast<uint32_t>(i); };
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::kMiscOff);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + C::kMiscOff + 4);
+  volatile unsigned* arrived = reinterpret_cast<volatile unsigned*>(base_ptr + C::kMiscOff + 8);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -275,14 +298,31 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Work item: head-major (the resident CTAs share one or two heads' Q, dO and dQ
   // accumulator in L2); within a head, key tile 0 (the heaviest if causal) first.
   const int n_kt = p.Npad / BN;
-  const int bh = static_cast<int>(blockIdx.x) / n_kt;
-  const int j = static_cast<int>(blockIdx.x) % n_kt;
+  const int n_tiles = p.BH * n_kt;
+  const int n_whole = n_tiles - p.n_split;
+  // this CTA's key tile and, for a split tile, which segment (-1: the whole tile)
+  int tile = static_cast<int>(blockIdx.x), seg = -1;
+  if (tile >= n_whole) {
+    const int c = tile - n_whole;                  // [larger segments][smaller segments]
+    const bool second_half = c >= p.n_split;
+    tile = n_whole + (second_half ? c - p.n_split : c);
+    const bool big_first = p.split_num < 8;        // segment 1 is the larger one
+    seg = (second_half == big_first) ? 0 : 1;
+  }
+  const int bh = tile / n_kt;
+  const int j = tile % n_kt;
   const int k0 = j * BN;
   const int n_q = (p.N + BM - 1) / BM;
   // query tiles [i_lo, i_hi) hold every query that may see a key of this tile
   const int k1 = min(k0 + BN, p.N) - 1;
-  const int i_lo = (wr < 0) ? 0 : max(0, k0 - wr) / BM;
-  const int i_hi = (wl < 0) ? n_q : min(n_q, (k1 + wl) / BM + 1);
+  const int i_lo_tile = (wr < 0) ? 0 : max(0, k0 - wr) / BM;
+  const int i_hi_tile = (wl < 0) ? n_q : min(n_q, (k1 + wl) / BM + 1);
+  // a split tile's segment walks a sub-range of the query tiles (no block mask then)
+  int i_lo = i_lo_tile, i_hi = i_hi_tile;
+  if (seg >= 0) {
+    const int a = split_point(i_hi_tile - i_lo_tile, p.split_num);
+    if (seg == 0) i_hi = i_lo_tile + a; else i_lo = i_lo_tile + a;
+  }
 
   // The block-mask column of this key tile as bits: warp w builds words w, w + 16, ...
   uint32_t* mask_bits = reinterpret_cast<uint32_t*>(base_ptr + C::kMaskOff);
@@ -308,6 +348,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(bar(C::kBarDQEmpty + h), 4);  // the 4 dQ warps
     }
     mbar_init(bar(C::kBarDKDV), 1);
+    mbar_init(bar(C::kBarSplitWritten), 8);  // the 8 P/dS warps
+    mbar_init(bar(C::kBarSplitDecided), 1);
     mbar_init(bar(C::kBarDrain), 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -602,16 +644,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (ok && nsteps > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarDKDV), 0, wd));
     if (ok && nsteps > 0) {
-      // warps 0-3 write dK (times scale), warps 4-7 write dV
+      // warps 0-3 write dK (times scale), warps 4-7 write dV; a split tile's segment
+      // writes its fp32 partial to its slot instead
       tc_fence_after();
       const uint32_t tm_acc = tmem + lane_off + (h == 0 ? C::kTmDK : C::kTmDV);
       uint16_t* out = (h == 0 ? p.dK : p.dV) + (static_cast<size_t>(bh) * p.N + key) * D;
       const float mul = (h == 0) ? p.scale : 1.0f;
+      const int ksplit = tile - n_whole;
+      // slot layout: [split tile][segment][dK, dV][128 key rows][D]
+      auto slot_row = [&](int sg) -> float* {
+        return p.part + ((static_cast<size_t>(ksplit) * 2 + sg) * 2 + h) * (BN * D) +
+               static_cast<size_t>(krow) * D;
+      };
 #pragma unroll 1
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t v[32];
         tmem_ld32(tm_acc + cc * 32, v);
         tmem_wait_ld();
+        if (seg >= 0) {
+          float4* dst = reinterpret_cast<float4*>(slot_row(seg) + cc * 32);
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            dst[u] = make_float4(__uint_as_float(v[4 * u]), __uint_as_float(v[4 * u + 1]),
+                                 __uint_as_float(v[4 * u + 2]), __uint_as_float(v[4 * u + 3]));
+          continue;
+        }
         uint32_t pk[16];
 #pragma unroll
         for (int k = 0; k < 16; ++k)
@@ -621,6 +678,48 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int u = 0; u < 4; ++u)
             dst[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+        }
+      }
+      if (seg >= 0) {
+        // Count this segment in once all 8 warps' rows are written (bounded waits); the
+        // second to arrive adds slot 0 and slot 1, in that order, and writes dK, dV.
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(C::kBarSplitWritten));
+        if (warp == 0) {
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarSplitWritten), 0, wd));
+          if (ok && lane == 0) {
+            __threadfence();
+            *arrived = atomicAdd(p.arrivals + ksplit, 1u);
+            mbar_arrive(bar(C::kBarSplitDecided));
+          }
+        }
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarSplitDecided), 0, wd));
+        if (ok && *arrived == 1u) {
+          __threadfence();
+          const float4* s0 = reinterpret_cast<const float4*>(slot_row(0));
+          const float4* s1 = reinterpret_cast<const float4*>(slot_row(1));
+#pragma unroll 1
+          for (int cc = 0; cc < D / 32; ++cc) {
+            float4 a[8], b[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              a[u] = __ldcg(s0 + cc * 8 + u);
+              b[u] = __ldcg(s1 + cc * 8 + u);
+            }
+            uint32_t pk[16];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+              pk[2 * u] = pack2<E>((a[u].x + b[u].x) * mul, (a[u].y + b[u].y) * mul);
+              pk[2 * u + 1] = pack2<E>((a[u].z + b[u].z) * mul, (a[u].w + b[u].w) * mul);
+            }
+            if (key < p.N) {
+              uint4* dst = reinterpret_cast<uint4*>(out + cc * 32);
+#pragma unroll
+              for (int u = 0; u < 4; ++u)
+                dst[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+            }
+          }
         }
       }
     }

@@ -377,6 +377,107 @@ FwdSplit fwd_split(int BH, int N, int wl, int wr, int sms) {
   return best;
 }
 
+// ---------------------------------------------------------------- backward tile split
+//
+// One backward CTA runs one key tile over all its query tiles ("steps"). When the
+// key tiles are few (B1 H8 N4096 d128: 256 tiles of 32 steps on 148 SMs, 1.73
+// waves) the last wave runs part empty. Cutting some tiles into two segments run
+// by two CTAs evens the waves; a split tile pays a partial-sum write and one sum.
+// The split is chosen by simulating the launch (CTAs start in grid order on the
+// first free SM: whole tiles, then the larger segments, then the smaller ones;
+// a CTA costs its steps plus one, a segment half a step more), for tiles of equal
+// step counts only (no causal or window bound, no block mask), and kept only when
+// the simulated time drops by more than 3%. Cached per shape.
+// The simulation leaves out what a segment costs beyond its steps (a second K/V load
+// and TMEM set-up, the fp32 partials written and read back), so two limits measured
+// on a B200 (d = 128, non-causal, backward time with and without the split) bound it:
+//   * only halves are tried: B1 H8 N4096 (108 tiles cut at 3/16) ran 3% slower;
+//   * tiles of fewer than kMinSplitSteps query tiles never split: 16 steps gained
+//     nothing (B1 H4 N2048 -3%, B1 H12 N2048 0%) and 8 steps lost (B1 H8 N1024 -20%),
+//     while 32 steps or more gained (B1 H2 N4096 +24%, B1 H16 N4096 +5%, B1 H3 N8192
+//     +19%, B1 H8 N8192 +8%).
+// Launches of more than kMaxSplitGrid key tiles (four waves of 148 SMs) never split,
+// and at most kMaxSplitTiles tiles split: the workspace makes room for that many.
+constexpr int kMaxSplitTiles = 160;
+constexpr long long kMaxSplitGrid = 4 * 148;
+constexpr int kMinSplitSteps = 32;
+
+struct BwdSplit {
+  int n_split, split_num;
+};
+
+double split_makespan(long long whole, int split, double whole_cost, double seg_a, double seg_b,
+                      int sms) {
+  std::priority_queue<double, std::vector<double>, std::greater<double>> free_at;
+  for (int i = 0; i < sms; ++i) free_at.push(0.0);
+  double end = 0.0;
+  auto run = [&](double cost) {
+    const double t = free_at.top() + cost;
+    free_at.pop();
+    free_at.push(t);
+    end = std::max(end, t);
+  };
+  for (long long i = 0; i < whole; ++i) run(whole_cost);
+  for (int i = 0; i < split; ++i) run(std::max(seg_a, seg_b));
+  for (int i = 0; i < split; ++i) run(std::min(seg_a, seg_b));
+  return end;
+}
+
+// Split tiles in the kernel's order need the larger segment first: segment 1 is the
+// larger when split_num < 8 (see bwd::Params).
+BwdSplit bwd_split(int BH, int N, bool uniform_tiles, int sms) {
+  BwdSplit none{0, 0};
+  const int n_kt = (N + 127) / 128;
+  const long long n_tiles = static_cast<long long>(BH) * n_kt;
+  if (!uniform_tiles || sms <= 0 || n_kt < kMinSplitSteps || n_tiles > 4ll * sms ||
+      n_tiles > kMaxSplitGrid)
+    return none;
+  static std::mutex mu;
+  static std::map<std::tuple<int, int, int>, BwdSplit> cache;  // at most 1024 shapes
+  const auto key = std::make_tuple(BH, N, sms);
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    auto it = cache.find(key);
+    if (it != cache.end()) return it->second;
+  }
+  const int steps = n_kt;
+  const double base = split_makespan(n_tiles, 0, steps + 1.0, 0, 0, sms);
+  BwdSplit best = none;
+  double best_t = base / 1.03;  // must beat the plain launch by more than 3%
+  const int max_split = static_cast<int>(std::min<long long>(n_tiles, kMaxSplitTiles));
+  const int ns_step = n_tiles < 64 ? 1 : 4;  // at most 64 simulated launches
+  for (int ns = ns_step; ns <= max_split; ns += ns_step)
+    for (int num : {8}) {
+      const int a = bwd::split_point(steps, num);
+      const double t = split_makespan(n_tiles - ns, ns, steps + 1.0, a + 1.5, steps - a + 1.5, sms);
+      if (t < best_t) {
+        best_t = t;
+        best = BwdSplit{ns, num};
+      }
+    }
+  std::lock_guard<std::mutex> lock(mu);
+  if (cache.size() >= 1024) cache.clear();
+  cache[key] = best;
+  return best;
+}
+
+// Split tiles whose partial sums the workspace makes room for: the most a shape can use.
+long long bwd_max_split(long long BH, int N) {
+  const long long n_kt = (static_cast<long long>(N) + 127) / 128;
+  if (n_kt < kMinSplitSteps || BH * n_kt > kMaxSplitGrid) return 0;
+  return std::min<long long>(BH * n_kt, kMaxSplitTiles);
+}
+
+// Workspace bytes: L2 [BH, Npad] | D [BH, Npad] | dQ accumulator [BH, N, d] (fp32) |
+// split-tile partials [S][2][2][128][d] (fp32) | arrival counters [S], for S split slots.
+size_t backward_ws_bytes(long long BH, int N, int d, long long S) {
+  const size_t bh = static_cast<size_t>(BH);
+  const size_t npad = (static_cast<size_t>(N) + 127) / 128 * 128;
+  const size_t s = static_cast<size_t>(S);
+  return 2 * round256(bh * npad * sizeof(float)) + round256(bh * N * d * sizeof(float)) +
+         round256(s * 4 * 128 * d * sizeof(float)) + round256(s * sizeof(unsigned));
+}
+
 int device_sms() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return 0;
@@ -451,11 +552,16 @@ struct BwdPlan {
   float* L2;
   float* Dv;
   float* dQacc;
+  float* part;         // partial dK/dV of split tiles
+  unsigned* arrivals;  // their arrival counters
+  int n_arrivals;
 };
 
+// split_ok = false: the workspace holds no split-tile slots (its size is the base
+// size, S = 0) and the main kernel splits no tile.
 fa_status bwd_plan(const void* const* ptrs, int nptrs, int B, int H, int N, int d,
                           float scale, int causal, void* workspace, size_t workspace_bytes,
-                          BwdPlan* plan) {
+                          BwdPlan* plan, bool split_ok = true) {
   fa_status st = check_shape(B, H, N, d, scale, causal);
   if (st != FA_OK) return st;
   plan->BH = B * H;
@@ -466,24 +572,32 @@ fa_status bwd_plan(const void* const* ptrs, int nptrs, int B, int H, int N, int 
   for (int i = 0; i < nptrs; ++i)
     if (ptrs[i] == nullptr || !aligned16(ptrs[i])) return FA_ERR_INVALID_ARG;
   if (workspace == nullptr || !aligned16(workspace)) return FA_ERR_INVALID_ARG;
-  if (workspace_bytes < fa_backward_workspace_size(B, H, N, d)) return FA_ERR_INVALID_ARG;
+  const long long smax = split_ok ? bwd_max_split(plan->BH, N) : 0;
+  if (workspace_bytes < backward_ws_bytes(plan->BH, N, d, smax)) return FA_ERR_INVALID_ARG;
   if ((st = prepare_device()) != FA_OK) return st;
-  // workspace: L2 [BH, Npad] | D [BH, Npad] | dQ accumulator [BH, N, d] (fp32)
+  // workspace layout: see backward_ws_bytes
   char* ws = static_cast<char*>(workspace);
   const size_t vec_bytes = round256(static_cast<size_t>(plan->BH) * plan->Npad * sizeof(float));
+  const size_t acc_bytes = round256(static_cast<size_t>(plan->BH) * N * d * sizeof(float));
+  const size_t part_bytes = round256(static_cast<size_t>(smax) * 4 * 128 * d * sizeof(float));
   plan->L2 = reinterpret_cast<float*>(ws);
   plan->Dv = reinterpret_cast<float*>(ws + vec_bytes);
   plan->dQacc = reinterpret_cast<float*>(ws + 2 * vec_bytes);
+  plan->part = reinterpret_cast<float*>(ws + 2 * vec_bytes + acc_bytes);
+  plan->arrivals = reinterpret_cast<unsigned*>(ws + 2 * vec_bytes + acc_bytes + part_bytes);
+  plan->n_arrivals = static_cast<int>(smax);
   return FA_OK;
 }
 
 template <Elt E>
 fa_status preprocess_impl(const void* O, const void* dO, const float* LSE, int B, int H,
                                  int N, int d, float scale, int causal, void* workspace,
-                                 size_t workspace_bytes, fa_stream_t stream) {
+                                 size_t workspace_bytes, fa_stream_t stream,
+                                 bool split_ok = true) {
   const void* ptrs[] = {O, dO, LSE};
   BwdPlan pl;
-  fa_status st = bwd_plan(ptrs, 3, B, H, N, d, scale, causal, workspace, workspace_bytes, &pl);
+  fa_status st = bwd_plan(ptrs, 3, B, H, N, d, scale, causal, workspace, workspace_bytes, &pl,
+                          split_ok);
   if (st != FA_OK || N == 0) return st;
   const long long rows = static_cast<long long>(pl.BH) * pl.Npad;
   const unsigned blocks = static_cast<unsigned>((rows + 7) / 8);
@@ -492,19 +606,20 @@ fa_status preprocess_impl(const void* O, const void* dO, const float* LSE, int B
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (d == 64)
     return launch(bwd::fa_bwd_pre_kernel<64, E>, blocks, 256, 0, s, O16, dO16, LSE, pl.L2, pl.Dv,
-                  pl.dQacc, N, pl.Npad, rows);
+                  pl.dQacc, N, pl.Npad, rows, pl.arrivals, pl.n_arrivals);
   return launch(bwd::fa_bwd_pre_kernel<128, E>, blocks, 256, 0, s, O16, dO16, LSE, pl.L2, pl.Dv,
-                pl.dQacc, N, pl.Npad, rows);
+                pl.dQacc, N, pl.Npad, rows, pl.arrivals, pl.n_arrivals);
 }
 
 template <Elt E>
 fa_status main_impl(const void* Q, const void* K, const void* V, const void* dO, void* dK,
                            void* dV, int B, int H, int N, int d, float scale, int causal,
                            const MaskSpec& mask, const DropSpec& drop, void* workspace,
-                           size_t workspace_bytes, fa_stream_t stream) {
+                           size_t workspace_bytes, fa_stream_t stream, bool split_ok = true) {
   const void* ptrs[] = {Q, K, V, dO, dK, dV};
   BwdPlan pl;
-  fa_status st = bwd_plan(ptrs, 6, B, H, N, d, scale, causal, workspace, workspace_bytes, &pl);
+  fa_status st = bwd_plan(ptrs, 6, B, H, N, d, scale, causal, workspace, workspace_bytes, &pl,
+                          split_ok);
   if (st != FA_OK || N == 0) return st;
   CUtensorMap mq, mk, mv, mdo;
   // Q and dO stream in half tiles of 64 rows; K and V are loaded as 128-row tiles
@@ -527,7 +642,16 @@ fa_status main_impl(const void* Q, const void* K, const void* V, const void* dO,
   p.blocks = mask.blocks;
   p.drop = drop.params;
   p.timeout_ns = watchdog_ns();
-  const dim3 grid(static_cast<unsigned>(pl.Npad / bwd::BN) * pl.BH);
+  const BwdSplit sp = pl.n_arrivals == 0 ? BwdSplit{0, 0}
+                                          : bwd_split(pl.BH, N,
+                                                      mask.wl < 0 && mask.wr < 0 &&
+                                                          mask.blocks == nullptr,
+                                                      device_sms());
+  p.n_split = std::min(sp.n_split, pl.n_arrivals);
+  p.split_num = sp.split_num;
+  p.part = pl.part;
+  p.arrivals = pl.arrivals;
+  const dim3 grid(static_cast<unsigned>(pl.Npad / bwd::BN) * pl.BH + p.n_split);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool g = mask.general();
   using bwd::Cfg;
@@ -550,10 +674,12 @@ fa_status main_impl(const void* Q, const void* K, const void* V, const void* dO,
 
 template <Elt E>
 fa_status dq_convert_impl(void* dQ, int B, int H, int N, int d, float scale, void* workspace,
-                                 size_t workspace_bytes, fa_stream_t stream) {
+                                 size_t workspace_bytes, fa_stream_t stream,
+                                 bool split_ok = true) {
   const void* ptrs[] = {dQ};
   BwdPlan pl;
-  fa_status st = bwd_plan(ptrs, 1, B, H, N, d, scale, 0, workspace, workspace_bytes, &pl);
+  fa_status st = bwd_plan(ptrs, 1, B, H, N, d, scale, 0, workspace, workspace_bytes, &pl,
+                          split_ok);
   if (st != FA_OK || N == 0) return st;
   const long long n4 = static_cast<long long>(pl.BH) * N * d / 4;
   const unsigned blocks = static_cast<unsigned>(std::min<long long>((n4 + 255) / 256, 148 * 16));
@@ -567,17 +693,20 @@ template <Elt E>
 fa_status backward_impl(const void* Q, const void* K, const void* V, const void* O, const void* dO,
                       const float* LSE, void* dQ, void* dK, void* dV, int B, int H, int N, int d,
                       float scale, int causal, const MaskSpec& mask, const DropSpec& drop,
-                      void* workspace, size_t workspace_bytes, fa_stream_t stream) {
+                      void* workspace, size_t workspace_bytes, fa_stream_t stream,
+                      bool split_ok = true) {
   const void* ptrs[] = {Q, K, V, O, dO, LSE, dQ, dK, dV};
   BwdPlan pl;
-  fa_status st = bwd_plan(ptrs, 9, B, H, N, d, scale, causal, workspace, workspace_bytes, &pl);
+  fa_status st = bwd_plan(ptrs, 9, B, H, N, d, scale, causal, workspace, workspace_bytes, &pl,
+                          split_ok);
   if (st != FA_OK || N == 0) return st;
-  st = preprocess_impl<E>(O, dO, LSE, B, H, N, d, scale, causal, workspace, workspace_bytes, stream);
+  st = preprocess_impl<E>(O, dO, LSE, B, H, N, d, scale, causal, workspace, workspace_bytes, stream,
+                          split_ok);
   if (st != FA_OK) return st;
   st = main_impl<E>(Q, K, V, dO, dK, dV, B, H, N, d, scale, causal, mask, drop, workspace,
-                    workspace_bytes, stream);
+                    workspace_bytes, stream, split_ok);
   if (st != FA_OK) return st;
-  return dq_convert_impl<E>(dQ, B, H, N, d, scale, workspace, workspace_bytes, stream);
+  return dq_convert_impl<E>(dQ, B, H, N, d, scale, workspace, workspace_bytes, stream, split_ok);
 }
 
 }  // namespace
@@ -599,9 +728,8 @@ const char* fa_status_string(fa_status s) {
 
 size_t fa_backward_workspace_size(int B, int H, int N, int d) {
   if (B < 1 || H < 1 || N < 1 || (d != 64 && d != 128)) return 0;
-  const size_t bh = static_cast<size_t>(B) * H;
-  const size_t npad = (static_cast<size_t>(N) + 127) / 128 * 128;
-  return 2 * round256(bh * npad * sizeof(float)) + round256(bh * N * d * sizeof(float));
+  const long long bh = static_cast<long long>(B) * H;
+  return backward_ws_bytes(bh, N, d, bwd_max_split(bh, N));
 }
 
 float fa_dropout_rate(float p_drop) {
@@ -741,7 +869,9 @@ fa_status fa_backward_noalloc(const void* Q, const void* K, const void* V, const
   fa_status st = check_shape(B, H, N, d, scale, causal);
   if (st != FA_OK) return st;
   if (N == 0) return FA_OK;
-  if (fa_backward_workspace_size(B, H, N, d) > kNoAllocScratchBytes) return FA_ERR_UNSUPPORTED;
+  // Without split-tile slots: the array holds L2, D and the dQ accumulator only.
+  if (backward_ws_bytes(static_cast<long long>(B) * H, N, d, 0) > kNoAllocScratchBytes)
+    return FA_ERR_UNSUPPORTED;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FA_ERR_CUDA;
   void* scratch = nullptr;
@@ -761,8 +891,11 @@ fa_status fa_backward_noalloc(const void* Q, const void* K, const void* V, const
   // The preprocess stage rewrites every byte of scratch the later stages read
   // (LSE*log2e, D, and the dQ accumulator it zeroes), so whatever an earlier call
   // left in the array does not matter.
-  return fa_backward(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, scale, causal, scratch,
-                     kNoAllocScratchBytes, stream);
+  MaskSpec m;
+  make_mask(N, causal, -1, -1, nullptr, &m);
+  return backward_impl<Elt::BF16>(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, scale, causal, m,
+                                  DropSpec{}, scratch, kNoAllocScratchBytes, stream,
+                                  /*split_ok=*/false);
 }
 
 fa_status fa_forward_dropout(const void* Q, const void* K, const void* V, void* O, float* LSE,

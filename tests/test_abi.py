@@ -47,9 +47,18 @@ def test_host_only_entry_points(libfa):
     assert libfa.fa_status_string(4) == b"kernel watchdog timeout"
     f = libfa.fa_backward_workspace_size
     f.restype = ctypes.c_size_t
-    # L2 and D padded to 128 rows, plus the fp32 dQ accumulator
+    # L2 and D padded to 128 rows and the fp32 dQ accumulator, each region rounded up
+    # to 256 bytes; launches of at most 592 key tiles with N padded to 4096 or more add
+    # room for the fp32 dK/dV partials (2 segments x 128 rows x d, twice) and arrival
+    # counters of min(key tiles, 160) split key tiles. 1024 key tiles, or short rows,
+    # get no split slots:
     assert f(1, 8, 16384, 128) == 2 * (8 * 16384 * 4) + 8 * 16384 * 128 * 4
     assert f(1, 1, 100, 64) == 2 * 512 + 25600
+    assert f(1, 2, 1000, 64) == 2 * 8192 + 512000
+    # 512 key tiles: 160 slots; 32 key tiles (N = 4000 pads to 4096): 32 slots
+    assert f(1, 8, 8192, 128) == (2 * (8 * 8192 * 4) + 8 * 8192 * 128 * 4
+                                  + 160 * 4 * 128 * 128 * 4 + 768)
+    assert f(1, 1, 4000, 64) == 2 * 16384 + 4000 * 64 * 4 + 32 * 4 * 128 * 64 * 4 + 256
     assert f(1, 1, 100, 96) == 0
     assert f(0, 1, 100, 64) == 0
 

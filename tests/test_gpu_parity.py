@@ -161,6 +161,21 @@ def test_bf16_small_full_parity(B, H, N, d, causal):
     check_full(q, k, v, do, 1.0 / math.sqrt(d), causal, TOL_BF16)
 
 
+# Non-causal launches of few key tiles with 32 or more query tiles each run some or
+# all of them as two CTAs, one per half of the query tiles, whose fp32 dK/dV partials
+# are summed by the second to end.
+SPLIT = [
+    (1, 1, 4000, 128, False),   # 32 key tiles, all split; ragged tail
+    (1, 5, 4000, 64, False),    # 160 key tiles, the last 12 split
+]
+
+
+@pytest.mark.parametrize("B,H,N,d,causal", SPLIT)
+def test_split_key_tiles_full_parity(B, H, N, d, causal):
+    q, k, v, do = make_inputs(B, H, N, d, torch.bfloat16, seed=41 + N + d)
+    check_full(q, k, v, do, 1.0 / math.sqrt(d), causal, TOL_BF16)
+
+
 @pytest.mark.parametrize("B,H,N,d,causal", [(1, 1, 256, 64, False), (1, 2, 200, 128, True),
                                             (2, 1, 1, 64, True), (1, 1, 100, 64, False)])
 def test_f32_small_full_parity(B, H, N, d, causal):
@@ -366,6 +381,17 @@ def test_dk_dv_deterministic():
     b = run_backward(q, k, v, o, lse, do, 0.088, True)
     assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
     assert torch.allclose(a[0].float(), b[0].float(), atol=1e-2)
+
+
+def test_split_key_tiles_are_deterministic():
+    """B1 H8 N8192 d128 (512 key tiles on 148 SMs) runs 68 key tiles as two CTAs each,
+    whose fp32 dK/dV partials are added in a fixed order: dK and dV are the same bits
+    every run."""
+    q, k, v, do = _dev(*make_inputs(1, 8, 8192, 128, torch.bfloat16, seed=13))
+    o, lse = run_forward(q, k, v, 0.088, False)
+    a = run_backward(q, k, v, o, lse, do, 0.088, False)
+    b = run_backward(q, k, v, o, lse, do, 0.088, False)
+    assert torch.equal(a[1], b[1]) and torch.equal(a[2], b[2])
 
 
 def test_argument_errors_launch_nothing():
