@@ -17,8 +17,9 @@
 // the CTA walks only the key tiles that some of its query rows can see.
 //
 // B200 mapping (one CTA per SM, 352 threads):
-//   * CTA = 2 query tiles of 128 rows (256 rows) of one (batch, head); the two tiles
-//     share every K/V tile that is loaded.
+//   * CTA = 2 query tiles of 128 rows (256 rows) of one (batch, head), or one; the two
+//     tiles share every K/V tile that is loaded. (fa_fwd_persistent_kernel, at the
+//     end of this file, walks a list of such items per CTA.)
 //   * warp 8: TMA producer for the Q tiles (once) and the K tiles (128 rows) through
 //     a ring of kKSlots shared-memory slots; warp 10: TMA producer for the V tiles
 //     (ring of kVSlots). Separate rings let K run further ahead of the MMAs than V.
@@ -84,7 +85,9 @@ struct Cfg {
   static constexpr int kBarSFree = kBarSFull + 2;                 // [2] S_t(j) read out
   static constexpr int kBarPFull = kBarSFree + 2;                 // [2] P_t(j) written
   static constexpr int kBarPVDone = kBarPFull + 2;                // [2] PV_t(j) complete
-  static constexpr int kBarDrain = kBarPVDone + 2;
+  static constexpr int kBarQEmpty = kBarPVDone + 2;               // [2] item's S_t done with Q_t
+  static constexpr int kBarOFree = kBarQEmpty + 2;                // [2] item's O_t read out
+  static constexpr int kBarDrain = kBarOFree + 2;
   static constexpr int kNumBars = kBarDrain + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;  // tmem base, abort flag
   static constexpr int kMaskOff = kMiscOff + 16;            // block-mask bits of both tiles
@@ -101,13 +104,19 @@ struct Params {
   float* LSE;
   int N;
   int BH;
-  // Work split: per head, pairs_ph CTAs own two consecutive query tiles each (tiles
-  // [singles_ph, n_qt)) and singles_ph CTAs own one (tiles [0, singles_ph)). All pair
-  // CTAs (n_pair_ctas = BH * pairs_ph) come first in the grid, so the single-tile
-  // CTAs (half the work) fill the last, partial wave.
+  // Work split: per head, pairs_ph items own two consecutive query tiles each (tiles
+  // [singles_ph, n_qt)) and singles_ph items own one (tiles [0, singles_ph)). All pair
+  // items (n_pair_items = BH * pairs_ph) come first in the list, heaviest first within
+  // a head, so the single-tile items (half the work) come last and even out the CTAs'
+  // loads. weight_major = 0: the list is head-major (a head's items are consecutive,
+  // so the CTAs busy at one time share one or two heads' K/V in L2); 1: rank-major
+  // (every head's heaviest item, then every head's second, ...), for causal or
+  // windowed launches whose K/V all fit in L2.
   int pairs_ph;
   int singles_ph;
-  int n_pair_ctas;
+  int n_pair_items;
+  int n_items;
+  int weight_major;
   float scale_log2;  // scale * log2(e)
   int wl;            // keys j >= i - wl are kept; < 0: no left bound
   int wr;            // keys j <= i + wr are kept; < 0: no right bound (causal: 0)
@@ -160,6 +169,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const Params p) {
   using C = Cfg<D>;
+  if (threadIdx.x == 0) FA_TRACE_CTA(0);
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -182,13 +192,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   // go first. Single-tile CTAs, on the lightest tiles, come after all pairs.
   int bh, qt0;
   bool own1;  // does this CTA own query tile 1 (qt0 + 1)?
-  if (static_cast<int>(blockIdx.x) < p.n_pair_ctas) {
+  if (static_cast<int>(blockIdx.x) < p.n_pair_items) {
     const int c = static_cast<int>(blockIdx.x);
     bh = c / p.pairs_ph;
     qt0 = p.singles_ph + 2 * (p.pairs_ph - 1 - c % p.pairs_ph);
     own1 = true;
   } else {
-    const int c = static_cast<int>(blockIdx.x) - p.n_pair_ctas;
+    const int c = static_cast<int>(blockIdx.x) - p.n_pair_items;
     bh = c / p.singles_ph;
     qt0 = p.singles_ph - 1 - c % p.singles_ph;
     own1 = false;
@@ -252,6 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Watchdog wd{abort_flag, p.timeout_ns};
+  if (threadIdx.x == 0) FA_TRACE_CTA(1);
 
   // Does query tile t see any key of key tile kt?
   auto member = [&](int kt, int t) -> bool {
@@ -434,6 +445,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (wq == 0) FA_TRACE_POINT(50, j, t);
       ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarSFull + t), j & 1, wd));
       if (wq == 0) FA_TRACE_POINT(51, j, t);
+      if (j == 0 && t == 0 && threadIdx.x == 0) FA_TRACE_CTA(2);
       if (!ok) break;
       tc_fence_after();
       uint32_t s[4][32];
@@ -583,6 +595,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       p.LSE[static_cast<size_t>(bh) * p.N + row] = -INFINITY;
     }
     if (ok && t_nk > 0) {
+      if (t == 0 && threadIdx.x == 0) FA_TRACE_CTA(3);
       tc_fence_after();
       const float norm = kDropout ? l : lr;
       const float inv_l = (norm > 0.0f) ? 1.0f / norm : 0.0f;
@@ -611,6 +624,537 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) FA_TRACE_CTA(4);
+  if (warp == kWarpMma) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmCols);
+  }
+}
+
+// The persistent form of the kernel above, for launches of many short items (few key
+// tiles each): min(items, SMs) CTAs, each walking a list of items and reusing its
+// buffers from one to the next (Q once the item's last S product has read it, O in
+// TMEM once the epilogue has read it out), so one item's epilogue overlaps the next
+// item's first loads and products. The same roles, barriers and arithmetic; no block
+// mask (its CTA would build the mask rows of every item it walks).
+template <int D, Elt E, bool kMasked, bool kDropout>
+__global__ void __launch_bounds__(kThreads, 1)
+    fa_fwd_persistent_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const Params p) {
+  using C = Cfg<D>;
+  if (threadIdx.x == 0) FA_TRACE_CTA(0);
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* base_ptr = smem_raw + (base - raw);
+  const uint32_t bars = base + C::kBarOff;
+  auto bar = [&](int i) -> uint32_t { return bars + 8u * static_cast<uint32_t>(i); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + C::kMiscOff + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  // Without a window's left bound (kMasked = false) it is a compile-time constant, so
+  // the general tile walk folds to the plain / causal one. Block masks never come here.
+  const int wl = kMasked ? p.wl : -1;
+  const int wr = p.wr;
+  const int n_kt = p.n_kt;
+
+  // Work items: item i < n_pair_items owns two consecutive query tiles, the others
+  // one. Every role of the CTA walks the same items, the k-th being k * G + b for even
+  // k and k * G + (G - 1 - b) for odd k (b = blockIdx.x, G = gridDim.x), so the heavy
+  // items at the front of the list are dealt out back and forth over the CTAs and one
+  // item's epilogue overlaps the next one's first loads and products.
+  auto item_of = [&](int k) -> int {
+    const int G = static_cast<int>(gridDim.x), b = static_cast<int>(blockIdx.x);
+    const int i = k * G + ((k & 1) ? (G - 1 - b) : b);
+    return i < p.n_items ? i : -1;
+  };
+  // An item's (batch, head), first query tile, whether it owns the second tile, the
+  // key tiles [lo[t], hi[t]) each tile's rows may see and how many of them a tile
+  // walks (nk), and the union [kt_lo, kt_hi) the CTA walks for it.
+  struct Work {
+    int bh, qt0, q0;
+    bool own1;
+    int lo[2], hi[2], nk[2];
+    int kt_lo, kt_hi;
+  };
+  auto member_w = [&](const Work& w, int kt, int t) -> bool {
+    return kt >= (t ? w.lo[1] : w.lo[0]) && kt < (t ? w.hi[1] : w.hi[0]);
+  };
+  auto decode = [&](int i, Work& w) {
+    int r;
+    if (i < p.n_pair_items) {
+      if (p.weight_major) { r = i / p.BH; w.bh = i % p.BH; }
+      else { w.bh = i / p.pairs_ph; r = i % p.pairs_ph; }
+      w.qt0 = p.singles_ph + 2 * (p.pairs_ph - 1 - r);
+      w.own1 = true;
+    } else {
+      const int c = i - p.n_pair_items;
+      if (p.weight_major) { r = c / p.BH; w.bh = c % p.BH; }
+      else { w.bh = c / p.singles_ph; r = c % p.singles_ph; }
+      w.qt0 = p.singles_ph - 1 - r;
+      w.own1 = false;
+    }
+    w.q0 = w.qt0 * BM;
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const int r0 = w.q0 + t * BM, r1 = min(r0 + BM, p.N) - 1;
+      w.lo[t] = (wl < 0) ? 0 : max(0, r0 - wl) / BN;
+      w.hi[t] = (wr < 0) ? n_kt : min(n_kt, (r1 + wr) / BN + 1);
+      if (r0 >= p.N || (t == 1 && !w.own1)) w.lo[t] = w.hi[t] = 0;
+    }
+    // the union of both ranges (contiguous: lo[1] <= hi[0])
+    w.kt_lo = (w.hi[0] > w.lo[0]) ? w.lo[0] : w.lo[1];
+    w.kt_hi = max(w.hi[0], w.hi[1]);
+#pragma unroll
+    for (int t = 0; t < 2; ++t) w.nk[t] = w.hi[t] - w.lo[t];
+  };
+
+  if (threadIdx.x == 0) {
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(bar(C::kBarQFull + t), 1);
+      mbar_init(bar(C::kBarQEmpty + t), 1);
+      mbar_init(bar(C::kBarSFull + t), 1);
+      mbar_init(bar(C::kBarSFree + t), 4);  // one arrival per softmax warp
+      mbar_init(bar(C::kBarPFull + t), 4);
+      mbar_init(bar(C::kBarPVDone + t), 1);
+      mbar_init(bar(C::kBarOFree + t), 4);
+    }
+    for (int s = 0; s < C::kKSlots; ++s) {
+      mbar_init(bar(C::kBarKFull + s), 1);
+      mbar_init(bar(C::kBarKEmpty + s), 1);
+    }
+    for (int s = 0; s < C::kVSlots; ++s) {
+      mbar_init(bar(C::kBarVFull + s), 1);
+      mbar_init(bar(C::kBarVEmpty + s), 1);
+    }
+    mbar_init(bar(C::kBarDrain), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(smem_u32(tmem_slot), C::kTmCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Watchdog wd{abort_flag, p.timeout_ns};
+  if (threadIdx.x == 0) FA_TRACE_CTA(1);
+
+  auto k_smem = [&](int g) -> uint32_t {
+    return base + C::kKOff + (g % C::kKSlots) * C::kTileBytes;
+  };
+  auto v_smem = [&](int g) -> uint32_t {
+    return base + C::kVOff + (g % C::kVSlots) * C::kTileBytes;
+  };
+  // first key tile >= kt that either query tile of the item sees (kt_hi if none)
+  auto next_kt = [&](const Work& w, int kt) -> int {
+    while (kt < w.kt_hi && !(member_w(w, kt, 0) || member_w(w, kt, 1))) ++kt;
+    return kt;
+  };
+
+  if (warp == kWarpTmaK || warp == kWarpTmaV) {
+    // ------------------------------------------------------------ producers
+    // (the whole warp runs the loop; one elected lane issues each copy)
+    // Warp 8 streams the K tiles of every item through its ring; warp 10 loads each
+    // item's Q tiles (once the previous item's S products have read them: QEmpty)
+    // and streams the V tiles. Ring indices run on across items.
+    const bool is_k = (warp == kWarpTmaK);
+    const CUtensorMap* map = is_k ? &tmK : &tmV;
+    const int nslots = is_k ? C::kKSlots : C::kVSlots;
+    const int bfull = is_k ? C::kBarKFull : C::kBarVFull;
+    const int bempty = is_k ? C::kBarKEmpty : C::kBarVEmpty;
+    if (lane == 0) tma_prefetch_desc(map);
+    if (!is_k && lane == 0) tma_prefetch_desc(&tmQ);
+    int issued = 0;       // ring index: tiles issued so far, over all items
+    int nq[2] = {0, 0};   // Q tile loads so far (their barrier phases)
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int item = item_of(k);
+      if (item < 0) break;
+      Work w;
+      decode(item, w);
+      if (!is_k) {
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+          if ((t ? w.nk[1] : w.nk[0]) == 0) continue;
+          const int n = t ? nq[1] : nq[0];
+          if (n > 0 && !mbar_wait_warp(bar(C::kBarQEmpty + t), (n - 1) & 1, wd)) { ok = false; break; }
+          const uint32_t dst = base + C::kQOff + t * C::kTileBytes;
+          mbar_arrive_expect_tx_e(bar(C::kBarQFull + t), C::kTileBytes);
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_load_3d_e(dst + c * C::kChunkBytes, &tmQ, bar(C::kBarQFull + t), c * 64,
+                          w.q0 + t * BM, w.bh);
+          if (t) ++nq[1]; else ++nq[0];
+        }
+        if (!ok) break;
+      }
+      for (int kt = next_kt(w, w.kt_lo); kt < w.kt_hi; kt = next_kt(w, kt + 1)) {
+        const int g = issued;
+        const int slot = g % nslots, rnd = g / nslots;
+        FA_TRACE_POINT(40, g, is_k ? 0 : 1);
+        if (rnd > 0 && !mbar_wait_warp(bar(bempty + slot), (rnd - 1) & 1, wd)) { ok = false; break; }
+        FA_TRACE_POINT(41, g, is_k ? 0 : 1);
+        const uint32_t dst = is_k ? k_smem(g) : v_smem(g);
+        mbar_arrive_expect_tx_e(bar(bfull + slot), C::kTileBytes);
+        for (int c = 0; c < C::kChunks; ++c)
+          tma_load_3d_e(dst + c * C::kChunkBytes, map, bar(bfull + slot), c * 64, kt * BN, w.bh);
+        issued = g + 1;
+      }
+    }
+    // Every issued copy must land before the CTA may exit.
+    for (int g = max(0, issued - nslots); g < issued; ++g)
+      drain_wait(bar(bfull + g % nslots), (g / nslots) & 1, p.timeout_ns);
+    // (warp 10 made every Q load: the last one's phase covers the earlier ones)
+#pragma unroll
+    for (int t = 0; t < 2; ++t) {
+      const int n = t ? nq[1] : nq[0];
+      if (n > 0) drain_wait(bar(C::kBarQFull + t), (n - 1) & 1, p.timeout_ns);
+    }
+    __syncwarp();
+  } else if (warp == kWarpMma) {
+    // ------------------------------------------------------------ MMA issuer
+    // (the whole warp runs the loop; one elected lane issues each MMA and commit)
+    FA_TRACE_POINT(0, 0, 0);
+    const uint32_t q_smem0 = base + C::kQOff, q_smem1 = base + C::kQOff + C::kTileBytes;
+    const uint32_t p_smem0 = base + C::kPOff, p_smem1 = base + C::kPOff + C::kPBytes;
+    auto wait_k = [&](int j) {
+      return mbar_wait_warp(bar(C::kBarKFull + j % C::kKSlots), (j / C::kKSlots) & 1, wd);
+    };
+    auto wait_v = [&](int j) {
+      return mbar_wait_warp(bar(C::kBarVFull + j % C::kVSlots), (j / C::kVSlots) & 1, wd);
+    };
+    // Counts over all items so far (their barrier phases): ns[t] / npv[t]: S_t and PV_t
+    // products issued; nq[t]: Q_t tiles consumed; no[t]: items whose O_t the softmax has
+    // read out. ns0 / npv0: ns / npv at the start of the current item.
+    int ns[2] = {0, 0}, npv[2] = {0, 0}, nq[2] = {0, 0}, no[2] = {0, 0};
+    int ns0[2] = {0, 0}, npv0[2] = {0, 0};
+    Work w;
+    auto member = [&](int kt, int t) -> bool { return member_w(w, kt, t); };
+    // S_t for the key tile at ring index j, for each query tile that sees it, each
+    // as soon as the softmax of that tile has read its previous S out of TMEM
+    auto issue_s_all = [&](int kt, int j) -> bool {
+      bool have_k = false;
+      for (int t = 0; t < 2; ++t) {
+        if (!member(kt, t)) continue;
+        FA_TRACE_POINT(42, ns[t], t);
+        if (ns[t] > 0 && !mbar_wait_warp(bar(C::kBarSFree + t), (ns[t] - 1) & 1, wd))
+          return false;
+        FA_TRACE_POINT(43, ns[t], t);
+        if (!have_k) {
+          if (!wait_k(j)) return false;
+          FA_TRACE_POINT(44, j, 0);
+          have_k = true;
+        }
+        tc_fence_after();
+        issue_s<D, E>(tmem + C::kTmS0 + t * 128, t ? q_smem1 : q_smem0, k_smem(j));
+        tc_commit_e(bar(C::kBarSFull + t));
+        FA_TRACE_POINT(45, ns[t], t);
+        ++ns[t];
+        // after the item's last S_t its Q_t buffer may be refilled
+        if (ns[t] - ns0[t] == w.nk[t]) tc_commit_e(bar(C::kBarQEmpty + t));
+      }
+      tc_commit_e(bar(C::kBarKEmpty + j % C::kKSlots));
+      return true;
+    };
+    bool ok = true;
+    int j = 0;  // ring index of the current key tile, over all items
+    for (int k = 0; ok; ++k) {
+      const int item = item_of(k);
+      if (item < 0) break;
+      decode(item, w);
+      for (int t = 0; t < 2 && ok; ++t)
+        if (w.nk[t] > 0) ok = mbar_wait_warp(bar(C::kBarQFull + t), nq[t]++ & 1, wd);
+      if (!ok) break;
+      FA_TRACE_POINT(58, k, 0);
+      ns0[0] = ns[0];
+      ns0[1] = ns[1];
+      npv0[0] = npv[0];
+      npv0[1] = npv[1];
+      int cur = next_kt(w, w.kt_lo);
+      if (cur < w.kt_hi) ok = issue_s_all(cur, j);
+      for (; cur < w.kt_hi && ok; ++j) {
+        // S for the next key tile before PV of this one
+        const int nxt = next_kt(w, cur + 1);
+        if (nxt < w.kt_hi && !issue_s_all(nxt, j + 1)) { ok = false; break; }
+        // O_t += P_t V_cur
+        bool have_v = false;
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (!member(cur, t)) continue;
+          // the item's first PV_t overwrites O_t: the previous item's O_t must be out
+          if (npv[t] == npv0[t] && no[t] > 0 &&
+              !mbar_wait_warp(bar(C::kBarOFree + t), (no[t] - 1) & 1, wd)) {
+            ok = false;
+            break;
+          }
+          FA_TRACE_POINT(46, npv[t], t);
+          if (!mbar_wait_warp(bar(C::kBarPFull + t), npv[t] & 1, wd)) { ok = false; break; }
+          FA_TRACE_POINT(47, npv[t], t);
+          if (!have_v) {
+            if (!wait_v(j)) { ok = false; break; }
+            FA_TRACE_POINT(48, j, 0);
+            have_v = true;
+          }
+          tc_fence_after();
+          issue_pv<D, E>(tmem + C::kTmO0 + t * D, t ? p_smem1 : p_smem0, v_smem(j),
+                         npv[t] > npv0[t]);
+          tc_commit_e(bar(C::kBarPVDone + t));
+          FA_TRACE_POINT(49, npv[t], t);
+          ++npv[t];
+        }
+        if (!ok) break;
+        tc_commit_e(bar(C::kBarVEmpty + j % C::kVSlots));
+        cur = nxt;
+      }
+      for (int t = 0; t < 2; ++t)
+        if (w.nk[t] > 0) ++no[t];
+    }
+    // No MMA may be in flight when TMEM is released.
+    tc_commit_e(bar(C::kBarDrain));
+    drain_wait(bar(C::kBarDrain), 0, p.timeout_ns);
+    __syncwarp();
+    FA_TRACE_POINT(99, 0, 0);
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int t = warp >> 2;
+    const int wq = warp & 3;
+    const int row_in_tile = wq * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const uint32_t tm_s = tmem + lane_off + C::kTmS0 + t * 128;
+    const uint32_t tm_o = tmem + lane_off + C::kTmO0 + t * D;
+    uint8_t* p_row = base_ptr + C::kPOff + t * C::kPBytes + row_in_tile * 128;
+    const float c = p.scale_log2;
+    // S_t and PV_t products of the items before this one (their barrier phases)
+    int n_prev = 0;
+    bool ok = true;
+    for (int ki = 0; ok; ++ki) {
+      const int item = item_of(ki);
+      if (item < 0) break;
+      Work w;
+      decode(item, w);
+      const int bh = w.bh;
+      const int r0 = w.q0 + t * BM;
+      const int row = r0 + row_in_tile;
+      float m_ref = -INFINITY;
+      float l = 0.0f;
+      // lr: the same sum over P as rounded for the PV product. O is divided by lr, so
+      // the weights it applies to V sum to exactly 1: the rounding of the largest
+      // p (up to 2^8 under the lagging reference max, so up to 2^-8 relative) then
+      // cancels instead of showing in O. LSE keeps the unrounded l. With dropout the
+      // rounded values carry the keep mask, so there O is divided by l.
+      float lr = 0.0f;
+      // this tile's range and count as scalars (no per-thread array indexing)
+      const int t_lo = t ? w.lo[1] : w.lo[0], t_hi = t ? w.hi[1] : w.hi[0];
+      const int t_nk = t ? w.nk[1] : w.nk[0];
+      auto t_member = [&](int kt) -> bool { return kt >= t_lo && kt < t_hi; };
+      // visible keys of this row: [k_lo, k_hi)
+      const int k_lo = (wl < 0) ? 0 : row - wl;
+      const int k_hi = (wr < 0) ? p.N : min(p.N, row + wr + 1);
+      const int r1 = r0 + BM - 1;
+      int kt = t_lo - 1;
+      for (int j = 0; j < t_nk && ok; ++j) {
+        do ++kt; while (!t_member(kt));
+        const int n = n_prev + j;
+        if (wq == 0) FA_TRACE_POINT(50, n, t);
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarSFull + t), n & 1, wd));
+        if (wq == 0) FA_TRACE_POINT(51, n, t);
+        if (ki == 0 && j == 0 && t == 0 && threadIdx.x == 0) FA_TRACE_CTA(2);
+        if (j == 0 && wq == 0) FA_TRACE_POINT(57, ki, t);
+        if (!ok) break;
+        tc_fence_after();
+        uint32_t s[4][32];
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) tmem_ld32(tm_s + cc * 32, s[cc]);
+        tmem_wait_ld();
+        // S_t is in registers: the MMA may overwrite it with the next S_t now
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(C::kBarSFree + t));
+        if (wq == 0) FA_TRACE_POINT(52, n, t);
+        const int kv0 = kt * BN;
+        // masking only where the tile crosses an edge of some row's visible range
+        const bool need_mask = (kv0 + BN > p.N) || (wr >= 0 && kv0 + BN - 1 > r0 + wr) ||
+                               (wl >= 0 && kv0 < r1 - wl);
+        if (need_mask) {
+          // key kv0 + k is visible iff 0 <= kv0 + k - k_lo < k_hi - k_lo
+          const int off = kv0 - k_lo;
+          const unsigned span = static_cast<unsigned>(max(k_hi - k_lo, 0));
+#pragma unroll
+          for (int k2 = 0; k2 < 128; ++k2)
+            if (static_cast<unsigned>(off + k2) >= span)
+              s[k2 / 32][k2 % 32] = __float_as_uint(-INFINITY);
+        }
+        // row max: per 32-column chunk a tree of three-input maxima (short dependency
+        // chains, few live temporaries), then across the four chunks
+        float cm[4];
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          float t1[11];
+#pragma unroll
+          for (int q = 0; q < 10; ++q)
+            t1[q] = fmax3(__uint_as_float(s[cc][3 * q]), __uint_as_float(s[cc][3 * q + 1]),
+                          __uint_as_float(s[cc][3 * q + 2]));
+          t1[10] = fmaxf(__uint_as_float(s[cc][30]), __uint_as_float(s[cc][31]));
+          const float a = fmax3(t1[0], t1[1], t1[2]), b = fmax3(t1[3], t1[4], t1[5]);
+          const float d2 = fmax3(t1[6], t1[7], t1[8]), e = fmaxf(t1[9], t1[10]);
+          cm[cc] = fmax3(a, b, fmaxf(d2, e));
+        }
+        const float mx = fmaxf(fmaxf(cm[0], cm[1]), fmaxf(cm[2], cm[3]));
+        const float m_new = fmaxf(m_ref, mx * c);
+        const bool need = m_new > m_ref + kRescaleThreshold;
+        // The reference max moves for the whole warp when any row needs it (TMEM
+        // accesses are warp-wide); O is rescaled below, after the scores are dead.
+        const bool move = __any_sync(0xffffffffu, need);
+        float alpha = 1.0f;
+        if (move) {
+          alpha = (m_ref == -INFINITY) ? 0.0f : ex2_approx(m_ref - m_new);
+          m_ref = m_new;
+          l *= alpha;
+          lr *= alpha;
+        }
+        // PV_t(j-1) must be complete before P_t is overwritten and O_t rescaled.
+        if (j > 0) {
+          if (wq == 0) FA_TRACE_POINT(53, n, t);
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarPVDone + t), (n - 1) & 1, wd));
+          if (wq == 0) FA_TRACE_POINT(54, n, t);
+          if (!ok) break;
+          tc_fence_after();
+        }
+        const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
+        const float2 c2 = make_float2(c, c), nm2 = make_float2(-m_use, -m_use);
+        float2 accr[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                         make_float2(0.f, 0.f)};
+        // dropout: this row's four words for the current 16 keys (byte b of word m is key
+        // 4m + b of the group)
+        [[maybe_unused]] uint32_t zw[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+        for (int cc = 0; cc < 4; ++cc) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            const float2 x = ffma2(make_float2(__uint_as_float(s[cc][2 * k]),
+                                               __uint_as_float(s[cc][2 * k + 1])), c2, nm2);
+            float2 pe;
+            constexpr int kPoly = C::kPolyPeriod;
+            if (kPoly > 0 && k % (kPoly > 0 ? kPoly : 1) == kPoly - 1) {
+              pe = exp2_poly2(x);  // a share of the exponentials on the FMA pipe
+            } else {
+              pe = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+            }
+            acc[k & 3] = fadd2(acc[k & 3], pe);  // l is the sum before dropout
+            if constexpr (kDropout) {
+              // One block covers 4 rows x 4 keys; the lanes of rows 4g..4g+3 share its
+              // counter. Every 16 keys, lane u (row mod 4) draws the block of keys
+              // 4u..4u+3 of the 16, and a 4 x 4 transpose across the four lanes hands
+              // each lane its own row's word of all four blocks.
+              if ((k & 7) == 0) {
+                const int u = lane & 3;
+                const uint4 w = philox4x32_10(
+                    make_uint4(static_cast<uint32_t>(((kv0 + 32 * cc + 2 * k) >> 2) + u),
+                               static_cast<uint32_t>(row >> 2), static_cast<uint32_t>(bh),
+                               p.drop.offset),
+                    p.drop.seed_lo, p.drop.seed_hi);
+                zw[0] = w.x;
+                zw[1] = w.y;
+                zw[2] = w.z;
+                zw[3] = w.w;
+                transpose4_lanes(zw, u);
+              }
+              // keys 2k, 2k + 1 of the chunk = keys 2(k mod 8), +1 of the group: word
+              // (k mod 8) / 2, bytes 2(k mod 2) and 2(k mod 2) + 1
+              const uint32_t wd = zw[(k & 7) >> 1] >> (16 * (k & 1));
+              pe.x = ((wd & 0xffu) >= p.drop.threshold) ? pe.x * p.drop.scale : 0.0f;
+              pe.y = (((wd >> 8) & 0xffu) >= p.drop.threshold) ? pe.y * p.drop.scale : 0.0f;
+            }
+            pk[k] = pack2<E>(pe.x, pe.y);
+            if constexpr (!kDropout) accr[k & 1] = fadd2(accr[k & 1], unpack2<E>(pk[k]));
+          }
+          // keys 32cc..32cc+31 = 16-byte units 4cc..4cc+3 of this row's 256 bytes:
+          // chunk (cc / 2), units (cc % 2) * 4 + u, 128-byte swizzle by the row
+          uint8_t* chunk = p_row + (cc >> 1) * C::kChunkBytes;
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            *reinterpret_cast<uint4*>(chunk + ((((cc & 1) * 4 + u) ^ (row_in_tile & 7)) * 16)) =
+                make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+        }
+        l += (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y) + (acc[2].x + acc[2].y) +
+             (acc[3].x + acc[3].y);
+        lr += (accr[0].x + accr[0].y) + (accr[1].x + accr[1].y);
+        if (move && j > 0) {
+          // bring the sum up to key tile j-1 to the new reference max before PV_t(j)
+#pragma unroll
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t o[32];
+            tmem_ld32(tm_o + cc * 32, o);
+            tmem_wait_ld();
+#pragma unroll
+            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+            tmem_st32(tm_o + cc * 32, o);
+          }
+          tmem_wait_st();
+        }
+        fence_proxy_async_smem();  // P (generic stores) before the MMA reads it
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(C::kBarPFull + t));
+        if (wq == 0) FA_TRACE_POINT(55, n, t);
+      }
+      if (!ok) break;
+      if (t_nk > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarPVDone + t), (n_prev + t_nk - 1) & 1, wd));
+        if (!ok) break;
+      }
+      n_prev += t_nk;
+      if (t_nk == 0 && row < p.N && (t == 0 || w.own1)) {
+        // a query tile that sees no key: O = 0, LSE = -inf
+        uint4* dst = reinterpret_cast<uint4*>(p.O + (static_cast<size_t>(bh) * p.N + row) * D);
+#pragma unroll
+        for (int v = 0; v < D / 8; ++v) dst[v] = make_uint4(0u, 0u, 0u, 0u);
+        p.LSE[static_cast<size_t>(bh) * p.N + row] = -INFINITY;
+      }
+      if (t_nk > 0) {
+        if (t == 0 && threadIdx.x == 0) FA_TRACE_CTA(3);
+        if (wq == 0) FA_TRACE_POINT(56, ki, t);
+        tc_fence_after();
+        const float norm = kDropout ? l : lr;
+        const float inv_l = (norm > 0.0f) ? 1.0f / norm : 0.0f;
+        uint16_t* orow = p.O + (static_cast<size_t>(bh) * p.N + row) * D;
+#pragma unroll
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t o[32];
+          tmem_ld32(tm_o + cc * 32, o);
+          tmem_wait_ld();
+          if (cc == D / 32 - 1) {
+            // O_t is in registers: the next item's first PV_t may overwrite it
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::kBarOFree + t));
+          }
+          uint32_t pk[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k)
+            pk[k] = pack2<E>(__uint_as_float(o[2 * k]) * inv_l, __uint_as_float(o[2 * k + 1]) * inv_l);
+          if (row < p.N) {
+            uint4* dst = reinterpret_cast<uint4*>(orow + cc * 32);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          }
+        }
+        if (row < p.N)
+          p.LSE[static_cast<size_t>(bh) * p.N + row] =
+              (l > 0.0f) ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0) FA_TRACE_CTA(4);
   if (warp == kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmCols);

@@ -146,8 +146,11 @@ cudaError_t set_smem(Kern k, size_t bytes) {
 
 template <int D, Elt E>
 cudaError_t set_smem_d() {
-  cudaError_t e = set_smem(fwd::fa_fwd_kernel<D, E, false>, fwd::Cfg<D>::kSmemBytes);
-  e = e ? e : set_smem(fwd::fa_fwd_kernel<D, E, true>, fwd::Cfg<D>::kSmemBytes);
+  constexpr size_t S = fwd::Cfg<D>::kSmemBytes;
+  cudaError_t e = set_smem(fwd::fa_fwd_kernel<D, E, false>, S);
+  e = e ? e : set_smem(fwd::fa_fwd_kernel<D, E, true>, S);
+  e = e ? e : set_smem(fwd::fa_fwd_persistent_kernel<D, E, false, false>, S);
+  e = e ? e : set_smem(fwd::fa_fwd_persistent_kernel<D, E, true, false>, S);
   e = e ? e : set_smem(bwd::fa_bwd_kernel<D, E, false>, bwd::Cfg<D>::kSmemBytes);
   e = e ? e : set_smem(bwd::fa_bwd_kernel<D, E, true>, bwd::Cfg<D>::kSmemBytes);
   return e;
@@ -160,6 +163,8 @@ cudaError_t set_smem_all() {
   if constexpr (E == Elt::BF16) {  // dropout instances (bf16, general masks)
     e = e ? e : set_smem(fwd::fa_fwd_kernel<64, E, true, true>, fwd::Cfg<64>::kSmemBytes);
     e = e ? e : set_smem(fwd::fa_fwd_kernel<128, E, true, true>, fwd::Cfg<128>::kSmemBytes);
+    e = e ? e : set_smem(fwd::fa_fwd_persistent_kernel<64, E, true, true>, fwd::Cfg<64>::kSmemBytes);
+    e = e ? e : set_smem(fwd::fa_fwd_persistent_kernel<128, E, true, true>, fwd::Cfg<128>::kSmemBytes);
     e = e ? e : set_smem(bwd::fa_bwd_kernel<64, E, true, true>, bwd::Cfg<64>::kSmemBytes);
     e = e ? e : set_smem(bwd::fa_bwd_kernel<128, E, true, true>, bwd::Cfg<128>::kSmemBytes);
   }
@@ -299,21 +304,41 @@ fa_status make_drop(float p_drop, uint64_t seed, uint32_t offset, DropSpec* d) {
 
 // ---------------------------------------------------------------- forward work split
 //
-// The forward CTA owns two query tiles (they share every K/V tile it loads). With
-// one CTA per SM, B*H*ceil(N/256) such CTAs often leave the last wave of the grid
-// mostly empty (B1 H8 N16384: 512 CTAs on 148 SMs = 3.46 waves). So per head the
-// lightest `singles` query tiles get a CTA of their own, launched after all pair
-// CTAs, where they fill that last wave at about half the cost of a pair. The split
-// is chosen by simulating the launch: CTAs start in grid order on the first free SM;
-// a pair costs the larger key-tile count of its two tiles, a single 0.74 of its own
-// (measured on B1 H8 N16384 d128: 1024 single-tile CTAs run at 0.77x the rate of
-// 512 pair CTAs). Cached per shape.
+// A forward item owns two query tiles (they share every K/V tile the CTA loads), or
+// one. Per head the lightest `singles` query tiles are single-tile items, listed after
+// all pair items, where they even out the CTAs' loads at about half the cost of a
+// pair. An item costs the larger key-tile count of its tiles (a pair) or 0.74 of its
+// own (a single: measured on B1 H8 N16384 d128, 1024 single-tile CTAs ran at 0.77x
+// the rate of 512 pair CTAs).
+// Launch forms:
+//   * one CTA per item, started in grid order on the first free SM. Each CTA pays
+//     its set-up, first loads and epilogue (about 4 us measured on a B200) and the
+//     next one on that SM starts about 1 us after it ends.
+//   * persistent (fa_fwd_persistent_kernel): min(items, SMs) CTAs deal the list out
+//     back and forth (CTA b takes items b, 2G - 1 - b, 2G + b, ...), so one item's
+//     epilogue overlaps the next item's first loads and products. Measured on a B200
+//     (forward TFLOP/s, one form against the other): short rows gain (B8 H12 N1024
+//     causal: d64 225 -> 273, d128 381 -> 434); long rows lose, the per-item
+//     bookkeeping slowing the issue loop (B1 H8 N4096 d128, one item per CTA either
+//     way: 906 -> 860) and the fixed deal balancing long causal rows worse than the
+//     hardware's first-free-SM order (B2 H16 N8192 d128 causal: 949 -> 898).
+// So the persistent form runs when items outnumber the SMs and average at most
+// kFwdPersistMaxTiles key tiles, without a block mask (its CTAs would build the mask
+// rows of every item they walk). The singles count is then chosen by simulating the
+// chosen form (an item costs 0.4 key tiles more for its epilogue in the persistent
+// form). Cached per shape.
 struct FwdSplit {
-  int pairs_ph, singles_ph;
+  int pairs_ph, singles_ph, weight_major, persistent;
 };
 
-double split_makespan(int BH, int n_qt, int singles, int sms,
-                      const std::vector<int>& key_tiles) {
+constexpr double kFwdItemOverhead = 0.4;
+constexpr double kFwdPersistMaxTiles = 16.0;
+// K and V of every head at most this large: rank-major item order (fits in L2)
+constexpr double kFwdWeightMajorBytes = 96.0 * (1 << 20);
+
+// Block-mask launches: one CTA per item, started in grid order on the first free SM.
+double fwd_makespan_grid(int BH, int n_qt, int singles, int sms,
+                         const std::vector<int>& key_tiles) {
   std::priority_queue<double, std::vector<double>, std::greater<double>> free_at;
   for (int i = 0; i < sms; ++i) free_at.push(0.0);
   double end = 0.0;
@@ -334,21 +359,49 @@ double split_makespan(int BH, int n_qt, int singles, int sms,
   return end;
 }
 
-FwdSplit fwd_split(int BH, int N, int wl, int wr, int sms) {
+// Persistent launches: the largest load any CTA takes when the items are dealt out
+// back and forth, in the kernel's order.
+double fwd_makespan_persistent(int BH, int n_qt, int singles, int sms, bool weight_major,
+                               const std::vector<int>& key_tiles) {
+  const int pairs = (n_qt - singles) / 2;
+  const long long n_pair = static_cast<long long>(BH) * pairs;
+  const long long n_items = n_pair + static_cast<long long>(BH) * singles;
+  const int G = static_cast<int>(std::min<long long>(n_items, sms));
+  if (G <= 0) return 0.0;
+  std::vector<double> load(G, 0.0);
+  for (long long i = 0; i < n_items; ++i) {
+    double cost;
+    if (i < n_pair) {
+      const long long r = weight_major ? i / BH : i % pairs;
+      const int t0 = singles + 2 * static_cast<int>(pairs - 1 - r);
+      cost = std::max(key_tiles[t0], key_tiles[t0 + 1]);
+    } else {
+      const long long c = i - n_pair;
+      const long long r = weight_major ? c / BH : c % singles;
+      cost = 0.74 * key_tiles[singles - 1 - static_cast<int>(r)];
+    }
+    const long long k = i / G, b = i % G;
+    load[(k & 1) ? G - 1 - b : b] += cost + kFwdItemOverhead;
+  }
+  return *std::max_element(load.begin(), load.end());
+}
+
+FwdSplit fwd_split(int BH, int N, int d, int wl, int wr, bool block_mask, int sms) {
   const int n_qt = (N + fwd::BM - 1) / fwd::BM;
   const int n_kt = (N + fwd::BN - 1) / fwd::BN;
   const int min_singles = n_qt % 2;
-  FwdSplit plain{(n_qt - min_singles) / 2, min_singles};
+  FwdSplit plain{(n_qt - min_singles) / 2, min_singles, 0, 0};
   if (sms <= 0) return plain;
-  // Singles only help while they fit in the last wave: at most about sms / BH per
-  // head are tried. The simulation replays every CTA per candidate, so the total
-  // (candidates x CTAs) is bounded too; beyond it the plain split is used.
+  // Singles only help while they fit in the last round: at most about sms / BH per
+  // head are tried. The simulation replays every item per candidate, so the total
+  // (candidates x items) is bounded too; beyond it the plain split is used.
   const int max_singles = std::min(n_qt, 2 * ((sms + BH - 1) / BH) + 1);
   const long long candidates = (max_singles - min_singles) / 2 + 1;
   if (candidates * BH * n_qt > (1ll << 22)) return plain;
   static std::mutex mu;
-  static std::map<std::tuple<int, int, int, int, int>, FwdSplit> cache;  // at most 1024 shapes
-  const auto key = std::make_tuple(BH, N, wl, wr, sms);
+  // at most 1024 shapes
+  static std::map<std::tuple<int, int, int, int, int, bool, int>, FwdSplit> cache;
+  const auto key = std::make_tuple(BH, N, d, wl, wr, block_mask, sms);
   {
     std::lock_guard<std::mutex> lock(mu);
     auto it = cache.find(key);
@@ -356,19 +409,34 @@ FwdSplit fwd_split(int BH, int N, int wl, int wr, int sms) {
   }
   // key tiles each query tile walks (window and causal; a block mask is ignored here)
   std::vector<int> key_tiles(n_qt);
+  bool uniform = true;
   for (int t = 0; t < n_qt; ++t) {
     const int r0 = t * fwd::BM, r1 = std::min(r0 + fwd::BM, N) - 1;
     const int lo = (wl < 0) ? 0 : std::max(0, r0 - wl) / fwd::BN;
     const int hi = (wr < 0) ? n_kt : std::min(n_kt, (r1 + wr) / fwd::BN + 1);
     key_tiles[t] = std::max(hi - lo, 1);
+    uniform = uniform && key_tiles[t] == key_tiles[0];
   }
-  FwdSplit best = plain;
-  double best_t = split_makespan(BH, n_qt, min_singles, sms, key_tiles);
+  // mean key tiles per item of the plain split
+  double work = 0.0;
+  for (int t = min_singles; t + 1 < n_qt; t += 2) work += std::max(key_tiles[t], key_tiles[t + 1]);
+  if (min_singles) work += key_tiles[0];
+  const long long plain_items = static_cast<long long>(BH) * ((n_qt + 1) / 2);
+  const bool persistent = !block_mask && plain_items > sms &&
+                          work / ((n_qt + 1) / 2) <= kFwdPersistMaxTiles;
+  const bool wm = persistent && !uniform &&
+                  static_cast<double>(BH) * N * d * 4.0 <= kFwdWeightMajorBytes;
+  auto cost = [&](int sg) {
+    return persistent ? fwd_makespan_persistent(BH, n_qt, sg, sms, wm, key_tiles)
+                      : fwd_makespan_grid(BH, n_qt, sg, sms, key_tiles);
+  };
+  FwdSplit best{plain.pairs_ph, plain.singles_ph, wm ? 1 : 0, persistent ? 1 : 0};
+  double best_t = cost(min_singles);
   for (int sg = min_singles + 2; sg <= max_singles; sg += 2) {
-    const double t = split_makespan(BH, n_qt, sg, sms, key_tiles);
+    const double t = cost(sg);
     if (t < best_t * 0.999) {
       best_t = t;
-      best = FwdSplit{(n_qt - sg) / 2, sg};
+      best = FwdSplit{(n_qt - sg) / 2, sg, wm ? 1 : 0, persistent ? 1 : 0};
     }
   }
   std::lock_guard<std::mutex> lock(mu);
@@ -496,6 +564,23 @@ namespace {
 // The bf16 and f16 entry points share these bodies; E picks the kernels' element
 // type and the tensor maps' data type.
 
+template <Elt E, bool kMasked, bool kDropout, bool kPersistent>
+fa_status launch_fwd(int d, dim3 grid, cudaStream_t s, const CUtensorMap& mq, const CUtensorMap& mk,
+                     const CUtensorMap& mv, const fwd::Params& p) {
+  constexpr int T = fwd::kThreads;
+  constexpr size_t S64 = fwd::Cfg<64>::kSmemBytes, S128 = fwd::Cfg<128>::kSmemBytes;
+  if constexpr (kPersistent) {
+    if (d == 64)
+      return launch(fwd::fa_fwd_persistent_kernel<64, E, kMasked, kDropout>, grid, T, S64, s,
+                    mq, mk, mv, p);
+    return launch(fwd::fa_fwd_persistent_kernel<128, E, kMasked, kDropout>, grid, T, S128, s,
+                  mq, mk, mv, p);
+  } else {
+    if (d == 64) return launch(fwd::fa_fwd_kernel<64, E, kMasked, kDropout>, grid, T, S64, s, mq, mk, mv, p);
+    return launch(fwd::fa_fwd_kernel<128, E, kMasked, kDropout>, grid, T, S128, s, mq, mk, mv, p);
+  }
+}
+
 template <Elt E>
 fa_status forward_impl(const void* Q, const void* K, const void* V, void* O, float* LSE, int B,
                      int H, int N, int d, float scale, int causal, const MaskSpec& mask,
@@ -515,10 +600,14 @@ fa_status forward_impl(const void* Q, const void* K, const void* V, void* O, flo
   p.LSE = LSE;
   p.N = N;
   p.BH = BH;
-  const FwdSplit split = fwd_split(BH, N, mask.wl, mask.wr, device_sms());
+  const bool block_mask = mask.blocks != nullptr;
+  const int sms = device_sms();
+  const FwdSplit split = fwd_split(BH, N, d, mask.wl, mask.wr, block_mask, sms);
   p.pairs_ph = split.pairs_ph;
   p.singles_ph = split.singles_ph;
-  p.n_pair_ctas = BH * split.pairs_ph;
+  p.n_pair_items = BH * split.pairs_ph;
+  p.n_items = BH * (split.pairs_ph + split.singles_ph);
+  p.weight_major = split.weight_major;
   p.scale_log2 = scale * 1.4426950408889634f;
   p.wl = mask.wl;
   p.wr = mask.wr;
@@ -526,23 +615,23 @@ fa_status forward_impl(const void* Q, const void* K, const void* V, void* O, flo
   p.n_kt = (N + fwd::BN - 1) / fwd::BN;
   p.drop = drop.params;
   p.timeout_ns = watchdog_ns();
-  const dim3 grid(static_cast<unsigned>(BH) * (split.pairs_ph + split.singles_ph));
+  // persistent: one CTA per SM at most; else one CTA per item
+  const bool pers = split.persistent != 0;
+  const dim3 grid(static_cast<unsigned>(pers ? std::min(p.n_items, sms) : p.n_items));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool g = mask.general();
-  constexpr int T = fwd::kThreads;
-  constexpr size_t S64 = fwd::Cfg<64>::kSmemBytes, S128 = fwd::Cfg<128>::kSmemBytes;
   if constexpr (E == Elt::BF16) {
     if (drop.on) {
-      if (d == 64) return launch(fwd::fa_fwd_kernel<64, E, true, true>, grid, T, S64, s, mq, mk, mv, p);
-      return launch(fwd::fa_fwd_kernel<128, E, true, true>, grid, T, S128, s, mq, mk, mv, p);
+      if (pers) return launch_fwd<E, true, true, true>(d, grid, s, mq, mk, mv, p);
+      return launch_fwd<E, true, true, false>(d, grid, s, mq, mk, mv, p);
     }
   } else if (drop.on) {
     return FA_ERR_UNSUPPORTED;
   }
-  if (d == 64 && !g) return launch(fwd::fa_fwd_kernel<64, E, false>, grid, T, S64, s, mq, mk, mv, p);
-  if (d == 64) return launch(fwd::fa_fwd_kernel<64, E, true>, grid, T, S64, s, mq, mk, mv, p);
-  if (!g) return launch(fwd::fa_fwd_kernel<128, E, false>, grid, T, S128, s, mq, mk, mv, p);
-  return launch(fwd::fa_fwd_kernel<128, E, true>, grid, T, S128, s, mq, mk, mv, p);
+  if (g && pers) return launch_fwd<E, true, false, true>(d, grid, s, mq, mk, mv, p);
+  if (g) return launch_fwd<E, true, false, false>(d, grid, s, mq, mk, mv, p);
+  if (pers) return launch_fwd<E, false, false, true>(d, grid, s, mq, mk, mv, p);
+  return launch_fwd<E, false, false, false>(d, grid, s, mq, mk, mv, p);
 }
 
 // Shared validation and set-up of the three backward stages. Fills the tensor maps
@@ -989,7 +1078,19 @@ int fa_trace_arm(int cta) {
   if (cudaMemcpyToSymbol(g_trace, zeros.data(), kTraceCap * sizeof(uint32_t)) != cudaSuccess)
     return -1;
   if (cudaMemcpyToSymbol(g_trace_cta, &cta, sizeof(cta)) != cudaSuccess) return -1;
+  static std::vector<unsigned long long> zeros_cta(kTraceCtas * 8u, 0ull);
+  if (cudaMemcpyToSymbol(g_trace_cta_ns, zeros_cta.data(), zeros_cta.size() * sizeof(unsigned long long)) !=
+      cudaSuccess)
+    return -1;
   return 0;
+}
+int fa_trace_cta_read(unsigned long long* out, int n_ctas) {
+  if (n_ctas < 0 || n_ctas > static_cast<int>(kTraceCtas)) return -1;
+  if (cudaDeviceSynchronize() != cudaSuccess) return -1;
+  if (cudaMemcpyFromSymbol(out, g_trace_cta_ns, static_cast<size_t>(n_ctas) * 8 * sizeof(unsigned long long)) !=
+      cudaSuccess)
+    return -1;
+  return n_ctas;
 }
 int fa_trace_read(uint32_t* slots, unsigned long long* ns) {
   if (cudaDeviceSynchronize() != cudaSuccess) return -1;

@@ -49,9 +49,26 @@ __device__ __forceinline__ void trace_point(uint32_t code, uint32_t a, uint32_t 
     }
   }
 }
+// Per-CTA timeline of every CTA (up to kTraceCtas): global timer at up to 7 stages
+// (slot < 7) and the SM id (slot 7), stored by whichever thread passes the stage.
+constexpr unsigned kTraceCtas = 16384u;
+__device__ unsigned long long g_trace_cta_ns[kTraceCtas * 8u];
+__device__ __forceinline__ void trace_cta(uint32_t slot) {
+  if (blockIdx.x >= kTraceCtas) return;
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  g_trace_cta_ns[blockIdx.x * 8u + (slot & 7u)] = t;
+  if (slot == 0u) {
+    uint32_t sm;
+    asm volatile("mov.u32 %0, %smid;" : "=r"(sm));
+    g_trace_cta_ns[blockIdx.x * 8u + 7u] = sm;
+  }
+}
 #define FA_TRACE_POINT(code, a, b) ::fa::trace_point((code), (a), (b))
+#define FA_TRACE_CTA(slot) ::fa::trace_cta(slot)
 #else
 #define FA_TRACE_POINT(code, a, b) ((void)0)
+#define FA_TRACE_CTA(slot) ((void)0)
 #endif
 
 // ---------------------------------------------------------------- mbarrier

@@ -42,6 +42,8 @@ CASES = [
     (2, 1, 384, 128, False, 0.1, 99, 2**31 + 5, (100, 50), None),
     (1, 2, 640, 64, True, 0.3, 7, 1, None, 0.6),
     (1, 1, 77, 128, False, 0.9, 5, 5, None, None),
+    # 192 items of 1 to 5 key tiles: the persistent forward
+    (2, 32, 640, 64, True, 0.2, 11, 0, None, None),
 ]
 
 

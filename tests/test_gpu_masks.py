@@ -73,6 +73,9 @@ WINDOW_CASES = [
     (2, 1, 640, 64, False, (-1, 129)),      # unbounded left, right past a tile edge
     (1, 1, 512, 128, True, (127, 0)),       # exactly one tile wide
     (1, 2, 384, 128, False, (5000, 5000)),  # wider than N: plain attention
+    # more items than SMs, few key tiles each: the persistent forward
+    (2, 32, 1024, 64, True, (100, 0)),
+    (1, 40, 1000, 128, False, (64, 64)),
 ]
 
 

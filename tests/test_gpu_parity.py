@@ -200,6 +200,25 @@ def test_f16_small_full_parity(B, H, N, d, causal):
     check_full(q, k, v, do, 1.0 / math.sqrt(d), causal, TOL_F16)
 
 
+# Launches of more items than SMs whose items average few key tiles run the
+# persistent forward: each CTA walks several items, reusing its Q, S, P and O
+# buffers (and the K/V rings) from one item to the next.
+PERSISTENT = [
+    # (B, H, N, d, causal, dtype)
+    (4, 16, 1024, 64, True, torch.bfloat16),    # 256 pair items, 1 to 8 key tiles each
+    (4, 16, 1024, 64, True, torch.float16),
+    (2, 40, 900, 128, True, torch.bfloat16),    # ragged tail; single-tile items too
+    (3, 64, 256, 128, False, torch.bfloat16),   # 192 items of 2 key tiles
+]
+
+
+@pytest.mark.parametrize("B,H,N,d,causal,dtype", PERSISTENT)
+def test_persistent_forward_full_parity(B, H, N, d, causal, dtype):
+    q, k, v, do = make_inputs(B, H, N, d, dtype, seed=61 + N + d + int(causal))
+    tol = TOL_F16 if dtype == torch.float16 else TOL_BF16
+    check_full(q, k, v, do, 1.0 / math.sqrt(d), causal, tol)
+
+
 def test_f16_large_logits_online_rescale():
     q, k, v, do = make_inputs(1, 2, 512, 128, torch.float16, seed=98, qk_gain=8.0)
     check_full(q, k, v, do, 1.0 / math.sqrt(128), True, TOL_F16)
