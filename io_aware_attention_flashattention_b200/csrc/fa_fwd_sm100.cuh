@@ -127,29 +127,29 @@ struct Params {
 };
 
 // S = Q_t K_j^T: M = 128 query rows, N = 128 keys, K = D; both operands K-major.
+// Per 64-column chunk, four K = 16 steps 32 bytes apart (2 descriptor units); the
+// chunks are kChunkBytes (1024 units) apart.
 template <int D, Elt E>
 __device__ __forceinline__ void issue_s(uint32_t tm_d, uint32_t q_smem, uint32_t k_smem) {
   constexpr uint32_t idesc = idesc_f32acc<E>(BM, BN, 0, 0);
+  constexpr uint64_t kChunk = Cfg<D>::kChunkBytes >> 4;
+  const uint64_t qa = sdesc_sw128(q_smem, 16, 1024), kb = sdesc_sw128(k_smem, 16, 1024);
 #pragma unroll
-  for (int kk = 0; kk < D / 16; ++kk) {
-    const uint32_t off = (kk / 4) * Cfg<D>::kChunkBytes + (kk % 4) * 32;
-    mma_ss_e(tm_d, sdesc_sw128(q_smem + off, 16, 1024), sdesc_sw128(k_smem + off, 16, 1024),
-             idesc, kk > 0 ? 1u : 0u);
-  }
+  for (int c = 0; c < D / 64; ++c)
+    mma_ss_x4<2, 2>(tm_d, qa + c * kChunk, kb + c * kChunk, idesc, c > 0 ? 1u : 0u);
 }
 
-// O += P V_j: A = P (128 x 128 keys, K-major in shared memory), B = V_j read MN-major.
+// O += P V_j: A = P (128 x 128 keys, K-major in shared memory), B = V_j read MN-major:
+// K = 16 keys step 16 rows x 128 bytes (128 descriptor units) down V, 32 bytes along P.
 template <int D, Elt E>
 __device__ __forceinline__ void issue_pv(uint32_t tm_o, uint32_t p_smem, uint32_t v_smem,
                                          bool accumulate) {
   constexpr uint32_t idesc = idesc_f32acc<E>(BM, D, 0, 1);
-#pragma unroll
-  for (int kk = 0; kk < BN / 16; ++kk) {
-    const uint32_t poff = (kk / 4) * Cfg<D>::kChunkBytes + (kk % 4) * 32;
-    mma_ss_e(tm_o, sdesc_sw128(p_smem + poff, 16, 1024),
-             sdesc_sw128(v_smem + kk * 16 * 128, Cfg<D>::kChunkBytes, 1024), idesc,
-             (accumulate || kk > 0) ? 1u : 0u);
-  }
+  constexpr uint64_t kChunk = Cfg<D>::kChunkBytes >> 4;
+  const uint64_t pa = sdesc_sw128(p_smem, 16, 1024);
+  const uint64_t vb = sdesc_sw128(v_smem, Cfg<D>::kChunkBytes, 1024);
+  mma_ss_x4<2, 128>(tm_o, pa, vb, idesc, accumulate ? 1u : 0u);
+  mma_ss_x4<2, 128>(tm_o, pa + kChunk, vb + 4 * 128, idesc, 1u);
 }
 
 // Drain wait: ignores the abort flag, bounded by its own limit. Used at teardown so

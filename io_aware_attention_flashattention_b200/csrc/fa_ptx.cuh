@@ -236,6 +236,63 @@ __device__ __forceinline__ void mma_ts_e(uint32_t d_tmem, uint32_t a_tmem, uint6
       : "memory");
 }
 
+// Four MMAs of one K chunk (K = 4 x 16) from one elected lane: MMA i takes the
+// descriptors a0 + i * SA and b0 + i * SB (in the descriptors' 16-byte address units;
+// shared-memory addresses stay below 256 KB, so the 14-bit start-address field never
+// carries into the next field) and accumulates if i > 0 or acc_first is set. Fewer
+// instructions in the issuing warp than four separate issues, each recomputing its
+// descriptors.
+template <uint32_t SA, uint32_t SB>
+__device__ __forceinline__ void mma_ss_x4(uint32_t d_tmem, uint64_t a0, uint64_t b0,
+                                          uint32_t idesc, uint32_t acc_first) {
+  asm volatile(
+      "{\n\t.reg .pred p, e, t;\n\t"
+      ".reg .b32 al, ah, bl, bh, x, y;\n\t"
+      ".reg .b64 a, b;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.b32 t, %4, %4;\n\t"
+      "mov.b64 {al, ah}, %1;\n\t"
+      "mov.b64 {bl, bh}, %2;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t"
+      "add.u32 x, al, %5;\n\tadd.u32 y, bl, %8;\n\t"
+      "mov.b64 a, {x, ah};\n\tmov.b64 b, {y, bh};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, t;\n\t"
+      "add.u32 x, al, %6;\n\tadd.u32 y, bl, %9;\n\t"
+      "mov.b64 a, {x, ah};\n\tmov.b64 b, {y, bh};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, t;\n\t"
+      "add.u32 x, al, %7;\n\tadd.u32 y, bl, %10;\n\t"
+      "mov.b64 a, {x, ah};\n\tmov.b64 b, {y, bh};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], a, b, %3, t;\n\t}" ::"r"(d_tmem),
+      "l"(a0), "l"(b0), "r"(idesc), "r"(acc_first), "n"(SA), "n"(2 * SA), "n"(3 * SA), "n"(SB),
+      "n"(2 * SB), "n"(3 * SB)
+      : "memory");
+}
+
+// The same with A in TMEM: MMA i reads A at column a_tmem + i * SA.
+template <uint32_t SA, uint32_t SB>
+__device__ __forceinline__ void mma_ts_x4(uint32_t d_tmem, uint32_t a_tmem, uint64_t b0,
+                                          uint32_t idesc, uint32_t acc_first) {
+  asm volatile(
+      "{\n\t.reg .pred p, e, t;\n\t"
+      ".reg .b32 bl, bh, x, y;\n\t"
+      ".reg .b64 b;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "setp.eq.b32 t, %4, %4;\n\t"
+      "mov.b64 {bl, bh}, %2;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t"
+      "add.u32 x, %1, %5;\n\tadd.u32 y, bl, %8;\n\tmov.b64 b, {y, bh};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [x], b, %3, t;\n\t"
+      "add.u32 x, %1, %6;\n\tadd.u32 y, bl, %9;\n\tmov.b64 b, {y, bh};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [x], b, %3, t;\n\t"
+      "add.u32 x, %1, %7;\n\tadd.u32 y, bl, %10;\n\tmov.b64 b, {y, bh};\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [x], b, %3, t;\n\t}" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b0), "r"(idesc), "r"(acc_first), "n"(SA), "n"(2 * SA), "n"(3 * SA),
+      "n"(SB), "n"(2 * SB), "n"(3 * SB)
+      : "memory");
+}
+
 __device__ __forceinline__ void tc_commit_e(uint32_t bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t"
