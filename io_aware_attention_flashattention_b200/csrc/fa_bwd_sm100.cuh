@@ -277,6 +277,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                   const Params p) {
   using C = Cfg<D>;
+  if (threadIdx.x == 0) FA_TRACE_CTA(0);
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -363,6 +364,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const Watchdog wd{abort_flag, p.timeout_ns};
+  if (threadIdx.x == 0) FA_TRACE_CTA(1);
   if (warp == kWarpMma) FA_TRACE_POINT(0, 0, 0);
 
   // Does some query of query tile i see a key of this tile?
@@ -463,6 +465,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         issue_xyT_half<D, E>(tm_s + 64 * h, k_smem, slot_smem(seqQ));
         tc_commit_e(bar(C::kBarS + h));
         FA_TRACE_POINT(8, s, h);
+        if (s == 0 && h == 0 && lane == 0) FA_TRACE_CTA(2);
       }
       return true;
     };
@@ -643,6 +646,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int u = 0; u < D / 8; ++u) dst[u] = make_uint4(0u, 0u, 0u, 0u);
     }
     if (ok && nsteps > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarDKDV), 0, wd));
+    if (threadIdx.x == 0) FA_TRACE_CTA(3);
     if (ok && nsteps > 0) {
       // warps 0-3 write dK (times scale), warps 4-7 write dV; a split tile's segment
       // writes its fp32 partial to its slot instead
@@ -783,6 +787,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  if (threadIdx.x == 0) FA_TRACE_CTA(4);
   if (warp == kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmCols);
