@@ -322,23 +322,28 @@ fa_status make_drop(float p_drop, uint64_t seed, uint32_t offset, DropSpec* d) {
 //     bookkeeping slowing the issue loop (B1 H8 N4096 d128, one item per CTA either
 //     way: 906 -> 860) and the fixed deal balancing long causal rows worse than the
 //     hardware's first-free-SM order (B2 H16 N8192 d128 causal: 949 -> 898).
-// So the persistent form runs when items outnumber the SMs and average at most
-// kFwdPersistMaxTiles key tiles, without a block mask (its CTAs would build the mask
-// rows of every item they walk). The singles count is then chosen by simulating the
-// chosen form (an item costs 0.4 key tiles more for its epilogue in the persistent
-// form). Cached per shape.
+// So both forms are simulated, each with its best singles count: one CTA per item as
+// above, and dealt back and forth with 0.4 key tiles of epilogue per item. The persistent
+// form runs when it has more items than SMs and its makespan, 5% longer for its slower
+// issue loop, beats that of one CTA per item (charged 1.5 key tiles per CTA for set-up,
+// first loads, epilogue and launch gap) by 4%, and never with a block mask (its CTAs would
+// build the mask rows of every item they walk). Those constants reproduce which form won
+// in the measurements above and in B1 H8 N8192 d128 causal (persistent +14%), B2 H16 N4096
+// d128 causal (+5%), B1 H8 N16384 d128 causal (0%) and non-causal (-6%). Cached per shape.
 struct FwdSplit {
   int pairs_ph, singles_ph, weight_major, persistent;
 };
 
-constexpr double kFwdItemOverhead = 0.4;
-constexpr double kFwdPersistMaxTiles = 16.0;
+constexpr double kFwdItemOverhead = 0.4;       // persistent: an item's epilogue, key tiles
+constexpr double kFwdGridCtaOverhead = 1.5;    // one CTA per item: set-up, first loads, epilogue, gap
+constexpr double kFwdPersistPenalty = 1.05;    // the persistent issue loop's slower key tiles
+constexpr double kFwdPersistMargin = 1.04;     // predicted gain the persistent form must beat
 // K and V of every head at most this large: rank-major item order (fits in L2)
 constexpr double kFwdWeightMajorBytes = 96.0 * (1 << 20);
 
 // Block-mask launches: one CTA per item, started in grid order on the first free SM.
 double fwd_makespan_grid(int BH, int n_qt, int singles, int sms,
-                         const std::vector<int>& key_tiles) {
+                         const std::vector<int>& key_tiles, double overhead = 0.0) {
   std::priority_queue<double, std::vector<double>, std::greater<double>> free_at;
   for (int i = 0; i < sms; ++i) free_at.push(0.0);
   double end = 0.0;
@@ -352,10 +357,10 @@ double fwd_makespan_grid(int BH, int n_qt, int singles, int sms,
   for (int h = 0; h < BH; ++h)
     for (int k = pairs - 1; k >= 0; --k) {
       const int t0 = singles + 2 * k;
-      run(std::max(key_tiles[t0], key_tiles[t0 + 1]));
+      run(std::max(key_tiles[t0], key_tiles[t0 + 1]) + overhead);
     }
   for (int h = 0; h < BH; ++h)
-    for (int t = singles - 1; t >= 0; --t) run(0.74 * key_tiles[t]);
+    for (int t = singles - 1; t >= 0; --t) run(0.74 * key_tiles[t] + overhead);
   return end;
 }
 
@@ -417,28 +422,31 @@ FwdSplit fwd_split(int BH, int N, int d, int wl, int wr, bool block_mask, int sm
     key_tiles[t] = std::max(hi - lo, 1);
     uniform = uniform && key_tiles[t] == key_tiles[0];
   }
-  // mean key tiles per item of the plain split
-  double work = 0.0;
-  for (int t = min_singles; t + 1 < n_qt; t += 2) work += std::max(key_tiles[t], key_tiles[t + 1]);
-  if (min_singles) work += key_tiles[0];
-  const long long plain_items = static_cast<long long>(BH) * ((n_qt + 1) / 2);
-  const bool persistent = !block_mask && plain_items > sms &&
-                          work / ((n_qt + 1) / 2) <= kFwdPersistMaxTiles;
-  const bool wm = persistent && !uniform &&
+  const bool wm = !block_mask && !uniform &&
                   static_cast<double>(BH) * N * d * 4.0 <= kFwdWeightMajorBytes;
-  auto cost = [&](int sg) {
-    return persistent ? fwd_makespan_persistent(BH, n_qt, sg, sms, wm, key_tiles)
-                      : fwd_makespan_grid(BH, n_qt, sg, sms, key_tiles);
-  };
-  FwdSplit best{plain.pairs_ph, plain.singles_ph, wm ? 1 : 0, persistent ? 1 : 0};
-  double best_t = cost(min_singles);
+  // each form's best singles count (one CTA per item: the makespan without the per-CTA
+  // cost, as first measured; persistent: with its per-item epilogue)
+  int sg_grid = min_singles, sg_pers = min_singles;
+  double t_grid = fwd_makespan_grid(BH, n_qt, min_singles, sms, key_tiles);
+  double t_pers = fwd_makespan_persistent(BH, n_qt, min_singles, sms, wm, key_tiles);
   for (int sg = min_singles + 2; sg <= max_singles; sg += 2) {
-    const double t = cost(sg);
-    if (t < best_t * 0.999) {
-      best_t = t;
-      best = FwdSplit{(n_qt - sg) / 2, sg, wm ? 1 : 0, persistent ? 1 : 0};
+    const double tg = fwd_makespan_grid(BH, n_qt, sg, sms, key_tiles);
+    if (tg < t_grid * 0.999) { t_grid = tg; sg_grid = sg; }
+    if (!block_mask) {
+      const double tp = fwd_makespan_persistent(BH, n_qt, sg, sms, wm, key_tiles);
+      if (tp < t_pers * 0.999) { t_pers = tp; sg_pers = sg; }
     }
   }
+  // the persistent form only where it is predicted to win by a margin, counting the one-CTA
+  // form's set-up, first loads, epilogue and launch gap and the persistent form's slower
+  // issue loop
+  const long long pers_items = static_cast<long long>(BH) * ((n_qt - sg_pers) / 2 + sg_pers);
+  const bool persistent =
+      !block_mask && pers_items > sms &&
+      fwd_makespan_grid(BH, n_qt, sg_grid, sms, key_tiles, kFwdGridCtaOverhead) >
+          kFwdPersistMargin * kFwdPersistPenalty * t_pers;
+  FwdSplit best = persistent ? FwdSplit{(n_qt - sg_pers) / 2, sg_pers, wm ? 1 : 0, 1}
+                             : FwdSplit{(n_qt - sg_grid) / 2, sg_grid, 0, 0};
   std::lock_guard<std::mutex> lock(mu);
   if (cache.size() >= 1024) cache.clear();
   cache[key] = best;
