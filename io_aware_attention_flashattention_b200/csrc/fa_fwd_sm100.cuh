@@ -164,6 +164,167 @@ __device__ __forceinline__ void drain_wait(uint32_t bar, uint32_t parity, uint64
   }
 }
 
+// The softmax work of one key tile for one query row (this thread, TMEM lane
+// row_in_tile of query tile t), once S_t has landed in TMEM: read S_t and release its
+// columns (SFree); mask the elements outside the row's visible keys [k_lo, k_hi) on
+// tiles that cross an edge; take the row max and move the reference max m_ref when it
+// grew by more than 2^8 (rescaling l, lr and, after the previous PV_t, O_t); p = 2^(s*c
+// - m_ref), their sum l and, rounded to 16 bits, P_t into the swizzled shared tile (with
+// dropout applied after the sum); then PFull. n counts this tile's S and PV products
+// before this one (their barrier phases); first: no PV_t of the item yet. Returns false
+// if a bounded wait gave up.
+template <int D, Elt E, bool kDropout>
+__device__ __forceinline__ bool softmax_key_tile(const Params& p, const Watchdog& wd,
+                                                 uint32_t tm_s, uint32_t tm_o, uint8_t* p_row,
+                                                 uint32_t bar_sfree, uint32_t bar_pvdone,
+                                                 uint32_t bar_pfull, int n, bool first, int kt,
+                                                 int r0, int row, int row_in_tile, int k_lo,
+                                                 int k_hi, int wl, int wr, int bh, int lane,
+                                                 int wq, int t, float& m_ref, float& l,
+                                                 float& lr) {
+  using C = Cfg<D>;
+  const float c = p.scale_log2;
+  const int r1 = r0 + BM - 1;
+  tc_fence_after();
+  uint32_t s[4][32];
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) tmem_ld32(tm_s + cc * 32, s[cc]);
+  tmem_wait_ld();
+  // S_t is in registers: the MMA may overwrite it with the next S_t now
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar_sfree);
+  if (wq == 0) FA_TRACE_POINT(52, n, t);
+  const int kv0 = kt * BN;
+  // masking only where the tile crosses an edge of some row's visible range
+  const bool need_mask = (kv0 + BN > p.N) || (wr >= 0 && kv0 + BN - 1 > r0 + wr) ||
+                         (wl >= 0 && kv0 < r1 - wl);
+  if (need_mask) {
+    // key kv0 + k is visible iff 0 <= kv0 + k - k_lo < k_hi - k_lo
+    const int off = kv0 - k_lo;
+    const unsigned span = static_cast<unsigned>(max(k_hi - k_lo, 0));
+#pragma unroll
+    for (int k = 0; k < 128; ++k)
+      if (static_cast<unsigned>(off + k) >= span) s[k / 32][k % 32] = __float_as_uint(-INFINITY);
+  }
+  // row max: per 32-column chunk a tree of three-input maxima (short dependency
+  // chains, few live temporaries), then across the four chunks
+  float cm[4];
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) {
+    float t1[11];
+#pragma unroll
+    for (int q = 0; q < 10; ++q)
+      t1[q] = fmax3(__uint_as_float(s[cc][3 * q]), __uint_as_float(s[cc][3 * q + 1]),
+                    __uint_as_float(s[cc][3 * q + 2]));
+    t1[10] = fmaxf(__uint_as_float(s[cc][30]), __uint_as_float(s[cc][31]));
+    const float a = fmax3(t1[0], t1[1], t1[2]), b = fmax3(t1[3], t1[4], t1[5]);
+    const float d2 = fmax3(t1[6], t1[7], t1[8]), e = fmaxf(t1[9], t1[10]);
+    cm[cc] = fmax3(a, b, fmaxf(d2, e));
+  }
+  const float mx = fmaxf(fmaxf(cm[0], cm[1]), fmaxf(cm[2], cm[3]));
+  const float m_new = fmaxf(m_ref, mx * c);
+  const bool need = m_new > m_ref + kRescaleThreshold;
+  // The reference max moves for the whole warp when any row needs it (TMEM
+  // accesses are warp-wide); O is rescaled below, after the scores are dead.
+  const bool move = __any_sync(0xffffffffu, need);
+  float alpha = 1.0f;
+  if (move) {
+    alpha = (m_ref == -INFINITY) ? 0.0f : ex2_approx(m_ref - m_new);
+    m_ref = m_new;
+    l *= alpha;
+    lr *= alpha;
+  }
+  // the previous PV_t must be complete before P_t is overwritten and O_t rescaled
+  if (!first) {
+    if (wq == 0) FA_TRACE_POINT(53, n, t);
+    const bool ok = __all_sync(0xffffffffu, mbar_wait(bar_pvdone, (n - 1) & 1, wd));
+    if (wq == 0) FA_TRACE_POINT(54, n, t);
+    if (!ok) return false;
+    tc_fence_after();
+  }
+  const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
+  const float2 c2 = make_float2(c, c), nm2 = make_float2(-m_use, -m_use);
+  float2 accr[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+  float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                   make_float2(0.f, 0.f)};
+  // dropout: this row's four words for the current 16 keys (byte b of word m is key
+  // 4m + b of the group)
+  [[maybe_unused]] uint32_t zw[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) {
+    uint32_t pk[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const float2 x = ffma2(make_float2(__uint_as_float(s[cc][2 * k]),
+                                         __uint_as_float(s[cc][2 * k + 1])), c2, nm2);
+      float2 pe;
+      constexpr int kPoly = C::kPolyPeriod;
+      if (kPoly > 0 && k % (kPoly > 0 ? kPoly : 1) == kPoly - 1) {
+        pe = exp2_poly2(x);  // a share of the exponentials on the FMA pipe
+      } else {
+        pe = make_float2(ex2_approx(x.x), ex2_approx(x.y));
+      }
+      acc[k & 3] = fadd2(acc[k & 3], pe);  // l is the sum before dropout
+      if constexpr (kDropout) {
+        // One block covers 4 rows x 4 keys; the lanes of rows 4g..4g+3 share its
+        // counter. Every 16 keys, lane u (row mod 4) draws the block of keys
+        // 4u..4u+3 of the 16, and a 4 x 4 transpose across the four lanes hands
+        // each lane its own row's word of all four blocks.
+        if ((k & 7) == 0) {
+          const int u = lane & 3;
+          const uint4 w = philox4x32_10(
+              make_uint4(static_cast<uint32_t>(((kv0 + 32 * cc + 2 * k) >> 2) + u),
+                         static_cast<uint32_t>(row >> 2), static_cast<uint32_t>(bh),
+                         p.drop.offset),
+              p.drop.seed_lo, p.drop.seed_hi);
+          zw[0] = w.x;
+          zw[1] = w.y;
+          zw[2] = w.z;
+          zw[3] = w.w;
+          transpose4_lanes(zw, u);
+        }
+        // keys 2k, 2k + 1 of the chunk = keys 2(k mod 8), +1 of the group: word
+        // (k mod 8) / 2, bytes 2(k mod 2) and 2(k mod 2) + 1
+        const uint32_t wd = zw[(k & 7) >> 1] >> (16 * (k & 1));
+        pe.x = ((wd & 0xffu) >= p.drop.threshold) ? pe.x * p.drop.scale : 0.0f;
+        pe.y = (((wd >> 8) & 0xffu) >= p.drop.threshold) ? pe.y * p.drop.scale : 0.0f;
+      }
+      pk[k] = pack2<E>(pe.x, pe.y);
+      if constexpr (!kDropout) accr[k & 1] = fadd2(accr[k & 1], unpack2<E>(pk[k]));
+    }
+    // keys 32cc..32cc+31 = 16-byte units 4cc..4cc+3 of this row's 256 bytes:
+    // chunk (cc / 2), units (cc % 2) * 4 + u, 128-byte swizzle by the row
+    uint8_t* chunk = p_row + (cc >> 1) * C::kChunkBytes;
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+      *reinterpret_cast<uint4*>(chunk + ((((cc & 1) * 4 + u) ^ (row_in_tile & 7)) * 16)) =
+          make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+  }
+  l += (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y) + (acc[2].x + acc[2].y) +
+       (acc[3].x + acc[3].y);
+  lr += (accr[0].x + accr[0].y) + (accr[1].x + accr[1].y);
+  if (move && !first) {
+    // bring the sum up to the previous key tile to the new reference max before this PV_t
+#pragma unroll
+    for (int cc = 0; cc < D / 32; ++cc) {
+      uint32_t o[32];
+      tmem_ld32(tm_o + cc * 32, o);
+      tmem_wait_ld();
+#pragma unroll
+      for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
+      tmem_st32(tm_o + cc * 32, o);
+    }
+    tmem_wait_st();
+  }
+  fence_proxy_async_smem();  // P (generic stores) before the MMA reads it
+  tc_fence_before();
+  __syncwarp();
+  if (lane == 0) mbar_arrive(bar_pfull);
+  if (wq == 0) FA_TRACE_POINT(55, n, t);
+  return true;
+}
+
 template <int D, Elt E, bool kMasked, bool kDropout = false>
 __global__ void __launch_bounds__(kThreads, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -417,7 +578,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tm_s = tmem + lane_off + C::kTmS0 + t * 128;
     const uint32_t tm_o = tmem + lane_off + C::kTmO0 + t * D;
     uint8_t* p_row = base_ptr + C::kPOff + t * C::kPBytes + row_in_tile * 128;
-    const float c = p.scale_log2;
     float m_ref = -INFINITY;
     float l = 0.0f;
     // lr: the same sum over P as rounded for the PV product. O is divided by lr, so
@@ -438,7 +598,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     // visible keys of this row: [k_lo, k_hi)
     const int k_lo = (wl < 0) ? 0 : row - wl;
     const int k_hi = (wr < 0) ? p.N : min(p.N, row + wr + 1);
-    const int r1 = r0 + BM - 1;
     int kt = t_lo - 1;
     for (int j = 0; j < t_nk && ok; ++j) {
       do ++kt; while (!t_member(kt));
@@ -447,143 +606,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (wq == 0) FA_TRACE_POINT(51, j, t);
       if (j == 0 && t == 0 && threadIdx.x == 0) FA_TRACE_CTA(2);
       if (!ok) break;
-      tc_fence_after();
-      uint32_t s[4][32];
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) tmem_ld32(tm_s + cc * 32, s[cc]);
-      tmem_wait_ld();
-      // S_t(j) is in registers: the MMA may overwrite it with S_t(j+1) now
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(C::kBarSFree + t));
-      if (wq == 0) FA_TRACE_POINT(52, j, t);
-      const int kv0 = kt * BN;
-      // masking only where the tile crosses an edge of some row's visible range
-      const bool need_mask = (kv0 + BN > p.N) || (wr >= 0 && kv0 + BN - 1 > r0 + wr) ||
-                             (wl >= 0 && kv0 < r1 - wl);
-      if (need_mask) {
-        // key kv0 + k is visible iff 0 <= kv0 + k - k_lo < k_hi - k_lo
-        const int off = kv0 - k_lo;
-        const unsigned span = static_cast<unsigned>(max(k_hi - k_lo, 0));
-#pragma unroll
-        for (int k = 0; k < 128; ++k)
-          if (static_cast<unsigned>(off + k) >= span) s[k / 32][k % 32] = __float_as_uint(-INFINITY);
+      if (!softmax_key_tile<D, E, kDropout>(p, wd, tm_s, tm_o, p_row, bar(C::kBarSFree + t),
+                                            bar(C::kBarPVDone + t), bar(C::kBarPFull + t), j,
+                                            j == 0, kt, r0, row, row_in_tile, k_lo, k_hi, wl,
+                                            wr, bh, lane, wq, t, m_ref, l, lr)) {
+        ok = false;
+        break;
       }
-      // row max: per 32-column chunk a tree of three-input maxima (short dependency
-      // chains, few live temporaries), then across the four chunks
-      float cm[4];
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        float t1[11];
-#pragma unroll
-        for (int q = 0; q < 10; ++q)
-          t1[q] = fmax3(__uint_as_float(s[cc][3 * q]), __uint_as_float(s[cc][3 * q + 1]),
-                        __uint_as_float(s[cc][3 * q + 2]));
-        t1[10] = fmaxf(__uint_as_float(s[cc][30]), __uint_as_float(s[cc][31]));
-        const float a = fmax3(t1[0], t1[1], t1[2]), b = fmax3(t1[3], t1[4], t1[5]);
-        const float d2 = fmax3(t1[6], t1[7], t1[8]), e = fmaxf(t1[9], t1[10]);
-        cm[cc] = fmax3(a, b, fmaxf(d2, e));
-      }
-      const float mx = fmaxf(fmaxf(cm[0], cm[1]), fmaxf(cm[2], cm[3]));
-      const float m_new = fmaxf(m_ref, mx * c);
-      const bool need = m_new > m_ref + kRescaleThreshold;
-      // The reference max moves for the whole warp when any row needs it (TMEM
-      // accesses are warp-wide); O is rescaled below, after the scores are dead.
-      const bool move = __any_sync(0xffffffffu, need);
-      float alpha = 1.0f;
-      if (move) {
-        alpha = (m_ref == -INFINITY) ? 0.0f : ex2_approx(m_ref - m_new);
-        m_ref = m_new;
-        l *= alpha;
-        lr *= alpha;
-      }
-      // PV_t(j-1) must be complete before P_t is overwritten and O_t rescaled.
-      if (j > 0) {
-        if (wq == 0) FA_TRACE_POINT(53, j, t);
-        ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarPVDone + t), (j - 1) & 1, wd));
-        if (wq == 0) FA_TRACE_POINT(54, j, t);
-        if (!ok) break;
-        tc_fence_after();
-      }
-      const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
-      const float2 c2 = make_float2(c, c), nm2 = make_float2(-m_use, -m_use);
-      float2 accr[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-      float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                       make_float2(0.f, 0.f)};
-      // dropout: this row's four words for the current 16 keys (byte b of word m is key
-      // 4m + b of the group)
-      [[maybe_unused]] uint32_t zw[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const float2 x = ffma2(make_float2(__uint_as_float(s[cc][2 * k]),
-                                             __uint_as_float(s[cc][2 * k + 1])), c2, nm2);
-          float2 pe;
-          constexpr int kPoly = C::kPolyPeriod;
-          if (kPoly > 0 && k % (kPoly > 0 ? kPoly : 1) == kPoly - 1) {
-            pe = exp2_poly2(x);  // a share of the exponentials on the FMA pipe
-          } else {
-            pe = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-          }
-          acc[k & 3] = fadd2(acc[k & 3], pe);  // l is the sum before dropout
-          if constexpr (kDropout) {
-            // One block covers 4 rows x 4 keys; the lanes of rows 4g..4g+3 share its
-            // counter. Every 16 keys, lane u (row mod 4) draws the block of keys
-            // 4u..4u+3 of the 16, and a 4 x 4 transpose across the four lanes hands
-            // each lane its own row's word of all four blocks.
-            if ((k & 7) == 0) {
-              const int u = lane & 3;
-              const uint4 w = philox4x32_10(
-                  make_uint4(static_cast<uint32_t>(((kv0 + 32 * cc + 2 * k) >> 2) + u),
-                             static_cast<uint32_t>(row >> 2), static_cast<uint32_t>(bh),
-                             p.drop.offset),
-                  p.drop.seed_lo, p.drop.seed_hi);
-              zw[0] = w.x;
-              zw[1] = w.y;
-              zw[2] = w.z;
-              zw[3] = w.w;
-              transpose4_lanes(zw, u);
-            }
-            // keys 2k, 2k + 1 of the chunk = keys 2(k mod 8), +1 of the group: word
-            // (k mod 8) / 2, bytes 2(k mod 2) and 2(k mod 2) + 1
-            const uint32_t wd = zw[(k & 7) >> 1] >> (16 * (k & 1));
-            pe.x = ((wd & 0xffu) >= p.drop.threshold) ? pe.x * p.drop.scale : 0.0f;
-            pe.y = (((wd >> 8) & 0xffu) >= p.drop.threshold) ? pe.y * p.drop.scale : 0.0f;
-          }
-          pk[k] = pack2<E>(pe.x, pe.y);
-          if constexpr (!kDropout) accr[k & 1] = fadd2(accr[k & 1], unpack2<E>(pk[k]));
-        }
-        // keys 32cc..32cc+31 = 16-byte units 4cc..4cc+3 of this row's 256 bytes:
-        // chunk (cc / 2), units (cc % 2) * 4 + u, 128-byte swizzle by the row
-        uint8_t* chunk = p_row + (cc >> 1) * C::kChunkBytes;
-#pragma unroll
-        for (int u = 0; u < 4; ++u)
-          *reinterpret_cast<uint4*>(chunk + ((((cc & 1) * 4 + u) ^ (row_in_tile & 7)) * 16)) =
-              make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-      }
-      l += (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y) + (acc[2].x + acc[2].y) +
-           (acc[3].x + acc[3].y);
-      lr += (accr[0].x + accr[0].y) + (accr[1].x + accr[1].y);
-      if (move && j > 0) {
-        // bring the sum up to key tile j-1 to the new reference max before PV_t(j)
-#pragma unroll
-        for (int cc = 0; cc < D / 32; ++cc) {
-          uint32_t o[32];
-          tmem_ld32(tm_o + cc * 32, o);
-          tmem_wait_ld();
-#pragma unroll
-          for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-          tmem_st32(tm_o + cc * 32, o);
-        }
-        tmem_wait_st();
-      }
-      fence_proxy_async_smem();  // P (generic stores) before the MMA reads it
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(bar(C::kBarPFull + t));
-      if (wq == 0) FA_TRACE_POINT(55, j, t);
     }
     if (ok && t_nk > 0)
       ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarPVDone + t), (t_nk - 1) & 1, wd));
@@ -926,7 +955,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tm_s = tmem + lane_off + C::kTmS0 + t * 128;
     const uint32_t tm_o = tmem + lane_off + C::kTmO0 + t * D;
     uint8_t* p_row = base_ptr + C::kPOff + t * C::kPBytes + row_in_tile * 128;
-    const float c = p.scale_log2;
     // S_t and PV_t products of the items before this one (their barrier phases)
     int n_prev = 0;
     bool ok = true;
@@ -953,7 +981,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       // visible keys of this row: [k_lo, k_hi)
       const int k_lo = (wl < 0) ? 0 : row - wl;
       const int k_hi = (wr < 0) ? p.N : min(p.N, row + wr + 1);
-      const int r1 = r0 + BM - 1;
       int kt = t_lo - 1;
       for (int j = 0; j < t_nk && ok; ++j) {
         do ++kt; while (!t_member(kt));
@@ -964,144 +991,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (ki == 0 && j == 0 && t == 0 && threadIdx.x == 0) FA_TRACE_CTA(2);
         if (j == 0 && wq == 0) FA_TRACE_POINT(57, ki, t);
         if (!ok) break;
-        tc_fence_after();
-        uint32_t s[4][32];
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) tmem_ld32(tm_s + cc * 32, s[cc]);
-        tmem_wait_ld();
-        // S_t is in registers: the MMA may overwrite it with the next S_t now
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(C::kBarSFree + t));
-        if (wq == 0) FA_TRACE_POINT(52, n, t);
-        const int kv0 = kt * BN;
-        // masking only where the tile crosses an edge of some row's visible range
-        const bool need_mask = (kv0 + BN > p.N) || (wr >= 0 && kv0 + BN - 1 > r0 + wr) ||
-                               (wl >= 0 && kv0 < r1 - wl);
-        if (need_mask) {
-          // key kv0 + k is visible iff 0 <= kv0 + k - k_lo < k_hi - k_lo
-          const int off = kv0 - k_lo;
-          const unsigned span = static_cast<unsigned>(max(k_hi - k_lo, 0));
-#pragma unroll
-          for (int k2 = 0; k2 < 128; ++k2)
-            if (static_cast<unsigned>(off + k2) >= span)
-              s[k2 / 32][k2 % 32] = __float_as_uint(-INFINITY);
+        if (!softmax_key_tile<D, E, kDropout>(p, wd, tm_s, tm_o, p_row, bar(C::kBarSFree + t),
+                                              bar(C::kBarPVDone + t), bar(C::kBarPFull + t),
+                                              n, j == 0, kt, r0, row, row_in_tile, k_lo, k_hi,
+                                              wl, wr, bh, lane, wq, t, m_ref, l, lr)) {
+          ok = false;
+          break;
         }
-        // row max: per 32-column chunk a tree of three-input maxima (short dependency
-        // chains, few live temporaries), then across the four chunks
-        float cm[4];
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          float t1[11];
-#pragma unroll
-          for (int q = 0; q < 10; ++q)
-            t1[q] = fmax3(__uint_as_float(s[cc][3 * q]), __uint_as_float(s[cc][3 * q + 1]),
-                          __uint_as_float(s[cc][3 * q + 2]));
-          t1[10] = fmaxf(__uint_as_float(s[cc][30]), __uint_as_float(s[cc][31]));
-          const float a = fmax3(t1[0], t1[1], t1[2]), b = fmax3(t1[3], t1[4], t1[5]);
-          const float d2 = fmax3(t1[6], t1[7], t1[8]), e = fmaxf(t1[9], t1[10]);
-          cm[cc] = fmax3(a, b, fmaxf(d2, e));
-        }
-        const float mx = fmaxf(fmaxf(cm[0], cm[1]), fmaxf(cm[2], cm[3]));
-        const float m_new = fmaxf(m_ref, mx * c);
-        const bool need = m_new > m_ref + kRescaleThreshold;
-        // The reference max moves for the whole warp when any row needs it (TMEM
-        // accesses are warp-wide); O is rescaled below, after the scores are dead.
-        const bool move = __any_sync(0xffffffffu, need);
-        float alpha = 1.0f;
-        if (move) {
-          alpha = (m_ref == -INFINITY) ? 0.0f : ex2_approx(m_ref - m_new);
-          m_ref = m_new;
-          l *= alpha;
-          lr *= alpha;
-        }
-        // PV_t(j-1) must be complete before P_t is overwritten and O_t rescaled.
-        if (j > 0) {
-          if (wq == 0) FA_TRACE_POINT(53, n, t);
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarPVDone + t), (n - 1) & 1, wd));
-          if (wq == 0) FA_TRACE_POINT(54, n, t);
-          if (!ok) break;
-          tc_fence_after();
-        }
-        const float m_use = (m_ref == -INFINITY) ? 0.0f : m_ref;
-        const float2 c2 = make_float2(c, c), nm2 = make_float2(-m_use, -m_use);
-        float2 accr[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-        float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                         make_float2(0.f, 0.f)};
-        // dropout: this row's four words for the current 16 keys (byte b of word m is key
-        // 4m + b of the group)
-        [[maybe_unused]] uint32_t zw[4] = {0u, 0u, 0u, 0u};
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            const float2 x = ffma2(make_float2(__uint_as_float(s[cc][2 * k]),
-                                               __uint_as_float(s[cc][2 * k + 1])), c2, nm2);
-            float2 pe;
-            constexpr int kPoly = C::kPolyPeriod;
-            if (kPoly > 0 && k % (kPoly > 0 ? kPoly : 1) == kPoly - 1) {
-              pe = exp2_poly2(x);  // a share of the exponentials on the FMA pipe
-            } else {
-              pe = make_float2(ex2_approx(x.x), ex2_approx(x.y));
-            }
-            acc[k & 3] = fadd2(acc[k & 3], pe);  // l is the sum before dropout
-            if constexpr (kDropout) {
-              // One block covers 4 rows x 4 keys; the lanes of rows 4g..4g+3 share its
-              // counter. Every 16 keys, lane u (row mod 4) draws the block of keys
-              // 4u..4u+3 of the 16, and a 4 x 4 transpose across the four lanes hands
-              // each lane its own row's word of all four blocks.
-              if ((k & 7) == 0) {
-                const int u = lane & 3;
-                const uint4 w = philox4x32_10(
-                    make_uint4(static_cast<uint32_t>(((kv0 + 32 * cc + 2 * k) >> 2) + u),
-                               static_cast<uint32_t>(row >> 2), static_cast<uint32_t>(bh),
-                               p.drop.offset),
-                    p.drop.seed_lo, p.drop.seed_hi);
-                zw[0] = w.x;
-                zw[1] = w.y;
-                zw[2] = w.z;
-                zw[3] = w.w;
-                transpose4_lanes(zw, u);
-              }
-              // keys 2k, 2k + 1 of the chunk = keys 2(k mod 8), +1 of the group: word
-              // (k mod 8) / 2, bytes 2(k mod 2) and 2(k mod 2) + 1
-              const uint32_t wd = zw[(k & 7) >> 1] >> (16 * (k & 1));
-              pe.x = ((wd & 0xffu) >= p.drop.threshold) ? pe.x * p.drop.scale : 0.0f;
-              pe.y = (((wd >> 8) & 0xffu) >= p.drop.threshold) ? pe.y * p.drop.scale : 0.0f;
-            }
-            pk[k] = pack2<E>(pe.x, pe.y);
-            if constexpr (!kDropout) accr[k & 1] = fadd2(accr[k & 1], unpack2<E>(pk[k]));
-          }
-          // keys 32cc..32cc+31 = 16-byte units 4cc..4cc+3 of this row's 256 bytes:
-          // chunk (cc / 2), units (cc % 2) * 4 + u, 128-byte swizzle by the row
-          uint8_t* chunk = p_row + (cc >> 1) * C::kChunkBytes;
-#pragma unroll
-          for (int u = 0; u < 4; ++u)
-            *reinterpret_cast<uint4*>(chunk + ((((cc & 1) * 4 + u) ^ (row_in_tile & 7)) * 16)) =
-                make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
-        }
-        l += (acc[0].x + acc[0].y) + (acc[1].x + acc[1].y) + (acc[2].x + acc[2].y) +
-             (acc[3].x + acc[3].y);
-        lr += (accr[0].x + accr[0].y) + (accr[1].x + accr[1].y);
-        if (move && j > 0) {
-          // bring the sum up to key tile j-1 to the new reference max before PV_t(j)
-#pragma unroll
-          for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t o[32];
-            tmem_ld32(tm_o + cc * 32, o);
-            tmem_wait_ld();
-#pragma unroll
-            for (int k = 0; k < 32; ++k) o[k] = __float_as_uint(__uint_as_float(o[k]) * alpha);
-            tmem_st32(tm_o + cc * 32, o);
-          }
-          tmem_wait_st();
-        }
-        fence_proxy_async_smem();  // P (generic stores) before the MMA reads it
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(bar(C::kBarPFull + t));
-        if (wq == 0) FA_TRACE_POINT(55, n, t);
       }
       if (!ok) break;
       if (t_nk > 0) {
