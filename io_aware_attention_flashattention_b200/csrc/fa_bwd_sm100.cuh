@@ -123,6 +123,11 @@ struct Params {
   int split_num;
   float* part;         // [n_split][2 segments][dK, dV][128 key rows][D] fp32
   unsigned* arrivals;  // [n_split] (zeroed by the preprocess)
+  // Grid order of the key tiles: head-major (0: the CTAs resident at one time share one
+  // or two heads' Q, dO and dQ accumulator in L2) or rank-major (1: every head's key tile
+  // 0, then every head's key tile 1, ...; for causal or windowed launches without splits
+  // whose Q, dO and dQ accumulator all fit in L2, so that the heaviest tiles start first).
+  int rank_major;
 };
 
 // The first segment's step count for a tile of `steps` steps.
@@ -310,8 +315,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool big_first = p.split_num < 8;        // segment 1 is the larger one
     seg = (second_half == big_first) ? 0 : 1;
   }
-  const int bh = tile / n_kt;
-  const int j = tile % n_kt;
+  const int bh = p.rank_major ? tile % p.BH : tile / n_kt;
+  const int j = p.rank_major ? tile / p.BH : tile % n_kt;
   const int k0 = j * BN;
   const int n_q = (p.N + BM - 1) / BM;
   // query tiles [i_lo, i_hi) hold every query that may see a key of this tile
