@@ -353,15 +353,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   // go first. Single-tile CTAs, on the lightest tiles, come after all pairs.
   int bh, qt0;
   bool own1;  // does this CTA own query tile 1 (qt0 + 1)?
+  // (weight_major: rank-major instead, every head's heaviest pair first)
   if (static_cast<int>(blockIdx.x) < p.n_pair_items) {
     const int c = static_cast<int>(blockIdx.x);
-    bh = c / p.pairs_ph;
-    qt0 = p.singles_ph + 2 * (p.pairs_ph - 1 - c % p.pairs_ph);
+    const int r = p.weight_major ? c / p.BH : c % p.pairs_ph;
+    bh = p.weight_major ? c % p.BH : c / p.pairs_ph;
+    qt0 = p.singles_ph + 2 * (p.pairs_ph - 1 - r);
     own1 = true;
   } else {
     const int c = static_cast<int>(blockIdx.x) - p.n_pair_items;
-    bh = c / p.singles_ph;
-    qt0 = p.singles_ph - 1 - c % p.singles_ph;
+    const int r = p.weight_major ? c / p.BH : c % p.singles_ph;
+    bh = p.weight_major ? c % p.BH : c / p.singles_ph;
+    qt0 = p.singles_ph - 1 - r;
     own1 = false;
   }
   const int q0 = qt0 * BM;
