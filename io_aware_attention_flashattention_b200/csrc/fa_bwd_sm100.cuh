@@ -86,7 +86,9 @@ struct Cfg {
   static constexpr int kBarDKDV = kBarDQEmpty + 2;
   static constexpr int kBarSplitWritten = kBarDKDV + 1;        // split tile: 8 warps' rows written
   static constexpr int kBarSplitDecided = kBarSplitWritten + 1;  // ... and the arrival counted
-  static constexpr int kBarDrain = kBarSplitDecided + 1;
+  static constexpr int kBarKVEmpty = kBarSplitDecided + 1;  // persistent: item's K/V read
+  static constexpr int kBarDKDVFree = kBarKVEmpty + 1;      // persistent: dK/dV read out
+  static constexpr int kBarDrain = kBarDKDVFree + 1;
   static constexpr int kNumBars = kBarDrain + 1;
   static constexpr int kMiscOff = kBarOff + kNumBars * 8;
   static constexpr int kMaskOff = kMiscOff + 16;  // block-mask column of this key tile, as bits
@@ -271,6 +273,91 @@ __global__ void __launch_bounds__(256)
     out.x = pack2<E>(v.x * scale, v.y * scale);
     out.y = pack2<E>(v.z * scale, v.w * scale);
     reinterpret_cast<uint2*>(dQ)[k] = out;
+  }
+}
+
+// P^T and dS^T of one half step for one key row (this thread, TMEM lane krow): from
+// S^T and dP^T in TMEM, P = 2^(S c - L2) and dS = P o (dP - D) (with dropout: P o Z s
+// for dV and P o (dP o Z s - D) for dS), both back to TMEM as 16-bit pairs over the
+// columns they came from, and dS also into the swizzled shared chunk (the dQ operand).
+// kM: test each query against the key's visible range [q_lo, q_hi): query qh0 + x is
+// visible iff qoff + x < q_span (unsigned).
+template <Elt E, bool kDropout, bool kM>
+__device__ __forceinline__ void p_ds_half(uint32_t tm_s, uint32_t tm_dp, const float4* Lv,
+                                          const float4* Dv4, float c, int key, int qh0, int bh,
+                                          const DropoutParams& drop, int lane, int qoff,
+                                          unsigned q_span, uint8_t* ds_row, int krow) {
+  uint32_t sv[2][16], dv[2][16];
+  tmem_ld16(tm_s, sv[0]);
+  tmem_ld16(tm_dp, dv[0]);
+  tmem_wait_ld();
+#pragma unroll
+  for (int cc = 0; cc < 4; ++cc) {
+    const int cur = cc & 1;
+    if (cc + 1 < 4) {  // the next chunk's loads overlap this chunk's arithmetic
+      tmem_ld16(tm_s + 16 * (cc + 1), sv[cur ^ 1]);
+      tmem_ld16(tm_dp + 16 * (cc + 1), dv[cur ^ 1]);
+    }
+    // Dropout bytes of this key for the chunk's 16 queries: byte e of zq[v] is
+    // query 16cc + 4v + e of the half. One block covers 4 queries x 4 keys, and
+    // the lanes of keys 4g..4g+3 share its counter: lane u draws the block of the
+    // query group (qh0 + 16cc) / 4 + u, regroups its bytes by key (zq[b] = byte b
+    // of words 0..3) and a 4 x 4 transpose across the four lanes hands each lane
+    // its own key's bytes of all four blocks.
+    [[maybe_unused]] uint32_t zq[4] = {0u, 0u, 0u, 0u};
+    if constexpr (kDropout) {
+      const int u = lane & 3;
+      const uint4 w = philox4x32_10(
+          make_uint4(static_cast<uint32_t>(key >> 2),
+                     static_cast<uint32_t>(((qh0 + cc * 16) >> 2) + u),
+                     static_cast<uint32_t>(bh), drop.offset),
+          drop.seed_lo, drop.seed_hi);
+      const uint32_t t0 = __byte_perm(w.x, w.y, 0x5140), t1 = __byte_perm(w.x, w.y, 0x7362);
+      const uint32_t t2 = __byte_perm(w.z, w.w, 0x5140), t3 = __byte_perm(w.z, w.w, 0x7362);
+      zq[0] = __byte_perm(t0, t2, 0x5410);
+      zq[1] = __byte_perm(t0, t2, 0x7632);
+      zq[2] = __byte_perm(t1, t3, 0x5410);
+      zq[3] = __byte_perm(t1, t3, 0x7632);
+      transpose4_lanes(zq, u);
+    }
+    uint32_t pk[8], dk[8];
+#pragma unroll
+    for (int v = 0; v < 4; ++v) {
+      const float4 L4 = Lv[cc * 4 + v];
+      const float4 D4 = Dv4[cc * 4 + v];
+      const float Ls[4] = {L4.x, L4.y, L4.z, L4.w};
+      const float Ds[4] = {D4.x, D4.y, D4.z, D4.w};
+      float pv[4], dsv[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int k = 4 * v + e;
+        float pe = ex2_approx(fmaf(__uint_as_float(sv[cur][k]), c, -Ls[e]));
+        if (kM && static_cast<unsigned>(qoff + cc * 16 + k) >= q_span) pe = 0.f;
+        if constexpr (kDropout) {
+          // dV takes P o Z * scale and dS = P o (dP o Z * scale - D), with
+          // scale = 1 / (1 - threshold / 256)
+          const float zs =
+              (((zq[v] >> (8 * e)) & 0xffu) >= drop.threshold) ? drop.scale : 0.0f;
+          pv[e] = pe * zs;
+          dsv[e] = pe * (__uint_as_float(dv[cur][k]) * zs - Ds[e]);
+        } else {
+          pv[e] = pe;
+          dsv[e] = pe * (__uint_as_float(dv[cur][k]) - Ds[e]);
+        }
+      }
+      pk[2 * v] = pack2<E>(pv[0], pv[1]);
+      pk[2 * v + 1] = pack2<E>(pv[2], pv[3]);
+      dk[2 * v] = pack2<E>(dsv[0], dsv[1]);
+      dk[2 * v + 1] = pack2<E>(dsv[2], dsv[3]);
+    }
+    tmem_st8(tm_s + 8 * cc, pk);
+    tmem_st8(tm_dp + 8 * cc, dk);
+    // dS into the swizzled shared chunk: 16 queries = 16-byte units 2cc, 2cc+1
+    *reinterpret_cast<uint4*>(ds_row + (((2 * cc) ^ (krow & 7)) * 16)) =
+        make_uint4(dk[0], dk[1], dk[2], dk[3]);
+    *reinterpret_cast<uint4*>(ds_row + (((2 * cc + 1) ^ (krow & 7)) * 16)) =
+        make_uint4(dk[4], dk[5], dk[6], dk[7]);
+    if (cc + 1 < 4) tmem_wait_ld();
   }
 }
 
@@ -557,85 +644,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int qoff = qh0 - q_lo;  // query qh0 + x is visible iff qoff + x < q_span (unsigned)
       // The element loop in two compiled forms: with the mask tests only on steps
       // that cross a mask edge, none on all the others.
-      auto p_ds = [&](auto masked) {
-        constexpr bool kM = decltype(masked)::value;
-        uint32_t sv[2][16], dv[2][16];
-        tmem_ld16(tm_s, sv[0]);
-        tmem_ld16(tm_dp, dv[0]);
-        tmem_wait_ld();
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          const int cur = cc & 1;
-          if (cc + 1 < 4) {  // the next chunk's loads overlap this chunk's arithmetic
-            tmem_ld16(tm_s + 16 * (cc + 1), sv[cur ^ 1]);
-            tmem_ld16(tm_dp + 16 * (cc + 1), dv[cur ^ 1]);
-          }
-          // Dropout bytes of this key for the chunk's 16 queries: byte e of zq[v] is
-          // query 16cc + 4v + e of the half. One block covers 4 queries x 4 keys, and
-          // the lanes of keys 4g..4g+3 share its counter: lane u draws the block of the
-          // query group (qh0 + 16cc) / 4 + u, regroups its bytes by key (zq[b] = byte b
-          // of words 0..3) and a 4 x 4 transpose across the four lanes hands each lane
-          // its own key's bytes of all four blocks.
-          [[maybe_unused]] uint32_t zq[4] = {0u, 0u, 0u, 0u};
-          if constexpr (kDropout) {
-            const int u = lane & 3;
-            const uint4 w = philox4x32_10(
-                make_uint4(static_cast<uint32_t>(key >> 2),
-                           static_cast<uint32_t>(((qh0 + cc * 16) >> 2) + u),
-                           static_cast<uint32_t>(bh), p.drop.offset),
-                p.drop.seed_lo, p.drop.seed_hi);
-            const uint32_t t0 = __byte_perm(w.x, w.y, 0x5140), t1 = __byte_perm(w.x, w.y, 0x7362);
-            const uint32_t t2 = __byte_perm(w.z, w.w, 0x5140), t3 = __byte_perm(w.z, w.w, 0x7362);
-            zq[0] = __byte_perm(t0, t2, 0x5410);
-            zq[1] = __byte_perm(t0, t2, 0x7632);
-            zq[2] = __byte_perm(t1, t3, 0x5410);
-            zq[3] = __byte_perm(t1, t3, 0x7632);
-            transpose4_lanes(zq, u);
-          }
-          uint32_t pk[8], dk[8];
-#pragma unroll
-          for (int v = 0; v < 4; ++v) {
-            const float4 L4 = Lv[cc * 4 + v];
-            const float4 D4 = Dv4[cc * 4 + v];
-            const float Ls[4] = {L4.x, L4.y, L4.z, L4.w};
-            const float Ds[4] = {D4.x, D4.y, D4.z, D4.w};
-            float pv[4], dsv[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int k = 4 * v + e;
-              float pe = ex2_approx(fmaf(__uint_as_float(sv[cur][k]), c, -Ls[e]));
-              if (kM && static_cast<unsigned>(qoff + cc * 16 + k) >= q_span) pe = 0.f;
-              if constexpr (kDropout) {
-                // dV takes P o Z * scale and dS = P o (dP o Z * scale - D), with
-                // scale = 1 / (1 - threshold / 256)
-                const float zs =
-                    (((zq[v] >> (8 * e)) & 0xffu) >= p.drop.threshold) ? p.drop.scale : 0.0f;
-                pv[e] = pe * zs;
-                dsv[e] = pe * (__uint_as_float(dv[cur][k]) * zs - Ds[e]);
-              } else {
-                pv[e] = pe;
-                dsv[e] = pe * (__uint_as_float(dv[cur][k]) - Ds[e]);
-              }
-            }
-            pk[2 * v] = pack2<E>(pv[0], pv[1]);
-            pk[2 * v + 1] = pack2<E>(pv[2], pv[3]);
-            dk[2 * v] = pack2<E>(dsv[0], dsv[1]);
-            dk[2 * v + 1] = pack2<E>(dsv[2], dsv[3]);
-          }
-          tmem_st8(tm_s + 8 * cc, pk);
-          tmem_st8(tm_dp + 8 * cc, dk);
-          // dS into the swizzled shared chunk: 16 queries = 16-byte units 2cc, 2cc+1
-          *reinterpret_cast<uint4*>(ds_row + (((2 * cc) ^ (krow & 7)) * 16)) =
-              make_uint4(dk[0], dk[1], dk[2], dk[3]);
-          *reinterpret_cast<uint4*>(ds_row + (((2 * cc + 1) ^ (krow & 7)) * 16)) =
-              make_uint4(dk[4], dk[5], dk[6], dk[7]);
-          if (cc + 1 < 4) tmem_wait_ld();
-        }
-      };
       if (mask)
-        p_ds(std::true_type{});
+        p_ds_half<E, kDropout, true>(tm_s, tm_dp, Lv, Dv4, c, key, qh0, bh, p.drop, lane, qoff,
+                                     q_span, ds_row, krow);
       else
-        p_ds(std::false_type{});
+        p_ds_half<E, kDropout, false>(tm_s, tm_dp, Lv, Dv4, c, key, qh0, bh, p.drop, lane, qoff,
+                                      q_span, ds_row, krow);
       tmem_wait_st();
       fence_proxy_async_smem();
       tc_fence_before();
@@ -732,6 +746,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+    if (threadIdx.x == 0) FA_TRACE_CTA(5);
   } else if (warp < kWarpTma) {
     // ------------------------------------------------------------ dQ readout
     const int wq = warp - kWarpDq;
@@ -787,6 +802,412 @@ __global__ void __launch_bounds__(kThreads, 1)
                        __uint_as_float(v[k / 8][(4 * k + 3) % 32]));
         }
       }
+    }
+    if (warp == kWarpDq && lane == 0) FA_TRACE_CTA(6);
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (threadIdx.x == 0) FA_TRACE_CTA(4);
+  if (warp == kWarpMma) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmCols);
+  }
+}
+
+// The persistent form of fa_bwd_kernel, for launches of many short key tiles:
+// min(tiles, SMs) CTAs, each walking a list of key tiles (items) and reusing its
+// buffers from one to the next: K/V once the item's last product has read them
+// (KVEmpty), dK/dV in TMEM once the epilogue has read them out (DKDVFree). Ring
+// indices and barrier phases run on across items, so the next item's first products
+// start while the P/dS warps write the last item's dK, dV and the dQ warps add its
+// last dQ. The same roles, products and arithmetic; no split tiles and no block mask.
+template <int D, Elt E, bool kMasked, bool kDropout>
+__global__ void __launch_bounds__(kThreads, 1)
+    fa_bwd_persistent_kernel(const __grid_constant__ CUtensorMap tmQ,
+                             const __grid_constant__ CUtensorMap tmK,
+                             const __grid_constant__ CUtensorMap tmV,
+                             const __grid_constant__ CUtensorMap tmdO, const Params p) {
+  using C = Cfg<D>;
+  if (threadIdx.x == 0) FA_TRACE_CTA(0);
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* base_ptr = smem_raw + (base - raw);
+  const uint32_t bars = base + C::kBarOff;
+  auto bar = [&](int i) -> uint32_t { return bars + 8u * static_cast<uint32_t>(i); };
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + C::kMiscOff);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(base_ptr + C::kMiscOff + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int wl = kMasked ? p.wl : -1;
+  const int wr = p.wr;
+  const int n_kt = p.Npad / BN;
+  const int n_tiles = p.BH * n_kt;
+  const int n_q = (p.N + BM - 1) / BM;
+
+  // Items: key tile i of the list (head-major or rank-major, as p.rank_major says); the
+  // k-th item of CTA b is k * G + b for even k and k * G + (G - 1 - b) for odd k.
+  auto item_of = [&](int k) -> int {
+    const int G = static_cast<int>(gridDim.x), b = static_cast<int>(blockIdx.x);
+    const int i = k * G + ((k & 1) ? (G - 1 - b) : b);
+    return i < n_tiles ? i : -1;
+  };
+  // An item's (batch, head), key tile and the query tiles [i_lo, i_hi) it walks.
+  struct Work {
+    int bh, j, k0, i_lo, i_hi;
+  };
+  auto decode = [&](int tile, Work& w) {
+    w.bh = p.rank_major ? tile % p.BH : tile / n_kt;
+    w.j = p.rank_major ? tile / p.BH : tile % n_kt;
+    w.k0 = w.j * BN;
+    const int k1 = min(w.k0 + BN, p.N) - 1;
+    w.i_lo = (wr < 0) ? 0 : max(0, w.k0 - wr) / BM;
+    w.i_hi = (wl < 0) ? n_q : min(n_q, (k1 + wl) / BM + 1);
+  };
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(C::kBarKV), 1);
+    mbar_init(bar(C::kBarKVEmpty), 1);
+    for (int s = 0; s < C::kSlots; ++s) {
+      mbar_init(bar(C::kBarFull + s), 1);
+      mbar_init(bar(C::kBarEmpty + s), 1);
+    }
+    for (int h = 0; h < 2; ++h) {
+      mbar_init(bar(C::kBarS + h), 1);
+      mbar_init(bar(C::kBarP + h), 4);        // the 4 warps of half h
+      mbar_init(bar(C::kBarDQFull + h), 1);
+      mbar_init(bar(C::kBarDQEmpty + h), 4);  // the 4 dQ warps
+    }
+    mbar_init(bar(C::kBarDKDV), 1);
+    mbar_init(bar(C::kBarDKDVFree), 8);  // the 8 P/dS warps
+    mbar_init(bar(C::kBarDrain), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == kWarpMma) {
+    tmem_alloc(smem_u32(tmem_slot), C::kTmCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const Watchdog wd{abort_flag, p.timeout_ns};
+  if (threadIdx.x == 0) FA_TRACE_CTA(1);
+
+  // ring of half tiles: seq = 4 * step + 2 * h + w over all the CTA's steps, w = 0 for
+  // dO (rows 64h.. of query tile i), w = 1 for Q (with L2 and D of those 64 queries)
+  auto seq_of = [](int s, int h, int w) { return 4 * s + 2 * h + w; };
+  auto slot_of = [&](int seq) { return seq % C::kSlots; };
+  auto round_of = [&](int seq) { return seq / C::kSlots; };
+  auto slot_smem = [&](int seq) -> uint32_t {
+    return base + C::kRingOff + slot_of(seq) * C::kHalfBytes;
+  };
+
+  if (warp == kWarpTma) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmdO);
+    }
+    int issued = 0;  // ring sequence numbers issued
+    int n_kv = 0;    // K/V loads so far (items with steps)
+    int s0 = 0;      // steps of the items before
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int item = item_of(k);
+      if (item < 0) break;
+      Work w;
+      decode(item, w);
+      const int nsteps = w.i_hi - w.i_lo;
+      if (nsteps == 0) continue;
+      // the previous item's products must be done with K and V
+      if (n_kv > 0 && !mbar_wait_warp(bar(C::kBarKVEmpty), (n_kv - 1) & 1, wd)) {
+        ok = false;
+        break;
+      }
+      mbar_arrive_expect_tx_e(bar(C::kBarKV), 2 * C::kTileBytes);
+      for (int c = 0; c < C::kChunks; ++c) {
+        tma_load_3d_e(base + C::kKOff + c * C::kChunkBytes, &tmK, bar(C::kBarKV), c * 64, w.k0,
+                      w.bh);
+        tma_load_3d_e(base + C::kVOff + c * C::kChunkBytes, &tmV, bar(C::kBarKV), c * 64, w.k0,
+                      w.bh);
+      }
+      ++n_kv;
+      for (int s = 0; s < nsteps && ok; ++s) {
+        const int i = w.i_lo + s;
+        for (int hw = 0; hw < 4 && ok; ++hw) {
+          const int h = hw >> 1, wv = hw & 1;
+          const int seq = seq_of(s0 + s, h, wv);
+          const int slot = slot_of(seq);
+          const int rnd = round_of(seq);
+          if (rnd > 0 && !mbar_wait_warp(bar(C::kBarEmpty + slot), (rnd - 1) & 1, wd)) {
+            ok = false;
+            break;
+          }
+          const uint32_t full = bar(C::kBarFull + slot);
+          const uint32_t dst = slot_smem(seq);
+          const int row0 = i * BM + 64 * h;
+          if (wv == 1) {
+            mbar_arrive_expect_tx_e(full, C::kHalfBytes + 2 * C::kVecBytes);
+            const uint32_t vec = base + C::kVecOff + slot * 2 * C::kVecBytes;
+            const size_t off = static_cast<size_t>(w.bh) * p.Npad + static_cast<size_t>(row0);
+            bulk_load_e(vec, p.L2 + off, C::kVecBytes, full);
+            bulk_load_e(vec + C::kVecBytes, p.Dv + off, C::kVecBytes, full);
+          } else {
+            mbar_arrive_expect_tx_e(full, C::kHalfBytes);
+          }
+          for (int c = 0; c < C::kChunks; ++c)
+            tma_load_3d_e(dst + c * C::kHalfChunkBytes, wv ? &tmQ : &tmdO, full, c * 64, row0,
+                          w.bh);
+          issued = seq + 1;
+        }
+      }
+      s0 += nsteps;
+    }
+    for (int seq = max(0, issued - C::kSlots); seq < issued; ++seq)
+      drain_wait(bar(C::kBarFull + slot_of(seq)), round_of(seq) & 1, p.timeout_ns);
+    if (n_kv > 0) drain_wait(bar(C::kBarKV), (n_kv - 1) & 1, p.timeout_ns);
+    __syncwarp();
+  } else if (warp == kWarpMma) {
+    // ------------------------------------------------------------ MMA issuer
+    const uint32_t k_smem = base + C::kKOff, v_smem = base + C::kVOff;
+    const uint32_t ds_smem = base + C::kDSOff;
+    const uint32_t tm_s = tmem + C::kTmS, tm_dp = tmem + C::kTmDP;
+    auto wait_full = [&](int seq) -> bool {
+      return mbar_wait_warp(bar(C::kBarFull + slot_of(seq)), round_of(seq) & 1, wd);
+    };
+    // S^T and dP^T of both halves of the CTA's step g (dP^T first: its columns free up
+    // earlier)
+    auto issue_sdp = [&](int g) -> bool {
+      for (int h = 0; h < 2; ++h) {
+        const int seqO = seq_of(g, h, 0), seqQ = seq_of(g, h, 1);
+        if (!(wait_full(seqO) && wait_full(seqQ))) return false;
+        tc_fence_after();
+        issue_xyT_half<D, E>(tm_dp + 64 * h, v_smem, slot_smem(seqO));
+        if (D == 128 && g > 0) {  // S^T_h shares columns with dQ^T_h of the step before
+          if (!mbar_wait_warp(bar(C::kBarDQEmpty + h), (g - 1) & 1, wd)) return false;
+          tc_fence_after();
+        }
+        issue_xyT_half<D, E>(tm_s + 64 * h, k_smem, slot_smem(seqQ));
+        tc_commit_e(bar(C::kBarS + h));
+      }
+      return true;
+    };
+    int n_kv = 0;  // items with steps so far
+    int g0 = 0;    // the CTA's step number of the item's first step
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int item = item_of(k);
+      if (item < 0) break;
+      Work w;
+      decode(item, w);
+      const int nsteps = w.i_hi - w.i_lo;
+      if (nsteps == 0) continue;
+      ok = mbar_wait_warp(bar(C::kBarKV), n_kv & 1, wd);
+      if (ok) ok = issue_sdp(g0);
+      for (int s = 0; s < nsteps && ok; ++s) {
+        const int g = g0 + s;
+        for (int h = 0; h < 2 && ok; ++h) {
+          const int seqO = seq_of(g, h, 0), seqQ = seq_of(g, h, 1);
+          if (!mbar_wait_warp(bar(C::kBarP + h), g & 1, wd)) { ok = false; break; }
+          // the item's first dV and dK overwrite the accumulators: the previous item's
+          // epilogue must have read them out
+          if (s == 0 && h == 0 && n_kv > 0 &&
+              !mbar_wait_warp(bar(C::kBarDKDVFree), (n_kv - 1) & 1, wd)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const bool acc = (s > 0) || (h > 0);
+          issue_acc_half<D, E>(tmem + C::kTmDV, tm_s + 64 * h, slot_smem(seqO), acc);   // dV
+          issue_acc_half<D, E>(tmem + C::kTmDK, tm_dp + 64 * h, slot_smem(seqQ), acc);  // dK
+          tc_commit_e(bar(C::kBarEmpty + slot_of(seqO)));
+          tc_commit_e(bar(C::kBarEmpty + slot_of(seqQ)));
+          if constexpr (D == 128) {
+            issue_dqT_half<E>(tm_s + 64 * h, k_smem, ds_smem + h * C::kChunkBytes);
+            tc_commit_e(bar(C::kBarDQFull + h));
+          }
+        }
+        if (!ok) break;
+        if constexpr (D == 64) {
+          if (g > 0) {  // the dQ columns are reused: the previous dQ must have been read
+            if (!mbar_wait_warp(bar(C::kBarDQEmpty), (g - 1) & 1, wd)) { ok = false; break; }
+            tc_fence_after();
+          }
+          issue_dq64<E>(tmem + C::kTmDQ64, ds_smem, k_smem);
+          tc_commit_e(bar(C::kBarDQFull));
+        }
+        if (s + 1 < nsteps) ok = issue_sdp(g + 1);
+      }
+      if (!ok) break;
+      tc_commit_e(bar(C::kBarDKDV));     // dK, dV complete
+      tc_commit_e(bar(C::kBarKVEmpty));  // K, V no longer read
+      ++n_kv;
+      g0 += nsteps;
+    }
+    tc_commit_e(bar(C::kBarDrain));
+    drain_wait(bar(C::kBarDrain), 0, p.timeout_ns);
+    __syncwarp();
+  } else if (warp < 8) {
+    // ------------------------------------------------------------ P^T, dS^T (key rows)
+    const int h = warp >> 2;                  // query half
+    const int krow = (warp & 3) * 32 + lane;  // key row within the tile = TMEM lane
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tm_s = tmem + lane_off + C::kTmS + 64 * h;
+    const uint32_t tm_dp = tmem + lane_off + C::kTmDP + 64 * h;
+    const float c = p.scale_log2;
+    uint8_t* ds_row = base_ptr + C::kDSOff + h * C::kChunkBytes + krow * 128;
+    const int dq_bar = (D == 128) ? C::kBarDQFull + h : C::kBarDQFull;
+    int n_kv = 0, g0 = 0;
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int item = item_of(k);
+      if (item < 0) break;
+      Work w;
+      decode(item, w);
+      const int nsteps = w.i_hi - w.i_lo;
+      const int key = w.k0 + krow;
+      uint16_t* out = (h == 0 ? p.dK : p.dV) + (static_cast<size_t>(w.bh) * p.N + key) * D;
+      if (nsteps == 0) {
+        // no query sees this key: dK = dV = 0 (warps 0-3 dK, warps 4-7 dV)
+        if (key < p.N) {
+          uint4* dst = reinterpret_cast<uint4*>(out);
+#pragma unroll
+          for (int u = 0; u < D / 8; ++u) dst[u] = make_uint4(0u, 0u, 0u, 0u);
+        }
+        continue;
+      }
+      const bool ragged_keys = w.k0 + BN > p.N;
+      // queries that see this key row: [q_lo, q_hi) (empty for a padding key)
+      const int q_lo = (wr < 0) ? 0 : key - wr;
+      const int q_hi = (key >= p.N) ? q_lo : ((wl < 0) ? p.Npad + BM : key + wl + 1);
+      const unsigned q_span = static_cast<unsigned>(q_hi - q_lo);
+      for (int s = 0; s < nsteps && ok; ++s) {
+        const int g = g0 + s;
+        const int qh0 = (w.i_lo + s) * BM + 64 * h;  // first query of this half
+        // the dQ product of the step before has read this dS chunk; L2 and D of this
+        // half arrived with its Q rows; then S^T and dP^T
+        if (g > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(dq_bar), (g - 1) & 1, wd));
+        const int seqQ = seq_of(g, h, 1);
+        if (ok)
+          ok = __all_sync(0xffffffffu,
+                          mbar_wait(bar(C::kBarFull + slot_of(seqQ)), round_of(seqQ) & 1, wd));
+        if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarS + h), g & 1, wd));
+        if (!ok) break;
+        tc_fence_after();
+        const float4* Lv = reinterpret_cast<const float4*>(
+            base_ptr + C::kVecOff + slot_of(seqQ) * 2 * C::kVecBytes);
+        const float4* Dv4 = Lv + 64 / 4;
+        const bool mask = ragged_keys || (wr >= 0 && w.k0 + BN - 1 - wr > qh0) ||
+                          (wl >= 0 && w.k0 + wl < qh0 + 63);
+        const int qoff = qh0 - q_lo;
+        if (mask)
+          p_ds_half<E, kDropout, true>(tm_s, tm_dp, Lv, Dv4, c, key, qh0, w.bh, p.drop, lane,
+                                       qoff, q_span, ds_row, krow);
+        else
+          p_ds_half<E, kDropout, false>(tm_s, tm_dp, Lv, Dv4, c, key, qh0, w.bh, p.drop, lane,
+                                        qoff, q_span, ds_row, krow);
+        tmem_wait_st();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(bar(C::kBarP + h));
+      }
+      if (!ok) break;
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarDKDV), n_kv & 1, wd));
+      if (!ok) break;
+      // warps 0-3 write dK (times scale), warps 4-7 write dV
+      tc_fence_after();
+      const uint32_t tm_acc = tmem + lane_off + (h == 0 ? C::kTmDK : C::kTmDV);
+      const float mul = (h == 0) ? p.scale : 1.0f;
+#pragma unroll 1
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t v[32];
+        tmem_ld32(tm_acc + cc * 32, v);
+        tmem_wait_ld();
+        uint32_t pk[16];
+#pragma unroll
+        for (int kk = 0; kk < 16; ++kk)
+          pk[kk] = pack2<E>(__uint_as_float(v[2 * kk]) * mul, __uint_as_float(v[2 * kk + 1]) * mul);
+        if (key < p.N) {
+          uint4* dst = reinterpret_cast<uint4*>(out + cc * 32);
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            dst[u] = make_uint4(pk[4 * u], pk[4 * u + 1], pk[4 * u + 2], pk[4 * u + 3]);
+        }
+      }
+      // dK and dV are out of TMEM: the next item's first products may overwrite them
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(bar(C::kBarDKDVFree));
+      ++n_kv;
+      g0 += nsteps;
+    }
+  } else if (warp < kWarpTma) {
+    // ------------------------------------------------------------ dQ readout
+    const int wq = warp - kWarpDq;
+    const uint32_t lane_off = static_cast<uint32_t>(wq * 32) << 16;
+    const int row = wq * 32 + lane;  // TMEM lane: head-dim element (D = 128) or query (D = 64)
+    int g0 = 0;
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int item = item_of(k);
+      if (item < 0) break;
+      Work w;
+      decode(item, w);
+      const int nsteps = w.i_hi - w.i_lo;
+      for (int s = 0; s < nsteps && ok; ++s) {
+        const int g = g0 + s;
+        const int q0 = (w.i_lo + s) * BM;
+        if constexpr (D == 128) {
+          for (int h = 0; h < 2 && ok; ++h) {
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarDQFull + h), g & 1, wd));
+            if (!ok) break;
+            tc_fence_after();
+            uint32_t v[2][32];
+            tmem_ld32(tmem + lane_off + C::kTmS + 64 * h, v[0]);
+            tmem_ld32(tmem + lane_off + C::kTmS + 64 * h + 32, v[1]);
+            tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar(C::kBarDQEmpty + h));
+            // element `row` of the head dimension for 64 queries: a warp covers 32
+            // consecutive elements of one query row (128 contiguous bytes) per add
+            float* dst = p.dQacc + (static_cast<size_t>(w.bh) * p.N + q0 + 64 * h) * D + row;
+            const int nq = min(64, p.N - (q0 + 64 * h));
+#pragma unroll
+            for (int qq = 0; qq < 64; ++qq)
+              if (qq < nq) red_add(dst + static_cast<size_t>(qq) * D, __uint_as_float(v[qq / 32][qq % 32]));
+          }
+        } else {
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(C::kBarDQFull), g & 1, wd));
+          if (!ok) break;
+          tc_fence_after();
+          uint32_t v[2][32];
+          tmem_ld32(tmem + lane_off + C::kTmDQ64, v[0]);
+          tmem_ld32(tmem + lane_off + C::kTmDQ64 + 32, v[1]);
+          tmem_wait_ld();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(bar(C::kBarDQEmpty));
+          const int q = q0 + row;
+          if (q < p.N) {
+            float* dst = p.dQacc + (static_cast<size_t>(w.bh) * p.N + q) * D;
+#pragma unroll
+            for (int kk = 0; kk < 16; ++kk)
+              red_add_v4(dst + 4 * kk, __uint_as_float(v[kk / 8][(4 * kk) % 32]),
+                         __uint_as_float(v[kk / 8][(4 * kk + 1) % 32]),
+                         __uint_as_float(v[kk / 8][(4 * kk + 2) % 32]),
+                         __uint_as_float(v[kk / 8][(4 * kk + 3) % 32]));
+          }
+        }
+      }
+      g0 += nsteps;
     }
   }
 

@@ -153,6 +153,8 @@ cudaError_t set_smem_d() {
   e = e ? e : set_smem(fwd::fa_fwd_persistent_kernel<D, E, true, false>, S);
   e = e ? e : set_smem(bwd::fa_bwd_kernel<D, E, false>, bwd::Cfg<D>::kSmemBytes);
   e = e ? e : set_smem(bwd::fa_bwd_kernel<D, E, true>, bwd::Cfg<D>::kSmemBytes);
+  e = e ? e : set_smem(bwd::fa_bwd_persistent_kernel<D, E, false, false>, bwd::Cfg<D>::kSmemBytes);
+  e = e ? e : set_smem(bwd::fa_bwd_persistent_kernel<D, E, true, false>, bwd::Cfg<D>::kSmemBytes);
   return e;
 }
 
@@ -167,6 +169,8 @@ cudaError_t set_smem_all() {
     e = e ? e : set_smem(fwd::fa_fwd_persistent_kernel<128, E, true, true>, fwd::Cfg<128>::kSmemBytes);
     e = e ? e : set_smem(bwd::fa_bwd_kernel<64, E, true, true>, bwd::Cfg<64>::kSmemBytes);
     e = e ? e : set_smem(bwd::fa_bwd_kernel<128, E, true, true>, bwd::Cfg<128>::kSmemBytes);
+    e = e ? e : set_smem(bwd::fa_bwd_persistent_kernel<64, E, true, true>, bwd::Cfg<64>::kSmemBytes);
+    e = e ? e : set_smem(bwd::fa_bwd_persistent_kernel<128, E, true, true>, bwd::Cfg<128>::kSmemBytes);
   }
   return e;
 }
@@ -721,6 +725,36 @@ fa_status preprocess_impl(const void* O, const void* dO, const float* LSE, int B
                 pl.dQacc, N, pl.Npad, rows, pl.arrivals, pl.n_arrivals);
 }
 
+template <Elt E, bool kMasked, bool kDropout, bool kPersistent>
+fa_status launch_bwd(int d, dim3 grid, cudaStream_t s, const CUtensorMap& mq, const CUtensorMap& mk,
+                     const CUtensorMap& mv, const CUtensorMap& mdo, const bwd::Params& p) {
+  constexpr int T = bwd::kThreads;
+  constexpr size_t S64 = bwd::Cfg<64>::kSmemBytes, S128 = bwd::Cfg<128>::kSmemBytes;
+  if constexpr (kPersistent) {
+    if (d == 64)
+      return launch(bwd::fa_bwd_persistent_kernel<64, E, kMasked, kDropout>, grid, T, S64, s, mq,
+                    mk, mv, mdo, p);
+    return launch(bwd::fa_bwd_persistent_kernel<128, E, kMasked, kDropout>, grid, T, S128, s, mq,
+                  mk, mv, mdo, p);
+  } else {
+    if (d == 64)
+      return launch(bwd::fa_bwd_kernel<64, E, kMasked, kDropout>, grid, T, S64, s, mq, mk, mv, mdo,
+                    p);
+    return launch(bwd::fa_bwd_kernel<128, E, kMasked, kDropout>, grid, T, S128, s, mq, mk, mv, mdo,
+                  p);
+  }
+}
+
+// The persistent backward (fa_bwd_persistent_kernel) runs for every launch of more key
+// tiles than SMs without a split tile or a block mask. Measured on a B200 (backward,
+// persistent against one CTA per tile): B8 H12 N1024 causal d64 240 -> 252, d128
+// 391 -> 428, B4 H16 N2048 d64 causal 341 -> 355, B1 H8 N4096 739 -> 746, B1 H8 N16384
+// 880 -> 892 and causal unchanged; no shape measured slower.
+bool bwd_persistent(int BH, int N, const MaskSpec& mask, int n_split, int sms) {
+  const long long n_tiles = static_cast<long long>(BH) * ((N + 127) / 128);
+  return mask.blocks == nullptr && n_split == 0 && sms > 0 && n_tiles > sms;
+}
+
 template <Elt E>
 fa_status main_impl(const void* Q, const void* K, const void* V, const void* dO, void* dK,
                            void* dV, int B, int H, int N, int d, float scale, int causal,
@@ -762,8 +796,8 @@ fa_status main_impl(const void* Q, const void* K, const void* V, const void* dO,
   p.part = pl.part;
   p.arrivals = pl.arrivals;
   // rank-major order for causal or windowed launches of more than one wave of key tiles
-  // whose Q, dO (16-bit) and fp32 dQ accumulator total at most 256 MiB: the one-CTA-per-
-  // tile launch then starts every head's heaviest tiles first. Measured on a B200
+  // whose Q, dO (16-bit) and fp32 dQ accumulator total at most 256 MiB: every head's
+  // heaviest key tiles then start first. Measured on a B200 with one CTA per tile
   // (backward, rank-major against head-major): B8 H12 N1024 d64 causal +8%, B8 H12 N1024
   // d128 +6%, B4 H12 N2048 +12%, B2 H16 N4096 +11%, B1 H8 N16384 (128 MiB) +3.5%, B2 H16
   // N8192 (256 MiB) +5%; B4 H16 N8192 (512 MiB, four times the L2) -5%.
@@ -773,25 +807,24 @@ fa_status main_impl(const void* Q, const void* K, const void* V, const void* dO,
                          static_cast<double>(pl.BH) * N * d * 8.0 <= kBwdRankMajorBytes
                      ? 1
                      : 0;
-  const dim3 grid(static_cast<unsigned>(pl.Npad / bwd::BN) * pl.BH + p.n_split);
+  const int sms = device_sms();
+  const bool pers = bwd_persistent(pl.BH, N, mask, p.n_split, sms);
+  const dim3 grid(pers ? static_cast<unsigned>(std::min<long long>(n_tiles, sms))
+                       : static_cast<unsigned>(n_tiles + p.n_split));
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const bool g = mask.general();
-  using bwd::Cfg;
-  constexpr int T = bwd::kThreads;
-  constexpr size_t S64 = Cfg<64>::kSmemBytes, S128 = Cfg<128>::kSmemBytes;
   if constexpr (E == Elt::BF16) {
     if (drop.on) {
-      if (d == 64)
-        return launch(bwd::fa_bwd_kernel<64, E, true, true>, grid, T, S64, s, mq, mk, mv, mdo, p);
-      return launch(bwd::fa_bwd_kernel<128, E, true, true>, grid, T, S128, s, mq, mk, mv, mdo, p);
+      if (pers) return launch_bwd<E, true, true, true>(d, grid, s, mq, mk, mv, mdo, p);
+      return launch_bwd<E, true, true, false>(d, grid, s, mq, mk, mv, mdo, p);
     }
   } else if (drop.on) {
     return FA_ERR_UNSUPPORTED;
   }
-  if (d == 64 && !g) return launch(bwd::fa_bwd_kernel<64, E, false>, grid, T, S64, s, mq, mk, mv, mdo, p);
-  if (d == 64) return launch(bwd::fa_bwd_kernel<64, E, true>, grid, T, S64, s, mq, mk, mv, mdo, p);
-  if (!g) return launch(bwd::fa_bwd_kernel<128, E, false>, grid, T, S128, s, mq, mk, mv, mdo, p);
-  return launch(bwd::fa_bwd_kernel<128, E, true>, grid, T, S128, s, mq, mk, mv, mdo, p);
+  if (g && pers) return launch_bwd<E, true, false, true>(d, grid, s, mq, mk, mv, mdo, p);
+  if (g) return launch_bwd<E, true, false, false>(d, grid, s, mq, mk, mv, mdo, p);
+  if (pers) return launch_bwd<E, false, false, true>(d, grid, s, mq, mk, mv, mdo, p);
+  return launch_bwd<E, false, false, false>(d, grid, s, mq, mk, mv, mdo, p);
 }
 
 template <Elt E>

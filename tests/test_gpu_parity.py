@@ -202,7 +202,9 @@ def test_f16_small_full_parity(B, H, N, d, causal):
 
 # Launches of more items than SMs whose items average few key tiles run the
 # persistent forward: each CTA walks several items, reusing its Q, S, P and O
-# buffers (and the K/V rings) from one item to the next.
+# buffers (and the K/V rings) from one item to the next. Their backward, with more
+# key tiles than SMs, runs the persistent backward the same way (K/V, dK/dV in TMEM,
+# the Q/dO ring).
 PERSISTENT = [
     # (B, H, N, d, causal, dtype)
     (4, 16, 1024, 64, True, torch.bfloat16),    # 256 pair items, 1 to 8 key tiles each
