@@ -506,7 +506,11 @@ def main():
     if not bf16:
         raise SystemExit("the benchmark times the bf16 tensor-core path")
 
-    names = ["fa_fwd_kernel", "fa_bwd_pre_kernel", "fa_bwd_kernel", "fa_bwd_dq_kernel"]
+    # the kernels this shape runs (one CTA per item or tile, or their persistent forms)
+    plan = api.fa_launch_plan(w.B, w.H, w.N, w.d, w.causal)
+    fwd_name = "fa_fwd_persistent_kernel" if plan["fwd_persistent"] else "fa_fwd_kernel"
+    bwd_name = "fa_bwd_persistent_kernel" if plan["bwd_persistent"] else "fa_bwd_kernel"
+    names = [fwd_name, "fa_bwd_pre_kernel", bwd_name, "fa_bwd_dq_kernel"]
     nev = len(names) + 1
 
     def step(ev=None):
@@ -573,12 +577,12 @@ def main():
     BH, N, d = w.B * w.H, w.N, w.d
     npad = (N + 127) // 128 * 128
     kern = {
-        "fa_fwd_kernel": {"flops": fwd_f, "bytes": 4 * BH * N * d * 2 + 4 * BH * N},
+        fwd_name: {"flops": fwd_f, "bytes": 4 * BH * N * d * 2 + 4 * BH * N},
         "fa_bwd_pre_kernel": {"bytes": 2 * BH * N * d * 2 + 4 * BH * N + 8 * BH * npad
                               + 4 * BH * N * d},
         # reads Q, K, V, dO and L2/D; writes dK, dV; read-modify-write of the fp32 dQ accumulator
-        "fa_bwd_kernel": {"flops": bwd_f, "bytes": 6 * BH * N * d * 2 + 8 * BH * npad
-                          + 2 * 4 * BH * N * d},
+        bwd_name: {"flops": bwd_f, "bytes": 6 * BH * N * d * 2 + 8 * BH * npad
+                   + 2 * 4 * BH * N * d},
         "fa_bwd_dq_kernel": {"bytes": 4 * BH * N * d + 2 * BH * N * d},
     }
     kernels = {}
@@ -695,7 +699,7 @@ def main():
         "ms_per_step": total_ms / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": workload_config(w, world),
-        "fwd_tflops": fwd_f / (kernels["fa_fwd_kernel"]["avg_ms"] * 1e-3) / 1e12,
+        "fwd_tflops": fwd_f / (kernels[names[0]]["avg_ms"] * 1e-3) / 1e12,
         "bwd_tflops": bwd_f / (sum(kernels[n]["avg_ms"] for n in names[1:]) * 1e-3) / 1e12,
         "frac_of_peak": {"fwd": None, "bwd": None, "peak_tflops": float(peaks["bf16_tflops"])},
         "roofline": roof,

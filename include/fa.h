@@ -229,6 +229,22 @@ fa_status fa_forward_dropout(const void* Q, const void* K, const void* V, void* 
                              int window_left, int window_right, const uint8_t* block_mask,
                              float p_drop, uint64_t seed, uint32_t offset, fa_stream_t stream);
 /*
+ * How the library distributes a plain call (no window, block mask or dropout) of this
+ * shape on the current GPU. A planning query: it launches nothing.
+ *   *fwd_persistent: 1 if fa_forward runs its persistent kernel (CTAs walking a list
+ *     of query-tile items), 0 if one CTA per item.
+ *   *bwd_persistent: 1 if the backward's main stage runs its persistent kernel (CTAs
+ *     walking a list of key tiles), 0 if one CTA per key tile.
+ *   *bwd_split: the number of key tiles the backward runs as two CTAs (0 when
+ *     persistent).
+ * Output pointers may be null. Returns FA_ERR_INVALID_ARG or FA_ERR_UNSUPPORTED for a
+ * shape the calls refuse, FA_ERR_CUDA without a usable sm_100 device.
+ */
+fa_status fa_launch_plan(int B, int H, int N, int d, int causal, int* fwd_persistent,
+                         int* bwd_persistent, int* bwd_split);
+
+/*
+ * The drop probability the dropout calls apply for `p_drop`:/*
  * The drop probability the dropout calls apply for `p_drop`: floor(256 p_drop) / 256
  * (for example 0.1 gives 25/256 = 0.09765625). Returns -1 for a p_drop those calls
  * refuse (outside [0, 1), NaN, or in (0, 1/256)). Host only; no CUDA call.

@@ -36,6 +36,7 @@ SIGNATURES = {
     "fa_backward_masked": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                 _i, _i, _i, _i, _f, _i, _i, _i, _vp, _vp, _sz, _vp]),
     "fa_dropout_rate": (_f, [_f]),
+    "fa_launch_plan": (_i, [_i, _i, _i, _i, _i, _vp, _vp, _vp]),
     "fa_forward_dropout": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _i, _i, _vp,
                                 _f, _u64, _u32, _vp]),
     "fa_backward_dropout": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,

@@ -29,6 +29,7 @@ __all__ = [
     "fa_backward_noalloc", "fa_forward_f16", "fa_backward_f16", "fa_forward_masked",
     "fa_backward_masked", "fa_forward_dropout", "fa_backward_dropout", "fa_forward_f32",
     "fa_backward_f32", "fa_get_status", "fa_watchdog_selftest", "fa_version", "fa_dropout_rate",
+    "fa_launch_plan",
     "forward", "backward", "attention", "FlashAttentionFunction",
 ]
 
@@ -158,6 +159,18 @@ def fa_backward_masked(Q, K, V, O, dO, LSE, dQ, dK, dV, scale: float, causal: bo
     check("fa_backward_masked", lib().fa_backward_masked(
         *ptrs, B, H, N, d, float(scale), int(bool(causal)), wl, wr, _block_mask(block_mask, N),
         ws, nbytes, _stream(stream)))
+
+
+def fa_launch_plan(B: int, H: int, N: int, d: int, causal: bool = False) -> dict:
+    """How a plain call of this shape is distributed on the current GPU (launches
+    nothing): ``fwd_persistent`` / ``bwd_persistent`` (persistent kernels, CTAs walking
+    a list of tiles) and ``bwd_split`` (key tiles run as two CTAs)."""
+    import ctypes
+    fp, bp, bs = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    check("fa_launch_plan", lib().fa_launch_plan(B, H, N, d, int(causal), ctypes.addressof(fp),
+                                                 ctypes.addressof(bp), ctypes.addressof(bs)))
+    return {"fwd_persistent": bool(fp.value), "bwd_persistent": bool(bp.value),
+            "bwd_split": bs.value}
 
 
 def fa_dropout_rate(p: float) -> float:

@@ -887,6 +887,30 @@ size_t fa_backward_workspace_size(int B, int H, int N, int d) {
   return backward_ws_bytes(bh, N, d, bwd_max_split(bh, N));
 }
 
+fa_status fa_launch_plan(int B, int H, int N, int d, int causal, int* fwd_persistent_out,
+                         int* bwd_persistent_out, int* bwd_split_out) {
+  fa_status st = check_shape(B, H, N, d, 1.0f, causal);
+  if (st != FA_OK) return st;
+  if ((st = prepare_device()) != FA_OK) return st;
+  const int BH = B * H, sms = device_sms();
+  int fp = 0, bp = 0, bs = 0;
+  if (N > 0) {
+    MaskSpec m;
+    if ((st = make_mask(N, causal, -1, -1, nullptr, &m)) != FA_OK) return st;
+    fp = fwd_split(BH, N, d, m.wl, m.wr, false, sms).persistent;
+    const long long smax = bwd_max_split(BH, N);
+    if (smax > 0) {
+      const BwdSplit sp = bwd_split(BH, N, m.wl < 0 && m.wr < 0, sms);
+      bs = static_cast<int>(std::min<long long>(sp.n_split, smax));
+    }
+    bp = bwd_persistent(BH, N, m, bs, sms) ? 1 : 0;
+  }
+  if (fwd_persistent_out) *fwd_persistent_out = fp;
+  if (bwd_persistent_out) *bwd_persistent_out = bp;
+  if (bwd_split_out) *bwd_split_out = bs;
+  return FA_OK;
+}
+
 float fa_dropout_rate(float p_drop) {
   const int t = drop_threshold(p_drop);
   if (t < 0 || (t == 0 && p_drop > 0.0f)) return -1.0f;

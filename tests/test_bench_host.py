@@ -60,7 +60,9 @@ def test_traffic_is_reported_only_for_the_profiled_sources(monkeypatch):
     path = os.path.join(bench.ROOT, "profiles", "traffic.json")
     with open(path) as f:
         table = json.load(f)
-    assert set(table) >= {"fa_fwd_kernel", "fa_bwd_kernel"}
+    # one forward and one backward main kernel (one-CTA or persistent form)
+    assert any(k.startswith("fa_fwd_") for k in table)
+    assert any(k.startswith("fa_bwd_") for k in table)
     for kernel, ent in table.items():
         assert ent["bytes_per_launch"] > 0 and len(ent["source_sha"]) == 16
         monkeypatch.setattr(bench, "kernel_source_sha", lambda: ent["source_sha"])

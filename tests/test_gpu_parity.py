@@ -475,3 +475,25 @@ def test_autograd_function_matches_oracle():
     assert_close_o("O", _np(out), O_ref, TOL_BF16["O"])
     for name, got, want in (("dQ", qc.grad, dQ), ("dK", kc.grad, dK), ("dV", vc.grad, dV)):
         assert_close(name, _np(got), want, grad_tol(TOL_BF16, want))
+
+
+def test_launch_plan_matches_the_measured_choices():
+    """The launch forms the host picks on a 148-SM B200 for the named shapes."""
+    props = torch.cuda.get_device_properties(0)
+    if props.multi_processor_count != 148:
+        pytest.skip("the expected plans are for 148 SMs")
+    plan = api.fa_launch_plan
+    # long rows: one CTA per forward item; more key tiles than SMs: persistent backward
+    assert plan(1, 8, 16384, 128, False) == {"fwd_persistent": False, "bwd_persistent": True,
+                                             "bwd_split": 0}
+    # GPT-2 shape: short causal rows run persistent in both directions
+    assert plan(8, 12, 1024, 64, True) == {"fwd_persistent": True, "bwd_persistent": True,
+                                           "bwd_split": 0}
+    # 512 key tiles of 64 steps: 68 split over two CTAs each, one CTA per tile
+    assert plan(1, 8, 8192, 128, False) == {"fwd_persistent": False, "bwd_persistent": False,
+                                            "bwd_split": 68}
+    # 256 items/tiles: the forward's 128 pairs fill one wave; the backward is persistent
+    assert plan(1, 8, 4096, 128, False) == {"fwd_persistent": False, "bwd_persistent": True,
+                                            "bwd_split": 0}
+    assert plan(1, 8, 0, 128, False) == {"fwd_persistent": False, "bwd_persistent": False,
+                                         "bwd_split": 0}
