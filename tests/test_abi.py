@@ -40,6 +40,19 @@ def test_binding_covers_the_header():
     assert set(declared_functions()) == set(_lib.SIGNATURES)
 
 
+def test_launch_plan_refuses_bad_shapes_before_any_device_call(libfa):
+    """fa_launch_plan validates the shape first: a refused shape returns its status
+    without touching a GPU (this host has none) and writes no output."""
+    f = _fn(libfa, "fa_launch_plan")
+    out = [ctypes.c_int(-7) for _ in range(3)]
+    ptrs = [ctypes.addressof(o) for o in out]
+    assert f(1, 1, 100, 96, 0, *ptrs) == 2        # d = 96: FA_ERR_UNSUPPORTED
+    assert f(0, 1, 100, 64, 0, *ptrs) == 1        # B = 0
+    assert f(1, 1, 100, 64, 2, *ptrs) == 1        # causal must be 0 or 1
+    assert f(1, 1, 2**30 + 1, 64, 0, *ptrs) == 2  # N beyond 2^30: FA_ERR_UNSUPPORTED
+    assert [o.value for o in out] == [-7, -7, -7]
+
+
 def test_host_only_entry_points(libfa):
     libfa.fa_version.restype = ctypes.c_char_p
     assert b"sm_100a" in libfa.fa_version()
