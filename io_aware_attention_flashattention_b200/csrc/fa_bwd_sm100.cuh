@@ -14,10 +14,12 @@
 //      rows, and rows that see no key (LSE = -inf), get L2 = +inf so that they
 //      contribute nothing), and zero the fp32 dQ accumulator.
 //   2. fa_bwd_kernel (one CTA per SM, 512 threads): the CTA owns one tile of 128
-//      keys K_j, V_j and streams the query tiles Q_i, dO_i (128 rows) through a
-//      ring of shared-memory slots with TMA. Each query tile is processed as two
-//      halves of 64 queries (h = 0, 1) so that the MMAs of one half overlap the
-//      elementwise work of the other.
+//      keys K_j, V_j (or, for a split tile, half of its query tiles) and streams the
+//      query tiles Q_i, dO_i (128 rows) through a ring of shared-memory slots with
+//      TMA. Each query tile is processed as two halves of 64 queries (h = 0, 1) so
+//      that the MMAs of one half overlap the elementwise work of the other.
+//      fa_bwd_persistent_kernel, at the end of this file, runs the same roles over a
+//      list of key tiles per CTA.
 //        warp 13 (MMA, one thread), per half h: S^T_h = K_j Q_ih^T and
 //          dP^T_h = V_j dO_ih^T into TMEM; dV += P^T_h dO_ih and dK += dS^T_h Q_ih
 //          with P^T_h and dS^T_h read from TMEM; for D = 128, dQ^T_h = K_j^T dS^T_h
