@@ -178,13 +178,16 @@ __device__ __forceinline__ bool softmax_key_tile(const Params& p, const Watchdog
                                                  uint32_t tm_s, uint32_t tm_o, uint8_t* p_row,
                                                  uint32_t bar_sfree, uint32_t bar_pvdone,
                                                  uint32_t bar_pfull, int n, bool first, int kt,
-                                                 int r0, int row, int row_in_tile, int k_lo,
-                                                 int k_hi, int wl, int wr, int bh, int lane,
+                                                 int r0, int row, int row_in_tile, int wl,
+                                                 int wr, int bh, int lane,
                                                  int wq, int t, float& m_ref, float& l,
                                                  float& lr) {
   using C = Cfg<D>;
   const float c = p.scale_log2;
   const int r1 = r0 + BM - 1;
+  // visible keys of this row: [k_lo, k_hi)
+  const int k_lo = (wl < 0) ? 0 : row - wl;
+  const int k_hi = (wr < 0) ? p.N : min(p.N, row + wr + 1);
   tc_fence_after();
   uint32_t s[4][32];
 #pragma unroll
@@ -598,9 +601,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       return blocks == nullptr || ((t_bits[kt >> 5] >> (kt & 31)) & 1u);
     };
     bool ok = t_nk > 0;
-    // visible keys of this row: [k_lo, k_hi)
-    const int k_lo = (wl < 0) ? 0 : row - wl;
-    const int k_hi = (wr < 0) ? p.N : min(p.N, row + wr + 1);
     int kt = t_lo - 1;
     for (int j = 0; j < t_nk && ok; ++j) {
       do ++kt; while (!t_member(kt));
@@ -611,7 +611,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       if (!softmax_key_tile<D, E, kDropout>(p, wd, tm_s, tm_o, p_row, bar(C::kBarSFree + t),
                                             bar(C::kBarPVDone + t), bar(C::kBarPFull + t), j,
-                                            j == 0, kt, r0, row, row_in_tile, k_lo, k_hi, wl,
+                                            j == 0, kt, r0, row, row_in_tile, wl,
                                             wr, bh, lane, wq, t, m_ref, l, lr)) {
         ok = false;
         break;
@@ -981,9 +981,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int t_lo = t ? w.lo[1] : w.lo[0], t_hi = t ? w.hi[1] : w.hi[0];
       const int t_nk = t ? w.nk[1] : w.nk[0];
       auto t_member = [&](int kt) -> bool { return kt >= t_lo && kt < t_hi; };
-      // visible keys of this row: [k_lo, k_hi)
-      const int k_lo = (wl < 0) ? 0 : row - wl;
-      const int k_hi = (wr < 0) ? p.N : min(p.N, row + wr + 1);
       int kt = t_lo - 1;
       for (int j = 0; j < t_nk && ok; ++j) {
         do ++kt; while (!t_member(kt));
@@ -996,7 +993,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         if (!softmax_key_tile<D, E, kDropout>(p, wd, tm_s, tm_o, p_row, bar(C::kBarSFree + t),
                                               bar(C::kBarPVDone + t), bar(C::kBarPFull + t),
-                                              n, j == 0, kt, r0, row, row_in_tile, k_lo, k_hi,
+                                              n, j == 0, kt, r0, row, row_in_tile,
                                               wl, wr, bh, lane, wq, t, m_ref, l, lr)) {
           ok = false;
           break;
