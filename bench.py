@@ -294,6 +294,25 @@ def oracle_sample(w, seconds: float, rng_seed: int = 0, inputs=None):
     return flops, dt, R, oracle.num_threads()
 
 
+def oracle_one_thread(seconds: float = 1.5) -> dict:
+    """The oracle on one host thread, on the two small workloads (the fp32 oracle-scale
+    one and the GPT-2 shape): TFLOP/s of a bounded row sample each, for comparison with
+    the all-core figure."""
+    import oracle
+    from io_aware_attention_flashattention_b200.inputs import WORKLOADS
+
+    n = oracle.num_threads()
+    out = {}
+    try:
+        oracle.default().set_num_threads(1)
+        for name in ("oracle_f32_n256_d64", "gpt2_causal_b8h12_n1024_d64"):
+            f, t, R, _ = oracle_sample(WORKLOADS[name], seconds, rng_seed=7)
+            out[name] = {"value": f / t / 1e12, "rows": R, "seconds": round(t, 2)}
+    finally:
+        oracle.default().set_num_threads(n)
+    return out
+
+
 def reference_arm(args, w):
     """--impl reference: the oracle on the host cores, each step a bounded sample."""
     rank = int(os.environ.get("RANK", "0"))
@@ -686,7 +705,8 @@ def main():
         f, t, R, threads = oracle_sample(w, args.cpu_seconds)
         cpu = {"value": f / t / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
                "sample": f"{R} random (head, query row) pairs of {w.name}, all visible keys: "
-                         f"oracle forward rows + dQ rows, fp64, {t:.1f} s"}
+                         f"oracle forward rows + dQ rows, fp64, {t:.1f} s",
+               "one_thread": oracle_one_thread()}
 
     if world > 1:
         barrier()
