@@ -221,6 +221,8 @@ __global__ void __launch_bounds__(256)
                       const float* __restrict__ LSE, float* __restrict__ L2,
                       float* __restrict__ Dv, float* __restrict__ dQacc, int N, int Npad,
                       long long total_rows, unsigned* __restrict__ arrivals, int n_arrivals) {
+  pdl_wait();  // the grid before this one (the forward) has completed
+  pdl_launch_dependents();
   if (blockIdx.x == 0)  // the main kernel's arrival counters of split tiles
     for (int k = threadIdx.x; k < n_arrivals; k += blockDim.x) arrivals[k] = 0u;
   const long long r = static_cast<long long>(blockIdx.x) * 8 + (threadIdx.x >> 5);
@@ -268,6 +270,8 @@ template <int D, Elt E>
 __global__ void __launch_bounds__(256)
     fa_bwd_dq_kernel(const float* __restrict__ dQacc, uint16_t* __restrict__ dQ, long long n4,
                      float scale) {
+  pdl_wait();  // the grid before this one (the main kernel) has completed
+  pdl_launch_dependents();
   for (long long k = static_cast<long long>(blockIdx.x) * blockDim.x + threadIdx.x; k < n4;
        k += static_cast<long long>(gridDim.x) * blockDim.x) {
     const float4 v = reinterpret_cast<const float4*>(dQacc)[k];
@@ -421,6 +425,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // The block-mask column of this key tile as bits: warp w builds words w, w + 16, ...
   uint32_t* mask_bits = reinterpret_cast<uint32_t*>(base_ptr + C::kMaskOff);
+  if (blocks != nullptr) pdl_wait();  // the mask may come from the grid before
   if (blocks != nullptr) {
     for (int wi = warp; wi < (n_q + 31) / 32; wi += kThreads / 32) {
       const int i = wi * 32 + lane;
@@ -457,6 +462,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // the grid before this one has completed: global memory is ours
   const Watchdog wd{abort_flag, p.timeout_ns};
   if (threadIdx.x == 0) FA_TRACE_CTA(1);
   if (warp == kWarpMma) FA_TRACE_POINT(0, 0, 0);
@@ -811,6 +817,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0) FA_TRACE_CTA(4);
+  pdl_launch_dependents();  // the next grid may launch: this CTA's work is done
   if (warp == kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmCols);
@@ -896,6 +903,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // the grid before this one has completed: global memory is ours
   const Watchdog wd{abort_flag, p.timeout_ns};
   if (threadIdx.x == 0) FA_TRACE_CTA(1);
 
@@ -1216,6 +1224,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0) FA_TRACE_CTA(4);
+  pdl_launch_dependents();  // the next grid may launch: this CTA's work is done
   if (warp == kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmCols);

@@ -388,6 +388,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   // Block mask rows of the two query tiles as bits in shared memory: warp w builds
   // words w, w + 11, ... with one byte per lane and a ballot.
   uint32_t* mask_bits = reinterpret_cast<uint32_t*>(base_ptr + C::kMaskOff);
+  if (blocks != nullptr) pdl_wait();  // the mask may come from the grid before
   if (blocks != nullptr) {
     const int nwords = (n_kt + 31) / 32;
     for (int w = warp; w < 2 * nwords; w += kThreads / 32) {
@@ -428,6 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // the grid before this one has completed: global memory is ours
   const Watchdog wd{abort_flag, p.timeout_ns};
   if (threadIdx.x == 0) FA_TRACE_CTA(1);
 
@@ -657,6 +659,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0) FA_TRACE_CTA(4);
+  pdl_launch_dependents();  // the next grid may launch: this CTA's work is done
   if (warp == kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmCols);
@@ -773,6 +776,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  pdl_wait();  // the grid before this one has completed: global memory is ours
   const Watchdog wd{abort_flag, p.timeout_ns};
   if (threadIdx.x == 0) FA_TRACE_CTA(1);
 
@@ -1051,6 +1055,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   if (threadIdx.x == 0) FA_TRACE_CTA(4);
+  pdl_launch_dependents();  // the next grid may launch: this CTA's work is done
   if (warp == kWarpMma) {
     tc_fence_after();
     tmem_dealloc(tmem, C::kTmCols);

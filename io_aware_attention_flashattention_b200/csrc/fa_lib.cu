@@ -32,6 +32,8 @@ namespace {
 __global__ void watchdog_selftest_kernel(unsigned long long timeout_ns) {
   __shared__ __align__(8) uint64_t bar;
   __shared__ int abort_flag;
+  pdl_wait();  // the status word is written below
+  pdl_launch_dependents();
   if (threadIdx.x == 0) {
     mbar_init(smem_u32(&bar), 1);
     abort_flag = 0;
@@ -123,15 +125,22 @@ std::mutex g_mutex;
 // Launches `kernel` and returns the status of this launch alone: an error left
 // pending by earlier, unrelated CUDA work is neither reported nor cleared. A
 // failed launch's own error is cleared, so that it does not surface later in the
-// caller's error checks.
+// caller's error checks. Launches allow programmatic stream serialization: the
+// kernel's set-up may overlap the tail of the kernel before it on the stream, and
+// every kernel waits for that one (pdl_wait) before touching global memory.
 template <typename... KArgs, typename... Args>
 fa_status launch(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
                  Args&&... args) {
+  cudaLaunchAttribute attr[1] = {};
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = grid;
   cfg.blockDim = block;
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
   if (e == cudaSuccess) return FA_OK;
   (void)cudaGetLastError();

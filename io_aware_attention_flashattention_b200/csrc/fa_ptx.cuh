@@ -178,6 +178,18 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
+// Programmatic dependent launch. Every kernel of this library is launched with
+// programmatic stream serialization, so it may start while the grid before it on
+// the stream is still running. pdl_wait blocks the calling thread until that grid
+// has completed and its memory writes are visible (at once when there is no such
+// grid); each kernel calls it before its first global memory access, read or write.
+// pdl_launch_dependents lets the grid after this one start launching once every CTA
+// of this grid has called it or exited; its CTAs then run their set-up and wait.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // Makes the mbarrier track completion of all prior tcgen05.mma of this thread.
 __device__ __forceinline__ void tc_commit(uint32_t bar) {
   asm volatile(

@@ -18,6 +18,8 @@
 #include <math.h>
 #include <stdint.h>
 
+#include "fa_ptx.cuh"  // pdl_wait, pdl_launch_dependents
+
 namespace fa {
 namespace f32 {
 
@@ -57,6 +59,8 @@ __global__ void __launch_bounds__(kWarps * 32)
     fa_f32_fwd_kernel(const float* __restrict__ Q, const float* __restrict__ K,
                       const float* __restrict__ V, float* __restrict__ O, float* __restrict__ LSE,
                       int N, float scale, int causal) {
+  pdl_wait();  // the grid before this one has completed
+  pdl_launch_dependents();
   constexpr int P = D + 4;
   constexpr int CPL = D / 32;  // output columns per lane
   __shared__ __align__(16) float sQ[kRowsPerBlock * P];
@@ -149,6 +153,8 @@ template <int D>
 __global__ void __launch_bounds__(kWarps * 32)
     fa_f32_bwd_dot_kernel(const float* __restrict__ O, const float* __restrict__ dO,
                           float* __restrict__ Dvec, long long rows) {
+  pdl_wait();  // the grid before this one has completed
+  pdl_launch_dependents();
   const long long r = static_cast<long long>(blockIdx.x) * kWarps + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (r >= rows) return;
@@ -167,6 +173,8 @@ __global__ void __launch_bounds__(kWarps * 32)
                            const float* __restrict__ LSE, const float* __restrict__ Dvec,
                            float* __restrict__ dK, float* __restrict__ dV, int N, float scale,
                            int causal) {
+  pdl_wait();  // the grid before this one has completed
+  pdl_launch_dependents();
   constexpr int P = D + 4;
   constexpr int CPL = D / 32;
   extern __shared__ __align__(16) float dsm[];  // dkdv_smem_bytes<D>() bytes
@@ -255,6 +263,8 @@ __global__ void __launch_bounds__(kWarps * 32)
                          const float* __restrict__ V, const float* __restrict__ dO,
                          const float* __restrict__ LSE, const float* __restrict__ Dvec,
                          float* __restrict__ dQ, int N, float scale, int causal) {
+  pdl_wait();  // the grid before this one has completed
+  pdl_launch_dependents();
   constexpr int P = D + 4;
   constexpr int CPL = D / 32;
   extern __shared__ __align__(16) float dsm[];  // dq_smem_bytes<D>() bytes
