@@ -31,6 +31,14 @@
  *   - Calls are asynchronous on `stream` (0 = the legacy default stream).
  *     Argument errors are returned synchronously and launch nothing. A failed
  *     launch returns FA_ERR_CUDA.
+ *   - Stream order holds as for any kernel. The library's kernels are launched
+ *     with programmatic stream serialization: each may be placed while the
+ *     kernel before it on the stream finishes, and waits for that kernel
+ *     (griddepcontrol.wait) before touching global memory. A kernel of the
+ *     caller's that follows on the stream and is itself launched with that
+ *     attribute may start once the library kernel's CTAs have done their work;
+ *     it must wait (griddepcontrol.wait / cudaGridDependencySynchronize) before
+ *     reading the call's outputs. Kernels launched without it see plain order.
  *   - Every wait inside a kernel is bounded (default 5 s; the environment
  *     variable FA_WATCHDOG_MS, read once per process, overrides it). A wait that
  *     runs out makes the kernel record the error in the device status word and
