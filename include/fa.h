@@ -236,6 +236,43 @@ fa_status fa_forward_dropout(const void* Q, const void* K, const void* V, void* 
                              int B, int H, int N, int d, float scale, int causal,
                              int window_left, int window_right, const uint8_t* block_mask,
                              float p_drop, uint64_t seed, uint32_t offset, fa_stream_t stream);
+fa_status fa_backward_dropout(const void* Q, const void* K, const void* V, const void* O,
+                              const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
+                              int B, int H, int N, int d, float scale, int causal,
+                              int window_left, int window_right, const uint8_t* block_mask,
+                              float p_drop, uint64_t seed, uint32_t offset, void* workspace,
+                              size_t workspace_bytes, fa_stream_t stream);
+
+/*
+ * The dropout calls for a range of a larger problem's heads: the Philox counter's
+ * third word is head_base + b * H + h instead of b * H + h, so a call on the flattened
+ * heads [head_base, head_base + B * H) of a [B', H', N, d] problem (given as a
+ * [1, B * H, N, d] slice, or any B, H with that product) draws exactly the keep masks
+ * the whole call draws for those heads. This is what lets a problem be split by heads
+ * over several GPUs with dropout. head_base = 0 is fa_forward_dropout /
+ * fa_backward_dropout; head_base < 0 is FA_ERR_INVALID_ARG. Other arguments, errors
+ * and ownership as for those calls.
+ */
+fa_status fa_forward_dropout_heads(const void* Q, const void* K, const void* V, void* O,
+                                   float* LSE, int B, int H, int N, int d, float scale,
+                                   int causal, int window_left, int window_right,
+                                   const uint8_t* block_mask, float p_drop, uint64_t seed,
+                                   uint32_t offset, int head_base, fa_stream_t stream);
+fa_status fa_backward_dropout_heads(const void* Q, const void* K, const void* V, const void* O,
+                                    const void* dO, const float* LSE, void* dQ, void* dK,
+                                    void* dV, int B, int H, int N, int d, float scale,
+                                    int causal, int window_left, int window_right,
+                                    const uint8_t* block_mask, float p_drop, uint64_t seed,
+                                    uint32_t offset, int head_base, void* workspace,
+                                    size_t workspace_bytes, fa_stream_t stream);
+
+/*
+ * The drop probability the dropout calls apply for `p_drop`: floor(256 p_drop) / 256
+ * (for example 0.1 gives 25/256 = 0.09765625). Returns -1 for a p_drop those calls
+ * refuse (outside [0, 1), NaN, or in (0, 1/256)). Host only; no CUDA call.
+ */
+float fa_dropout_rate(float p_drop);
+
 /*
  * How the library distributes a plain call (no window, block mask or dropout) of this
  * shape on the current GPU. A planning query: it launches nothing.
@@ -250,20 +287,6 @@ fa_status fa_forward_dropout(const void* Q, const void* K, const void* V, void* 
  */
 fa_status fa_launch_plan(int B, int H, int N, int d, int causal, int* fwd_persistent,
                          int* bwd_persistent, int* bwd_split);
-
-/*
- * The drop probability the dropout calls apply for `p_drop`:/*
- * The drop probability the dropout calls apply for `p_drop`: floor(256 p_drop) / 256
- * (for example 0.1 gives 25/256 = 0.09765625). Returns -1 for a p_drop those calls
- * refuse (outside [0, 1), NaN, or in (0, 1/256)). Host only; no CUDA call.
- */
-float fa_dropout_rate(float p_drop);
-fa_status fa_backward_dropout(const void* Q, const void* K, const void* V, const void* O,
-                              const void* dO, const float* LSE, void* dQ, void* dK, void* dV,
-                              int B, int H, int N, int d, float scale, int causal,
-                              int window_left, int window_right, const uint8_t* block_mask,
-                              float p_drop, uint64_t seed, uint32_t offset, void* workspace,
-                              size_t workspace_bytes, fa_stream_t stream);
 
 /*
  * fp32 entry points: the same operation and arguments with fp32 tensors

@@ -42,6 +42,11 @@ SIGNATURES = {
     "fa_backward_dropout": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                  _i, _i, _i, _i, _f, _i, _i, _i, _vp, _f, _u64, _u32,
                                  _vp, _sz, _vp]),
+    "fa_forward_dropout_heads": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _i, _i,
+                                      _vp, _f, _u64, _u32, _i, _vp]),
+    "fa_backward_dropout_heads": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                       _i, _i, _i, _i, _f, _i, _i, _i, _vp, _f, _u64, _u32,
+                                       _i, _vp, _sz, _vp]),
     "fa_forward_f32": (_i, [_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _f, _i, _vp]),
     "fa_backward_f32": (_i, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                              _i, _i, _i, _i, _f, _i, _vp, _sz, _vp]),

@@ -184,26 +184,38 @@ def fa_dropout_rate(p: float) -> float:
 
 
 def _dropout(dropout):
+    """(p, seed, offset, head_base) from dropout = (p, seed, offset) or (p, seed, offset,
+    head_base); head_base (default 0) as for fa_forward_dropout_heads."""
     if dropout is None:
-        return 0.0, 0, 0
-    p, seed, offset = dropout
-    return float(p), int(seed) & ((1 << 64) - 1), int(offset) & 0xFFFFFFFF
+        return 0.0, 0, 0, 0
+    p, seed, offset, *rest = dropout
+    if len(rest) > 1:
+        raise ValueError("dropout is (p, seed, offset) or (p, seed, offset, head_base)")
+    head_base = int(rest[0]) if rest else 0
+    return float(p), int(seed) & ((1 << 64) - 1), int(offset) & 0xFFFFFFFF, head_base
 
 
 @_on_one_device
 def fa_forward_dropout(Q, K, V, O, LSE, scale: float, causal: bool, dropout, window=None,
                        block_mask=None, stream=None) -> None:
     """fa_forward_masked with dropout=(p, seed, offset) on P (Philox-4x32-10 mask, one
-    byte per element; the drop rate is p rounded down to a multiple of 1/256)."""
+    byte per element; the drop rate is p rounded down to a multiple of 1/256). A fourth
+    element, head_base, draws the masks of heads head_base + b*H + h of a larger
+    problem (fa_forward_dropout_heads)."""
     B, H, N, d = _shape(Q)
     bf = torch.bfloat16
     args = [_need("Q", Q, bf, (B, H, N, d)), _need("K", K, bf, (B, H, N, d)),
             _need("V", V, bf, (B, H, N, d)), _need("O", O, bf, (B, H, N, d)),
             _need("LSE", LSE, torch.float32, (B, H, N))]
     wl, wr = _window(window)
-    check("fa_forward_dropout", lib().fa_forward_dropout(
-        *args, B, H, N, d, float(scale), int(bool(causal)), wl, wr, _block_mask(block_mask, N),
-        *_dropout(dropout), _stream(stream)))
+    p, seed, offset, head_base = _dropout(dropout)
+    common = (*args, B, H, N, d, float(scale), int(bool(causal)), wl, wr,
+              _block_mask(block_mask, N), p, seed, offset)
+    if head_base:
+        check("fa_forward_dropout_heads",
+              lib().fa_forward_dropout_heads(*common, head_base, _stream(stream)))
+    else:
+        check("fa_forward_dropout", lib().fa_forward_dropout(*common, _stream(stream)))
 
 
 @_on_one_device
@@ -212,9 +224,15 @@ def fa_backward_dropout(Q, K, V, O, dO, LSE, dQ, dK, dV, scale: float, causal: b
     ptrs, (B, H, N, d), ws, nbytes = _bwd_args(Q, K, V, O, dO, LSE, dQ, dK, dV, workspace,
                                                torch.bfloat16)
     wl, wr = _window(window)
-    check("fa_backward_dropout", lib().fa_backward_dropout(
-        *ptrs, B, H, N, d, float(scale), int(bool(causal)), wl, wr, _block_mask(block_mask, N),
-        *_dropout(dropout), ws, nbytes, _stream(stream)))
+    p, seed, offset, head_base = _dropout(dropout)
+    common = (*ptrs, B, H, N, d, float(scale), int(bool(causal)), wl, wr,
+              _block_mask(block_mask, N), p, seed, offset)
+    if head_base:
+        check("fa_backward_dropout_heads", lib().fa_backward_dropout_heads(
+            *common, head_base, ws, nbytes, _stream(stream)))
+    else:
+        check("fa_backward_dropout", lib().fa_backward_dropout(
+            *common, ws, nbytes, _stream(stream)))
 
 
 @_on_one_device

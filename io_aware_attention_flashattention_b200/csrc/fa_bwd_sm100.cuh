@@ -287,10 +287,12 @@ __global__ void __launch_bounds__(256)
 // for dV and P o (dP o Z s - D) for dS), both back to TMEM as 16-bit pairs over the
 // columns they came from, and dS also into the swizzled shared chunk (the dQ operand).
 // kM: test each query against the key's visible range [q_lo, q_hi): query qh0 + x is
-// visible iff qoff + x < q_span (unsigned).
+// visible iff qoff + x < q_span (unsigned). ctr_head: the dropout counter's head word
+// (the call's head_base + the flattened head).
 template <Elt E, bool kDropout, bool kM>
 __device__ __forceinline__ void p_ds_half(uint32_t tm_s, uint32_t tm_dp, const float4* Lv,
-                                          const float4* Dv4, float c, int key, int qh0, int bh,
+                                          const float4* Dv4, float c, int key, int qh0,
+                                          uint32_t ctr_head,
                                           const DropoutParams& drop, int lane, int qoff,
                                           unsigned q_span, uint8_t* ds_row, int krow) {
   uint32_t sv[2][16], dv[2][16];
@@ -316,7 +318,7 @@ __device__ __forceinline__ void p_ds_half(uint32_t tm_s, uint32_t tm_dp, const f
       const uint4 w = philox4x32_10(
           make_uint4(static_cast<uint32_t>(key >> 2),
                      static_cast<uint32_t>(((qh0 + cc * 16) >> 2) + u),
-                     static_cast<uint32_t>(bh), drop.offset),
+                     ctr_head, drop.offset),
           drop.seed_lo, drop.seed_hi);
       const uint32_t t0 = __byte_perm(w.x, w.y, 0x5140), t1 = __byte_perm(w.x, w.y, 0x7362);
       const uint32_t t2 = __byte_perm(w.z, w.w, 0x5140), t3 = __byte_perm(w.z, w.w, 0x7362);
@@ -622,6 +624,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q_lo = (wr < 0) ? 0 : key - wr;
     const int q_hi = (key >= p.N) ? q_lo : ((wl < 0) ? p.Npad + BM : key + wl + 1);
     const unsigned q_span = static_cast<unsigned>(q_hi - q_lo);
+    const uint32_t ctr_head = p.drop.head_base + static_cast<uint32_t>(bh);  // dropout
     bool ok = true;
     int i = i_lo - 1;
     for (int s = 0; s < nsteps && ok; ++s) {
@@ -653,11 +656,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       // The element loop in two compiled forms: with the mask tests only on steps
       // that cross a mask edge, none on all the others.
       if (mask)
-        p_ds_half<E, kDropout, true>(tm_s, tm_dp, Lv, Dv4, c, key, qh0, bh, p.drop, lane, qoff,
-                                     q_span, ds_row, krow);
+        p_ds_half<E, kDropout, true>(tm_s, tm_dp, Lv, Dv4, c, key, qh0, ctr_head, p.drop, lane,
+                                     qoff, q_span, ds_row, krow);
       else
-        p_ds_half<E, kDropout, false>(tm_s, tm_dp, Lv, Dv4, c, key, qh0, bh, p.drop, lane, qoff,
-                                      q_span, ds_row, krow);
+        p_ds_half<E, kDropout, false>(tm_s, tm_dp, Lv, Dv4, c, key, qh0, ctr_head, p.drop, lane,
+                                      qoff, q_span, ds_row, krow);
       tmem_wait_st();
       fence_proxy_async_smem();
       tc_fence_before();
@@ -1097,6 +1100,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int q_lo = (wr < 0) ? 0 : key - wr;
       const int q_hi = (key >= p.N) ? q_lo : ((wl < 0) ? p.Npad + BM : key + wl + 1);
       const unsigned q_span = static_cast<unsigned>(q_hi - q_lo);
+      const uint32_t ctr_head = p.drop.head_base + static_cast<uint32_t>(w.bh);  // dropout
       for (int s = 0; s < nsteps && ok; ++s) {
         const int g = g0 + s;
         const int qh0 = (w.i_lo + s) * BM + 64 * h;  // first query of this half
@@ -1117,10 +1121,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                           (wl >= 0 && w.k0 + wl < qh0 + 63);
         const int qoff = qh0 - q_lo;
         if (mask)
-          p_ds_half<E, kDropout, true>(tm_s, tm_dp, Lv, Dv4, c, key, qh0, w.bh, p.drop, lane,
+          p_ds_half<E, kDropout, true>(tm_s, tm_dp, Lv, Dv4, c, key, qh0, ctr_head, p.drop, lane,
                                        qoff, q_span, ds_row, krow);
         else
-          p_ds_half<E, kDropout, false>(tm_s, tm_dp, Lv, Dv4, c, key, qh0, w.bh, p.drop, lane,
+          p_ds_half<E, kDropout, false>(tm_s, tm_dp, Lv, Dv4, c, key, qh0, ctr_head, p.drop, lane,
                                         qoff, q_span, ds_row, krow);
         tmem_wait_st();
         fence_proxy_async_smem();

@@ -179,7 +179,7 @@ __device__ __forceinline__ bool softmax_key_tile(const Params& p, const Watchdog
                                                  uint32_t bar_sfree, uint32_t bar_pvdone,
                                                  uint32_t bar_pfull, int n, bool first, int kt,
                                                  int r0, int row, int row_in_tile, int wl,
-                                                 int wr, int bh, int lane,
+                                                 int wr, uint32_t ctr_head, int lane,
                                                  int wq, int t, float& m_ref, float& l,
                                                  float& lr) {
   using C = Cfg<D>;
@@ -278,8 +278,7 @@ __device__ __forceinline__ bool softmax_key_tile(const Params& p, const Watchdog
           const int u = lane & 3;
           const uint4 w = philox4x32_10(
               make_uint4(static_cast<uint32_t>(((kv0 + 32 * cc + 2 * k) >> 2) + u),
-                         static_cast<uint32_t>(row >> 2), static_cast<uint32_t>(bh),
-                         p.drop.offset),
+                         static_cast<uint32_t>(row >> 2), ctr_head, p.drop.offset),
               p.drop.seed_lo, p.drop.seed_hi);
           zw[0] = w.x;
           zw[1] = w.y;
@@ -602,6 +601,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (kt < t_lo || kt >= t_hi) return false;
       return blocks == nullptr || ((t_bits[kt >> 5] >> (kt & 31)) & 1u);
     };
+    // the dropout counter's head word: the call's head_base + the flattened head
+    const uint32_t ctr_head = p.drop.head_base + static_cast<uint32_t>(bh);
     bool ok = t_nk > 0;
     int kt = t_lo - 1;
     for (int j = 0; j < t_nk && ok; ++j) {
@@ -614,7 +615,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!softmax_key_tile<D, E, kDropout>(p, wd, tm_s, tm_o, p_row, bar(C::kBarSFree + t),
                                             bar(C::kBarPVDone + t), bar(C::kBarPFull + t), j,
                                             j == 0, kt, r0, row, row_in_tile, wl,
-                                            wr, bh, lane, wq, t, m_ref, l, lr)) {
+                                            wr, ctr_head, lane, wq, t, m_ref, l, lr)) {
         ok = false;
         break;
       }
@@ -971,6 +972,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       Work w;
       decode(item, w);
       const int bh = w.bh;
+      const uint32_t ctr_head = p.drop.head_base + static_cast<uint32_t>(bh);  // dropout
       const int r0 = w.q0 + t * BM;
       const int row = r0 + row_in_tile;
       float m_ref = -INFINITY;
@@ -998,7 +1000,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!softmax_key_tile<D, E, kDropout>(p, wd, tm_s, tm_o, p_row, bar(C::kBarSFree + t),
                                               bar(C::kBarPVDone + t), bar(C::kBarPFull + t),
                                               n, j == 0, kt, r0, row, row_in_tile,
-                                              wl, wr, bh, lane, wq, t, m_ref, l, lr)) {
+                                              wl, wr, ctr_head, lane, wq, t, m_ref, l, lr)) {
           ok = false;
           break;
         }

@@ -299,9 +299,9 @@ int drop_threshold(float p_drop) {
   return static_cast<int>(std::min(t, 255.0));
 }
 
-fa_status make_drop(float p_drop, uint64_t seed, uint32_t offset, DropSpec* d) {
+fa_status make_drop(float p_drop, uint64_t seed, uint32_t offset, int head_base, DropSpec* d) {
   const int ti = drop_threshold(p_drop);
-  if (ti < 0) return FA_ERR_INVALID_ARG;
+  if (ti < 0 || head_base < 0) return FA_ERR_INVALID_ARG;
   // A rate in (0, 1/256) has threshold 0: it would silently drop nothing.
   if (ti == 0 && p_drop > 0.0f) return FA_ERR_UNSUPPORTED;
   d->on = ti > 0;
@@ -312,6 +312,8 @@ fa_status make_drop(float p_drop, uint64_t seed, uint32_t offset, DropSpec* d) {
   d->params.seed_lo = static_cast<uint32_t>(seed);
   d->params.seed_hi = static_cast<uint32_t>(seed >> 32);
   d->params.offset = offset;
+  // head_base + bh stays below 2^31 + 2^27: the shape checks keep B*H below 2^27
+  d->params.head_base = static_cast<uint32_t>(head_base);
   return FA_OK;
 }
 
@@ -1090,9 +1092,18 @@ fa_status fa_forward_dropout(const void* Q, const void* K, const void* V, void* 
                              int B, int H, int N, int d, float scale, int causal,
                              int window_left, int window_right, const uint8_t* block_mask,
                              float p_drop, uint64_t seed, uint32_t offset, fa_stream_t stream) {
+  return fa_forward_dropout_heads(Q, K, V, O, LSE, B, H, N, d, scale, causal, window_left,
+                                  window_right, block_mask, p_drop, seed, offset, 0, stream);
+}
+
+fa_status fa_forward_dropout_heads(const void* Q, const void* K, const void* V, void* O,
+                                   float* LSE, int B, int H, int N, int d, float scale,
+                                   int causal, int window_left, int window_right,
+                                   const uint8_t* block_mask, float p_drop, uint64_t seed,
+                                   uint32_t offset, int head_base, fa_stream_t stream) {
   MaskSpec m;
   DropSpec dr;
-  fa_status st = make_drop(p_drop, seed, offset, &dr);
+  fa_status st = make_drop(p_drop, seed, offset, head_base, &dr);
   if (st != FA_OK) return st;
   if ((st = make_mask(N, causal, window_left, window_right, block_mask, &m)) != FA_OK) return st;
   return forward_impl<Elt::BF16>(Q, K, V, O, LSE, B, H, N, d, scale, causal, m, dr, stream);
@@ -1104,9 +1115,21 @@ fa_status fa_backward_dropout(const void* Q, const void* K, const void* V, const
                               int window_left, int window_right, const uint8_t* block_mask,
                               float p_drop, uint64_t seed, uint32_t offset, void* workspace,
                               size_t workspace_bytes, fa_stream_t stream) {
+  return fa_backward_dropout_heads(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, scale, causal,
+                                   window_left, window_right, block_mask, p_drop, seed, offset,
+                                   0, workspace, workspace_bytes, stream);
+}
+
+fa_status fa_backward_dropout_heads(const void* Q, const void* K, const void* V, const void* O,
+                                    const void* dO, const float* LSE, void* dQ, void* dK,
+                                    void* dV, int B, int H, int N, int d, float scale,
+                                    int causal, int window_left, int window_right,
+                                    const uint8_t* block_mask, float p_drop, uint64_t seed,
+                                    uint32_t offset, int head_base, void* workspace,
+                                    size_t workspace_bytes, fa_stream_t stream) {
   MaskSpec m;
   DropSpec dr;
-  fa_status st = make_drop(p_drop, seed, offset, &dr);
+  fa_status st = make_drop(p_drop, seed, offset, head_base, &dr);
   if (st != FA_OK) return st;
   if ((st = make_mask(N, causal, window_left, window_right, block_mask, &m)) != FA_OK) return st;
   return backward_impl<Elt::BF16>(Q, K, V, O, dO, LSE, dQ, dK, dV, B, H, N, d, scale, causal, m,

@@ -588,13 +588,15 @@ __device__ __forceinline__ void transpose4_lanes(uint32_t (&a)[4], int u) {
 }
 
 // Dropout on P: key j of query row i in head bh is kept iff byte (j mod 4) of word
-// (i mod 4) of philox4x32_10((j / 4, i / 4, bh, offset), seed) is at least
+// (i mod 4) of philox4x32_10((j / 4, i / 4, head_base + bh, offset), seed) is at least
 // `threshold` (= floor(256 p), so the drop probability is threshold / 256); kept
-// values are scaled by `scale` = 256 / (256 - threshold).
+// values are scaled by `scale` = 256 / (256 - threshold). head_base is 0 except for a
+// call on a range of a larger problem's heads, which draws that problem's masks.
 struct DropoutParams {
   uint32_t threshold;
   float scale;
   uint32_t seed_lo, seed_hi, offset;
+  uint32_t head_base;
 };
 
 }  // namespace fa

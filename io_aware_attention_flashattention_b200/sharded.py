@@ -16,8 +16,9 @@ Two forms:
     ``gather_heads`` assembles the full output on every rank when the caller wants
     it (an all-gather of outputs, outside the attention computation itself).
 
-Dropout is not offered here: its keep mask is keyed by the head index within the
-call, so a shard would draw a different mask than the unsharded call.
+Dropout: the keep mask is keyed by the head index, so each shard passes its first
+flattened head as head_base (fa_forward_dropout_heads) and draws exactly the masks
+the unsharded call draws for its heads.
 """
 from __future__ import annotations
 
@@ -73,11 +74,21 @@ def _mask_on(block_mask, dev):
     return None if block_mask is None else block_mask.to(dev, non_blocking=True)
 
 
+def _shard_dropout(dropout, a: int):
+    """The dropout tuple for the shard whose first flattened head is ``a``."""
+    if dropout is None:
+        return None
+    p, seed, offset, *rest = dropout
+    return (p, seed, offset, (int(rest[0]) if rest else 0) + a)
+
+
 def forward_sharded(q, k, v, devices, causal: bool = False, scale=None, window=None,
-                    block_mask=None):
+                    block_mask=None, dropout=None):
     """(O, LSE) of the whole problem, computed in head shards on ``devices`` (a list of
     CUDA devices; one may appear more than once). Inputs and outputs live on q's
-    device; each shard's inputs are copied to its GPU and its outputs copied back."""
+    device; each shard's inputs are copied to its GPU and its outputs copied back.
+    ``dropout`` = (p, seed, offset) as for api.forward draws the unsharded call's
+    masks."""
     devs = _devices(devices)
     B, H, N, d = q.shape
     o = torch.empty_like(q)
@@ -87,17 +98,18 @@ def forward_sharded(q, k, v, devices, causal: bool = False, scale=None, window=N
             continue
         with torch.cuda.device(dev):
             qs, ks, vs = (_piece(t, a, b, dev) for t in (q, k, v))
-            os_, ls = api.forward(qs, ks, vs, causal, scale, window, _mask_on(block_mask, dev))
+            os_, ls = api.forward(qs, ks, vs, causal, scale, window, _mask_on(block_mask, dev),
+                                  _shard_dropout(dropout, a))
             _flat(o)[a:b].copy_(os_[0], non_blocking=True)
             _flat(lse)[a:b].copy_(ls[0], non_blocking=True)
     return o, lse
 
 
 def backward_sharded(q, k, v, o, lse, do, devices, causal: bool = False, scale=None,
-                     window=None, block_mask=None):
+                     window=None, block_mask=None, dropout=None):
     """(dQ, dK, dV) of the loss <dO, O>, computed in head shards on ``devices``, with
-    the same masks as the forward. Each shard's backward workspace is allocated on
-    its own GPU."""
+    the same masks and dropout as the forward. Each shard's backward workspace is
+    allocated on its own GPU."""
     devs = _devices(devices)
     B, H, N, d = q.shape
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
@@ -108,7 +120,7 @@ def backward_sharded(q, k, v, o, lse, do, devices, causal: bool = False, scale=N
             qs, ks, vs, os_, dos = (_piece(t, a, b, dev) for t in (q, k, v, o, do))
             ls = _piece(lse, a, b, dev)
             g = api.backward(qs, ks, vs, os_, ls, dos, causal, scale, None, window,
-                             _mask_on(block_mask, dev))
+                             _mask_on(block_mask, dev), _shard_dropout(dropout, a))
             for dst, src in zip((dq, dk, dv), g):
                 _flat(dst)[a:b].copy_(src[0], non_blocking=True)
     return dq, dk, dv
@@ -118,26 +130,28 @@ class ShardedAttentionFunction(torch.autograd.Function):
     """Differentiable head-sharded attention."""
 
     @staticmethod
-    def forward(ctx, q, k, v, devices, causal=False, scale=None, window=None, block_mask=None):
+    def forward(ctx, q, k, v, devices, causal=False, scale=None, window=None, block_mask=None,
+                dropout=None):
         q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
-        o, lse = forward_sharded(q, k, v, devices, causal, scale, window, block_mask)
+        o, lse = forward_sharded(q, k, v, devices, causal, scale, window, block_mask, dropout)
         ctx.save_for_backward(q, k, v, o, lse)
-        ctx.args = (devices, causal, scale, window, block_mask)
+        ctx.args = (devices, causal, scale, window, block_mask, dropout)
         return o
 
     @staticmethod
     def backward(ctx, do):
         q, k, v, o, lse = ctx.saved_tensors
-        devices, causal, scale, window, block_mask = ctx.args
+        devices, causal, scale, window, block_mask, dropout = ctx.args
         dq, dk, dv = backward_sharded(q, k, v, o, lse, do.contiguous(), devices, causal, scale,
-                                      window, block_mask)
-        return dq, dk, dv, None, None, None, None, None
+                                      window, block_mask, dropout)
+        return dq, dk, dv, None, None, None, None, None, None
 
 
 def attention_sharded(q, k, v, devices, causal: bool = False, scale=None, window=None,
-                      block_mask=None):
+                      block_mask=None, dropout=None):
     """Differentiable attention whose heads are computed on ``devices``."""
-    return ShardedAttentionFunction.apply(q, k, v, devices, causal, scale, window, block_mask)
+    return ShardedAttentionFunction.apply(q, k, v, devices, causal, scale, window, block_mask,
+                                          dropout)
 
 
 def gather_heads(local: torch.Tensor, B: int, H: int, group=None) -> torch.Tensor:

@@ -126,6 +126,9 @@ def test_host_validation_of_every_entry_point(libfa):
         assert drop(P, P, P, P, P, 1, 1, 256, 64, 0.1, 0, -1, -1, None, p, 7, 0, None) == 1
     # a rate below 1/256 would round down to no dropout at all: refused
     assert drop(P, P, P, P, P, 1, 1, 256, 64, 0.1, 0, -1, -1, None, 0.003, 7, 0, None) == 2
+    dheads = _fn(libfa, "fa_forward_dropout_heads")
+    assert dheads(P, P, P, P, P, 1, 1, 256, 64, 0.1, 0, -1, -1, None, 0.1, 7, 0, -1, None) == 1
+    assert dheads(P, P, P, P, P, 1, 1, 256, 64, 0.1, 0, -1, -1, None, 1.5, 7, 0, 3, None) == 1
     ws = _fn(libfa, "fa_backward_workspace_size")(1, 2, 384, 64)
     bwd = _fn(libfa, "fa_backward")
     assert bwd(P, P, P, P, P, P, P, P, P, 1, 2, 384, 64, 0.1, 0, P, ws - 1, None) == 1
@@ -144,6 +147,9 @@ def test_host_validation_of_every_entry_point(libfa):
     bdrop_ok = bdrop(P, P, P, P, P, P, P, P, P, 1, 2, 384, 64, 0.1, 0, -1, -1, None, 0.001, 1, 0,
                      P, ws, None)
     assert bdrop_ok == 2
+    bheads = _fn(libfa, "fa_backward_dropout_heads")
+    assert bheads(P, P, P, P, P, P, P, P, P, 1, 2, 384, 64, 0.1, 0, -1, -1, None, 0.1, 1, 0,
+                  -5, P, ws, None) == 1
 
 
 def test_dropout_rate_is_the_byte_threshold(libfa):

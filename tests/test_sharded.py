@@ -122,3 +122,62 @@ def test_sharded_equals_unsharded_and_oracle(B, H, N, d, causal, nshards):
     out.backward(doc)
     assert torch.equal(out.detach(), o)
     assert torch.equal(ka.grad, dk) and torch.equal(va.grad, dv)
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("B,H,N,d,causal,nshards", [(1, 5, 640, 128, True, 2),
+                                                     (2, 3, 300, 64, False, 3)])
+def test_sharded_dropout_draws_the_unsharded_masks(B, H, N, d, causal, nshards):
+    """Each shard passes its first flattened head as head_base, so the sharded call
+    draws the unsharded call's keep masks: O, LSE, dK and dV bit for bit, dQ within 2
+    ulps (fp32 atomic adds); and a different head_base draws other masks."""
+    from io_aware_attention_flashattention_b200 import api
+    from io_aware_attention_flashattention_b200.sharded import (attention_sharded,
+                                                                backward_sharded,
+                                                                forward_sharded)
+    from test_gpu_parity import _np
+
+    n_gpu = torch.cuda.device_count()
+    devices = [f"cuda:{i % n_gpu}" for i in range(nshards)]
+    q, k, v, do = make_inputs(B, H, N, d, torch.bfloat16, seed=700 + N)
+    qc, kc, vc, doc = (t.cuda() for t in (q, k, v, do))
+    drop = (0.2, 4321, 9)
+    o, lse = forward_sharded(qc, kc, vc, devices, causal, dropout=drop)
+    dq, dk, dv = backward_sharded(qc, kc, vc, o, lse, doc, devices, causal, dropout=drop)
+    o1, lse1 = api.forward(qc, kc, vc, causal, dropout=drop)
+    dq1, dk1, dv1 = api.backward(qc, kc, vc, o1, lse1, doc, causal, dropout=drop)
+    torch.cuda.synchronize()
+    assert api.fa_get_status() == 0
+    for a, b in ((o, o1), (lse, lse1), (dk, dk1), (dv, dv1)):
+        assert torch.equal(a, b)
+    g, w = _np(dq), _np(dq1)
+    ulp = np.exp2(np.floor(np.log2(np.maximum(np.maximum(np.abs(g), np.abs(w)), 1e-30))) - 7)
+    assert np.all(np.abs(g - w) <= 2 * ulp + 1e-5 * np.abs(w).max())
+    # the last head alone, as its own call with head_base = its flattened index
+    last = B * H - 1
+    qs, ks, vs = (t.reshape(B * H, N, d)[last:].unsqueeze(0).contiguous() for t in (qc, kc, vc))
+    os_, _ = api.forward(qs, ks, vs, causal, dropout=drop + (last,))
+    assert torch.equal(os_[0, 0], o.reshape(B * H, N, d)[last])
+    # with head_base 0 that head draws head 0's mask instead: a different output
+    o0, _ = api.forward(qs, ks, vs, causal, dropout=drop)
+    assert not torch.equal(o0[0, 0], os_[0, 0])
+    # the autograd form
+    qa, ka, va = (t.clone().requires_grad_() for t in (qc, kc, vc))
+    out = attention_sharded(qa, ka, va, devices, causal, dropout=drop)
+    out.backward(doc)
+    assert torch.equal(out.detach(), o)
+    assert torch.equal(ka.grad, dk) and torch.equal(va.grad, dv)
+
+
+def test_dropout_tuple_takes_an_optional_head_base():
+    from io_aware_attention_flashattention_b200 import api
+    from io_aware_attention_flashattention_b200.sharded import _shard_dropout
+
+    assert api._dropout(None) == (0.0, 0, 0, 0)
+    assert api._dropout((0.1, 5, 6)) == (0.1, 5, 6, 0)
+    assert api._dropout((0.1, 5, 6, 40)) == (0.1, 5, 6, 40)
+    with pytest.raises(ValueError):
+        api._dropout((0.1, 5, 6, 1, 2))
+    assert _shard_dropout(None, 3) is None
+    assert _shard_dropout((0.1, 5, 6), 3) == (0.1, 5, 6, 3)
+    assert _shard_dropout((0.1, 5, 6, 10), 3) == (0.1, 5, 6, 13)
