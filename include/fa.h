@@ -90,8 +90,9 @@ fa_status fa_forward(const void* Q, const void* K, const void* V, void* O, float
  *   (fp32 [B,H,N,d]) + room for S split key tiles: fp32 dK and dV partials of
  *   both halves (fp32 [S,2,2,128,d]) and an arrival counter each (u32 [S]);
  *   each region rounded up to 256 bytes. S = min(T, 160) when T <= 592 and
- *   Npad >= 4096 (32 query tiles per key tile), else 0. (A launch of few key tiles runs some of them as two CTAs, one per
- *   half of the query tiles, to fill the SMs' last wave.)
+ *   Npad >= 4096 (32 query tiles per key tile), else 0. (A launch of few key
+ *   tiles runs some of them as two CTAs, one per half of the query tiles, to
+ *   fill the SMs' last wave.)
  * Returns 0 for a shape that is invalid or empty.
  */
 size_t fa_backward_workspace_size(int B, int H, int N, int d);

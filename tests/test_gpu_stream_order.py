@@ -32,7 +32,8 @@ def _assert_dq_close(got, want):
     assert torch.isfinite(g).all()
     bound = 2.0 ** -6 * w.abs() + 1e-6 * float(w.abs().max())
     worst = float(((g - w).abs() - bound).max())
-    assert worst <= 0.0, f"dQ differs from the one-call-at-a-time run by more than 2 ulp ({worst:.3e})"
+    assert worst <= 0.0, (
+        f"dQ differs from the one-call-at-a-time run by more than 2 ulp ({worst:.3e})")
 
 
 def _chain(sets, B, H, N, d, causal, sync, fwd, bwd, dtype=torch.bfloat16, **kw):
